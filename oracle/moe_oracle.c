@@ -1,0 +1,391 @@
+/*
+ * moe_oracle.c -- plain, slow, single-threaded CPU definition of one
+ * DeepSeek-V3-style MoE layer forward.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA path (combine_expert_ffn_b200/csrc),
+ * and nothing in the product path may call it.
+ *
+ * What it computes, step by step, and where each step comes from:
+ *   1. router affinity  s_i = sigmoid(x . e_i (+ o_i))   -- affinities feed
+ *      top-k gating ["MoE + Expert-Parallel Overlap (Exp08)", Implemented];
+ *      the sigmoid form is DeepSeek-V3's (that page gives the V4
+ *      Sqrt(Softplus) form, which this layer does not use).  o_i is an
+ *      optional per-expert logit offset (the skewed-load workload).
+ *   2. selection bias  b_i = s_i + bias_i  (auxiliary-loss-free balancing:
+ *      "per-expert bias updates", Exp08 Implemented) -- used to choose
+ *      experts only, never to weight them.
+ *   3. node-limited routing: experts are split into G contiguous groups
+ *      (stand-ins for nodes; "four experts per GPU", deepnotes "The real
+ *      cluster, and the mesh DeepSeek actually disclosed"); a token's experts
+ *      lie in at most M groups ("moe-node-limited-routing", opening
+ *      definition).  Group score = sum of the group's top-(K/M) biased
+ *      affinities; the M best groups are kept; ties go to the lower index.
+ *   4. top-K experts by b inside the kept groups, ordered by descending b
+ *      then ascending index; gate w_j = s_j / sum_j s_j over the K chosen
+ *      UNBIASED affinities (no routed scaling factor, no epsilon).
+ *   5. dispatch: a stable counting sort of the T*K token copies by expert
+ *      (tokens ascending inside each expert segment), with per-expert counts,
+ *      offsets and the group-to-group send matrix ("send matrices",
+ *      shivam2003 "5. Tail latency controls step time").  Source group of
+ *      token t is t / (T/G).
+ *   6. expert FFN: SwiGLU  y = W_d (SiLU(W_g x) * (W_u x)); the shared
+ *      experts are always on with weight 1 ("shared experts (always active) +
+ *      fine-grained routed experts", Exp08 Implemented).
+ *   7. combine: out_t = sum_shared FFN_s(x_t) + sum_j w_j FFN_{e_j}(x_t).
+ *
+ * Arithmetic: dot products accumulate in double from the exact bf16/fp32
+ * inputs; sigmoid and SiLU use libm exp() in double.  The selection steps
+ * (2-4) and the gate weights are done in fp32 exactly as written above, so
+ * that a GPU given the same fp32 affinities must reproduce them bit for bit.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_EBADARG 1
+#define ORC_EINDEX 2
+#define ORC_ENOMEM 3
+
+static double bf16_value(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* b_i "beats" b_j: larger value, ties to the lower index. */
+static int beats(float bi, int i, float bj, int j)
+{
+    return bi > bj || (bi == bj && i < j);
+}
+
+/* ------------------------------------------------------------------ 1 */
+/* scores[r*E + i] = sigmoid(sum_k x[rows[r], k] * e[i, k] + off[i]) for the
+ * listed token rows (rows == NULL: rows 0..n_rows-1).  Rounded once to fp32. */
+int oracle_router_scores(int n_rows, const int64_t *rows, int d, int E,
+                         const uint16_t *x, const float *e, const float *off,
+                         float *scores)
+{
+    if (n_rows < 0 || d <= 0 || E <= 0 || !x || !e || !scores)
+        return ORC_EBADARG;
+    for (int r = 0; r < n_rows; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        const uint16_t *xt = x + t * (int64_t)d;
+        for (int i = 0; i < E; ++i) {
+            const float *ei = e + (int64_t)i * d;
+            double acc = 0.0;
+            for (int k = 0; k < d; ++k)
+                acc += bf16_value(xt[k]) * (double)ei[k];
+            if (off)
+                acc += (double)off[i];
+            scores[(int64_t)r * E + i] = (float)(1.0 / (1.0 + exp(-acc)));
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ 2-4 */
+/* Node-limited top-K selection for n_rows tokens whose fp32 affinities are
+ * scores[n_rows, E].  Writes topk_idx[n_rows, K] and topk_w[n_rows, K].
+ * If group_score != NULL it also receives the fp32 group scores [n_rows, G]. */
+int oracle_select(int n_rows, int E, int G, int K, int M,
+                  const float *scores, const float *bias,
+                  int32_t *topk_idx, float *topk_w, float *group_score)
+{
+    if (n_rows < 0 || E <= 0 || G <= 0 || K <= 0 || M <= 0 || E % G || K % M)
+        return ORC_EBADARG;
+    const int gsz = E / G, kpg = K / M;
+    if (kpg > gsz || M > G || !scores || !bias || !topk_idx || !topk_w)
+        return ORC_EBADARG;
+
+    float *b = malloc(sizeof(float) * E);
+    float *gs = malloc(sizeof(float) * G);
+    char *taken = malloc(E);
+    char *gkeep = malloc(G);
+    if (!b || !gs || !taken || !gkeep) {
+        free(b); free(gs); free(taken); free(gkeep);
+        return ORC_ENOMEM;
+    }
+    for (int t = 0; t < n_rows; ++t) {
+        const float *s = scores + (int64_t)t * E;
+        /* step 2: biased affinity, one fp32 add */
+        for (int i = 0; i < E; ++i)
+            b[i] = s[i] + bias[i];
+
+        /* step 3a: group score = sum of the group's kpg largest b, added in
+         * the order they are picked (descending b, ties to lower index) */
+        memset(taken, 0, E);
+        for (int g = 0; g < G; ++g) {
+            float sum = 0.0f;
+            for (int r = 0; r < kpg; ++r) {
+                int best = -1;
+                for (int i = g * gsz; i < (g + 1) * gsz; ++i)
+                    if (!taken[i] && (best < 0 || beats(b[i], i, b[best], best)))
+                        best = i;
+                taken[best] = 1;
+                sum = (r == 0) ? b[best] : sum + b[best];
+            }
+            gs[g] = sum;
+        }
+        if (group_score)
+            memcpy(group_score + (int64_t)t * G, gs, sizeof(float) * G);
+
+        /* step 3b: keep the M best groups (ties to the lower group index) */
+        memset(gkeep, 0, G);
+        for (int r = 0; r < M; ++r) {
+            int best = -1;
+            for (int g = 0; g < G; ++g)
+                if (!gkeep[g] && (best < 0 || beats(gs[g], g, gs[best], best)))
+                    best = g;
+            gkeep[best] = 1;
+        }
+
+        /* step 4: top-K experts by b among the kept groups, in pick order */
+        memset(taken, 0, E);
+        int32_t *idx = topk_idx + (int64_t)t * K;
+        for (int j = 0; j < K; ++j) {
+            int best = -1;
+            for (int i = 0; i < E; ++i)
+                if (gkeep[i / gsz] && !taken[i] &&
+                    (best < 0 || beats(b[i], i, b[best], best)))
+                    best = i;
+            taken[best] = 1;
+            idx[j] = best;
+        }
+
+        /* gate weights over the chosen UNBIASED affinities, fp32, slot order */
+        float denom = 0.0f;
+        for (int j = 0; j < K; ++j)
+            denom += s[idx[j]];
+        for (int j = 0; j < K; ++j)
+            topk_w[(int64_t)t * K + j] = s[idx[j]] / denom;
+    }
+    free(b); free(gs); free(taken); free(gkeep);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ 5 */
+/* Stable counting-sort dispatch of the T*K copies by expert.
+ *   counts[E], offsets[E+1], send[G*G] (copies src-group -> expert-group),
+ *   send_tok[G*G] (tokens src-group -> expert-group, each token counted once
+ *   per destination group), perm_token[T*K] (token of each permuted row),
+ *   inv_perm[T*K] (row of copy (t, j)).
+ * Returns ORC_EINDEX for an expert id out of range or repeated in a token. */
+int oracle_dispatch(int T, int E, int G, int K, const int32_t *topk_idx,
+                    int32_t *counts, int32_t *offsets, int32_t *send,
+                    int32_t *send_tok, int32_t *perm_token, int32_t *inv_perm)
+{
+    if (T < 0 || E <= 0 || G <= 0 || K <= 0 || E % G || (T > 0 && T % G))
+        return ORC_EBADARG;
+    const int gsz = E / G, tpg = T > 0 ? T / G : 1;
+    for (int64_t c = 0; c < (int64_t)T * K; ++c)
+        if (topk_idx[c] < 0 || topk_idx[c] >= E)
+            return ORC_EINDEX;
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < K; ++j)
+            for (int q = 0; q < j; ++q)
+                if (topk_idx[(int64_t)t * K + j] == topk_idx[(int64_t)t * K + q])
+                    return ORC_EINDEX;
+
+    memset(counts, 0, sizeof(int32_t) * E);
+    for (int64_t c = 0; c < (int64_t)T * K; ++c)
+        counts[topk_idx[c]]++;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e)
+        offsets[e + 1] = offsets[e] + counts[e];
+
+    int32_t *cursor = malloc(sizeof(int32_t) * E);
+    char *hit = malloc(G);
+    if (!cursor || !hit) {
+        free(cursor); free(hit);
+        return ORC_ENOMEM;
+    }
+    memcpy(cursor, offsets, sizeof(int32_t) * E);
+    memset(send, 0, sizeof(int32_t) * G * G);
+    memset(send_tok, 0, sizeof(int32_t) * G * G);
+    for (int t = 0; t < T; ++t) {
+        int src = t / tpg;
+        memset(hit, 0, G);
+        for (int j = 0; j < K; ++j) {
+            int e = topk_idx[(int64_t)t * K + j];
+            int row = cursor[e]++;
+            perm_token[row] = t;
+            inv_perm[(int64_t)t * K + j] = row;
+            send[src * G + e / gsz]++;
+            hit[e / gsz] = 1;
+        }
+        for (int g = 0; g < G; ++g)
+            send_tok[src * G + g] += hit[g];
+    }
+    free(cursor); free(hit);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ 6 */
+/* One SwiGLU FFN applied to one bf16 row, added into y[d] with weight w:
+ *   y += w * Wd (SiLU(Wg x) * (Wu x)),  Wg/Wu [f_ff, d], Wd [d, ld_d] with
+ *   the f_ff columns starting at column col0 (ld_d = row stride of Wd).
+ * If round_h is set, h is rounded to bf16 (nearest even) before Wd. */
+static void swiglu_row_acc(int d, int f_ff, const uint16_t *x,
+                           const uint16_t *Wg, const uint16_t *Wu,
+                           const uint16_t *Wd, int ld_d, int col0,
+                           double w, int round_h, double *h, double *y)
+{
+    for (int f = 0; f < f_ff; ++f) {
+        double u = 0.0, v = 0.0;
+        const uint16_t *g = Wg + (int64_t)f * d, *p = Wu + (int64_t)f * d;
+        for (int k = 0; k < d; ++k) {
+            double xk = bf16_value(x[k]);
+            u += xk * bf16_value(g[k]);
+            v += xk * bf16_value(p[k]);
+        }
+        h[f] = u / (1.0 + exp(-u)) * v;
+        if (round_h) {
+            float hf = (float)h[f];
+            uint32_t bits;
+            memcpy(&bits, &hf, 4);
+            bits += 0x7FFFu + ((bits >> 16) & 1u);
+            bits &= 0xFFFF0000u;
+            memcpy(&hf, &bits, 4);
+            h[f] = hf;
+        }
+    }
+    for (int o = 0; o < d; ++o) {
+        double acc = 0.0;
+        const uint16_t *dr = Wd + (int64_t)o * ld_d + col0;
+        for (int f = 0; f < f_ff; ++f)
+            acc += h[f] * bf16_value(dr[f]);
+        y[o] += w * acc;
+    }
+}
+
+/* y[d] = FFN_e(x_row) for one routed expert (Wg/Wu [d_ff,d], Wd [d,d_ff]). */
+int oracle_ffn_row(int d, int d_ff, const uint16_t *x_row, const uint16_t *Wg,
+                   const uint16_t *Wu, const uint16_t *Wd, int round_h, double *y)
+{
+    if (d <= 0 || d_ff <= 0 || !x_row || !Wg || !Wu || !Wd || !y)
+        return ORC_EBADARG;
+    double *h = malloc(sizeof(double) * d_ff);
+    if (!h)
+        return ORC_ENOMEM;
+    memset(y, 0, sizeof(double) * d);
+    swiglu_row_acc(d, d_ff, x_row, Wg, Wu, Wd, d_ff, 0, 1.0, round_h, h, y);
+    free(h);
+    return ORC_OK;
+}
+
+/* y[d] = sum over the n_shared shared experts of FFN_s(x_row); shared
+ * weights Wsg/Wsu [n_shared, d_ff_s, d], Wsd [n_shared, d, d_ff_s]. */
+int oracle_shared_row(int d, int n_shared, int d_ff_s, const uint16_t *x_row,
+                      const uint16_t *Wsg, const uint16_t *Wsu,
+                      const uint16_t *Wsd, int round_h, double *y)
+{
+    if (d <= 0 || n_shared < 0 || d_ff_s <= 0 || !x_row || !y)
+        return ORC_EBADARG;
+    memset(y, 0, sizeof(double) * d);
+    if (n_shared == 0)
+        return ORC_OK;
+    if (!Wsg || !Wsu || !Wsd)
+        return ORC_EBADARG;
+    double *h = malloc(sizeof(double) * d_ff_s);
+    if (!h)
+        return ORC_ENOMEM;
+    for (int s = 0; s < n_shared; ++s)
+        swiglu_row_acc(d, d_ff_s, x_row,
+                       Wsg + (int64_t)s * d_ff_s * d, Wsu + (int64_t)s * d_ff_s * d,
+                       Wsd + (int64_t)s * d * d_ff_s, d_ff_s, 0, 1.0, round_h, h, y);
+    free(h);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ 7 */
+/* out[t, :] = y_shared[t, :] + sum_j w[t,j] * y_perm[inv_perm[t,j], :]
+ * in double from bf16 rows (y_shared may be NULL). */
+int oracle_combine(int T, int d, int K, int64_t n_perm_rows,
+                   const uint16_t *y_perm, const int32_t *inv_perm,
+                   const float *topk_w, const uint16_t *y_shared, double *out)
+{
+    if (T < 0 || d <= 0 || K <= 0 || !y_perm || !inv_perm || !topk_w || !out)
+        return ORC_EBADARG;
+    for (int t = 0; t < T; ++t) {
+        double *o = out + (int64_t)t * d;
+        for (int k = 0; k < d; ++k)
+            o[k] = y_shared ? bf16_value(y_shared[(int64_t)t * d + k]) : 0.0;
+        for (int j = 0; j < K; ++j) {
+            int64_t row = inv_perm[(int64_t)t * K + j];
+            if (row < 0 || row >= n_perm_rows)
+                return ORC_EINDEX;
+            double w = (double)topk_w[(int64_t)t * K + j];
+            for (int k = 0; k < d; ++k)
+                o[k] += w * bf16_value(y_perm[row * d + k]);
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ 1-7 */
+/* The whole layer for a list of token rows (routing is per token, so any
+ * sample of tokens can be evaluated alone).  Routed expert weights come as
+ * per-expert pointer arrays (Wg[e], Wu[e]: [d_ff, d]; Wd[e]: [d, d_ff]); an
+ * entry may be NULL if no listed token selects that expert.
+ * Outputs: out[n_rows, d] (double), topk_idx/topk_w [n_rows, K],
+ * scores [n_rows, E] (may be NULL). */
+int oracle_layer_rows(int n_rows, const int64_t *rows,
+                      int d, int E, int G, int K, int M, int d_ff,
+                      int n_shared, int d_ff_s,
+                      const uint16_t *x, const float *e, const float *off,
+                      const float *bias,
+                      const uint16_t *const *Wg, const uint16_t *const *Wu,
+                      const uint16_t *const *Wd,
+                      const uint16_t *Wsg, const uint16_t *Wsu, const uint16_t *Wsd,
+                      int round_h, double *out, int32_t *topk_idx, float *topk_w,
+                      float *scores_out)
+{
+    if (n_rows < 0 || !rows || !x || !e || !bias || !Wg || !Wu || !Wd || !out ||
+        !topk_idx || !topk_w)
+        return ORC_EBADARG;
+    int rc = ORC_OK;
+    float *scores = malloc(sizeof(float) * (size_t)E * (n_rows > 0 ? n_rows : 1));
+    double *y = malloc(sizeof(double) * d);
+    if (!scores || !y) {
+        rc = ORC_ENOMEM;
+        goto done;
+    }
+    rc = oracle_router_scores(n_rows, rows, d, E, x, e, off, scores);
+    if (rc)
+        goto done;
+    rc = oracle_select(n_rows, E, G, K, M, scores, bias, topk_idx, topk_w, NULL);
+    if (rc)
+        goto done;
+    for (int r = 0; r < n_rows; ++r) {
+        const uint16_t *xr = x + rows[r] * (int64_t)d;
+        double *o = out + (int64_t)r * d;
+        rc = oracle_shared_row(d, n_shared, d_ff_s, xr, Wsg, Wsu, Wsd, round_h, o);
+        if (rc)
+            goto done;
+        for (int j = 0; j < K; ++j) {
+            int ex = topk_idx[(int64_t)r * K + j];
+            if (!Wg[ex] || !Wu[ex] || !Wd[ex]) {
+                rc = ORC_EBADARG;
+                goto done;
+            }
+            rc = oracle_ffn_row(d, d_ff, xr, Wg[ex], Wu[ex], Wd[ex], round_h, y);
+            if (rc)
+                goto done;
+            double w = (double)topk_w[(int64_t)r * K + j];
+            for (int k = 0; k < d; ++k)
+                o[k] += w * y[k];
+        }
+    }
+    if (scores_out)
+        memcpy(scores_out, scores, sizeof(float) * (size_t)E * n_rows);
+done:
+    free(scores);
+    free(y);
+    return rc;
+}
