@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Throughput of the MoE layer forward on B200 (tokens/s), with rooflines.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3] [--impl ours|reference]
+
+One step = one whole layer forward (route -> dispatch -> expert FFN ->
+combine) over one batch of seeded synthetic tokens of the named workload,
+inputs resident in HBM.  The stages are issued as the four ABI calls that
+moe_forward makes, with CUDA events between them on the launching stream, so
+the timed region also yields each stage's device time.  `e2e` times the
+public moe_forward call on pinned HOST buffers with the host->device copy of
+x and the device->host copy of the output inside the timed region.
+
+Multi-GPU: the layer does not shard (one GPU per layer instance), so N > 1
+runs N independent replicas, one per rank, each on its own batch; the job's
+value is all ranks' tokens / the slowest rank's time.
+
+`--impl reference` times the CPU oracle, as it stands, on the host cores over a
+bounded sample of tokens of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200; grouped-GEMM % bf16 peak; permute/combine % HBM"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 CUDA-core peak for the router logits: 148 SMs x 128 FMA lanes x 2 FLOP x clock
+FP32_LANES = 148 * 128 * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+def algorithmic(sh):
+    """Per-token algorithmic work of each stage (bytes or FLOPs)."""
+    T, d, E, K, ff = sh.T, sh.d, sh.E, sh.K, sh.d_ff
+    shared_ff = sh.n_shared * sh.d_ff_shared
+    return {
+        # route: read x row (bf16) + write K idx/w; router weights read once per batch
+        "route_flop": 2.0 * E * d,
+        # dispatch: read x once, write K copies (bf16) + 3 int32 index words per copy
+        "dispatch_bytes": 2.0 * d * (1 + K) + 4.0 * 3 * K,
+        # expert FFN: 6 d d_ff per token-expert (gate, up, down), routed + shared
+        "ffn_flop": 6.0 * d * (ff * K + shared_ff),
+        # combine: read K y rows + y_shared + K (idx, w), write out
+        "combine_bytes": 2.0 * d * (K + 2) + 8.0 * K,
+    }
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemm_sm100.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "combine_expert_ffn_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def traffic_from_profile(sh):
+    """DRAM bytes per launch pair of the expert FFN from a committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "expert_ffn_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_sha256") != kernel_source_hash() or d.get("workload") != sh.name:
+        return None
+    return d.get("dram_bytes_per_step")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_tokens_per_s(sh, inp, n_tokens, seed_offset=0):
+    """Times the oracle (single thread) on `n_tokens` sampled tokens; returns (tok/s, seconds)."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    rows = (np.linspace(0, sh.T - 1, n_tokens).astype(np.int64) + seed_offset) % sh.T
+    x_h, e_h, b_h = inp["x"].cpu(), inp["router_w"].cpu(), inp["bias"].cpu()
+    off = inp.get("logit_offset")
+    off_h = off.cpu() if off is not None else None
+    scores = oracle.router_scores(x_h, e_h, off_h, rows=rows)
+    idx, _ = oracle.select(scores, b_h, sh.G, sh.K, sh.M)
+    g, u, d = [None] * sh.E, [None] * sh.E, [None] * sh.E
+    for e in sorted(set(int(v) for v in idx.ravel())):
+        g[e], u[e], d[e] = inp["w_gate"][e].cpu(), inp["w_up"][e].cpu(), inp["w_down"][e].cpu()
+    sg, su, sd = inp["ws_gate"].cpu(), inp["ws_up"].cpu(), inp["ws_down"].cpu()
+    t0 = time.perf_counter()
+    oracle.layer_rows(rows, sh, x_h, e_h, b_h, g, u, d, sg, su, sd, logit_offset=off_h)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt
+
+
+def run_reference(args, sh, world, rank):
+    if rank != 0:
+        return 0
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.make_inputs(sh, dev)
+    n = args.ref_tokens
+    vals, total = [], 0.0
+    for i in range(args.warmup + args.steps):
+        v, dt = oracle_tokens_per_s(sh, inp, n, seed_offset=i)
+        if i >= args.warmup:
+            vals.append(v)
+            total += dt
+    value = n * args.steps / total
+    sample = f"{n} tokens per step of the {sh.name} workload (routing + {sh.K} routed + {sh.n_shared} shared SwiGLU FFN per token), single thread"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator)",
+        "config": {"workload": sh.name, **sh.as_dict(), "tokens_per_step": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- ours
+def run_ours(args, sh, world, rank, local):
+    import combine_expert_ffn_b200 as moe
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sh_rank = sh.replace(seed=sh.seed) if world == 1 else sh
+    inp = synth.make_inputs(sh_rank, dev)
+    if world > 1 and rank > 0:   # replicas: each rank its own batch of tokens
+        inp["x"] = synth.normal(sh.seed + 1000 * rank, synth.TENSOR_IDS["x"], (sh.T, sh.d),
+                                sh.x_sigma, torch.bfloat16, dev)
+    cfg = moe.MoeConfig.of(sh)
+    ws = moe.alloc_workspace(cfg, dev)
+    o = moe.forward_outputs(cfg, dev)
+    T, K, E, G, d = sh.T, sh.K, sh.E, sh.G, sh.d
+    # stage buffers (the same intermediates moe_forward keeps in its workspace)
+    scores = torch.empty(T, E, dtype=torch.float32, device=dev)
+    perm_token = torch.empty(T * K, dtype=torch.int32, device=dev)
+    inv_perm = torch.empty(T, K, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
+    y_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
+    y_sh = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                      o["topk_idx"], o["topk_w"], scores, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_dispatch(cfg, inp["x"], o["topk_idx"], o["counts"], o["offsets"], o["send"],
+                         o["send_tok"], perm_token, inv_perm, x_perm, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        moe.moe_expert_ffn(cfg, x_perm, o["offsets"], inp["w_gate"], inp["w_up"], inp["w_down"],
+                           y_perm, inp["x"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], y_sh,
+                           ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        moe.moe_combine(cfg, y_perm, inv_perm, o["topk_w"], y_sh, o["out"], stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if moe.moe_read_device_status(ws) != moe.MOE_OK:
+        raise RuntimeError("device status after warm-up: %d" % moe.moe_read_device_status(ws))
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.25)  # let the sampler take its first sample
+    n0 = moe.moe_launch_count()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = moe.moe_launch_count() - n0
+    clk = clocks.stop()
+    barrier(world)
+    ms_total = max_over_ranks(start.elapsed_time(end), world)
+    stage_ms = {k: 0.0 for k in ("route", "dispatch", "expert_ffn", "combine")}
+    for ev in evs:
+        for j, k in enumerate(stage_ms):
+            stage_ms[k] += ev[j].elapsed_time(ev[j + 1])
+    stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
+    status = moe.moe_read_device_status(ws)
+    if status != moe.MOE_OK:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    ms_step = ms_total / args.steps
+    value = world * T * args.steps / (ms_total / 1e3)
+
+    # ---- end to end through moe_forward with pinned host buffers
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    out_dev = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_forward(cfg, x_dev, inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                        inp["w_gate"], inp["w_up"], inp["w_down"], inp["ws_gate"], inp["ws_up"],
+                        inp["ws_down"], out_dev, ws=ws, stream=stream)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    if not torch.equal(out_host, o["out"].cpu()) and world == 1:
+        raise RuntimeError("moe_forward and the staged calls disagree")
+
+    if rank != 0:
+        return 0
+
+    peaks = load_peaks()
+    alg = algorithmic(sh)
+    ffn_s = stage_ms["expert_ffn"] / 1e3
+    ffn_tflops = alg["ffn_flop"] * T / ffn_s / 1e12
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    hbm = peaks["hbm_gbs"]
+    clock_for_alu = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    route_tflops = alg["route_flop"] * T / (stage_ms["route"] / 1e3) / 1e12
+    fp32_peak = FP32_LANES * clock_for_alu * 1e6 / 1e12
+    disp_gbs = alg["dispatch_bytes"] * T / (stage_ms["dispatch"] / 1e3) / 1e9
+    comb_gbs = alg["combine_bytes"] * T / (stage_ms["combine"] / 1e3) / 1e9
+    traffic = traffic_from_profile(sh)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded counter-based generator, random-init weights)",
+        "config": {"workload": sh.name, **sh.as_dict(), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
+                         % ((3 * sh.E * sh.d * sh.d_ff + 3 * sh.n_shared * sh.d * sh.d_ff_shared) * 2 / 1e9)},
+        "roofline": {"bound": "tensor", "kernel": "expert FFN: grouped_ffn_gemm_kernel<SwiGLU> + <store> (2 launches)",
+                     "achieved": ffn_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": ffn_tflops / tensor_peak,
+                     "peak_kind": f"{peaks['source']} bf16 sustained (burst {peaks['bf16_tflops']})",
+                     "frac_of_burst": ffn_tflops / peaks["bf16_tflops"],
+                     "traffic": traffic},
+        "stages": {
+            "ms": stage_ms,
+            "route": {"bound": "alu", "achieved": route_tflops, "unit": "TFLOP/s (fp32 FMA)",
+                      "peak": fp32_peak, "frac": route_tflops / fp32_peak},
+            "dispatch": {"bound": "hbm", "achieved": disp_gbs, "unit": "GB/s", "peak": hbm,
+                         "frac": disp_gbs / hbm},
+            "combine": {"bound": "hbm", "achieved": comb_gbs, "unit": "GB/s", "peak": hbm,
+                        "frac": comb_gbs / hbm},
+        },
+        "gpu_launches": int(launches),
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
+                "d2h_bytes_per_step": T * d * 2},
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_tokens
+        v, dt = oracle_tokens_per_s(sh, inp, n)
+        line["cpu_baseline"] = {
+            "value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of the {sh.name} workload, whole layer per token, single thread, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="v3", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=24)
+    ap.add_argument("--ref-tokens", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    sh = synth.config(args.config)
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, sh, world, rank)
+        return run_ours(args, sh, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

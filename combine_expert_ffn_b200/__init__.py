@@ -1,0 +1,213 @@
+"""Python binding of libmoe, the B200 (sm_100a) MoE-layer forward library.
+
+Argument marshalling only: every function below forwards torch tensors'
+device pointers and the current CUDA stream to the C entry point of the same
+name in ``include/moe.h`` and raises :class:`MoeError` on a nonzero status.
+All arithmetic happens in the library's CUDA kernels; there is no CPU or
+PyTorch fallback.  If ``libmoe.so`` is missing the import fails -- build it
+with ``python -m combine_expert_ffn_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: run `python -m combine_expert_ffn_b200.build`")
+
+_lib = C.CDLL(LIB_PATH)
+
+STATUS = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+    3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
+    6: "MOE_ERR_DEVICE_FAULT", 7: "MOE_ERR_NO_DEVICE",
+}
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_WORKSPACE_TOO_SMALL, \
+    MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_FAULT, MOE_ERR_NO_DEVICE = range(8)
+
+EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_launch_count",
+           "moe_read_device_status", "moe_clear_device_status", "moe_route", "moe_route_select",
+           "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
+           "moe_selftest_bounded_wait")
+
+
+class MoeConfig(C.Structure):
+    """Mirror of ``moe_config``."""
+    _fields_ = [(n, C.c_int32) for n in
+                ("T", "d", "E", "G", "K", "M", "d_ff", "n_shared", "d_ff_shared")]
+
+    @classmethod
+    def of(cls, shape) -> "MoeConfig":
+        """From any object with the nine size attributes (e.g. ``synth.MoeShape``)."""
+        return cls(*(int(getattr(shape, n)) for n, _ in cls._fields_))
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn}: {STATUS.get(status, status)} ({moe_status_string(status)})")
+
+
+_P, _S, _I64 = C.c_void_p, C.c_size_t, C.c_int64
+_CP = C.POINTER(MoeConfig)
+_sig = {
+    "moe_check_config": (C.c_int, [_CP]),
+    "moe_workspace_size": (_S, [_CP]),
+    "moe_status_string": (C.c_char_p, [C.c_int]),
+    "moe_launch_count": (C.c_uint64, []),
+    "moe_read_device_status": (C.c_int, [_P, _P, _P]),
+    "moe_clear_device_status": (C.c_int, [_P, _P]),
+    "moe_route": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "moe_route_select": (C.c_int, [_CP, _P, _P, _P, _P, _P]),
+    "moe_dispatch": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "moe_expert_ffn": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "moe_combine": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
+    "moe_forward": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                              _P, _P, _P, _P, _S, _P]),
+    "moe_selftest_bounded_wait": (C.c_int, [_I64, _P, _P]),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype, _f.argtypes = _res, _args
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _cfg(cfg):
+    return C.byref(cfg if isinstance(cfg, MoeConfig) else MoeConfig.of(cfg))
+
+
+def _ok(fn, st):
+    if st != MOE_OK:
+        raise MoeError(fn, st)
+
+
+def _ws(ws):
+    return (None, 0) if ws is None else (ws.data_ptr(), ws.numel() * ws.element_size())
+
+
+# ----------------------------------------------------------------- queries
+def moe_check_config(cfg) -> int:
+    return _lib.moe_check_config(_cfg(cfg))
+
+
+def moe_workspace_size(cfg) -> int:
+    return _lib.moe_workspace_size(_cfg(cfg))
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(int(status)).decode()
+
+
+def moe_launch_count() -> int:
+    return _lib.moe_launch_count()
+
+
+def alloc_workspace(cfg, device="cuda") -> torch.Tensor:
+    """Device workspace of moe_workspace_size(cfg) bytes (torch blocks are 512-byte aligned)."""
+    n = moe_workspace_size(cfg)
+    if n == 0:
+        raise MoeError("moe_workspace_size", moe_check_config(cfg) or MOE_ERR_UNSUPPORTED_SHAPE)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def moe_read_device_status(ws, stream=None) -> int:
+    out = C.c_int32(-1)
+    _ok("moe_read_device_status", _lib.moe_read_device_status(_ptr(ws), C.byref(out), _stream(stream)))
+    return out.value
+
+
+def moe_clear_device_status(ws, stream=None) -> None:
+    _ok("moe_clear_device_status", _lib.moe_clear_device_status(_ptr(ws), _stream(stream)))
+
+
+# ----------------------------------------------------------------- stages
+def moe_route(cfg, x, router_w, logit_offset, bias, topk_idx, topk_w, scores=None, ws=None,
+              stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_route", _lib.moe_route(_cfg(cfg), _ptr(x), _ptr(router_w), _ptr(logit_offset),
+                                    _ptr(bias), _ptr(topk_idx), _ptr(topk_w), _ptr(scores), wp, wn,
+                                    _stream(stream)))
+
+
+def moe_route_select(cfg, scores, bias, topk_idx, topk_w, stream=None) -> None:
+    _ok("moe_route_select", _lib.moe_route_select(_cfg(cfg), _ptr(scores), _ptr(bias),
+                                                  _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
+
+
+def moe_dispatch(cfg, x, topk_idx, counts, offsets, send, send_tok, perm_token, inv_perm, x_perm,
+                 ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_dispatch", _lib.moe_dispatch(_cfg(cfg), _ptr(x), _ptr(topk_idx), _ptr(counts),
+                                          _ptr(offsets), _ptr(send), _ptr(send_tok),
+                                          _ptr(perm_token), _ptr(inv_perm), _ptr(x_perm), wp, wn,
+                                          _stream(stream)))
+
+
+def moe_expert_ffn(cfg, x_perm, offsets, w_gate, w_up, w_down, y_perm, x, ws_gate, ws_up, ws_down,
+                   y_shared, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_expert_ffn", _lib.moe_expert_ffn(_cfg(cfg), _ptr(x_perm), _ptr(offsets), _ptr(w_gate),
+                                              _ptr(w_up), _ptr(w_down), _ptr(y_perm), _ptr(x),
+                                              _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down),
+                                              _ptr(y_shared), wp, wn, _stream(stream)))
+
+
+def moe_combine(cfg, y_perm, inv_perm, topk_w, y_shared, out, stream=None) -> None:
+    _ok("moe_combine", _lib.moe_combine(_cfg(cfg), _ptr(y_perm), _ptr(inv_perm), _ptr(topk_w),
+                                        _ptr(y_shared), _ptr(out), _stream(stream)))
+
+
+def moe_forward(cfg, x, router_w, logit_offset, bias, w_gate, w_up, w_down, ws_gate, ws_up,
+                ws_down, out, topk_idx=None, topk_w=None, counts=None, offsets=None, send=None,
+                send_tok=None, ws=None, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_forward", _lib.moe_forward(_cfg(cfg), _ptr(x), _ptr(router_w), _ptr(logit_offset),
+                                        _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                        _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(out),
+                                        _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(offsets),
+                                        _ptr(send), _ptr(send_tok), wp, wn, _stream(stream)))
+
+
+def moe_selftest_bounded_wait(timeout_ns, ws, stream=None) -> None:
+    _ok("moe_selftest_bounded_wait",
+        _lib.moe_selftest_bounded_wait(int(timeout_ns), _ptr(ws), _stream(stream)))
+
+
+# ----------------------------------------------------------------- convenience
+def forward_outputs(cfg, device="cuda"):
+    """Allocates the outputs of moe_forward (out, topk_idx, topk_w, counts, offsets, send, send_tok)."""
+    c = cfg if isinstance(cfg, MoeConfig) else MoeConfig.of(cfg)
+    return {
+        "out": torch.empty(c.T, c.d, dtype=torch.bfloat16, device=device),
+        "topk_idx": torch.empty(c.T, c.K, dtype=torch.int32, device=device),
+        "topk_w": torch.empty(c.T, c.K, dtype=torch.float32, device=device),
+        "counts": torch.empty(c.E, dtype=torch.int32, device=device),
+        "offsets": torch.empty(c.E + 1, dtype=torch.int32, device=device),
+        "send": torch.empty(c.G, c.G, dtype=torch.int32, device=device),
+        "send_tok": torch.empty(c.G, c.G, dtype=torch.int32, device=device),
+    }

@@ -1,0 +1,318 @@
+// api.cu -- the C ABI of libmoe (declared in include/moe.h).
+//
+// Host code only: argument validation, the workspace layout, and the launch
+// sequence of each entry point.  Every compute entry point enqueues kernels
+// on the caller's stream and returns; nothing here allocates device memory,
+// synchronises, or copies between host and device (except
+// moe_read_device_status, whose purpose is that copy).
+#include <atomic>
+#include <cstring>
+
+#include "kernels.h"
+
+namespace moe {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr int64_t kWaitTimeoutNs = 2000000000LL;  // 2 s per device wait
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+    size_t status, scores, hist_t, base_t, send_part, sendtok_part;
+    size_t topk_idx, topk_w, counts, offsets, send, send_tok, perm_token, inv_perm;
+    size_t x_perm, h, y_perm, h_sh, y_sh;
+    size_t total;
+};
+
+Layout layout(const moe_config &c) {
+    Layout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes, 256);
+        return at;
+    };
+    const size_t T = (size_t)c.T, E = (size_t)c.E, K = (size_t)c.K, G = (size_t)c.G;
+    const size_t nblk = (size_t)dispatch_nblk(c.T);
+    L.status = take(256);
+    L.scores = take(4 * T * E);
+    L.hist_t = take(4 * E * nblk);
+    L.base_t = take(4 * E * nblk);
+    L.send_part = take(4 * nblk * G * G);
+    L.sendtok_part = take(4 * nblk * G * G);
+    L.topk_idx = take(4 * T * K);
+    L.topk_w = take(4 * T * K);
+    L.counts = take(4 * E);
+    L.offsets = take(4 * (E + 1));
+    L.send = take(4 * G * G);
+    L.send_tok = take(4 * G * G);
+    L.perm_token = take(4 * T * K);
+    L.inv_perm = take(4 * T * K);
+    L.x_perm = take(2 * T * K * (size_t)c.d);
+    L.h = take(2 * T * K * (size_t)c.d_ff);
+    L.y_perm = take(2 * T * K * (size_t)c.d);
+    L.h_sh = take(2 * T * (size_t)c.n_shared * (size_t)c.d_ff_shared);
+    L.y_sh = take(2 * T * (size_t)c.d);
+    L.total = off;
+    return L;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The current device must be an sm_100 part (checked once per device).
+moe_status check_device() {
+    static std::atomic<int> ok_cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_NO_DEVICE;
+    if (dev < 0 || dev >= 64) return MOE_ERR_NO_DEVICE;
+    int v = ok_cache[dev].load();
+    if (v == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return MOE_ERR_NO_DEVICE;
+        v = (major == 10 && minor == 0) ? 1 : 2;
+        ok_cache[dev].store(v);
+    }
+    return v == 1 ? MOE_OK : MOE_ERR_NO_DEVICE;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_check_config(const moe_config *c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->G <= 0 || c->K <= 0 || c->M <= 0 ||
+        c->d_ff <= 0 || c->n_shared < 0 || c->d_ff_shared < 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->E % c->G || c->K % c->M || c->M > c->G || c->K / c->M > c->E / c->G)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->K > 32 || c->E > 1024 || c->G > 64) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T % c->G) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d % 64 || c->d_ff % 64) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->n_shared > 0 && (c->d_ff_shared <= 0 || c->d_ff_shared % 64))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((int64_t)c->T * c->K >= (1LL << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((int64_t)c->n_shared * c->d_ff_shared >= (1LL << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_config *c) {
+    if (moe_check_config(c) != MOE_OK) return 0;
+    return layout(*c).total;
+}
+
+const char *moe_status_string(int s) {
+    switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument (NULL required pointer or misaligned buffer)";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported layer sizes";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than moe_workspace_size()";
+    case MOE_ERR_CUDA: return "a CUDA call failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+    case MOE_ERR_DEVICE_FAULT: return "a kernel found an invalid index in its inputs";
+    case MOE_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown status";
+    }
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+moe_status moe_read_device_status(const void *ws, int32_t *host_status, void *stream) {
+    if (!ws || !host_status) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_device();
+    if (st) return st;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemcpyAsync(host_status, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cuda_status(cudaStreamSynchronize(s));
+}
+
+moe_status moe_clear_device_status(void *ws, void *stream) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_device();
+    if (st) return st;
+    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), as_stream(stream)));
+}
+
+moe_status moe_route_select(const moe_config *c, const float *scores, const float *bias,
+                            int32_t *topk_idx, float *topk_w, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->T > 0 && (!scores || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx,
+                                           topk_w, as_stream(stream)));
+}
+
+moe_status moe_route(const moe_config *c, const void *x, const float *router_w,
+                     const float *logit_offset, const float *bias, int32_t *topk_idx,
+                     float *topk_w, float *scores, void *ws, size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->T > 0 && (!x || !router_w || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout(*c);
+    if (!scores) {
+        if (!ws) return MOE_ERR_INVALID_ARG;
+        if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+        scores = at<float>(ws, L.scores);
+    }
+    if ((st = check_device())) return st;
+    cudaStream_t s = as_stream(stream);
+    cudaError_t e = launch_router_logits(x, router_w, logit_offset, c->T, c->d, c->E, scores, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(
+        launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s));
+}
+
+moe_status moe_dispatch(const moe_config *c, const void *x, const int32_t *topk_idx,
+                        int32_t *counts, int32_t *offsets, int32_t *send, int32_t *send_tok,
+                        int32_t *perm_token, int32_t *inv_perm, void *x_perm, void *ws,
+                        size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!counts || !offsets || !send || !ws) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0 && (!topk_idx || !perm_token || !inv_perm)) return MOE_ERR_INVALID_ARG;
+    if (x_perm && (!x || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout(*c);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),
+                  at<int32_t>(ws, L.send_part), at<int32_t>(ws, L.sendtok_part)};
+    return cuda_status(launch_dispatch(x, topk_idx, c->T, c->d, c->E, c->G, c->K, counts, offsets,
+                                       send, send_tok, perm_token, inv_perm, x_perm, dw,
+                                       at<int32_t>(ws, L.status), as_stream(stream)));
+}
+
+moe_status moe_expert_ffn(const moe_config *c, const void *x_perm, const int32_t *offsets,
+                          const void *w_gate, const void *w_up, const void *w_down, void *y_perm,
+                          const void *x, const void *ws_gate, const void *ws_up,
+                          const void *ws_down, void *y_shared, void *ws, size_t ws_bytes,
+                          void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0) {
+        if (!x_perm || !offsets || !w_gate || !w_up || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
+        if (c->n_shared > 0 && (!x || !ws_gate || !ws_up || !ws_down || !y_shared))
+            return MOE_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {x_perm, w_gate, w_up, w_down, y_perm, x, ws_gate, ws_up, ws_down, y_shared};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout(*c);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    FfnArgs a{};
+    a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
+    a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
+    a.x_perm = x_perm; a.offsets = offsets;
+    a.w_gate = w_gate; a.w_up = w_up; a.w_down = w_down;
+    a.h = at<void>(ws, L.h); a.y_perm = y_perm;
+    a.x = x; a.ws_gate = ws_gate; a.ws_up = ws_up; a.ws_down = ws_down;
+    a.h_shared = at<void>(ws, L.h_sh); a.y_shared = y_shared;
+    a.status = at<int32_t>(ws, L.status);
+    a.timeout_ns = kWaitTimeoutNs;
+    return cuda_status(launch_expert_ffn(a, as_stream(stream)));
+}
+
+moe_status moe_combine(const moe_config *c, const void *y_perm, const int32_t *inv_perm,
+                       const float *topk_w, const void *y_shared, void *out, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->T > 0 && (!y_perm || !inv_perm || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_perm) || !aligned16(y_shared) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_shared, c->T, c->d, c->K,
+                                      (int64_t)c->T * c->K, out, as_stream(stream)));
+}
+
+moe_status moe_forward(const moe_config *c, const void *x, const float *router_w,
+                       const float *logit_offset, const float *bias, const void *w_gate,
+                       const void *w_up, const void *w_down, const void *ws_gate,
+                       const void *ws_up, const void *ws_down, void *out, int32_t *topk_idx,
+                       float *topk_w, int32_t *counts, int32_t *offsets, int32_t *send,
+                       int32_t *send_tok, void *ws, size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0) {
+        if (!x || !router_w || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+        if (c->n_shared > 0 && (!ws_gate || !ws_up || !ws_down)) return MOE_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout(*c);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    if (c->T == 0) return MOE_OK;
+
+    cudaStream_t s = as_stream(stream);
+    if (!topk_idx) topk_idx = at<int32_t>(ws, L.topk_idx);
+    if (!topk_w) topk_w = at<float>(ws, L.topk_w);
+    if (!counts) counts = at<int32_t>(ws, L.counts);
+    if (!offsets) offsets = at<int32_t>(ws, L.offsets);
+    if (!send) send = at<int32_t>(ws, L.send);
+    if (!send_tok) send_tok = at<int32_t>(ws, L.send_tok);
+    float *scores = at<float>(ws, L.scores);
+    int32_t *perm_token = at<int32_t>(ws, L.perm_token);
+    int32_t *inv_perm = at<int32_t>(ws, L.inv_perm);
+    void *x_perm = at<void>(ws, L.x_perm);
+    void *y_perm = at<void>(ws, L.y_perm);
+    void *y_sh = c->n_shared > 0 ? at<void>(ws, L.y_sh) : nullptr;
+    int32_t *status = at<int32_t>(ws, L.status);
+
+    if (launch_router_logits(x, router_w, logit_offset, c->T, c->d, c->E, scores, s)) return MOE_ERR_CUDA;
+    if (launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
+        return MOE_ERR_CUDA;
+    DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),
+                  at<int32_t>(ws, L.send_part), at<int32_t>(ws, L.sendtok_part)};
+    if (launch_dispatch(x, topk_idx, c->T, c->d, c->E, c->G, c->K, counts, offsets, send, send_tok,
+                        perm_token, inv_perm, x_perm, dw, status, s))
+        return MOE_ERR_CUDA;
+    FfnArgs a{};
+    a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
+    a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
+    a.x_perm = x_perm; a.offsets = offsets;
+    a.w_gate = w_gate; a.w_up = w_up; a.w_down = w_down;
+    a.h = at<void>(ws, L.h); a.y_perm = y_perm;
+    a.x = x; a.ws_gate = ws_gate; a.ws_up = ws_up; a.ws_down = ws_down;
+    a.h_shared = at<void>(ws, L.h_sh); a.y_shared = y_sh;
+    a.status = status;
+    a.timeout_ns = kWaitTimeoutNs;
+    if (launch_expert_ffn(a, s)) return MOE_ERR_CUDA;
+    return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_sh, c->T, c->d, c->K,
+                                      (int64_t)c->T * c->K, out, s));
+}
+
+moe_status moe_selftest_bounded_wait(int64_t timeout_ns, void *ws, void *stream) {
+    if (!ws || timeout_ns < 1000 || timeout_ns > 10000000000LL) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_device();
+    if (st) return st;
+    return cuda_status(launch_bounded_wait_selftest(timeout_ns, static_cast<int32_t *>(ws),
+                                                    as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,268 @@
+// dispatch.cu -- token copies -> expert-contiguous rows (stable counting sort).
+//
+// The dispatch all-to-all ("moe-node-limited-routing", "Why all to all
+// dominates MoE step time") becomes a local permutation on one GPU: the T*K
+// copies (t, j) are sorted by expert, tokens ascending inside each segment,
+// with per-expert counts and offsets and the group-to-group send matrices
+// ("send matrices", shivam2003 "5. Tail latency controls step time").
+//
+// Four kernels, none using global atomics, so every output is deterministic:
+//   count   : per 256-token block, a bitmask per expert (bit = token in the
+//             block chose it) -> block histograms + partial send matrices
+//   scan    : warp per expert, prefix over blocks -> counts, block bases;
+//             block 0 also sums the partial send matrices
+//   scatter : per block, rank of a copy = popcount of the expert's mask below
+//             its token; row = offsets[e] + base + rank -> perm, inv_perm;
+//             offsets = exclusive scan of counts (recomputed per block)
+//   gather  : x_perm[row] = x[t], reading each x row once and writing it K
+//             times with 16-byte vector accesses
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+constexpr int BLK = DISPATCH_BLOCK;       // tokens per block = threads per CTA
+constexpr int WORDS = BLK / 32;           // mask words per expert
+
+// Rebuilds the block's expert masks in smem: masks[e * WORDS + w] bit l set if
+// token (block * BLK + 32 w + l) chose expert e.  Returns nothing; flags bad
+// ids and repeated experts of a token in `status`.
+__device__ __forceinline__ void build_masks(const int32_t *__restrict__ topk_idx, int T, int E,
+                                            int K, uint32_t *masks, int32_t *status,
+                                            bool flag_errors) {
+    const int tid = threadIdx.x;
+    for (int i = tid; i < E * WORDS; i += BLK) masks[i] = 0u;
+    __syncthreads();
+    const int t = blockIdx.x * BLK + tid;
+    if (t < T) {
+        const uint32_t bit = 1u << (tid & 31);
+        const int w = tid >> 5;
+        for (int j = 0; j < K; ++j) {
+            const int e = topk_idx[(size_t)t * K + j];
+            if (e < 0 || e >= E) {
+                if (flag_errors) record_status(status, MOE_ERR_DEVICE_FAULT);
+                continue;
+            }
+            const uint32_t old = atomicOr(&masks[e * WORDS + w], bit);
+            if ((old & bit) && flag_errors) record_status(status, MOE_ERR_DEVICE_FAULT);
+        }
+    }
+    __syncthreads();
+}
+}  // namespace
+
+__global__ void __launch_bounds__(BLK)
+dispatch_count_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int G, int K,
+                      int32_t *__restrict__ hist_t, int32_t *__restrict__ send_part,
+                      int32_t *__restrict__ sendtok_part, int32_t *status) {
+    extern __shared__ uint32_t dsm[];
+    uint32_t *masks = dsm;                                   // [E * WORDS]
+    int32_t *send_s = reinterpret_cast<int32_t *>(dsm + E * WORDS);  // [G*G]
+    int32_t *sendtok_s = send_s + G * G;                     // [G*G]
+    const int tid = threadIdx.x, nblk = gridDim.x, blk = blockIdx.x;
+    for (int i = tid; i < 2 * G * G; i += BLK) send_s[i] = 0;
+    build_masks(topk_idx, T, E, K, masks, status, true);
+
+    const int t = blk * BLK + tid;
+    if (t < T) {
+        const int gsz = E / G, src = t / (T / G);
+        uint64_t hit = 0;
+        for (int j = 0; j < K; ++j) {
+            const int e = topk_idx[(size_t)t * K + j];
+            if (e < 0 || e >= E) continue;
+            const int g = e / gsz;
+            atomicAdd(&send_s[src * G + g], 1);
+            hit |= 1ull << g;
+        }
+        while (hit) {
+            const int g = __ffsll((long long)hit) - 1;
+            hit &= hit - 1;
+            atomicAdd(&sendtok_s[src * G + g], 1);
+        }
+    }
+    for (int e = tid; e < E; e += BLK) {
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < WORDS; ++w) c += __popc(masks[e * WORDS + w]);
+        hist_t[(size_t)e * nblk + blk] = c;
+    }
+    __syncthreads();
+    for (int i = tid; i < G * G; i += BLK) {
+        send_part[(size_t)blk * G * G + i] = send_s[i];
+        sendtok_part[(size_t)blk * G * G + i] = sendtok_s[i];
+    }
+}
+
+// Warp per expert: exclusive prefix of hist_t[e, :] over the blocks.
+__global__ void __launch_bounds__(256)
+dispatch_scan_kernel(const int32_t *__restrict__ hist_t, int nblk, int E, int G,
+                     const int32_t *__restrict__ send_part,
+                     const int32_t *__restrict__ sendtok_part, int32_t *__restrict__ base_t,
+                     int32_t *__restrict__ counts, int32_t *__restrict__ send,
+                     int32_t *__restrict__ send_tok) {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int e = blockIdx.x * 8 + warp;
+    if (e < E) {
+        const int32_t *h = hist_t + (size_t)e * nblk;
+        int32_t *bo = base_t + (size_t)e * nblk;
+        int carry = 0;
+        for (int b0 = 0; b0 < nblk; b0 += 32) {
+            const int b = b0 + lane;
+            const int v = b < nblk ? h[b] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (b < nblk) bo[b] = carry + incl - v;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) counts[e] = carry;
+    }
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < G * G; i += blockDim.x) {
+            int a = 0, c = 0;
+            for (int b = 0; b < nblk; ++b) {
+                a += send_part[(size_t)b * G * G + i];
+                c += sendtok_part[(size_t)b * G * G + i];
+            }
+            send[i] = a;
+            if (send_tok) send_tok[i] = c;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(BLK)
+dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int K,
+                        const int32_t *__restrict__ counts, const int32_t *__restrict__ base_t,
+                        int32_t *__restrict__ offsets, int32_t *__restrict__ perm_token,
+                        int32_t *__restrict__ inv_perm) {
+    extern __shared__ uint32_t dsm[];
+    uint32_t *masks = dsm;                                          // [E * WORDS]
+    int32_t *offs = reinterpret_cast<int32_t *>(dsm + E * WORDS);   // [E + 1]
+    int32_t *wsum = offs + E + 1;                                   // [BLK / 32]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nblk = gridDim.x, blk = blockIdx.x;
+
+    // offsets = exclusive scan of counts: each thread owns a run of experts
+    const int per = (E + BLK - 1) / BLK;
+    int run = 0;
+    for (int i = 0; i < per; ++i) {
+        const int e = tid * per + i;
+        if (e < E) run += counts[e];
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    build_masks(topk_idx, T, E, K, masks, nullptr, false);  // contains __syncthreads
+    int wpre = 0;
+    for (int w = 0; w < warp; ++w) wpre += wsum[w];
+    int acc = wpre + incl - run;
+    for (int i = 0; i < per; ++i) {
+        const int e = tid * per + i;
+        if (e < E) {
+            offs[e] = acc;
+            acc += counts[e];
+        }
+    }
+    if (tid == BLK - 1) offs[E] = wpre + incl;
+    __syncthreads();
+    if (blk == 0)
+        for (int e = tid; e <= E; e += BLK) offsets[e] = offs[e];
+
+    const int t = blk * BLK + tid;
+    if (t >= T) return;
+    const int w = tid >> 5;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j = 0; j < K; ++j) {
+        const int e = topk_idx[(size_t)t * K + j];
+        if (e < 0 || e >= E) {
+            inv_perm[(size_t)t * K + j] = -1;
+            continue;
+        }
+        int rank = __popc(masks[e * WORDS + w] & below);
+        for (int q = 0; q < w; ++q) rank += __popc(masks[e * WORDS + q]);
+        const int row = offs[e] + base_t[(size_t)e * nblk + blk] + rank;
+        perm_token[row] = t;
+        inv_perm[(size_t)t * K + j] = row;
+    }
+}
+
+// Thread per 16-byte chunk of a token row: one load, K stores.
+__global__ void __launch_bounds__(256)
+dispatch_gather_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ inv_perm, int T,
+                       int chunks, int K, int64_t n_rows, uint4 *__restrict__ x_perm) {
+    const int64_t total = (int64_t)T * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        const uint4 v = __ldg(x + i);
+        for (int j = 0; j < K; ++j) {
+            const int row = __ldg(inv_perm + t * K + j);
+            if (row >= 0 && row < n_rows) x_perm[(int64_t)row * chunks + c] = v;
+        }
+    }
+}
+
+cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d, int E, int G,
+                            int K, int32_t *counts, int32_t *offsets, int32_t *send,
+                            int32_t *send_tok, int32_t *perm_token, int32_t *inv_perm,
+                            void *x_perm, const DispatchWs &ws, int32_t *status, cudaStream_t st) {
+    const int nblk = dispatch_nblk(T);
+    cudaError_t err;
+    if (T == 0) {
+        // no copies: zero the outputs that still have entries
+        if ((err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st))) return err;
+        if ((err = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st))) return err;
+        if ((err = cudaMemsetAsync(send, 0, sizeof(int32_t) * G * G, st))) return err;
+        if (send_tok && (err = cudaMemsetAsync(send_tok, 0, sizeof(int32_t) * G * G, st))) return err;
+        return cudaSuccess;
+    }
+    const size_t smem_count = sizeof(uint32_t) * (E * WORDS + 2 * G * G);
+    const size_t smem_scatter = sizeof(uint32_t) * (E * WORDS + E + 1 + BLK / 32);
+    if (smem_count > 48 * 1024 &&
+        (err = cudaFuncSetAttribute(dispatch_count_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_count)))
+        return err;
+    if (smem_scatter > 48 * 1024 &&
+        (err = cudaFuncSetAttribute(dispatch_scatter_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_scatter)))
+        return err;
+    dispatch_count_kernel<<<nblk, BLK, smem_count, st>>>(topk_idx, T, E, G, K, ws.hist_t,
+                                                         ws.send_part, ws.sendtok_part, status);
+    count_launch();
+    if ((err = cudaGetLastError())) return err;
+    dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(ws.hist_t, nblk, E, G, ws.send_part,
+                                                      ws.sendtok_part, ws.base_t, counts, send,
+                                                      send_tok);
+    count_launch();
+    if ((err = cudaGetLastError())) return err;
+    dispatch_scatter_kernel<<<nblk, BLK, smem_scatter, st>>>(topk_idx, T, E, K, counts, ws.base_t,
+                                                             offsets, perm_token, inv_perm);
+    count_launch();
+    if ((err = cudaGetLastError())) return err;
+    if (x_perm) {
+        const int chunks = d / 8;
+        const int64_t total = (int64_t)T * chunks;
+        int sms = 148;
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t want = (total + 255) / 256;
+        const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+        dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4 *>(x), inv_perm, T,
+                                                     chunks, K, (int64_t)T * K,
+                                                     static_cast<uint4 *>(x_perm));
+        count_launch();
+        if ((err = cudaGetLastError())) return err;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace moe

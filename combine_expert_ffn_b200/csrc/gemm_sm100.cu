@@ -1,0 +1,529 @@
+// gemm_sm100.cu -- grouped expert FFN on the 5th-generation tensor cores.
+//
+// Per routed expert e with rows R_e = [offsets[e], offsets[e+1]) of x_perm
+// and for the shared experts on all T rows of x:
+//   GEMM1:  h = SiLU(X W_g^T) * (X W_u^T)     (SwiGLU fused in the epilogue)
+//   GEMM2:  y = h W_d^T
+// ("shared experts (always active) + fine-grained routed experts", "MoE +
+// Expert-Parallel Overlap (Exp08)", Implemented; the pages' per token-expert
+// cost is 6 d d_ff FLOPs, same page, Implemented / overlap simulator.)
+//
+// One persistent kernel per GEMM, one CTA per SM, 192 threads:
+//   warp 0      TMA producer: A tile 128 x 64 and B tile 256 x 64 (bf16,
+//               128-byte swizzle) per stage into a 4-stage smem ring
+//   warp 1      TMEM owner (512 columns = two 128 x 256 fp32 accumulators)
+//               and single-thread tcgen05.mma issuer (M=128, N=256, K=16)
+//   warps 2..5  epilogue: tcgen05.ld -> SwiGLU or plain -> bf16 -> global
+// The accumulator is double-buffered so the epilogue of tile i overlaps the
+// mainloop of tile i+1.  Tiles: for every expert, ceil(R_e/128) row tiles x
+// the output column tiles; row tiles of one expert are adjacent in the tile
+// order so the expert's weight tiles are read from HBM about once and served
+// from L2 to its other row tiles.  Row tiles may run past the segment end
+// into the next expert's rows (or past the buffer, where TMA fills zeros):
+// those rows are computed and never stored.  Every wait is bounded; on
+// running out the kernel records MOE_ERR_DEVICE_TIMEOUT, drains its own TMA
+// loads and MMAs, frees TMEM and returns.
+#include "kernels.h"
+
+#include <mutex>
+
+namespace moe {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int BN_ACC = 256;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN_ACC * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int MAX_E = 1024;
+constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 1024;
+constexpr uint32_t IDESC = idesc_bf16_f32<BM, BN_ACC>();
+
+enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
+
+template <int EPI>
+struct Cfg {
+    static constexpr int BN_OUT = EPI == EPI_SWIGLU ? 128 : 256;  // output columns per tile
+};
+
+struct Maps {
+    CUtensorMap a_r;   // routed A  [rows_r, k_r]           box 64 x 128
+    CUtensorMap a_s;   // shared A  [T, k_s]                box 64 x 128
+    CUtensorMap b0_r;  // routed B  gate | down  3-D        box 64 x (128 | 256) x 1
+    CUtensorMap b1_r;  // routed B  up (SwiGLU only)
+    CUtensorMap b0_s;  // shared B  gate | down
+    CUtensorMap b1_s;  // shared B  up
+};
+
+struct Params {
+    const int32_t *offsets;  // [E+1]
+    int E;
+    int T;                   // shared rows; 0 = no shared experts
+    int n_out_r, n_out_s;    // output columns
+    int k_r, k_s;            // reduction lengths
+    int kseg_s;              // shared B is split along k into experts of this width
+    __nv_bfloat16 *out_r;
+    __nv_bfloat16 *out_s;
+    int32_t *status;
+    int64_t timeout_ns;
+};
+
+struct Tile {
+    int row0;        // first A row
+    int rows_valid;  // rows to store
+    int n0;          // first output column
+    int e;           // expert (routed) or -1 (shared)
+    int kblocks;
+};
+
+template <int EPI>
+__device__ __forceinline__ Tile decode_tile(int idx, const int *tile_base, const int *seg,
+                                            const Params &p, int ntr, int mt_s, int nt_s) {
+    constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
+    Tile t;
+    if (idx < ntr) {
+        int lo = 0, hi = p.E;  // tile_base[lo] <= idx < tile_base[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tile_base[mid] <= idx) lo = mid; else hi = mid;
+        }
+        const int cnt = seg[lo + 1] - seg[lo];
+        const int mt = (cnt + BM - 1) / BM;
+        const int local = idx - tile_base[lo];
+        const int n = local / mt, m = local - n * mt;
+        t.row0 = seg[lo] + m * BM;
+        t.rows_valid = min(BM, cnt - m * BM);
+        t.n0 = n * BN_OUT;
+        t.e = lo;
+        t.kblocks = p.k_r / BK;
+    } else {
+        const int local = idx - ntr;
+        const int m = local / nt_s, n = local - m * nt_s;  // column tiles fastest
+        t.row0 = m * BM;
+        t.rows_valid = min(BM, p.T - m * BM);
+        t.n0 = n * BN_OUT;
+        t.e = -1;
+        t.kblocks = p.k_s / BK;
+    }
+    return t;
+}
+
+// Bounded wait used while winding down: ignores the abort flag, so that
+// copies and MMAs already in flight are waited for before the CTA exits.
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int64_t timeout_ns,
+                                           int32_t *status) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if ((int64_t)(globaltimer_ns() - t0) > timeout_ns) {
+            record_status(status, MOE_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return g / (1.0f + __expf(-g)) * u;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
+    constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ int tile_base[MAX_E + 1];
+    __shared__ int seg[MAX_E + 1];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t smem0 = smem_u32(smem);
+    volatile int *abort_flag = &abort_s;
+
+    // ---------------------------------------------------------- prologue
+    if (warp == 0) {
+        // tile_base[e] = sum over experts < e of (row tiles x column tiles)
+        const int nt_r = (p.n_out_r + BN_OUT - 1) / BN_OUT;
+        int carry = 0;
+        for (int e0 = 0; e0 < p.E; e0 += 32) {
+            const int e = e0 + lane;
+            int lo = 0, cnt = 0;
+            if (e < p.E) {
+                lo = p.offsets[e];
+                cnt = p.offsets[e + 1] - lo;
+                seg[e] = lo;
+            }
+            const int v = ((cnt + BM - 1) / BM) * nt_r;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (e < p.E) tile_base[e] = carry + incl - v;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) {
+            tile_base[p.E] = carry;
+            seg[p.E] = p.offsets[p.E];
+            tma_prefetch_desc(&maps.a_r);
+            tma_prefetch_desc(&maps.b0_r);
+            if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
+            if (p.T > 0) {
+                tma_prefetch_desc(&maps.a_s);
+                tma_prefetch_desc(&maps.b0_s);
+                if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_s);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(smem_u32(&full_bar[s]), 1);
+                mbar_init(smem_u32(&empty_bar[s]), 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(smem_u32(&tfull_bar[b]), 1);
+                mbar_init(smem_u32(&tempty_bar[b]), 128);
+            }
+            mbar_init(smem_u32(&done_bar), 1);
+            abort_s = 0;
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc<TMEM_COLS>(smem_u32(&tmem_base_s));
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_s;
+
+    const int ntr = tile_base[p.E];
+    const int mt_s = p.T > 0 ? (p.T + BM - 1) / BM : 0;
+    const int nt_s = p.T > 0 ? (p.n_out_s + BN_OUT - 1) / BN_OUT : 0;
+    const int total = ntr + mt_s * nt_s;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t n_issued = 0;
+            for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+                const Tile t = decode_tile<EPI>(idx, tile_base, seg, p, ntr, mt_s, nt_s);
+                bool ok = true;
+                for (int kb = 0; kb < t.kblocks; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
+                                           p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    const uint32_t a_dst = smem0 + stage * STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + A_BYTES;
+                    const int k = kb * BK;
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    if (t.e >= 0) {
+                        tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
+                            tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_r, fb, k, t.n0, t.e);
+                        } else {
+                            tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
+                        }
+                    } else {
+                        tma_load_2d(a_dst, &maps.a_s, fb, k, t.row0);
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_3d(b_dst, &maps.b0_s, fb, k, t.n0, 0);
+                            tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_s, fb, k, t.n0, 0);
+                        } else {
+                            const int s = k / p.kseg_s;
+                            tma_load_3d(b_dst, &maps.b0_s, fb, k - s * p.kseg_s, t.n0, s);
+                        }
+                    }
+                    ++n_issued;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            // wind down: every load issued into a stage has landed
+            for (int s = 0; s < STAGES; ++s) {
+                if (n_issued > (uint32_t)s) {
+                    const uint32_t uses = (n_issued - 1 - s) / STAGES + 1;
+                    drain_wait(smem_u32(&full_bar[s]), (uses - 1) & 1u, p.timeout_ns, p.status);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+                const Tile t = decode_tile<EPI>(idx, tile_base, seg, p, ntr, mt_s, nt_s);
+                if (!mbar_wait_bounded(smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag,
+                                       p.status, p.timeout_ns))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN_ACC;
+                bool ok = true;
+                for (int kb = 0; kb < t.kblocks; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.status,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem0 + stage * STAGE_BYTES;
+                    const uint64_t a_desc = smem_desc_sw128(a_addr);
+                    const uint64_t b_desc = smem_desc_sw128(a_addr + A_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < BK / 16; ++ks)
+                        tc_mma_bf16(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks, IDESC,
+                                    (kb | ks) != 0 ? 1u : 0u);
+                    tc_commit(smem_u32(&empty_bar[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&tfull_bar[acc]));
+                if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+            }
+            // wind down: every MMA issued has completed
+            tc_commit(smem_u32(&done_bar));
+            drain_wait(smem_u32(&done_bar), 0, p.timeout_ns, p.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue
+        const int q = warp & 3;            // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;     // accumulator row = tile row
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+            const Tile t = decode_tile<EPI>(idx, tile_base, seg, p, ntr, mt_s, nt_s);
+            if (!mbar_wait_bounded(smem_u32(&tfull_bar[acc]), acc_phase, abort_flag, p.status,
+                                   p.timeout_ns))
+                break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
+            const bool shared = t.e < 0;
+            const int n_out = shared ? p.n_out_s : p.n_out_r;
+            __nv_bfloat16 *orow = (shared ? p.out_s : p.out_r) + (size_t)(t.row0 + row) * n_out;
+            const bool row_ok = row < t.rows_valid;
+            if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < BN_OUT; c += 32) {
+                    uint32_t g[32], u[32];
+                    tmem_ld32(taddr + c, g);
+                    tmem_ld32(taddr + BN_ACC / 2 + c, u);
+                    tc_wait_ld();
+                    if (row_ok && t.n0 + c < n_out) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + t.n0 + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 o;
+                            o.x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
+                                              silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
+                            o.y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
+                                              silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
+                            o.z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
+                                              silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
+                            o.w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
+                                              silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
+                            dst[v] = o;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN_OUT; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr + c, r);
+                    tc_wait_ld();
+                    if (row_ok && t.n0 + c < n_out) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + t.n0 + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                            dst[v] = o;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty_bar[acc]));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    // ---------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<TMEM_COLS>(tmem_base);
+    }
+}
+
+// Bounded-wait self-test: one thread waits on a barrier that never completes.
+__global__ void bounded_wait_selftest_kernel(int32_t *status, int64_t timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_s;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_s = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(smem_u32(&bar), 0, &abort_s, status, timeout_ns);
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 map over [rows, cols] row-major, box 64 (cols) x box_rows.
+bool map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {BK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over [n_mat, rows, cols], box 64 (cols) x box_rows x 1.
+bool map_3d(CUtensorMap *m, const void *base, uint64_t n_mat, uint64_t rows, uint64_t cols,
+            uint32_t box_rows) {
+    const cuuint64_t dims[3] = {cols, rows, n_mat};
+    const cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+    const cuuint32_t box[3] = {BK, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return sms;
+}
+
+template <int EPI>
+cudaError_t launch_one(const Maps &maps, const Params &p, cudaStream_t st) {
+    cudaError_t err = cudaFuncSetAttribute(grouped_ffn_gemm_kernel<EPI>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+    if (err != cudaSuccess) return err;
+    grouped_ffn_gemm_kernel<EPI><<<sm_count(), NUM_THREADS, SMEM_DYN, st>>>(maps, p);
+    count_launch();
+    return cudaGetLastError();
+}
+}  // namespace
+}  // namespace gemm
+
+cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
+    using namespace gemm;
+    if (!encode_fn()) return cudaErrorNotSupported;
+    const uint64_t rows_r = (uint64_t)a.T * a.K;
+    const bool has_shared = a.n_shared > 0 && a.T > 0;
+    const int ffs = a.n_shared * a.d_ff_shared;
+    if (rows_r == 0) return cudaSuccess;
+
+    // GEMM1: h = SwiGLU(x_perm) per expert; h_shared = SwiGLU(x) for the shared experts
+    Maps m1;
+    bool ok = map_2d(&m1.a_r, a.x_perm, rows_r, a.d, BM) &&
+              map_3d(&m1.b0_r, a.w_gate, a.E, a.d_ff, a.d, BN_ACC / 2) &&
+              map_3d(&m1.b1_r, a.w_up, a.E, a.d_ff, a.d, BN_ACC / 2);
+    if (has_shared)
+        ok = ok && map_2d(&m1.a_s, a.x, a.T, a.d, BM) &&
+             map_3d(&m1.b0_s, a.ws_gate, 1, ffs, a.d, BN_ACC / 2) &&
+             map_3d(&m1.b1_s, a.ws_up, 1, ffs, a.d, BN_ACC / 2);
+    else
+        m1.a_s = m1.a_r, m1.b0_s = m1.b0_r, m1.b1_s = m1.b1_r;
+    if (!ok) return cudaErrorInvalidValue;
+    Params p1{};
+    p1.offsets = a.offsets;
+    p1.E = a.E;
+    p1.T = has_shared ? a.T : 0;
+    p1.n_out_r = a.d_ff;
+    p1.n_out_s = ffs;
+    p1.k_r = a.d;
+    p1.k_s = a.d;
+    p1.kseg_s = a.d;
+    p1.out_r = static_cast<__nv_bfloat16 *>(a.h);
+    p1.out_s = static_cast<__nv_bfloat16 *>(a.h_shared);
+    p1.status = a.status;
+    p1.timeout_ns = a.timeout_ns;
+    cudaError_t err = launch_one<EPI_SWIGLU>(m1, p1, st);
+    if (err != cudaSuccess) return err;
+
+    // GEMM2: y_perm = h W_d^T per expert; y_shared = h_shared Ws_d^T (k split per shared expert)
+    Maps m2;
+    ok = map_2d(&m2.a_r, a.h, rows_r, a.d_ff, BM) &&
+         map_3d(&m2.b0_r, a.w_down, a.E, a.d, a.d_ff, BN_ACC);
+    if (has_shared)
+        ok = ok && map_2d(&m2.a_s, a.h_shared, a.T, ffs, BM) &&
+             map_3d(&m2.b0_s, a.ws_down, a.n_shared, a.d, a.d_ff_shared, BN_ACC);
+    else
+        m2.a_s = m2.a_r, m2.b0_s = m2.b0_r;
+    m2.b1_r = m2.b0_r;
+    m2.b1_s = m2.b0_s;
+    if (!ok) return cudaErrorInvalidValue;
+    Params p2 = p1;
+    p2.n_out_r = a.d;
+    p2.n_out_s = a.d;
+    p2.k_r = a.d_ff;
+    p2.k_s = ffs;
+    p2.kseg_s = a.d_ff_shared;
+    p2.out_r = static_cast<__nv_bfloat16 *>(a.y_perm);
+    p2.out_s = static_cast<__nv_bfloat16 *>(a.y_shared);
+    return launch_one<EPI_STORE>(m2, p2, st);
+}
+
+cudaError_t launch_bounded_wait_selftest(int64_t timeout_ns, int32_t *status, cudaStream_t st) {
+    gemm::bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(status, timeout_ns);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,59 @@
+// kernels.h -- internal launch functions of libmoe (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// Counts one kernel launch (process-wide, for moe_launch_count()).
+void count_launch();
+
+// route.cu
+cudaError_t launch_router_logits(const void *x, const float *e, const float *off, int T, int d,
+                                 int E, float *scores, cudaStream_t st);
+cudaError_t launch_route_select(const float *scores, const float *bias, int T, int E, int G,
+                                int K, int M, int32_t *topk_idx, float *topk_w, cudaStream_t st);
+
+// dispatch.cu
+struct DispatchWs {
+    int32_t *hist_t;       // [E, nblk] copies of expert e in token block b
+    int32_t *base_t;       // [E, nblk] exclusive prefix of hist_t along b
+    int32_t *send_part;    // [nblk, G*G]
+    int32_t *sendtok_part; // [nblk, G*G]
+};
+constexpr int DISPATCH_BLOCK = 256;  // tokens per dispatch block
+inline int dispatch_nblk(int T) { return (T + DISPATCH_BLOCK - 1) / DISPATCH_BLOCK; }
+cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d, int E, int G,
+                            int K, int32_t *counts, int32_t *offsets, int32_t *send,
+                            int32_t *send_tok, int32_t *perm_token, int32_t *inv_perm,
+                            void *x_perm, const DispatchWs &ws, int32_t *status, cudaStream_t st);
+
+// combine.cu
+cudaError_t launch_combine(const void *y_perm, const int32_t *inv_perm, const float *topk_w,
+                           const void *y_shared, int T, int d, int K, int64_t n_rows, void *out,
+                           cudaStream_t st);
+
+// gemm_sm100.cu
+struct FfnArgs {
+    int T, d, E, K, d_ff, n_shared, d_ff_shared;
+    const void *x_perm;
+    const int32_t *offsets;
+    const void *w_gate, *w_up, *w_down;
+    void *h;        // [T*K, d_ff] bf16 scratch
+    void *y_perm;   // [T*K, d] bf16
+    const void *x;  // [T, d]
+    const void *ws_gate, *ws_up, *ws_down;
+    void *h_shared; // [T, n_shared*d_ff_shared] bf16 scratch
+    void *y_shared; // [T, d]
+    int32_t *status;
+    int64_t timeout_ns;
+};
+cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st);
+cudaError_t launch_bounded_wait_selftest(int64_t timeout_ns, int32_t *status, cudaStream_t st);
+
+}  // namespace moe

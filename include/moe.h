@@ -1,0 +1,207 @@
+/*
+ * moe.h -- C ABI of libmoe: one DeepSeek-V3-style MoE layer forward on one
+ * B200 (sm_100a).
+ *
+ * The layer (sources are the pages' titles and sections):
+ *   route     s_i = sigmoid(x . e_i [+ o_i]); b_i = s_i + bias_i picks experts
+ *             only ("MoE + Expert-Parallel Overlap (Exp08)", Implemented:
+ *             top-k gating, per-expert bias balancing); node-limited top-K:
+ *             the E experts form G contiguous groups standing in for nodes
+ *             ("moe-node-limited-routing", opening definition; deepnotes
+ *             "The real cluster, and the mesh DeepSeek actually disclosed":
+ *             four experts per GPU), the M groups with the largest sum of
+ *             their top-(K/M) b are kept, the top-K b inside them are chosen
+ *             (ties to the lower index), gates w_j = s_j / sum s over the K
+ *             chosen UNBIASED affinities.
+ *   dispatch  the token copies are sorted by expert into expert-contiguous
+ *             rows (stable: tokens ascending inside a segment) with counts,
+ *             offsets and the group-to-group send matrices (the dispatch
+ *             all-to-all of "moe-node-limited-routing", "Why all to all
+ *             dominates MoE step time", becomes a local permutation; "send
+ *             matrices", shivam2003 "5. Tail latency controls step time").
+ *   expert    y = W_d (SiLU(W_g x) * (W_u x)) per expert on its rows, plus
+ *             the always-on shared experts on every token (Exp08,
+ *             Implemented: shared + fine-grained routed experts).
+ *   combine   out_t = shared_t + sum_j w_j y_(t,j) back in token order (the
+ *             combine all-to-all, same section).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are DEVICE pointers to dense row-major arrays; bf16 data is
+ *     passed as `void *` (IEEE bfloat16 bit patterns).  The caller owns every
+ *     buffer; the library never allocates, frees, or keeps a pointer after
+ *     the call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     compute entry point only enqueues kernels: it returns before they run,
+ *     performs no host<->device copy and no synchronisation.
+ *   - A nonzero moe_status means nothing was enqueued (argument errors) or a
+ *     launch failed (MOE_ERR_CUDA).  Faults found by the kernels themselves
+ *     (an expert id out of range, a bounded wait that ran out) are written to
+ *     the status word at the start of the workspace; read it with
+ *     moe_read_device_status() after the stream has run.
+ *   - Buffers must be 16-byte aligned; the workspace 256-byte aligned.
+ *   - Sizes supported: E % G == 0, K % M == 0, K/M <= E/G, M <= G, K <= 32,
+ *     E <= 1024, G <= 64, T % G == 0, d % 64 == 0, d_ff % 64 == 0,
+ *     d_ff_shared % 64 == 0, T*K < 2^31, T >= 0 (T == 0 is a no-op).
+ *     Anything else returns MOE_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layer sizes. */
+typedef struct moe_config {
+    int32_t T;           /* tokens in the batch                               */
+    int32_t d;           /* hidden size                                       */
+    int32_t E;           /* routed experts                                    */
+    int32_t G;           /* expert groups (emulated nodes), E/G experts each  */
+    int32_t K;           /* routed experts per token                          */
+    int32_t M;           /* max groups a token may use                        */
+    int32_t d_ff;        /* routed expert intermediate size                   */
+    int32_t n_shared;    /* always-on shared experts (0 allowed)              */
+    int32_t d_ff_shared; /* shared expert intermediate size                   */
+} moe_config;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,         /* NULL required pointer, bad alignment   */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,   /* sizes outside the supported set above  */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < moe_workspace_size(cfg)     */
+    MOE_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed      */
+    MOE_ERR_DEVICE_TIMEOUT = 5,      /* device status: a bounded wait ran out  */
+    MOE_ERR_DEVICE_FAULT = 6,        /* device status: bad index in the inputs */
+    MOE_ERR_NO_DEVICE = 7            /* no sm_100 device is current            */
+} moe_status;
+
+/* Validates sizes only (no CUDA call).  MOE_OK or MOE_ERR_UNSUPPORTED_SHAPE /
+ * MOE_ERR_INVALID_ARG (cfg == NULL). */
+MOE_API moe_status moe_check_config(const moe_config *cfg);
+
+/* Bytes of device workspace every entry point that takes `ws` may use for
+ * this configuration; 0 if the configuration is unsupported.  Monotone in T. */
+MOE_API size_t moe_workspace_size(const moe_config *cfg);
+
+/* Static English text for a status code (never NULL). */
+MOE_API const char *moe_status_string(int status);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams).  For accounting; not synchronised with the GPU. */
+MOE_API uint64_t moe_launch_count(void);
+
+/* Copies the workspace status word to *host_status after synchronising
+ * `stream` (the only entry point that synchronises).  MOE_OK if no kernel
+ * recorded a fault since the last moe_clear_device_status(). */
+MOE_API moe_status moe_read_device_status(const void *ws, int32_t *host_status, void *stream);
+
+/* Enqueues a reset of the workspace status word to MOE_OK. */
+MOE_API moe_status moe_clear_device_status(void *ws, void *stream);
+
+/*
+ * Router (affinity + node-limited top-K).
+ *   x            [T, d]   bf16
+ *   router_w     [E, d]   fp32  (e_i rows)
+ *   logit_offset [E]      fp32 or NULL: added to x . e_i before the sigmoid
+ *   bias         [E]      fp32: selection-only balance bias (NULL = zeros)
+ *   topk_idx     [T, K]   int32 out: chosen experts, descending b_i then
+ *                               ascending index
+ *   topk_w       [T, K]   fp32 out: gates, sum to 1 over the K slots
+ *   scores       [T, E]   fp32 out or NULL: the affinities s
+ * fp32 accumulation of x . e_i; s = 1 / (1 + expf(-L)).
+ */
+MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *router_w,
+                     const float *logit_offset, const float *bias,
+                     int32_t *topk_idx, float *topk_w, float *scores,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/* Selection only, from given fp32 affinities scores[T, E]: exactly the
+ * selection and gate steps of moe_route.  Same fp32 operations in the same
+ * order as the written-out definition, so equal inputs give equal bits. */
+MOE_API moe_status moe_route_select(const moe_config *cfg, const float *scores, const float *bias,
+                            int32_t *topk_idx, float *topk_w, void *stream);
+
+/*
+ * Dispatch: stable counting sort of the T*K token copies by expert.
+ *   topk_idx   [T, K]   int32 in (distinct experts per token, each < E)
+ *   counts     [E]      int32 out: copies per expert
+ *   offsets    [E+1]    int32 out: exclusive prefix sum of counts
+ *   send       [G, G]   int32 out: copies from source group (t / (T/G)) to
+ *                               expert group (e / (E/G)); sums to T*K
+ *   send_tok   [G, G]   int32 out (or NULL): tokens from source group to
+ *                               expert group, one per token and group
+ *   perm_token [T*K]    int32 out: token of each permuted row
+ *   inv_perm   [T, K]   int32 out: permuted row of copy (t, j)
+ *   x_perm     [T*K, d] bf16 out (or NULL): x_perm[row] = x[perm_token[row]]
+ * Bad ids are skipped and flagged MOE_ERR_DEVICE_FAULT in the status word.
+ */
+MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int32_t *topk_idx,
+                        int32_t *counts, int32_t *offsets, int32_t *send, int32_t *send_tok,
+                        int32_t *perm_token, int32_t *inv_perm, void *x_perm,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Expert FFN: grouped SwiGLU over the expert segments plus the shared experts.
+ *   x_perm    [T*K, d]             bf16 expert-contiguous rows
+ *   offsets   [E+1]                int32 segment starts (offsets[E] == T*K)
+ *   w_gate    [E, d_ff, d]         bf16     w_up [E, d_ff, d]   bf16
+ *   w_down    [E, d, d_ff]         bf16
+ *   y_perm    [T*K, d]             bf16 out: y_perm[r] = FFN_e(x_perm[r])
+ *   x         [T, d]               bf16 (shared-expert input; may be NULL
+ *                                  only when n_shared == 0)
+ *   ws_gate   [n_shared, d_ff_shared, d]   ws_up same   bf16
+ *   ws_down   [n_shared, d, d_ff_shared]   bf16
+ *   y_shared  [T, d]               bf16 out: sum of the shared FFNs
+ * tcgen05 tensor cores, fp32 accumulation; the intermediate h = SiLU(gate) *
+ * up is rounded to bf16 (nearest even) before the down projection.
+ */
+MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                          const void *w_gate, const void *w_up, const void *w_down,
+                          void *y_perm, const void *x, const void *ws_gate,
+                          const void *ws_up, const void *ws_down, void *y_shared,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Combine: out[t] = y_shared[t] + sum_j topk_w[t,j] * y_perm[inv_perm[t,j]],
+ * fp32 accumulation, rounded to bf16.  y_shared may be NULL (treated as 0).
+ */
+MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *inv_perm,
+                       const float *topk_w, const void *y_shared, void *out, void *stream);
+
+/*
+ * The whole layer: route -> dispatch -> expert FFN -> combine on `stream`.
+ *   out [T, d] bf16 out.  topk_idx [T,K], topk_w [T,K], counts [E],
+ *   offsets [E+1], send [G,G], send_tok [G,G] are optional outputs (NULL:
+ *   kept in the workspace).  Intermediates live in the workspace.
+ */
+MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float *router_w,
+                       const float *logit_offset, const float *bias,
+                       const void *w_gate, const void *w_up, const void *w_down,
+                       const void *ws_gate, const void *ws_up, const void *ws_down,
+                       void *out, int32_t *topk_idx, float *topk_w, int32_t *counts,
+                       int32_t *offsets, int32_t *send, int32_t *send_tok,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Self-test of the bounded device waits: launches one kernel that waits on
+ * an mbarrier no thread ever arrives on, with a limit of `timeout_ns`
+ * nanoseconds (1e3 .. 1e10).  The kernel must give up, record
+ * MOE_ERR_DEVICE_TIMEOUT in the status word and return; the context stays
+ * usable.  Uses only the status word of `ws` (>= 256 bytes).
+ */
+MOE_API moe_status moe_selftest_bounded_wait(int64_t timeout_ns, void *ws, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -217,7 +217,41 @@ def make_inputs(shape: MoeShape, device="cpu", weights: bool = True) -> dict:
         out["w_gate"] = normal(sd, TENSOR_IDS["w_gate"], (E, ff, d), _inv_sqrt(d), torch.bfloat16, device)
         out["w_up"] = normal(sd, TENSOR_IDS["w_up"], (E, ff, d), _inv_sqrt(d), torch.bfloat16, device)
         out["w_down"] = normal(sd, TENSOR_IDS["w_down"], (E, d, ff), _inv_sqrt(ff), torch.bfloat16, device)
-        out["ws_gate"] = normal(sd, TENSOR_IDS["ws_gate"], (ns, ffs, d), _inv_sqrt(d), torch.bfloat16, device)
-        out["ws_up"] = normal(sd, TENSOR_IDS["ws_up"], (ns, ffs, d), _inv_sqrt(d), torch.bfloat16, device)
-        out["ws_down"] = normal(sd, TENSOR_IDS["ws_down"], (ns, d, ffs), _inv_sqrt(ffs), torch.bfloat16, device)
+        if ns > 0:
+            out["ws_gate"] = normal(sd, TENSOR_IDS["ws_gate"], (ns, ffs, d), _inv_sqrt(d), torch.bfloat16, device)
+            out["ws_up"] = normal(sd, TENSOR_IDS["ws_up"], (ns, ffs, d), _inv_sqrt(d), torch.bfloat16, device)
+            out["ws_down"] = normal(sd, TENSOR_IDS["ws_down"], (ns, d, ffs), _inv_sqrt(ffs), torch.bfloat16, device)
+        else:
+            out["ws_gate"] = out["ws_up"] = out["ws_down"] = None
     return out
+
+
+def uniform01(seed: int, tid: int, shape, device="cpu") -> torch.Tensor:
+    """fp32 uniform on (0, 1): (24-bit integer + 0.5) * 2^-24, exact in fp32."""
+    n = 1
+    for s in shape:
+        n *= int(s)
+    out = torch.empty(n, dtype=torch.float32, device=device)
+    for s in range(0, n, _CHUNK):
+        m = min(_CHUNK, n - s)
+        idx = torch.arange(s, s + m, dtype=torch.int64, device=device)
+        a, _ = _words(seed, tid, idx)
+        out[s:s + m] = ((a >> 8).to(torch.float32) + 0.5) * (2.0 ** -24)
+    return out.view(*shape)
+
+
+def random_routing(seed: int, T: int, E: int, K: int, zipf_s: float = 0.0,
+                   device="cpu") -> torch.Tensor:
+    """[T, K] int32: K distinct experts per token drawn without replacement.
+
+    Weighted sampling by the Efraimidis-Spirakis keys u^(1/p_e) with Zipf(s)
+    weights p_e (uniform when s == 0); an input for testing the dispatch
+    alone on skewed or balanced expert loads.
+    """
+    u = uniform01(seed, TENSOR_IDS["scores"] + 100, (T, E), device).double()
+    if zipf_s > 0:
+        p = torch.arange(1, E + 1, dtype=torch.float64, device=device).pow(-zipf_s)
+        keys = torch.log(u) / p
+    else:
+        keys = torch.log(u)
+    return torch.topk(keys, K, dim=1).indices.to(torch.int32)

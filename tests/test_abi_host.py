@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load and export every entry point ``include/moe.h``
+declares, and validate its arguments before touching CUDA.  No call here
+reaches a kernel launch: each one is rejected by validation first.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+import synth
+from tests import harness as H
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from combine_expert_ffn_b200 import build
+    build.build()
+    import combine_expert_ffn_b200 as m
+    return m
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API[^;(]*?\b(moe_\w+)\(", text, flags=re.S)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for s in ("moe_route", "moe_route_select", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+              "moe_forward", "moe_workspace_size"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(moe):
+    lib = C.CDLL(moe.LIB_PATH)
+    for s in declared_symbols():
+        assert hasattr(lib, s), s
+    assert sorted(moe.EXPORTS) == declared_symbols()
+
+
+@pytest.mark.parametrize("name", list(H.SHAPES))
+def test_known_workloads_are_supported(moe, name):
+    cfg = moe.MoeConfig.of(H.shape(name))
+    assert moe.moe_check_config(cfg) == moe.MOE_OK
+    assert moe.moe_workspace_size(cfg) > 0
+
+
+BAD = [
+    dict(E=15),                    # E % G
+    dict(K=3),                     # K % M
+    dict(M=8),                     # M > G
+    dict(K=32, M=2),               # K/M > E/G
+    dict(d=100),                   # d % 64
+    dict(d_ff=96),                 # d_ff % 64
+    dict(d_ff_shared=32),          # d_ff_shared % 64
+    dict(T=63),                    # T % G
+    dict(E=2048, G=4),             # E > 1024
+    dict(K=64, M=2, E=64, G=2),    # K > 32
+    dict(T=-4),
+    dict(d=0),
+]
+
+
+@pytest.mark.parametrize("kw", BAD)
+def test_unsupported_shapes_are_rejected(moe, kw):
+    cfg = moe.MoeConfig.of(synth.config("tiny").replace(**kw))
+    assert moe.moe_check_config(cfg) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert moe.moe_workspace_size(cfg) == 0
+
+
+def test_null_config(moe):
+    assert moe._lib.moe_check_config(None) == moe.MOE_ERR_INVALID_ARG
+    assert moe._lib.moe_workspace_size(None) == 0
+
+
+def test_workspace_grows_with_tokens(moe):
+    base = synth.config("v3")
+    sizes = [moe.moe_workspace_size(moe.MoeConfig.of(base.replace(T=t))) for t in (0, 8, 64, 1024, 8192, 32768)]
+    assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+    # the forward intermediates dominate: x_perm + y_perm + h + y_shared at least
+    sh = base
+    floor = 2 * sh.T * sh.K * sh.d * 2 + sh.T * sh.K * sh.d_ff * 2 + sh.T * sh.d * 2
+    assert moe.moe_workspace_size(moe.MoeConfig.of(sh)) >= floor
+
+
+def test_status_strings(moe):
+    for code in range(8):
+        assert moe.moe_status_string(code)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+def test_entry_points_validate_before_cuda(moe):
+    cfg = moe.MoeConfig.of(synth.config("tiny"))
+    ws_n = moe.moe_workspace_size(cfg)
+    lib, fake = moe._lib, 1 << 20
+    P = C.c_void_p
+    # NULL required pointers
+    assert lib.moe_route(C.byref(cfg), None, P(fake), None, None, P(fake), P(fake), P(fake),
+                         None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_select(C.byref(cfg), None, None, P(fake), P(fake), None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(C.byref(cfg), None, P(fake), P(fake), None, P(fake), None) == moe.MOE_ERR_INVALID_ARG
+    # misaligned buffer
+    assert lib.moe_combine(C.byref(cfg), P(fake + 2), P(fake), P(fake), None, P(fake), None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small
+    args = [P(fake)] * 9
+    assert lib.moe_dispatch(C.byref(cfg), *args, P(fake), ws_n - 1, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert lib.moe_forward(C.byref(cfg), *([P(fake)] * 17), P(fake), ws_n - 1, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    # misaligned workspace
+    assert lib.moe_dispatch(C.byref(cfg), *args, P(fake + 16), ws_n, None) == moe.MOE_ERR_INVALID_ARG
+    # unsupported shape wins over everything else
+    bad = moe.MoeConfig.of(synth.config("tiny").replace(E=15))
+    assert lib.moe_forward(C.byref(bad), *([None] * 17), None, 0, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    # self-test limits
+    assert lib.moe_selftest_bounded_wait(10, P(fake), None) == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a GPU")
+def test_no_device_is_reported(moe):
+    assert moe._lib.moe_clear_device_status(C.c_void_p(1 << 20), None) == moe.MOE_ERR_NO_DEVICE
