@@ -5,7 +5,7 @@ device pointers and the current CUDA stream to the C entry point of the same
 name in ``include/moe.h`` and raises :class:`MoeError` on a nonzero status.
 All arithmetic happens in the library's CUDA kernels; there is no CPU or
 PyTorch fallback.  If ``libmoe.so`` is missing the import fails -- build it
-with ``python -m combine_expert_ffn_b200.build``.
+with ``python combine_expert_ffn_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: run `python -m combine_expert_ffn_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: run `python combine_expert_ffn_b200/build.py`")
 
 _lib = C.CDLL(LIB_PATH)
 

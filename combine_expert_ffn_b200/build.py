@@ -1,6 +1,9 @@
 """Builds libmoe.so in-tree with nvcc for sm_100a.
 
-    python -m combine_expert_ffn_b200.build [--force] [--verbose]
+    python combine_expert_ffn_b200/build.py [--force] [--verbose]
+
+(Run it as a script or load it by path: importing the package itself loads
+libmoe.so and fails while the library is missing.)
 
 The CUDA runtime is linked statically and the driver entry point
 (cuTensorMapEncodeTiled) is resolved at run time, so the library loads on a

@@ -127,6 +127,8 @@ int oracle_select(int n_rows, int E, int G, int K, int M,
                 for (int i = g * gsz; i < (g + 1) * gsz; ++i)
                     if (!taken[i] && (best < 0 || beats(b[i], i, b[best], best)))
                         best = i;
+                if (best < 0)
+                    break; /* unreachable: kpg <= gsz was checked */
                 taken[best] = 1;
                 sum = (r == 0) ? b[best] : sum + b[best];
             }
@@ -142,6 +144,8 @@ int oracle_select(int n_rows, int E, int G, int K, int M,
             for (int g = 0; g < G; ++g)
                 if (!gkeep[g] && (best < 0 || beats(gs[g], g, gs[best], best)))
                     best = g;
+            if (best < 0)
+                break; /* unreachable: M <= G was checked */
             gkeep[best] = 1;
         }
 
@@ -154,6 +158,8 @@ int oracle_select(int n_rows, int E, int G, int K, int M,
                 if (gkeep[i / gsz] && !taken[i] &&
                     (best < 0 || beats(b[i], i, b[best], best)))
                     best = i;
+            if (best < 0)
+                break; /* unreachable: K <= M * gsz was checked */
             taken[best] = 1;
             idx[j] = best;
         }
@@ -285,12 +291,12 @@ int oracle_shared_row(int d, int n_shared, int d_ff_s, const uint16_t *x_row,
                       const uint16_t *Wsg, const uint16_t *Wsu,
                       const uint16_t *Wsd, int round_h, double *y)
 {
-    if (d <= 0 || n_shared < 0 || d_ff_s <= 0 || !x_row || !y)
+    if (d <= 0 || n_shared < 0 || !x_row || !y)
         return ORC_EBADARG;
     memset(y, 0, sizeof(double) * d);
     if (n_shared == 0)
         return ORC_OK;
-    if (!Wsg || !Wsu || !Wsd)
+    if (d_ff_s <= 0 || !Wsg || !Wsu || !Wsd)
         return ORC_EBADARG;
     double *h = malloc(sizeof(double) * d_ff_s);
     if (!h)

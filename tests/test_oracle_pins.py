@@ -341,3 +341,20 @@ def test_round_h_only_perturbs_at_bf16_level(orc):
     y1 = orc.ffn_row(x, Wg, Wu, Wd, round_h=True)
     rel = np.linalg.norm(y1 - y0) / np.linalg.norm(y0)
     assert 0 < rel < 8e-3
+
+
+def test_layer_without_shared_experts(orc):
+    """n_shared = 0: the layer is the gate-weighted routed sum alone."""
+    shape = synth.MoeShape("nosh", T=8, d=32, E=8, G=4, K=2, M=2, d_ff=16, n_shared=0,
+                           d_ff_shared=0, x_sigma=1, e_sigma=1, bias_sigma=0)
+    rng = np.random.default_rng(12)
+    x, e, Wg, Wu, Wd, _ = _layer_inputs(shape.replace(n_shared=1, d_ff_shared=8), rng)
+    bias = np.zeros(8, np.float32)
+    empty = torch.zeros(1, 8, 32, dtype=torch.bfloat16)
+    out, idx, w, _ = orc.layer_rows(range(8), shape, x, e, bias, Wg, Wu, Wd, empty, empty,
+                                    torch.zeros(1, 32, 8, dtype=torch.bfloat16))
+    xs = _bf16_np(x)
+    want = np.stack([sum(float(w[t, j]) * _swiglu_np(xs[t], _bf16_np(Wg[idx[t, j]]), _bf16_np(Wu[idx[t, j]]),
+                                                     _bf16_np(Wd[idx[t, j]])) for j in range(2))
+                     for t in range(8)])
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-13)
