@@ -33,7 +33,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_WORKSPACE_TOO_SM
 EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_launch_count",
            "moe_read_device_status", "moe_clear_device_status", "moe_route", "moe_route_select",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
-           "moe_selftest_bounded_wait")
+           "moe_selftest_bounded_wait", "moe_dispatch_noalloc")
 
 
 class MoeConfig(C.Structure):
@@ -73,6 +73,7 @@ _sig = {
     "moe_forward": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _S, _P]),
     "moe_selftest_bounded_wait": (C.c_int, [_I64, _P, _P]),
+    "moe_dispatch_noalloc": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -196,6 +197,15 @@ def moe_forward(cfg, x, router_w, logit_offset, bias, w_gate, w_up, w_down, ws_g
 def moe_selftest_bounded_wait(timeout_ns, ws, stream=None) -> None:
     _ok("moe_selftest_bounded_wait",
         _lib.moe_selftest_bounded_wait(int(timeout_ns), _ptr(ws), _stream(stream)))
+
+
+def moe_dispatch_noalloc(cfg, x, topk_idx, counts, offsets, send, send_tok, perm_token, inv_perm,
+                         x_perm, device_status=None, stream=None) -> None:
+    """moe_dispatch with its scratch in the library's static device array (no workspace)."""
+    _ok("moe_dispatch_noalloc",
+        _lib.moe_dispatch_noalloc(_cfg(cfg), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                  _ptr(send), _ptr(send_tok), _ptr(perm_token), _ptr(inv_perm),
+                                  _ptr(x_perm), _ptr(device_status), _stream(stream)))
 
 
 # ----------------------------------------------------------------- convenience

@@ -150,6 +150,37 @@ MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int3
                         void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * moe_dispatch for callers that cannot allocate device memory.  No passage of
+ * the pages has a counterpart: this entry point exists for deployment only.
+ * Callers such as a serving runtime that owns the whole HBM budget through
+ * its own pool, or a latency-critical path that cannot afford cudaMalloc's
+ * implicit device synchronisation, get the same results as moe_dispatch
+ * (same kernels, bit for bit) without passing a workspace.
+ *   Arguments are those of moe_dispatch, without ws / ws_bytes, plus
+ *   device_status: a device int32 (or NULL) that receives the first fault a
+ *   kernel finds (MOE_ERR_DEVICE_FAULT for a bad expert id); the caller
+ *   clears it.  With NULL, faults are not reported.
+ *   Scratch: a fixed 4 MiB static device array, held by every GPU that loads
+ *   the library until the process exits.  This call needs
+ *   256 + 2 * r(4 E n) + 2 * r(4 n G^2) bytes of it, n = ceil(T / 256) and
+ *   r() rounding up to 256; larger sizes return MOE_ERR_WORKSPACE_TOO_SMALL
+ *   before anything is launched (the five named workloads need at most
+ *   0.3 MiB).  It allocates and frees nothing.
+ *   First call on a device: it looks up the array's device address with
+ *   cudaGetSymbolAddress (once per device, with that device current); make
+ *   that first call before any stream capture.
+ *   Every call uses the same array: nothing in it has to start at zero
+ *   (each call writes every scratch word before reading it), but calls whose
+ *   kernels overlap on the GPU -- on two streams, or from two threads --
+ *   race on it and give wrong results.  Serialise them.
+ */
+MOE_API moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
+                                        const int32_t *topk_idx, int32_t *counts,
+                                        int32_t *offsets, int32_t *send, int32_t *send_tok,
+                                        int32_t *perm_token, int32_t *inv_perm, void *x_perm,
+                                        int32_t *device_status, void *stream);
+
+/*
  * Expert FFN: grouped SwiGLU over the expert segments plus the shared experts.
  *   x_perm    [T*K, d]             bf16 expert-contiguous rows
  *   offsets   [E+1]                int32 segment starts (offsets[E] == T*K)
