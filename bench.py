@@ -294,10 +294,25 @@ def run_ours(args, sh, world, rank, local):
     if status != moe.MOE_OK:
         raise RuntimeError(f"device status {status} after the timed region")
 
-    ms_step = ms_total / args.steps
-    value = world * T * args.steps / (ms_total / 1e3)
-
     # ---- end to end through moe_forward with pinned host buffers
+    e2e = e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world) if not args.no_e2e else None
+    if rank != 0:
+        return 0
+    line = report(args, sh, world, ms_total, stage_ms, launches, clk, e2e)
+    if world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_tokens
+        v, dt = oracle_tokens_per_s(sh, inp, n)
+        line["cpu_baseline"] = {
+            "value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of the {sh.name} workload, whole layer per token, single thread, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world):
+    """moe_forward on pinned host buffers: H2D of x and D2H of out inside the timed region."""
+    import combine_expert_ffn_b200 as moe
+    T, d = sh.T, sh.d
     x_host = inp["x"].cpu().pin_memory()
     out_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty_like(inp["x"])
@@ -324,10 +339,14 @@ def run_ours(args, sh, world, rank, local):
     e2e_value = world * T * args.steps / (e2e_ms / 1e3)
     if not torch.equal(out_host, o["out"].cpu()) and world == 1:
         raise RuntimeError("moe_forward and the staged calls disagree")
+    return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
+            "d2h_bytes_per_step": T * d * 2}
 
-    if rank != 0:
-        return 0
 
+def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
+    T = sh.T
+    ms_step = ms_total / args.steps
+    value = world * T * args.steps / (ms_total / 1e3)
     peaks = load_peaks()
     alg = algorithmic(sh)
     ffn_s = stage_ms["expert_ffn"] / 1e3
@@ -365,30 +384,23 @@ def run_ours(args, sh, world, rank, local):
                         "frac": comb_gbs / hbm},
         },
         "gpu_launches": int(launches),
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
-                "d2h_bytes_per_step": T * d * 2},
+        "e2e": e2e,
         "clocks": clk,
     }
-    if world == 1 and not args.no_cpu_baseline:
-        n = args.cpu_tokens
-        v, dt = oracle_tokens_per_s(sh, inp, n)
-        line["cpu_baseline"] = {
-            "value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens of the {sh.name} workload, whole layer per token, single thread, {dt:.1f} s"}
-    print(json.dumps(line), flush=True)
-    return 0
+    return line
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="v3", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--config", default="v3", choices=sorted(synth.CONFIGS) + sorted(synth.PROFILE_CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=24)
     ap.add_argument("--ref-tokens", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

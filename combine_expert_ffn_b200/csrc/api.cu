@@ -22,7 +22,7 @@ constexpr int64_t kWaitTimeoutNs = 2000000000LL;  // 2 s per device wait
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-    size_t status, scores, hist_t, base_t, send_part, sendtok_part;
+    size_t status, scores, e_split, hist_t, base_t, send_part, sendtok_part;
     size_t topk_idx, topk_w, counts, offsets, send, send_tok, perm_token, inv_perm;
     size_t x_perm, h, y_perm, h_sh, y_sh;
     size_t total;
@@ -40,6 +40,7 @@ Layout layout(const moe_config &c) {
     const size_t nblk = (size_t)dispatch_nblk(c.T);
     L.status = take(256);
     L.scores = take(4 * T * E);
+    L.e_split = take(2 * 3 * E * (size_t)c.d);
     L.hist_t = take(4 * E * nblk);
     L.base_t = take(4 * E * nblk);
     L.send_part = take(4 * nblk * G * G);
@@ -167,18 +168,18 @@ moe_status moe_route(const moe_config *c, const void *x, const float *router_w,
                      float *topk_w, float *scores, void *ws, size_t ws_bytes, void *stream) {
     moe_status st = moe_check_config(c);
     if (st) return st;
+    if (!ws) return MOE_ERR_INVALID_ARG;
     if (c->T > 0 && (!x || !router_w || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_INVALID_ARG;
     const Layout L = layout(*c);
-    if (!scores) {
-        if (!ws) return MOE_ERR_INVALID_ARG;
-        if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
-        scores = at<float>(ws, L.scores);
-    }
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if (!scores) scores = at<float>(ws, L.scores);
     if ((st = check_device())) return st;
     cudaStream_t s = as_stream(stream);
-    cudaError_t e = launch_router_logits(x, router_w, logit_offset, c->T, c->d, c->E, scores, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, at<void>(ws, L.e_split),
+                                scores, at<int32_t>(ws, L.status), kWaitTimeoutNs, s))
+        return MOE_ERR_CUDA;
     return cuda_status(
         launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s));
 }
@@ -284,7 +285,9 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
     void *y_sh = c->n_shared > 0 ? at<void>(ws, L.y_sh) : nullptr;
     int32_t *status = at<int32_t>(ws, L.status);
 
-    if (launch_router_logits(x, router_w, logit_offset, c->T, c->d, c->E, scores, s)) return MOE_ERR_CUDA;
+    if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, at<void>(ws, L.e_split),
+                                scores, status, kWaitTimeoutNs, s))
+        return MOE_ERR_CUDA;
     if (launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
         return MOE_ERR_CUDA;
     DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),

@@ -1,6 +1,6 @@
 // common.cuh -- device helpers shared by the libmoe kernels (sm_100a only).
 //
-// PTX wrappers for mbarriers, TMA tile loads (never with cluster multicast),
+// PTX wrappers for mbarriers, TMA tile loads (each into one CTA's own smem),
 // tcgen05 (TMEM alloc / MMA / commit / load), bounded waits that record a
 // status code instead of hanging, and small bf16 / warp utilities.
 #pragma once
@@ -99,7 +99,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 
 // ----------------------------------------------------------------- TMA
 // Tile loads global -> shared, completion signalled on `bar` by byte count.
-// Plain (non-multicast) form only.
+// Plain form: the tile lands in this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int32_t c0, int32_t c1) {
     asm volatile(

@@ -15,7 +15,9 @@
 //               and single-thread tcgen05.mma issuer (M=128, N=256, K=16)
 //   warps 2..5  epilogue: tcgen05.ld -> SwiGLU or plain -> bf16 -> global
 // The accumulator is double-buffered so the epilogue of tile i overlaps the
-// mainloop of tile i+1.  Tiles: for every expert, ceil(R_e/128) row tiles x
+// mainloop of tile i+1.  (Token rows on the MMA's M side and weight rows on N:
+// measured on B200, weights-stationary tiles with tokens on N -- 1-CTA or CTA
+// pair -- lost 20-45% to TMA issue throughput despite doing less MMA work.)  Tiles: for every expert, ceil(R_e/128) row tiles x
 // the output column tiles; row tiles of one expert are adjacent in the tile
 // order so the expert's weight tiles are read from HBM about once and served
 // from L2 to its other row tiles.  Row tiles may run past the segment end
@@ -25,7 +27,6 @@
 // loads and MMAs, frees TMEM and returns.
 #include "kernels.h"
 
-#include <mutex>
 
 namespace moe {
 namespace gemm {
@@ -41,13 +42,14 @@ constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
 constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 1024;
-constexpr uint32_t IDESC = idesc_bf16_f32<BM, BN_ACC>();
 
 enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
 
 template <int EPI>
 struct Cfg {
-    static constexpr int BN_OUT = EPI == EPI_SWIGLU ? 128 : 256;  // output columns per tile
+    static constexpr int BN_OUT = EPI == EPI_STORE ? 256 : 128;    // output columns per tile
+    static constexpr int BN_MMA = 256;                              // MMA N
+    static constexpr uint32_t TX = A_BYTES + BN_MMA * BK * 2;      // bytes per stage
 };
 
 struct Maps {
@@ -62,6 +64,7 @@ struct Maps {
 struct Params {
     const int32_t *offsets;  // [E+1]
     int E;
+    int rows_r;              // rows of the routed A buffer (T*K)
     int T;                   // shared rows; 0 = no shared experts
     int n_out_r, n_out_s;    // output columns
     int k_r, k_s;            // reduction lengths
@@ -82,7 +85,8 @@ struct Tile {
 
 template <int EPI>
 __device__ __forceinline__ Tile decode_tile(int idx, const int *tile_base, const int *seg,
-                                            const Params &p, int ntr, int mt_s, int nt_s) {
+                                            const int *segc, const Params &p, int ntr, int mt_s,
+                                            int nt_s) {
     constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
     Tile t;
     if (idx < ntr) {
@@ -91,7 +95,7 @@ __device__ __forceinline__ Tile decode_tile(int idx, const int *tile_base, const
             const int mid = (lo + hi) >> 1;
             if (tile_base[mid] <= idx) lo = mid; else hi = mid;
         }
-        const int cnt = seg[lo + 1] - seg[lo];
+        const int cnt = segc[lo];
         const int mt = (cnt + BM - 1) / BM;
         const int local = idx - tile_base[lo];
         const int n = local / mt, m = local - n * mt;
@@ -127,7 +131,7 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int64_
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) {
-    return g / (1.0f + __expf(-g)) * u;
+    return g * __frcp_rn(1.0f + __expf(-g)) * u;
 }
 
 template <int EPI>
@@ -143,7 +147,8 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_base[MAX_E + 1];
-    __shared__ int seg[MAX_E + 1];
+    __shared__ int seg[MAX_E];
+    __shared__ int segc[MAX_E];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -162,7 +167,15 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             if (e < p.E) {
                 lo = p.offsets[e];
                 cnt = p.offsets[e + 1] - lo;
+                // a segment outside [0, rows_r] or of negative length is
+                // treated as empty and reported
+                if (lo < 0 || cnt < 0 || lo + cnt > p.rows_r) {
+                    record_status(p.status, MOE_ERR_DEVICE_FAULT);
+                    lo = 0;
+                    cnt = 0;
+                }
                 seg[e] = lo;
+                segc[e] = cnt;
             }
             const int v = ((cnt + BM - 1) / BM) * nt_r;
             int incl = v;
@@ -176,7 +189,6 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         }
         if (lane == 0) {
             tile_base[p.E] = carry;
-            seg[p.E] = p.offsets[p.E];
             tma_prefetch_desc(&maps.a_r);
             tma_prefetch_desc(&maps.b0_r);
             if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
@@ -220,7 +232,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             uint32_t phase = 0;
             uint32_t n_issued = 0;
             for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-                const Tile t = decode_tile<EPI>(idx, tile_base, seg, p, ntr, mt_s, nt_s);
+                const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
                 bool ok = true;
                 for (int kb = 0; kb < t.kblocks; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
@@ -232,7 +244,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                     const uint32_t a_dst = smem0 + stage * STAGE_BYTES;
                     const uint32_t b_dst = a_dst + A_BYTES;
                     const int k = kb * BK;
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    mbar_arrive_expect_tx(fb, Cfg<EPI>::TX);
                     if (t.e >= 0) {
                         tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
                         if (EPI == EPI_SWIGLU) {
@@ -273,7 +285,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             int acc = 0;
             uint32_t acc_phase = 0;
             for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-                const Tile t = decode_tile<EPI>(idx, tile_base, seg, p, ntr, mt_s, nt_s);
+                const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
                 if (!mbar_wait_bounded(smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag,
                                        p.status, p.timeout_ns))
                     break;
@@ -292,7 +304,8 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                     const uint64_t b_desc = smem_desc_sw128(a_addr + A_BYTES);
 #pragma unroll
                     for (int ks = 0; ks < BK / 16; ++ks)
-                        tc_mma_bf16(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks, IDESC,
+                        tc_mma_bf16(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks,
+                                    idesc_bf16_f32<BM, Cfg<EPI>::BN_MMA>(),
                                     (kb | ks) != 0 ? 1u : 0u);
                     tc_commit(smem_u32(&empty_bar[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -313,7 +326,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            const Tile t = decode_tile<EPI>(idx, tile_base, seg, p, ntr, mt_s, nt_s);
+            const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
             if (!mbar_wait_bounded(smem_u32(&tfull_bar[acc]), acc_phase, abort_flag, p.status,
                                    p.timeout_ns))
                 break;
@@ -398,48 +411,15 @@ __global__ void bounded_wait_selftest_kernel(int32_t *status, int64_t timeout_ns
 
 // ---------------------------------------------------------------- host side
 namespace {
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
 // 2-D bf16 map over [rows, cols] row-major, box 64 (cols) x box_rows.
 bool map_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {BK, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tensor_map_2d_bf16(m, base, rows, cols, BK, box_rows);
 }
 
 // 3-D bf16 map over [n_mat, rows, cols], box 64 (cols) x box_rows x 1.
 bool map_3d(CUtensorMap *m, const void *base, uint64_t n_mat, uint64_t rows, uint64_t cols,
             uint32_t box_rows) {
-    const cuuint64_t dims[3] = {cols, rows, n_mat};
-    const cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
-    const cuuint32_t box[3] = {BK, box_rows, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
-                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tensor_map_3d_bf16(m, base, n_mat, rows, cols, BK, box_rows);
 }
 
 int sm_count() {
@@ -463,7 +443,7 @@ cudaError_t launch_one(const Maps &maps, const Params &p, cudaStream_t st) {
 
 cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     using namespace gemm;
-    if (!encode_fn()) return cudaErrorNotSupported;
+    if (!tensor_maps_available()) return cudaErrorNotSupported;
     const uint64_t rows_r = (uint64_t)a.T * a.K;
     const bool has_shared = a.n_shared > 0 && a.T > 0;
     const int ffs = a.n_shared * a.d_ff_shared;
@@ -484,6 +464,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     Params p1{};
     p1.offsets = a.offsets;
     p1.E = a.E;
+    p1.rows_r = (int)rows_r;
     p1.T = has_shared ? a.T : 0;
     p1.n_out_r = a.d_ff;
     p1.n_out_s = ffs;

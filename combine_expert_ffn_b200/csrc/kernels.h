@@ -13,9 +13,14 @@ namespace moe {
 // Counts one kernel launch (process-wide, for moe_launch_count()).
 void count_launch();
 
+// tmap.cu: bf16 tensor maps, 128-byte swizzle, box = box_cols x box_rows (x 1)
+bool tensor_maps_available();
+bool tensor_map_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                        uint32_t box_cols, uint32_t box_rows);
+bool tensor_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t n_mat, uint64_t rows,
+                        uint64_t cols, uint32_t box_cols, uint32_t box_rows);
+
 // route.cu
-cudaError_t launch_router_logits(const void *x, const float *e, const float *off, int T, int d,
-                                 int E, float *scores, cudaStream_t st);
 cudaError_t launch_route_select(const float *scores, const float *bias, int T, int E, int G,
                                 int K, int M, int32_t *topk_idx, float *topk_w, cudaStream_t st);
 
@@ -54,6 +59,12 @@ struct FfnArgs {
     int64_t timeout_ns;
 };
 cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st);
+// router_tc.cu: router affinities on the tensor cores; e (fp32 [E, d]) is
+// split into three bf16 parts in e_split ([3, E, d] bf16 scratch);
+// scores = sigmoid(x.e + off).
+cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *off, int T, int d,
+                                    int E, void *e_split, float *scores, int32_t *status,
+                                    int64_t timeout_ns, cudaStream_t st);
 cudaError_t launch_bounded_wait_selftest(int64_t timeout_ns, int32_t *status, cudaStream_t st);
 
 }  // namespace moe

@@ -116,8 +116,12 @@ MOE_API moe_status moe_clear_device_status(void *ws, void *stream);
  *   topk_idx     [T, K]   int32 out: chosen experts, descending b_i then
  *                               ascending index
  *   topk_w       [T, K]   fp32 out: gates, sum to 1 over the K slots
- *   scores       [T, E]   fp32 out or NULL: the affinities s
- * fp32 accumulation of x . e_i; s = 1 / (1 + expf(-L)).
+ *   scores       [T, E]   fp32 out or NULL (then kept in the workspace):
+ *                               the affinities s
+ *   ws, ws_bytes          workspace of moe_workspace_size(cfg) bytes (required)
+ * L = x . e_i on the tensor cores: e_i is split into three bf16 parts whose
+ * sum reproduces the fp32 value to ~2^-27 relative, the products are exact,
+ * and the accumulation is fp32; s = 1 / (1 + expf(-L)).
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *router_w,
                      const float *logit_offset, const float *bias,

@@ -31,7 +31,12 @@ __all__ = [
 ]
 
 _M32 = 0xFFFFFFFF
-_CHUNK = 1 << 20  # elements generated per pass (bounds int64 temporaries)
+_CHUNK = 1 << 20       # elements generated per pass on the CPU (bounds int64 temporaries)
+_CHUNK_GPU = 1 << 26   # ... and on a GPU (fewer, larger launches)
+
+
+def _chunk(device) -> int:
+    return _CHUNK_GPU if torch.device(device).type == "cuda" else _CHUNK
 
 
 @dataclass(frozen=True)
@@ -88,6 +93,13 @@ CONFIGS = {
                      x_sigma=1.0, e_sigma=_inv_sqrt(7168), bias_sigma=0.5, zipf_s=1.2),
 }
 
+# Reduced workloads for profiler captures: the V3 layer's dimensions and rows
+# per expert (T*K/E = 256) with fewer experts, so that a capture holds a few
+# GB on the device; DRAM traffic per token is that of the full layer.
+PROFILE_CONFIGS = {
+    "v3_e32": CONFIGS["v3"].replace(name="v3_e32", T=1024, E=32),
+}
+
 # Fixed tensor ids: salt of the counter-based generator.
 TENSOR_IDS = {
     "x": 1, "router_w": 2, "bias": 3, "w_gate": 4, "w_up": 5, "w_down": 6,
@@ -97,7 +109,7 @@ TENSOR_IDS = {
 
 
 def config(name: str) -> MoeShape:
-    return CONFIGS[name]
+    return CONFIGS[name] if name in CONFIGS else PROFILE_CONFIGS[name]
 
 
 # ---------------------------------------------------------------- hashing
@@ -148,8 +160,9 @@ def normal_slice(seed: int, tid: int, start: int, count: int, sigma: float,
         out.zero_()
         return out
     c = torch.tensor(_scale32(sigma), dtype=torch.float32, device=device)
-    for s in range(0, count, _CHUNK):
-        n = min(_CHUNK, count - s)
+    step = _chunk(device)
+    for s in range(0, count, step):
+        n = min(step, count - s)
         idx = torch.arange(start + s, start + s + n, dtype=torch.int64, device=device)
         a, b = _words(seed, tid, idx)
         acc = (a & 0xFFFF) + (a >> 16) + (b & 0xFFFF) + (b >> 16)
@@ -232,8 +245,9 @@ def uniform01(seed: int, tid: int, shape, device="cpu") -> torch.Tensor:
     for s in shape:
         n *= int(s)
     out = torch.empty(n, dtype=torch.float32, device=device)
-    for s in range(0, n, _CHUNK):
-        m = min(_CHUNK, n - s)
+    step = _chunk(device)
+    for s in range(0, n, step):
+        m = min(step, n - s)
         idx = torch.arange(s, s + m, dtype=torch.int64, device=device)
         a, _ = _words(seed, tid, idx)
         out[s:s + m] = ((a >> 8).to(torch.float32) + 0.5) * (2.0 ** -24)

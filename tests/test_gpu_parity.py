@@ -106,8 +106,9 @@ def test_route_affinities_and_selection(orc, name, n_sample):
     sh = H.shape(name)
     inp = inputs(name)
     idx, w, s = _i32(sh.T, sh.K), _f32(sh.T, sh.K), _f32(sh.T, sh.E)
-    moe.moe_route(moe.MoeConfig.of(sh), inp["x"], inp["router_w"], inp.get("logit_offset"),
-                  inp["bias"], idx, w, scores=s)
+    cfg = moe.MoeConfig.of(sh)
+    moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"], idx, w,
+                  scores=s, ws=moe.alloc_workspace(cfg))
     rows = np.arange(sh.T) if n_sample is None else \
         np.unique(np.linspace(0, sh.T - 1, n_sample).astype(np.int64))
     ref_s = orc.router_scores(inp["x"].cpu(), inp["router_w"].cpu(), H.host(inp.get("logit_offset")),
@@ -239,6 +240,24 @@ def test_expert_ffn_segment_edges(orc):
     sh = synth.MoeShape("edges", T=sum(counts), d=192, E=len(counts), G=1, K=1, M=1, d_ff=192,
                         n_shared=1, d_ff_shared=192, x_sigma=1, e_sigma=1, bias_sigma=0)
     _ffn_case(orc, sh, counts)
+
+
+def test_expert_ffn_flags_bad_offsets():
+    """Offsets outside the buffer or decreasing are reported; nothing is written out of bounds."""
+    sh = H.RAGGED2.replace(T=64, n_shared=0, d_ff_shared=0)
+    cfg = moe.MoeConfig.of(sh)
+    n = sh.T * sh.K
+    x_perm = synth.normal(1, 21, (n, sh.d), 1.0, torch.bfloat16, DEV)
+    wg = synth.normal(1, 23, (sh.E, sh.d_ff, sh.d), 0.1, torch.bfloat16, DEV)
+    wd = synth.normal(1, 25, (sh.E, sh.d, sh.d_ff), 0.1, torch.bfloat16, DEV)
+    offsets = torch.linspace(0, n, sh.E + 1, device=DEV).to(torch.int32)
+    offsets[7] = offsets[9] + 5          # a decreasing pair
+    guard = torch.zeros(n + 64, sh.d, dtype=torch.bfloat16, device=DEV)
+    y_perm = guard[:n]
+    ws = moe.alloc_workspace(cfg)
+    moe.moe_expert_ffn(cfg, x_perm, offsets, wg, wg, wd, y_perm, None, None, None, None, None, ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_ERR_DEVICE_FAULT
+    assert int(guard[n:].view(torch.int16).abs().sum()) == 0   # the tail guard is untouched
 
 
 @pytest.mark.parametrize("name", ["ragged", "ragged2", "noshared", "tiny"])
