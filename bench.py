@@ -81,16 +81,21 @@ def kernel_source_hash():
 
 
 def traffic_from_profile(sh):
-    """DRAM bytes per launch pair of the expert FFN from a committed ncu summary,
-    if it was taken on the current kernel source; else None."""
-    p = os.path.join(ROOT, "profiles", "expert_ffn_traffic.json")
+    """DRAM bytes per step of the expert FFN (both GEMM launches) from the committed
+    ncu summary, if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "expert_ffn_traffic.txt")
     if not os.path.exists(p):
         return None
+    d = {}
     with open(p) as f:
-        d = json.load(f)
+        for line in f:
+            if line.startswith("#") or ":" not in line:
+                continue
+            k, v = line.split(":", 1)
+            d[k.strip()] = v.strip()
     if d.get("source_sha256") != kernel_source_hash() or d.get("workload") != sh.name:
         return None
-    return d.get("dram_bytes_per_step")
+    return int(d["dram_bytes_per_step"])
 
 
 class ClockSampler:
@@ -158,13 +163,19 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v, world):
+def max_over_ranks(v, world, device="cuda"):
+    """The slowest rank's time (every rank gets the same value)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank, world, steps, ms_max):
+    """Whole-job throughput: every replica's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -336,7 +347,7 @@ def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    e2e_value = job_tokens_per_s(T, world, args.steps, e2e_ms)
     if not torch.equal(out_host, o["out"].cpu()) and world == 1:
         raise RuntimeError("moe_forward and the staged calls disagree")
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
@@ -346,7 +357,7 @@ def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world):
 def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
     T = sh.T
     ms_step = ms_total / args.steps
-    value = world * T * args.steps / (ms_total / 1e3)
+    value = job_tokens_per_s(T, world, args.steps, ms_total)
     peaks = load_peaks()
     alg = algorithmic(sh)
     ffn_s = stage_ms["expert_ffn"] / 1e3
