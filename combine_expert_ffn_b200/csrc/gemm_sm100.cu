@@ -41,7 +41,8 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
-constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 1024;
+constexpr int STORE_BUF = 32 * 32 * 2;     // one warp's 32 rows x 32 columns of bf16
+constexpr int SMEM_DYN = STAGES * STAGE_BYTES + 4 * 2 * STORE_BUF + 1024;
 
 enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
 
@@ -59,6 +60,8 @@ struct Maps {
     CUtensorMap b1_r;  // routed B  up (SwiGLU only)
     CUtensorMap b0_s;  // shared B  gate | down
     CUtensorMap b1_s;  // shared B  up
+    CUtensorMap o_r;   // routed output [rows_r, n_out_r]    box 32 x 32, for full tiles
+    CUtensorMap o_s;   // shared output [T, n_out_s]         box 32 x 32
 };
 
 struct Params {
@@ -189,6 +192,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         }
         if (lane == 0) {
             tile_base[p.E] = carry;
+            tma_prefetch_desc(&maps.o_r);
             tma_prefetch_desc(&maps.a_r);
             tma_prefetch_desc(&maps.b0_r);
             if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
@@ -321,8 +325,15 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         __syncwarp();
     } else {
         // ------------------------------------------------------ epilogue
+        // A full tile (128 valid rows) leaves through TMA stores: each warp
+        // stages its 32 rows x 32 columns (64-byte rows) in shared memory and
+        // one lane stores the box, so global writes are whole 64-byte row
+        // pieces.  Rows of a partial tile that belong to the next expert must
+        // not be written, so partial tiles use masked direct stores.
         const int q = warp & 3;            // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;     // accumulator row = tile row
+        const uint32_t stage_buf0 = smem0 + STAGES * STAGE_BYTES + (warp - 2) * 2 * STORE_BUF;
+        int sb = 0;                        // staging buffer toggle
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
@@ -335,55 +346,68 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             const bool shared = t.e < 0;
             const int n_out = shared ? p.n_out_s : p.n_out_r;
             __nv_bfloat16 *orow = (shared ? p.out_s : p.out_r) + (size_t)(t.row0 + row) * n_out;
+            const CUtensorMap *omap = shared ? &maps.o_s : &maps.o_r;
+            const bool full = t.rows_valid == BM;
             const bool row_ok = row < t.rows_valid;
-            if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
-                for (int c = 0; c < BN_OUT; c += 32) {
+            for (int c = 0; c < BN_OUT; c += 32) {
+                uint4 o[4];
+                if (EPI == EPI_SWIGLU) {
                     uint32_t g[32], u[32];
                     tmem_ld32(taddr + c, g);
                     tmem_ld32(taddr + BN_ACC / 2 + c, u);
                     tc_wait_ld();
-                    if (row_ok && t.n0 + c < n_out) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + t.n0 + c);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint4 o;
-                            o.x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
-                                              silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
-                            o.y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
-                                              silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
-                            o.z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
-                                              silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
-                            o.w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
-                                              silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
-                            dst[v] = o;
-                        }
+                    for (int v = 0; v < 4; ++v) {
+                        o[v].x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
+                                             silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
+                        o[v].y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
+                                             silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
+                        o[v].z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
+                                             silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
+                        o[v].w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
+                                             silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
                     }
-                }
-            } else {
-#pragma unroll 1
-                for (int c = 0; c < BN_OUT; c += 32) {
+                } else {
                     uint32_t r[32];
                     tmem_ld32(taddr + c, r);
                     tc_wait_ld();
-                    if (row_ok && t.n0 + c < n_out) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + t.n0 + c);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-                            o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-                            o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-                            o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-                            dst[v] = o;
-                        }
+                    for (int v = 0; v < 4; ++v) {
+                        o[v].x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                        o[v].y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                        o[v].z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                        o[v].w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
                     }
+                }
+                if (t.n0 + c >= n_out) continue;     // whole chunk past the last column
+                if (full) {
+                    // staging buffer sb: the store that last read it must be done
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    const uint32_t buf = stage_buf0 + sb * STORE_BUF;
+                    uint4 *sp = reinterpret_cast<uint4 *>(smem + (buf - smem0)) + lane * 4;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) sp[v] = o[v];
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(omap, buf, t.n0 + c, t.row0 + q * 32);
+                        bulk_commit_group();
+                    }
+                    sb ^= 1;
+                } else if (row_ok) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + t.n0 + c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = o[v];
                 }
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty_bar[acc]));
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
+        if (lane == 0) bulk_wait_group_all();  // every staged store has landed
+        __syncwarp();
     }
 
     // ---------------------------------------------------------- teardown
@@ -460,6 +484,12 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
              map_3d(&m1.b1_s, a.ws_up, 1, ffs, a.d, BN_ACC / 2);
     else
         m1.a_s = m1.a_r, m1.b0_s = m1.b0_r, m1.b1_s = m1.b1_r;
+    // output maps for the full-tile TMA stores (box 32 x 32, no swizzle)
+    ok = ok && tensor_map_2d_bf16(&m1.o_r, a.h, rows_r, a.d_ff, 32, 32, 0);
+    if (has_shared)
+        ok = ok && tensor_map_2d_bf16(&m1.o_s, a.h_shared, a.T, ffs, 32, 32, 0);
+    else
+        m1.o_s = m1.o_r;
     if (!ok) return cudaErrorInvalidValue;
     Params p1{};
     p1.offsets = a.offsets;
@@ -489,6 +519,11 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
         m2.a_s = m2.a_r, m2.b0_s = m2.b0_r;
     m2.b1_r = m2.b0_r;
     m2.b1_s = m2.b0_s;
+    ok = ok && tensor_map_2d_bf16(&m2.o_r, a.y_perm, rows_r, a.d, 32, 32, 0);
+    if (has_shared)
+        ok = ok && tensor_map_2d_bf16(&m2.o_s, a.y_shared, a.T, a.d, 32, 32, 0);
+    else
+        m2.o_s = m2.o_r;
     if (!ok) return cudaErrorInvalidValue;
     Params p2 = p1;
     p2.n_out_r = a.d;

@@ -13,12 +13,14 @@ namespace moe {
 // Counts one kernel launch (process-wide, for moe_launch_count()).
 void count_launch();
 
-// tmap.cu: bf16 tensor maps, 128-byte swizzle, box = box_cols x box_rows (x 1)
+// tmap.cu: bf16 tensor maps, box = box_cols x box_rows (x 1), swizzle of
+// swizzle_bytes (64 or 128 = the box's row length in bytes; 0 = none)
 bool tensor_maps_available();
 bool tensor_map_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
-                        uint32_t box_cols, uint32_t box_rows);
+                        uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes = 128);
 bool tensor_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t n_mat, uint64_t rows,
-                        uint64_t cols, uint32_t box_cols, uint32_t box_rows);
+                        uint64_t cols, uint32_t box_cols, uint32_t box_rows,
+                        uint32_t swizzle_bytes = 128);
 
 // route.cu
 cudaError_t launch_route_select(const float *scores, const float *bias, int T, int E, int G,

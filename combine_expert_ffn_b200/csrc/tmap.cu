@@ -1,5 +1,5 @@
-// tmap.cu -- host-side TMA tensor-map encoding for bf16 tiles with 128-byte
-// swizzle (cuTensorMapEncodeTiled, resolved through the runtime's driver
+// tmap.cu -- host-side TMA tensor-map encoding for bf16 tiles with 64- or
+// 128-byte swizzle (cuTensorMapEncodeTiled, resolved through the runtime's driver
 // entry point so that the library needs no link-time libcuda).
 #include <mutex>
 
@@ -30,8 +30,15 @@ EncodeTiledFn encode_fn() {
 
 bool tensor_maps_available() { return encode_fn() != nullptr; }
 
+namespace {
+CUtensorMapSwizzle swizzle_for(uint32_t bytes) {
+    return bytes == 0 ? CU_TENSOR_MAP_SWIZZLE_NONE
+                      : bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+}
+}  // namespace
+
 bool tensor_map_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
-                        uint32_t box_cols, uint32_t box_rows) {
+                        uint32_t box_cols, uint32_t box_rows, uint32_t swizzle_bytes) {
     if (!encode_fn()) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
@@ -39,12 +46,13 @@ bool tensor_map_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_
     const cuuint32_t estr[2] = {1, 1};
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       swizzle_for(swizzle_bytes), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool tensor_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t n_mat, uint64_t rows,
-                        uint64_t cols, uint32_t box_cols, uint32_t box_rows) {
+                        uint64_t cols, uint32_t box_cols, uint32_t box_rows,
+                        uint32_t swizzle_bytes) {
     if (!encode_fn()) return false;
     const cuuint64_t dims[3] = {cols, rows, n_mat};
     const cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
@@ -52,7 +60,7 @@ bool tensor_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t n_mat, uint64
     const cuuint32_t estr[3] = {1, 1, 1};
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       swizzle_for(swizzle_bytes), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
