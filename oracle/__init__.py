@@ -46,9 +46,18 @@ def lib():
         _lib.oracle_combine.argtypes = [i32, i32, i32, i64, P, P, P, P, P]
         _lib.oracle_layer_rows.argtypes = [i32, P, i32, i32, i32, i32, i32, i32, i32, i32,
                                            P, P, P, P, P, P, P, P, P, P, i32, P, P, P, P]
+        _lib.oracle_router_affinity.argtypes = [i32, P, i32, i32, P, P, P, i32, P]
+        _lib.oracle_layer_rows_ex.argtypes = [i32, P, i32, i32, i32, i32, i32, i32, i32, i32,
+                                              P, P, P, P, i32, P, P, P, P, P, P, P, i32, P, P,
+                                              P, P]
+        _lib.oracle_hash_route.argtypes = [i32, P, i32, i32, i32, i32, P, P]
+        _lib.oracle_lowbias32.argtypes = [C.c_uint32]
+        _lib.oracle_lowbias32.restype = C.c_uint32
+        _lib.oracle_bias_update.argtypes = [i32, i32, i32, P, C.c_float, P]
         for f in ("oracle_router_scores", "oracle_select", "oracle_dispatch",
                   "oracle_ffn_row", "oracle_shared_row", "oracle_combine",
-                  "oracle_layer_rows"):
+                  "oracle_layer_rows", "oracle_router_affinity", "oracle_layer_rows_ex",
+                  "oracle_hash_route", "oracle_bias_update"):
             getattr(_lib, f).restype = C.c_int
     return _lib
 
@@ -80,8 +89,13 @@ def _check(rc, what):
         raise RuntimeError(f"{what} failed with oracle status {rc}")
 
 
-def router_scores(x, e, logit_offset=None, rows=None):
-    """fp32 affinities sigmoid(x[rows] . e_i + o_i), shape [n_rows, E]."""
+AFFINITY_SIGMOID, AFFINITY_SQRT_SOFTPLUS = 0, 1
+ROUTER_SIGMOID, ROUTER_SQRT_SOFTPLUS, ROUTER_HASH = 0, 1, 2
+
+
+def router_scores(x, e, logit_offset=None, rows=None, affinity=AFFINITY_SIGMOID):
+    """fp32 affinities f(x[rows] . e_i + o_i), shape [n_rows, E]; f = sigmoid
+    (affinity 0) or sqrt(softplus) (affinity 1)."""
     x = _np(x, np.uint16)
     e = _np(e, np.float32)
     off = None if logit_offset is None else _np(logit_offset, np.float32)
@@ -90,9 +104,32 @@ def router_scores(x, e, logit_offset=None, rows=None):
     r = None if rows is None else _np(np.asarray(rows, dtype=np.int64), np.int64)
     n = T if r is None else len(r)
     out = np.empty((n, E), np.float32)
-    _check(lib().oracle_router_scores(n, _p(r), d, E, _p(x), _p(e), _p(off), _p(out)),
-           "oracle_router_scores")
+    _check(lib().oracle_router_affinity(n, _p(r), d, E, _p(x), _p(e), _p(off), int(affinity),
+                                        _p(out)), "oracle_router_affinity")
     return out
+
+
+def lowbias32(v):
+    return int(lib().oracle_lowbias32(C.c_uint32(int(v) & 0xFFFFFFFF)))
+
+
+def hash_route(token_ids, E, G, K, M):
+    """Hash router: returns (topk_idx int32 [n,K], topk_w fp32 [n,K]) for int64 token ids."""
+    ids = _np(np.asarray(token_ids, dtype=np.int64), np.int64)
+    n = len(ids)
+    idx = np.empty((n, K), np.int32)
+    w = np.empty((n, K), np.float32)
+    _check(lib().oracle_hash_route(n, _p(ids), E, G, K, M, _p(idx), _p(w)), "oracle_hash_route")
+    return idx, w
+
+
+def bias_update(counts, T, K, gamma, bias):
+    """Returns bias + gamma * sign(T*K/E - counts) (fp32), the input left as is."""
+    c = _np(np.asarray(counts, dtype=np.int32), np.int32)
+    b = np.array(_np(bias, np.float32), copy=True)
+    _check(lib().oracle_bias_update(len(c), int(T), int(K), _p(c), C.c_float(gamma), _p(b)),
+           "oracle_bias_update")
+    return b
 
 
 def select(scores, bias, G, K, M, want_group_score=False):
@@ -159,18 +196,21 @@ def combine(y_perm, inv_perm, topk_w, y_shared=None):
 
 
 def layer_rows(rows, shape, x, router_w, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
-               logit_offset=None, round_h=False):
+               logit_offset=None, round_h=False, router=ROUTER_SIGMOID, token_ids=None):
     """The whole layer for the token rows ``rows``.
 
     ``w_gate``/``w_up``/``w_down`` are sequences of per-expert host matrices
     (entries may be None for experts no listed token selects).
+    ``router`` is ROUTER_SIGMOID, ROUTER_SQRT_SOFTPLUS or ROUTER_HASH (the
+    last keyed by ``token_ids[row]``, or the row index when None).
     Returns (out float64 [n,d], topk_idx [n,K], topk_w [n,K], scores [n,E]).
     """
     r = _np(np.asarray(rows, dtype=np.int64), np.int64)
     x = _np(x, np.uint16)
-    e = _np(router_w, np.float32)
-    b = _np(bias, np.float32)
+    e = None if router_w is None else _np(router_w, np.float32)
+    b = None if bias is None else _np(bias, np.float32)
     off = None if logit_offset is None else _np(logit_offset, np.float32)
+    tid = None if token_ids is None else _np(np.asarray(token_ids, dtype=np.int64), np.int64)
     keep = []
 
     def parr(mats):
@@ -189,11 +229,12 @@ def layer_rows(rows, shape, x, router_w, bias, w_gate, w_up, w_down, ws_gate, ws
     idx = np.empty((n, shape.K), np.int32)
     w = np.empty((n, shape.K), np.float32)
     sc = np.empty((n, shape.E), np.float32)
-    rc = lib().oracle_layer_rows(n, _p(r), shape.d, shape.E, shape.G, shape.K, shape.M,
-                                 shape.d_ff, shape.n_shared, shape.d_ff_shared,
-                                 _p(x), _p(e), _p(off), _p(b),
-                                 C.cast(g, C.c_void_p), C.cast(u, C.c_void_p),
-                                 C.cast(dn, C.c_void_p), _p(sg), _p(su), _p(sd),
-                                 int(round_h), _p(out), _p(idx), _p(w), _p(sc))
-    _check(rc, "oracle_layer_rows")
+    sc.fill(np.nan)
+    rc = lib().oracle_layer_rows_ex(n, _p(r), shape.d, shape.E, shape.G, shape.K, shape.M,
+                                    shape.d_ff, shape.n_shared, shape.d_ff_shared,
+                                    _p(x), _p(e), _p(off), _p(b), int(router), _p(tid),
+                                    C.cast(g, C.c_void_p), C.cast(u, C.c_void_p),
+                                    C.cast(dn, C.c_void_p), _p(sg), _p(su), _p(sd),
+                                    int(round_h), _p(out), _p(idx), _p(w), _p(sc))
+    _check(rc, "oracle_layer_rows_ex")
     return out, idx, w, sc

@@ -65,13 +65,29 @@ static int beats(float bi, int i, float bj, int j)
 }
 
 /* ------------------------------------------------------------------ 1 */
-/* scores[r*E + i] = sigmoid(sum_k x[rows[r], k] * e[i, k] + off[i]) for the
- * listed token rows (rows == NULL: rows 0..n_rows-1).  Rounded once to fp32. */
-int oracle_router_scores(int n_rows, const int64_t *rows, int d, int E,
-                         const uint16_t *x, const float *e, const float *off,
-                         float *scores)
+/* Router affinity of either kind from a double-precision logit:
+ *   kind 0: sigmoid(L)                 (DeepSeek-V3)
+ *   kind 1: sqrt(softplus(L)),  softplus(L) = log(1 + e^L)  ("MoE +
+ *           Expert-Parallel Overlap (Exp08)", Implemented: top-k gating over
+ *           Sqrt(Softplus(.)) affinities, the V4 change)
+ * Rounded once to fp32. */
+static float affinity_of(double L, int kind)
 {
-    if (n_rows < 0 || d <= 0 || E <= 0 || !x || !e || !scores)
+    if (kind == 1) {
+        const double sp = L > 0.0 ? L + log1p(exp(-L)) : log1p(exp(L));
+        return (float)sqrt(sp);
+    }
+    return (float)(1.0 / (1.0 + exp(-L)));
+}
+
+/* scores[r*E + i] = affinity(sum_k x[rows[r], k] * e[i, k] + off[i]) of the
+ * given kind (0 or 1) for the listed token rows (rows == NULL: rows
+ * 0..n_rows-1), the sum in double. */
+int oracle_router_affinity(int n_rows, const int64_t *rows, int d, int E,
+                           const uint16_t *x, const float *e, const float *off,
+                           int kind, float *scores)
+{
+    if (n_rows < 0 || d <= 0 || E <= 0 || !x || !e || !scores || kind < 0 || kind > 1)
         return ORC_EBADARG;
     for (int r = 0; r < n_rows; ++r) {
         int64_t t = rows ? rows[r] : r;
@@ -83,10 +99,19 @@ int oracle_router_scores(int n_rows, const int64_t *rows, int d, int E,
                 acc += bf16_value(xt[k]) * (double)ei[k];
             if (off)
                 acc += (double)off[i];
-            scores[(int64_t)r * E + i] = (float)(1.0 / (1.0 + exp(-acc)));
+            scores[(int64_t)r * E + i] = affinity_of(acc, kind);
         }
     }
     return ORC_OK;
+}
+
+/* scores[r*E + i] = sigmoid(sum_k x[rows[r], k] * e[i, k] + off[i]) for the
+ * listed token rows (rows == NULL: rows 0..n_rows-1).  Rounded once to fp32. */
+int oracle_router_scores(int n_rows, const int64_t *rows, int d, int E,
+                         const uint16_t *x, const float *e, const float *off,
+                         float *scores)
+{
+    return oracle_router_affinity(n_rows, rows, d, E, x, e, off, 0, scores);
 }
 
 /* ------------------------------------------------------------------ 2-4 */
@@ -341,19 +366,27 @@ int oracle_combine(int T, int d, int K, int64_t n_perm_rows,
  * entry may be NULL if no listed token selects that expert.
  * Outputs: out[n_rows, d] (double), topk_idx/topk_w [n_rows, K],
  * scores [n_rows, E] (may be NULL). */
-int oracle_layer_rows(int n_rows, const int64_t *rows,
-                      int d, int E, int G, int K, int M, int d_ff,
-                      int n_shared, int d_ff_s,
-                      const uint16_t *x, const float *e, const float *off,
-                      const float *bias,
-                      const uint16_t *const *Wg, const uint16_t *const *Wu,
-                      const uint16_t *const *Wd,
-                      const uint16_t *Wsg, const uint16_t *Wsu, const uint16_t *Wsd,
-                      int round_h, double *out, int32_t *topk_idx, float *topk_w,
-                      float *scores_out)
+int oracle_hash_route(int n_rows, const int64_t *token_ids, int E, int G, int K, int M,
+                      int32_t *topk_idx, float *topk_w);
+
+/* The layer for the listed rows with a chosen router:
+ *   router 0: sigmoid affinities + node-limited top-K (DeepSeek-V3)
+ *   router 1: sqrt(softplus) affinities + the same selection (V4)
+ *   router 2: hash router keyed by token_ids[rows[r]] (or rows[r] when
+ *             token_ids is NULL); e, off, bias unused, scores_out untouched. */
+int oracle_layer_rows_ex(int n_rows, const int64_t *rows,
+                         int d, int E, int G, int K, int M, int d_ff,
+                         int n_shared, int d_ff_s,
+                         const uint16_t *x, const float *e, const float *off,
+                         const float *bias, int router, const int64_t *token_ids,
+                         const uint16_t *const *Wg, const uint16_t *const *Wu,
+                         const uint16_t *const *Wd,
+                         const uint16_t *Wsg, const uint16_t *Wsu, const uint16_t *Wsd,
+                         int round_h, double *out, int32_t *topk_idx, float *topk_w,
+                         float *scores_out)
 {
-    if (n_rows < 0 || !rows || !x || !e || !bias || !Wg || !Wu || !Wd || !out ||
-        !topk_idx || !topk_w)
+    if (n_rows < 0 || !rows || !x || !Wg || !Wu || !Wd || !out || !topk_idx || !topk_w ||
+        router < 0 || router > 2 || (router < 2 && (!e || !bias)))
         return ORC_EBADARG;
     int rc = ORC_OK;
     float *scores = malloc(sizeof(float) * (size_t)E * (n_rows > 0 ? n_rows : 1));
@@ -362,10 +395,17 @@ int oracle_layer_rows(int n_rows, const int64_t *rows,
         rc = ORC_ENOMEM;
         goto done;
     }
-    rc = oracle_router_scores(n_rows, rows, d, E, x, e, off, scores);
-    if (rc)
-        goto done;
-    rc = oracle_select(n_rows, E, G, K, M, scores, bias, topk_idx, topk_w, NULL);
+    if (router == 2) {
+        for (int r = 0; r < n_rows && !rc; ++r) {
+            const int64_t id = token_ids ? token_ids[rows[r]] : rows[r];
+            rc = oracle_hash_route(1, &id, E, G, K, M, topk_idx + (int64_t)r * K,
+                                   topk_w + (int64_t)r * K);
+        }
+    } else {
+        rc = oracle_router_affinity(n_rows, rows, d, E, x, e, off, router, scores);
+        if (!rc)
+            rc = oracle_select(n_rows, E, G, K, M, scores, bias, topk_idx, topk_w, NULL);
+    }
     if (rc)
         goto done;
     for (int r = 0; r < n_rows; ++r) {
@@ -388,10 +428,117 @@ int oracle_layer_rows(int n_rows, const int64_t *rows,
                 o[k] += w * y[k];
         }
     }
-    if (scores_out)
+    if (scores_out && router != 2)
         memcpy(scores_out, scores, sizeof(float) * (size_t)E * n_rows);
 done:
     free(scores);
     free(y);
     return rc;
+}
+
+int oracle_layer_rows(int n_rows, const int64_t *rows,
+                      int d, int E, int G, int K, int M, int d_ff,
+                      int n_shared, int d_ff_s,
+                      const uint16_t *x, const float *e, const float *off,
+                      const float *bias,
+                      const uint16_t *const *Wg, const uint16_t *const *Wu,
+                      const uint16_t *const *Wd,
+                      const uint16_t *Wsg, const uint16_t *Wsu, const uint16_t *Wsd,
+                      int round_h, double *out, int32_t *topk_idx, float *topk_w,
+                      float *scores_out)
+{
+    return oracle_layer_rows_ex(n_rows, rows, d, E, G, K, M, d_ff, n_shared, d_ff_s, x, e, off,
+                                bias, 0, NULL, Wg, Wu, Wd, Wsg, Wsu, Wsd, round_h, out, topk_idx,
+                                topk_w, scores_out);
+}
+
+/* ------------------------------------------------------------------ hash router */
+/* "a hash router for early-layer emulation" (Exp08, Implemented).  The page
+ * gives no formula; the reading used here keeps the node limit: the token's
+ * M groups and, inside each, its K/M experts are drawn without replacement by
+ * a partial Fisher-Yates shuffle driven by the public "lowbias32" integer hash
+ * (C. Wellons) of the token id; every gate is 1/K. */
+static uint32_t lowbias32(uint32_t x)
+{
+    x ^= x >> 16;
+    x *= 0x7FEB352Du;
+    x ^= x >> 15;
+    x *= 0x846CA68Bu;
+    x ^= x >> 16;
+    return x;
+}
+
+uint32_t oracle_lowbias32(uint32_t x) { return lowbias32(x); }
+
+/* m distinct values of [0, n) in draw order: step i swaps position i with
+ * position i + (hash(seed ^ i * 0x9E3779B9) mod (n - i)) of the virtual array
+ * a[k] = k and takes the value that lands at i. */
+static int partial_shuffle(uint32_t n, uint32_t m, uint32_t seed, int32_t *out)
+{
+    uint32_t pos[64], val[64];
+    int used = 0;
+    if (m > n || m > 32)
+        return ORC_EBADARG;
+    for (uint32_t i = 0; i < m; ++i) {
+        const uint32_t j = i + lowbias32(seed ^ (i * 0x9E3779B9u)) % (n - i);
+        uint32_t vi = i, vj = j;
+        int si = -1, sj = -1;
+        for (int q = 0; q < used; ++q) {
+            if (pos[q] == i) { vi = val[q]; si = q; }
+            if (pos[q] == j) { vj = val[q]; sj = q; }
+        }
+        if (si < 0) { pos[used] = i; si = used++; }
+        if (sj < 0 && j != i) { pos[used] = j; sj = used++; }
+        val[si] = vj;
+        if (j != i)
+            val[sj] = vi;
+        out[i] = (int32_t)vj;
+    }
+    return ORC_OK;
+}
+
+int oracle_hash_route(int n_rows, const int64_t *token_ids, int E, int G, int K, int M,
+                      int32_t *topk_idx, float *topk_w)
+{
+    if (n_rows < 0 || E <= 0 || G <= 0 || K <= 0 || M <= 0 || E % G || K % M || M > G ||
+        K / M > E / G || G > 64 || K > 32 || !topk_idx || !topk_w)
+        return ORC_EBADARG;
+    const int gsz = E / G, kpg = K / M;
+    for (int r = 0; r < n_rows; ++r) {
+        const uint64_t tau = token_ids ? (uint64_t)token_ids[r] : (uint64_t)r;
+        const uint32_t s0 = lowbias32((uint32_t)tau ^ lowbias32((uint32_t)(tau >> 32) ^ 0x68E31DA4u));
+        int32_t groups[64], local[32];
+        if (partial_shuffle((uint32_t)G, (uint32_t)M, s0, groups))
+            return ORC_EBADARG;
+        for (int gi = 0; gi < M; ++gi) {
+            const uint32_t g = (uint32_t)groups[gi];
+            if (partial_shuffle((uint32_t)gsz, (uint32_t)kpg, lowbias32(s0 ^ ((g + 1u) * 0x85EBCA6Bu)), local))
+                return ORC_EBADARG;
+            for (int q = 0; q < kpg; ++q) {
+                topk_idx[(int64_t)r * K + gi * kpg + q] = (int32_t)(g * gsz) + local[q];
+                topk_w[(int64_t)r * K + gi * kpg + q] = 1.0f / (float)K;
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ bias update */
+/* Auxiliary-loss-free balancing: "per-expert bias updates" (Exp08,
+ * Implemented).  The step rule (DeepSeek-V3's sign rule; the step size is not
+ * on the pages, so it is a parameter): an expert above the mean load
+ * T*K/E moves down by gamma, one below moves up, one at the mean stays:
+ *   bias_i <- bias_i + gamma * sign(T*K/E - counts_i)     (one fp32 add)
+ * The comparison is exact: counts_i * E against T * K in integers. */
+int oracle_bias_update(int E, int T, int K, const int32_t *counts, float gamma, float *bias)
+{
+    if (E <= 0 || T < 0 || K <= 0 || !counts || !bias)
+        return ORC_EBADARG;
+    const int64_t total = (int64_t)T * K;
+    for (int i = 0; i < E; ++i) {
+        const int64_t c = (int64_t)counts[i] * E;
+        const float step = c < total ? gamma : (c > total ? -gamma : 0.0f);
+        bias[i] = bias[i] + step;
+    }
+    return ORC_OK;
 }
