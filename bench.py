@@ -310,6 +310,8 @@ def run_ours(args, sh, world, rank, local):
     if rank != 0:
         return 0
     line = report(args, sh, world, ms_total, stage_ms, launches, clk, e2e)
+    if not args.no_variants:
+        line["variants"] = variants_leg(sh, inp, dev, stream)
     if world == 1 and not args.no_cpu_baseline:
         n = args.cpu_tokens
         v, dt = oracle_tokens_per_s(sh, inp, n)
@@ -352,6 +354,59 @@ def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world):
         raise RuntimeError("moe_forward and the staged calls disagree")
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
             "d2h_bytes_per_step": T * d * 2}
+
+
+def variants_leg(sh, inp, dev, stream, reps=20):
+    """Device times of the routing variants and the bias update (CUDA events,
+    mean over `reps` back-to-back launches after 3 warm-ups): the route stage
+    under each router, moe_forward under each router, and moe_bias_update.
+    Not part of the headline step."""
+    import combine_expert_ffn_b200 as moe
+    T, K, E = sh.T, sh.K, sh.E
+    ids = synth.token_ids(sh.seed, T, device=dev)
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    bias = inp["bias"].clone()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    out = {}
+    names = {moe.MOE_ROUTER_SIGMOID: "sigmoid", moe.MOE_ROUTER_SQRT_SOFTPLUS: "sqrt_softplus",
+             moe.MOE_ROUTER_HASH: "hash"}
+    for r, name in names.items():
+        cfg = moe.MoeConfig.of(sh, router=r)
+        ws = moe.alloc_workspace(cfg, dev)
+        o = moe.forward_outputs(cfg, dev)
+        if r == moe.MOE_ROUTER_HASH:
+            route = lambda: moe.moe_route_hash(cfg, ids, idx, w, stream)  # noqa: E731
+        else:
+            route = lambda: moe.moe_route(cfg, inp["x"], inp["router_w"],  # noqa: E731
+                                          inp.get("logit_offset"), inp["bias"], idx, w, None,
+                                          ws, stream)
+        fwd = lambda: moe.moe_forward(cfg, inp["x"], inp["router_w"],  # noqa: E731
+                                      inp.get("logit_offset"), inp["bias"], inp["w_gate"],
+                                      inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                                      inp.get("ws_up"), inp.get("ws_down"), o["out"],
+                                      counts=o["counts"], ws=ws, stream=stream, token_ids=ids)
+        route_ms, fwd_ms = timed(route), timed(fwd)
+        if moe.moe_read_device_status(ws, stream) != moe.MOE_OK:
+            raise RuntimeError(f"device status after the {name} router variant")
+        out[name] = {"route_ms": route_ms, "forward_ms": fwd_ms,
+                     "forward_tokens_per_s": T / (fwd_ms / 1e3)}
+        if r == moe.MOE_ROUTER_SIGMOID:
+            out["bias_update_ms"] = timed(lambda: moe.moe_bias_update(cfg, o["counts"], 1e-3,
+                                                                      bias, stream))
+        del ws, o
+    return out
 
 
 def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
@@ -412,6 +467,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the router-variant and bias-update timings")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -33,18 +33,24 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_WORKSPACE_TOO_SM
 EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_launch_count",
            "moe_read_device_status", "moe_clear_device_status", "moe_route", "moe_route_select",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
-           "moe_selftest_bounded_wait", "moe_dispatch_noalloc")
+           "moe_selftest_bounded_wait", "moe_dispatch_noalloc", "moe_route_hash",
+           "moe_bias_update")
+
+MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
 
 
 class MoeConfig(C.Structure):
     """Mirror of ``moe_config``."""
     _fields_ = [(n, C.c_int32) for n in
-                ("T", "d", "E", "G", "K", "M", "d_ff", "n_shared", "d_ff_shared")]
+                ("T", "d", "E", "G", "K", "M", "d_ff", "n_shared", "d_ff_shared", "router")]
 
     @classmethod
-    def of(cls, shape) -> "MoeConfig":
-        """From any object with the nine size attributes (e.g. ``synth.MoeShape``)."""
-        return cls(*(int(getattr(shape, n)) for n, _ in cls._fields_))
+    def of(cls, shape, router=None) -> "MoeConfig":
+        """From any object with the nine size attributes (e.g. ``synth.MoeShape``);
+        the router is ``router``, else the object's ``router``, else the sigmoid."""
+        if router is None:
+            router = getattr(shape, "router", MOE_ROUTER_SIGMOID)
+        return cls(*(int(getattr(shape, n)) for n, _ in cls._fields_[:-1]), int(router))
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -71,7 +77,9 @@ _sig = {
     "moe_expert_ffn": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_combine": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
-                              _P, _P, _P, _P, _S, _P]),
+                              _P, _P, _P, _P, _P, _S, _P]),
+    "moe_route_hash": (C.c_int, [_CP, _P, _P, _P, _P]),
+    "moe_bias_update": (C.c_int, [_CP, _P, C.c_float, _P, _P]),
     "moe_selftest_bounded_wait": (C.c_int, [_I64, _P, _P]),
     "moe_dispatch_noalloc": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
@@ -155,6 +163,16 @@ def moe_route(cfg, x, router_w, logit_offset, bias, topk_idx, topk_w, scores=Non
                                     _stream(stream)))
 
 
+def moe_route_hash(cfg, token_ids, topk_idx, topk_w, stream=None) -> None:
+    _ok("moe_route_hash", _lib.moe_route_hash(_cfg(cfg), _ptr(token_ids), _ptr(topk_idx),
+                                              _ptr(topk_w), _stream(stream)))
+
+
+def moe_bias_update(cfg, counts, gamma, bias, stream=None) -> None:
+    _ok("moe_bias_update", _lib.moe_bias_update(_cfg(cfg), _ptr(counts), C.c_float(gamma),
+                                                _ptr(bias), _stream(stream)))
+
+
 def moe_route_select(cfg, scores, bias, topk_idx, topk_w, stream=None) -> None:
     _ok("moe_route_select", _lib.moe_route_select(_cfg(cfg), _ptr(scores), _ptr(bias),
                                                   _ptr(topk_idx), _ptr(topk_w), _stream(stream)))
@@ -185,10 +203,11 @@ def moe_combine(cfg, y_perm, inv_perm, topk_w, y_shared, out, stream=None) -> No
 
 def moe_forward(cfg, x, router_w, logit_offset, bias, w_gate, w_up, w_down, ws_gate, ws_up,
                 ws_down, out, topk_idx=None, topk_w=None, counts=None, offsets=None, send=None,
-                send_tok=None, ws=None, stream=None) -> None:
+                send_tok=None, ws=None, stream=None, token_ids=None) -> None:
     wp, wn = _ws(ws)
     _ok("moe_forward", _lib.moe_forward(_cfg(cfg), _ptr(x), _ptr(router_w), _ptr(logit_offset),
-                                        _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                        _ptr(bias), _ptr(token_ids), _ptr(w_gate), _ptr(w_up),
+                                        _ptr(w_down),
                                         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(out),
                                         _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(offsets),
                                         _ptr(send), _ptr(send_tok), wp, wn, _stream(stream)))

@@ -103,6 +103,8 @@ moe_status moe_check_config(const moe_config *c) {
     if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->G <= 0 || c->K <= 0 || c->M <= 0 ||
         c->d_ff <= 0 || c->n_shared < 0 || c->d_ff_shared < 0)
         return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->router < MOE_ROUTER_SIGMOID || c->router > MOE_ROUTER_HASH)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->E % c->G || c->K % c->M || c->M > c->G || c->K / c->M > c->E / c->G)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->K > 32 || c->E > 1024 || c->G > 64) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -169,6 +171,7 @@ moe_status moe_route(const moe_config *c, const void *x, const float *router_w,
     moe_status st = moe_check_config(c);
     if (st) return st;
     if (!ws) return MOE_ERR_INVALID_ARG;
+    if (c->router == MOE_ROUTER_HASH) return MOE_ERR_INVALID_ARG;
     if (c->T > 0 && (!x || !router_w || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_INVALID_ARG;
     const Layout L = layout(*c);
@@ -177,11 +180,31 @@ moe_status moe_route(const moe_config *c, const void *x, const float *router_w,
     if (!scores) scores = at<float>(ws, L.scores);
     if ((st = check_device())) return st;
     cudaStream_t s = as_stream(stream);
-    if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, at<void>(ws, L.e_split),
-                                scores, at<int32_t>(ws, L.status), kWaitTimeoutNs, s))
+    if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, c->router,
+                                at<void>(ws, L.e_split), scores, at<int32_t>(ws, L.status),
+                                kWaitTimeoutNs, s))
         return MOE_ERR_CUDA;
     return cuda_status(
         launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s));
+}
+
+moe_status moe_route_hash(const moe_config *c, const int64_t *token_ids, int32_t *topk_idx,
+                          float *topk_w, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->T > 0 && (!topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_hash_route(token_ids, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w,
+                                         as_stream(stream)));
+}
+
+moe_status moe_bias_update(const moe_config *c, const int32_t *counts, float gamma, float *bias,
+                           void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!counts || !bias || !(gamma - gamma == 0.0f)) return MOE_ERR_INVALID_ARG;  // finite
+    if ((st = check_device())) return st;
+    return cuda_status(launch_bias_update(counts, c->E, c->T, c->K, gamma, bias, as_stream(stream)));
 }
 
 moe_status moe_dispatch(const moe_config *c, const void *x, const int32_t *topk_idx,
@@ -249,7 +272,8 @@ moe_status moe_combine(const moe_config *c, const void *y_perm, const int32_t *i
 }
 
 moe_status moe_forward(const moe_config *c, const void *x, const float *router_w,
-                       const float *logit_offset, const float *bias, const void *w_gate,
+                       const float *logit_offset, const float *bias, const int64_t *token_ids,
+                       const void *w_gate,
                        const void *w_up, const void *w_down, const void *ws_gate,
                        const void *ws_up, const void *ws_down, void *out, int32_t *topk_idx,
                        float *topk_w, int32_t *counts, int32_t *offsets, int32_t *send,
@@ -258,7 +282,8 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
     if (st) return st;
     if (!ws) return MOE_ERR_INVALID_ARG;
     if (c->T > 0) {
-        if (!x || !router_w || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+        if (!x || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+        if (c->router != MOE_ROUTER_HASH && !router_w) return MOE_ERR_INVALID_ARG;
         if (c->n_shared > 0 && (!ws_gate || !ws_up || !ws_down)) return MOE_ERR_INVALID_ARG;
     }
     const void *ptrs[] = {x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out};
@@ -285,11 +310,16 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
     void *y_sh = c->n_shared > 0 ? at<void>(ws, L.y_sh) : nullptr;
     int32_t *status = at<int32_t>(ws, L.status);
 
-    if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, at<void>(ws, L.e_split),
-                                scores, status, kWaitTimeoutNs, s))
-        return MOE_ERR_CUDA;
-    if (launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
-        return MOE_ERR_CUDA;
+    if (c->router == MOE_ROUTER_HASH) {
+        if (launch_hash_route(token_ids, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
+            return MOE_ERR_CUDA;
+    } else {
+        if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, c->router,
+                                    at<void>(ws, L.e_split), scores, status, kWaitTimeoutNs, s))
+            return MOE_ERR_CUDA;
+        if (launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
+            return MOE_ERR_CUDA;
+    }
     DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),
                   at<int32_t>(ws, L.send_part), at<int32_t>(ws, L.sendtok_part)};
     if (launch_dispatch(x, topk_idx, c->T, c->d, c->E, c->G, c->K, counts, offsets, send, send_tok,

@@ -63,10 +63,17 @@ struct FfnArgs {
 cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st);
 // router_tc.cu: router affinities on the tensor cores; e (fp32 [E, d]) is
 // split into three bf16 parts in e_split ([3, E, d] bf16 scratch);
-// scores = sigmoid(x.e + off).
+// scores = f(x.e + off), f = sigmoid (affinity 0) or sqrt(softplus) (1).
 cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *off, int T, int d,
-                                    int E, void *e_split, float *scores, int32_t *status,
-                                    int64_t timeout_ns, cudaStream_t st);
+                                    int E, int affinity, void *e_split, float *scores,
+                                    int32_t *status, int64_t timeout_ns, cudaStream_t st);
+
+// route_variants.cu: the hash router (token ids -> K experts in M groups,
+// gates 1/K; token_ids NULL = row index) and the per-expert bias update.
+cudaError_t launch_hash_route(const int64_t *token_ids, int T, int E, int G, int K, int M,
+                              int32_t *topk_idx, float *topk_w, cudaStream_t st);
+cudaError_t launch_bias_update(const int32_t *counts, int E, int T, int K, float gamma,
+                               float *bias, cudaStream_t st);
 cudaError_t launch_bounded_wait_selftest(int64_t timeout_ns, int32_t *status, cudaStream_t st);
 
 }  // namespace moe

@@ -1,9 +1,10 @@
 // router_tc.cu -- router affinities on the tensor cores.
 //
-//   s_i = sigmoid(x . e_i + o_i)      x bf16 [T, d], e fp32 [E, d]
+//   s_i = f(x . e_i + o_i)      x bf16 [T, d], e fp32 [E, d]
 // (top-k gating over expert affinities, "MoE + Expert-Parallel Overlap
-// (Exp08)", Implemented; the sigmoid form is DeepSeek-V3's; o_i is the
-// optional per-expert logit offset of the skewed-load workload.)
+// (Exp08)", Implemented; f is DeepSeek-V3's sigmoid, or the V4 form
+// sqrt(softplus(L)) named there; o_i is the optional per-expert logit offset
+// of the skewed-load workload.)
 //
 // The fp32 weights are split into three bf16 parts, e = hi + mid + lo to
 // about 2^-27 relative (each subtraction exact in fp32), so every product
@@ -19,7 +20,7 @@
 //               per stage, 3 stages of 64 KB
 //   warp 1      TMEM owner (4 buffers x 128 columns), single-thread MMA issuer
 //   warps 2..5  epilogue: per k block, TMEM -> registers (+=); per tile,
-//               sigmoid -> fp32 scores
+//               f -> fp32 scores
 #include "kernels.h"
 
 #include <algorithm>
@@ -44,6 +45,7 @@ struct Maps {
 
 struct Params {
     int T, E, d;
+    int affinity;  // 0: sigmoid, 1: sqrt(softplus)
     const float *off;
     float *scores;
     int32_t *status;
@@ -60,6 +62,12 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int64_
         }
     }
     return true;
+}
+
+// softplus(L) = log(1 + e^L), evaluated without overflow on either side
+__device__ __forceinline__ float sqrt_softplus(float L) {
+    const float sp = L > 0.f ? L + log1pf(expf(-L)) : log1pf(expf(L));
+    return sqrtf(sp);
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -221,7 +229,7 @@ router_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
                     if (col < p.E) {
                         float L = acc[c];
                         if (p.off) L += p.off[col];
-                        out[col] = 1.0f / (1.0f + expf(-L));
+                        out[col] = p.affinity == 1 ? sqrt_softplus(L) : 1.0f / (1.0f + expf(-L));
                     }
                 }
             }
@@ -256,8 +264,8 @@ __global__ void router_split_kernel(const float *__restrict__ e, int64_t n,
 }  // namespace router
 
 cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *off, int T, int d,
-                                    int E, void *e_split, float *scores, int32_t *status,
-                                    int64_t timeout_ns, cudaStream_t st) {
+                                    int E, int affinity, void *e_split, float *scores,
+                                    int32_t *status, int64_t timeout_ns, cudaStream_t st) {
     using namespace router;
     if (T == 0) return cudaSuccess;
     int dev = 0, sms = 148;
@@ -273,7 +281,7 @@ cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *
     if (!tensor_map_2d_bf16(&m.x, x, T, d, BK, BM) ||
         !tensor_map_3d_bf16(&m.parts, e_split, 3, E, d, BK, BN))
         return cudaErrorInvalidValue;
-    Params p{T, E, d, off, scores, status, timeout_ns};
+    Params p{T, E, d, affinity, off, scores, status, timeout_ns};
     err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
     if (err != cudaSuccess) return err;
     const int tiles = ((T + BM - 1) / BM) * ((E + BN - 1) / BN);

@@ -24,6 +24,10 @@
  *             Implemented: shared + fine-grained routed experts).
  *   combine   out_t = shared_t + sum_j w_j y_(t,j) back in token order (the
  *             combine all-to-all, same section).
+ * Variants (same passage of Exp08, Implemented): the V4 affinity
+ * sqrt(softplus(L)) in place of the sigmoid, a hash router for early layers,
+ * and the per-expert bias update that balances the load without an
+ * auxiliary loss (moe_config.router, moe_route_hash, moe_bias_update).
  *
  * Conventions for every entry point:
  *   - Tensors are DEVICE pointers to dense row-major arrays; bf16 data is
@@ -60,7 +64,14 @@
 extern "C" {
 #endif
 
-/* Layer sizes. */
+/* Router of the layer (moe_config.router). */
+typedef enum moe_router {
+    MOE_ROUTER_SIGMOID = 0,       /* s = sigmoid(L) (DeepSeek-V3); the default */
+    MOE_ROUTER_SQRT_SOFTPLUS = 1, /* s = sqrt(log(1 + e^L)) (the V4 form)      */
+    MOE_ROUTER_HASH = 2           /* experts from a hash of the token id       */
+} moe_router;
+
+/* Layer sizes and router.  A zero-initialised `router` is the sigmoid. */
 typedef struct moe_config {
     int32_t T;           /* tokens in the batch                               */
     int32_t d;           /* hidden size                                       */
@@ -71,6 +82,7 @@ typedef struct moe_config {
     int32_t d_ff;        /* routed expert intermediate size                   */
     int32_t n_shared;    /* always-on shared experts (0 allowed)              */
     int32_t d_ff_shared; /* shared expert intermediate size                   */
+    int32_t router;      /* moe_router; other values: UNSUPPORTED_SHAPE       */
 } moe_config;
 
 typedef enum moe_status {
@@ -108,10 +120,11 @@ MOE_API moe_status moe_read_device_status(const void *ws, int32_t *host_status, 
 MOE_API moe_status moe_clear_device_status(void *ws, void *stream);
 
 /*
- * Router (affinity + node-limited top-K).
+ * Router (affinity + node-limited top-K) for cfg->router SIGMOID or
+ * SQRT_SOFTPLUS (HASH: MOE_ERR_INVALID_ARG; use moe_route_hash).
  *   x            [T, d]   bf16
  *   router_w     [E, d]   fp32  (e_i rows)
- *   logit_offset [E]      fp32 or NULL: added to x . e_i before the sigmoid
+ *   logit_offset [E]      fp32 or NULL: added to x . e_i before the affinity
  *   bias         [E]      fp32: selection-only balance bias (NULL = zeros)
  *   topk_idx     [T, K]   int32 out: chosen experts, descending b_i then
  *                               ascending index
@@ -121,7 +134,9 @@ MOE_API moe_status moe_clear_device_status(void *ws, void *stream);
  *   ws, ws_bytes          workspace of moe_workspace_size(cfg) bytes (required)
  * L = x . e_i on the tensor cores: e_i is split into three bf16 parts whose
  * sum reproduces the fp32 value to ~2^-27 relative, the products are exact,
- * and the accumulation is fp32; s = 1 / (1 + expf(-L)).
+ * and the accumulation is fp32; s = 1 / (1 + expf(-L)), or for SQRT_SOFTPLUS
+ * s = sqrtf(softplus(L)) with softplus(L) = L + log1pf(expf(-L)) for L > 0,
+ * log1pf(expf(L)) otherwise (no overflow on either side).
  */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *router_w,
                      const float *logit_offset, const float *bias,
@@ -133,6 +148,35 @@ MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const float *
  * order as the written-out definition, so equal inputs give equal bits. */
 MOE_API moe_status moe_route_select(const moe_config *cfg, const float *scores, const float *bias,
                             int32_t *topk_idx, float *topk_w, void *stream);
+
+/*
+ * Hash router ("a hash router for early-layer emulation", Exp08,
+ * Implemented; the page gives no formula, this is the library's reading):
+ * the node limit is kept -- a token takes M of the G groups and K/M experts
+ * in each, drawn without replacement by a partial Fisher-Yates shuffle driven
+ * by the lowbias32 integer hash of its 64-bit id; every gate is 1/K.
+ *   token_ids  [T]     int64, or NULL: the row index t is the id
+ *   topk_idx   [T, K]  int32 out: slots grouped by group in draw order
+ *   topk_w     [T, K]  fp32 out: 1/K
+ * Deterministic: equal ids give equal routes, on any batch position.
+ * cfg->router is not consulted.
+ */
+MOE_API moe_status moe_route_hash(const moe_config *cfg, const int64_t *token_ids,
+                                  int32_t *topk_idx, float *topk_w, void *stream);
+
+/*
+ * Per-expert bias update of auxiliary-loss-free balancing ("per-expert bias
+ * updates", Exp08, Implemented; the sign rule of DeepSeek-V3, its step size a
+ * parameter): every expert above the mean load T*K/E moves its bias down by
+ * gamma, every expert below it moves up, one exactly at the mean keeps it:
+ *   bias[i] = bias[i] + gamma * sign(T*K/E - counts[i])   (one fp32 add)
+ * The comparison is exact (counts[i] * E against T * K in 64-bit integers).
+ *   counts  [E]  int32: copies per expert, as moe_dispatch / moe_forward write
+ *   gamma        fp32 step (finite)
+ *   bias    [E]  fp32 in/out
+ */
+MOE_API moe_status moe_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,
+                                   float *bias, void *stream);
 
 /*
  * Dispatch: stable counting sort of the T*K token copies by expert.
@@ -217,9 +261,12 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const 
  *   out [T, d] bf16 out.  topk_idx [T,K], topk_w [T,K], counts [E],
  *   offsets [E+1], send [G,G], send_tok [G,G] are optional outputs (NULL:
  *   kept in the workspace).  Intermediates live in the workspace.
+ *   The route is cfg->router's: moe_route's for SIGMOID and SQRT_SOFTPLUS
+ *   (router_w required, token_ids ignored), moe_route_hash's for HASH
+ *   (token_ids [T] int64 or NULL; router_w, logit_offset, bias ignored).
  */
 MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float *router_w,
-                       const float *logit_offset, const float *bias,
+                       const float *logit_offset, const float *bias, const int64_t *token_ids,
                        const void *w_gate, const void *w_up, const void *w_down,
                        const void *ws_gate, const void *ws_up, const void *ws_down,
                        void *out, int32_t *topk_idx, float *topk_w, int32_t *counts,

@@ -27,7 +27,7 @@ import torch
 
 __all__ = [
     "MoeShape", "CONFIGS", "TENSOR_IDS", "config", "normal", "normal_slice",
-    "zipf_logit_offset", "make_inputs", "expert_slice",
+    "zipf_logit_offset", "make_inputs", "expert_slice", "token_ids",
 ]
 
 _M32 = 0xFFFFFFFF
@@ -104,8 +104,11 @@ PROFILE_CONFIGS = {
 TENSOR_IDS = {
     "x": 1, "router_w": 2, "bias": 3, "w_gate": 4, "w_up": 5, "w_down": 6,
     "ws_gate": 7, "ws_up": 8, "ws_down": 9, "zipf_perm": 10, "y_perm": 11,
-    "y_shared": 12, "scores": 13,
+    "y_shared": 12, "scores": 13, "token_ids": 14,
 }
+
+# Vocabulary of DeepSeek-V3's tokenizer: the id range of synthetic token ids.
+VOCAB = 129280
 
 
 def config(name: str) -> MoeShape:
@@ -269,3 +272,12 @@ def random_routing(seed: int, T: int, E: int, K: int, zipf_s: float = 0.0,
     else:
         keys = torch.log(u)
     return torch.topk(keys, K, dim=1).indices.to(torch.int32)
+
+
+def token_ids(seed: int, T: int, vocab: int = VOCAB, device="cpu") -> torch.Tensor:
+    """[T] int64 token ids with a Zipf-like (log-uniform) frequency over
+    [0, vocab): id = floor(vocab^u) - 1 for u uniform on (0, 1), so small ids
+    (frequent words) repeat often and large ones rarely, as in text."""
+    u = uniform01(seed, TENSOR_IDS["token_ids"], (T,), device).double()
+    ids = torch.floor(torch.pow(float(vocab), u)).to(torch.int64) - 1
+    return ids.clamp_(0, vocab - 1)

@@ -64,25 +64,32 @@ def expert_mats_host(inp: dict, experts, E: int):
     return g, u, d
 
 
-def oracle_layer_sample(orc, sh: synth.MoeShape, inp: dict, rows):
+def oracle_layer_sample(orc, sh: synth.MoeShape, inp: dict, rows, router: int = 0,
+                        token_ids=None):
     """Oracle layer output for the token rows `rows` of device inputs `inp`.
 
     Only the x rows and the experts those tokens choose (by the oracle's own
-    routing) are copied to the host.
+    routing) are copied to the host.  `router`: 0 sigmoid, 1 sqrt(softplus),
+    2 hash keyed by `token_ids` (host int64 [T] or None for the row index).
     """
     rows = np.asarray(rows, dtype=np.int64)
     x_h = inp["x"].cpu()
     e_h = inp["router_w"].cpu()
     b_h = inp["bias"].cpu()
     off_h = host(inp.get("logit_offset"))
-    scores = orc.router_scores(x_h, e_h, off_h, rows=rows)
-    idx, _ = orc.select(scores, b_h, sh.G, sh.K, sh.M)
+    if router == 2:
+        keys = rows if token_ids is None else np.asarray(token_ids, dtype=np.int64)[rows]
+        idx, _ = orc.hash_route(keys, sh.E, sh.G, sh.K, sh.M)
+    else:
+        scores = orc.router_scores(x_h, e_h, off_h, rows=rows, affinity=router)
+        idx, _ = orc.select(scores, b_h, sh.G, sh.K, sh.M)
     g, u, d = expert_mats_host(inp, idx.ravel(), sh.E)
     ns = sh.n_shared
     Sg = inp["ws_gate"].cpu() if ns else torch.zeros(1, 64, sh.d, dtype=torch.bfloat16)
     Su = inp["ws_up"].cpu() if ns else torch.zeros(1, 64, sh.d, dtype=torch.bfloat16)
     Sd = inp["ws_down"].cpu() if ns else torch.zeros(1, sh.d, 64, dtype=torch.bfloat16)
-    return orc.layer_rows(rows, sh, x_h, e_h, b_h, g, u, d, Sg, Su, Sd, logit_offset=off_h)
+    return orc.layer_rows(rows, sh, x_h, e_h, b_h, g, u, d, Sg, Su, Sd, logit_offset=off_h,
+                          router=router, token_ids=token_ids)
 
 
 def near_tie_certified(sh: synth.MoeShape, s_orc: np.ndarray, bias: np.ndarray,

@@ -114,14 +114,39 @@ def test_entry_points_validate_before_cuda(moe):
     # workspace too small
     args = [P(fake)] * 9
     assert lib.moe_dispatch(C.byref(cfg), *args, P(fake), ws_n - 1, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
-    assert lib.moe_forward(C.byref(cfg), *([P(fake)] * 17), P(fake), ws_n - 1, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert lib.moe_forward(C.byref(cfg), *([P(fake)] * 18), P(fake), ws_n - 1, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
     # misaligned workspace
     assert lib.moe_dispatch(C.byref(cfg), *args, P(fake + 16), ws_n, None) == moe.MOE_ERR_INVALID_ARG
     # unsupported shape wins over everything else
     bad = moe.MoeConfig.of(synth.config("tiny").replace(E=15))
-    assert lib.moe_forward(C.byref(bad), *([None] * 17), None, 0, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_forward(C.byref(bad), *([None] * 18), None, 0, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     # self-test limits
     assert lib.moe_selftest_bounded_wait(10, P(fake), None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_router_variants_validate_before_cuda(moe):
+    sh = synth.config("tiny")
+    assert moe.moe_check_config(moe.MoeConfig.of(sh, router=3)) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert moe.moe_check_config(moe.MoeConfig.of(sh, router=-1)) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    for r in (moe.MOE_ROUTER_SIGMOID, moe.MOE_ROUTER_SQRT_SOFTPLUS, moe.MOE_ROUTER_HASH):
+        assert moe.moe_check_config(moe.MoeConfig.of(sh, router=r)) == moe.MOE_OK
+    assert moe.MoeConfig.of(sh).router == moe.MOE_ROUTER_SIGMOID
+    lib, fake, P = moe._lib, 1 << 20, C.c_void_p
+    hcfg = moe.MoeConfig.of(sh, router=moe.MOE_ROUTER_HASH)
+    ws_n = moe.moe_workspace_size(hcfg)
+    # the learned router refuses a hash configuration
+    assert lib.moe_route(C.byref(hcfg), P(fake), P(fake), None, None, P(fake), P(fake), None,
+                         P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_hash(C.byref(hcfg), None, None, P(fake), None) == moe.MOE_ERR_INVALID_ARG
+    cfg = moe.MoeConfig.of(sh)
+    for g in (float("nan"), float("inf"), float("-inf")):
+        assert lib.moe_bias_update(C.byref(cfg), P(fake), g, P(fake), None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(C.byref(cfg), None, 1e-3, P(fake), None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(C.byref(cfg), P(fake), 1e-3, None, None) == moe.MOE_ERR_INVALID_ARG
+    # moe_forward: the learned routers need router_w, the hash router does not
+    args = [P(fake)] * 18
+    args[1] = None  # router_w
+    assert lib.moe_forward(C.byref(cfg), *args, P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a GPU")

@@ -1,0 +1,212 @@
+"""Parity of the routing variants (CUDA path through the C ABI vs the oracle).
+
+"MoE + Expert-Parallel Overlap (Exp08)", Implemented: sqrt(softplus)
+affinities, a hash router for early layers, per-expert bias updates.
+Bars: affinities within 1e-5 absolute; selection bit-exact given the same fp32
+affinities and certified near ties otherwise; hash routes and bias updates
+bit-exact; layer outputs within the layer's Frobenius / per-element bars.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import combine_expert_ffn_b200 as moe
+else:  # collected on CPU-only machines, skipped by the marker filter
+    moe = None
+
+DEV = "cuda"
+SQRT_SOFTPLUS, HASH = 1, 2
+
+
+@pytest.fixture(autouse=True)
+def _free_gpu():
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+_cache = {}
+
+
+def inputs(name):
+    if name not in _cache:
+        _cache.clear()
+        gc.collect()
+        torch.cuda.empty_cache()
+        _cache[name] = synth.make_inputs(H.shape(name), DEV)
+    return _cache[name]
+
+
+def _rows(T, n_sample):
+    return np.arange(T) if n_sample is None else \
+        np.unique(np.linspace(0, T - 1, n_sample).astype(np.int64))
+
+
+# ---------------------------------------------------------------- sqrt(softplus)
+@pytest.mark.parametrize("name,n_sample", [("tiny", None), ("ragged", None), ("ragged2", None),
+                                           ("mid", 256), ("v3", 64), ("skew", 64)])
+def test_sqrt_softplus_route(orc, name, n_sample):
+    sh = H.shape(name)
+    inp = inputs(name)
+    cfg = moe.MoeConfig.of(sh, router=SQRT_SOFTPLUS)
+    idx = torch.empty(sh.T, sh.K, dtype=torch.int32, device=DEV)
+    w = torch.empty(sh.T, sh.K, dtype=torch.float32, device=DEV)
+    s = torch.empty(sh.T, sh.E, dtype=torch.float32, device=DEV)
+    ws = moe.alloc_workspace(cfg)
+    moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"], idx, w,
+                  scores=s, ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    rows = _rows(sh.T, n_sample)
+    ref_s = orc.router_scores(inp["x"].cpu(), inp["router_w"].cpu(),
+                              H.host(inp.get("logit_offset")), rows=rows, affinity=SQRT_SOFTPLUS)
+    gs = s.cpu().numpy()
+    assert np.abs(gs[rows] - ref_s).max() <= H.TOL_AFFINITY
+    # the selection step on the GPU's own affinities: bit-exact, every token
+    bias = inp["bias"].cpu()
+    sel_idx, sel_w = orc.select(gs, bias, sh.G, sh.K, sh.M)
+    np.testing.assert_array_equal(idx.cpu().numpy(), sel_idx)
+    np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), sel_w.view(np.uint32))
+    # ... and on the oracle's: equal up to certified near ties
+    ref_idx, _ = orc.select(ref_s, bias, sh.G, sh.K, sh.M)
+    gi = idx.cpu().numpy()[rows]
+    flips = 0
+    for r in range(len(rows)):
+        if not np.array_equal(gi[r], ref_idx[r]):
+            flips += 1
+            assert H.near_tie_certified(sh, ref_s[r], bias.numpy(), gi[r], ref_idx[r])
+    assert flips <= max(1, len(rows) // 100)
+
+
+def test_sqrt_softplus_extreme_logits(orc):
+    """Logit offsets push L into both tails of softplus (no overflow, no NaN)."""
+    sh = H.RAGGED2.replace(T=128)
+    inp = synth.make_inputs(sh, DEV, weights=False)
+    off = torch.linspace(-60, 60, sh.E, device=DEV)
+    cfg = moe.MoeConfig.of(sh, router=SQRT_SOFTPLUS)
+    idx = torch.empty(sh.T, sh.K, dtype=torch.int32, device=DEV)
+    w = torch.empty(sh.T, sh.K, dtype=torch.float32, device=DEV)
+    s = torch.empty(sh.T, sh.E, dtype=torch.float32, device=DEV)
+    moe.moe_route(cfg, inp["x"], inp["router_w"], off, inp["bias"], idx, w, scores=s,
+                  ws=moe.alloc_workspace(cfg))
+    ref_s = orc.router_scores(inp["x"].cpu(), inp["router_w"].cpu(), off.cpu(),
+                              affinity=SQRT_SOFTPLUS)
+    gs = s.cpu().numpy()
+    assert np.isfinite(gs).all() and (gs > 0).all()
+    np.testing.assert_allclose(gs, ref_s, rtol=2e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("name,n_sample", [("ragged", None), ("ragged2", None), ("v3", 6)])
+def test_forward_sqrt_softplus(orc, name, n_sample):
+    sh = H.shape(name)
+    inp = inputs(name)
+    cfg = moe.MoeConfig.of(sh, router=SQRT_SOFTPLUS)
+    ws = moe.alloc_workspace(cfg)
+    o = moe.forward_outputs(cfg)
+    moe.moe_forward(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                    inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                    inp.get("ws_up"), inp.get("ws_down"), o["out"], o["topk_idx"], o["topk_w"],
+                    o["counts"], o["offsets"], o["send"], o["send_tok"], ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    rows = _rows(sh.T, n_sample)
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows, router=SQRT_SOFTPLUS)
+    gi = o["topk_idx"].cpu().numpy()[rows]
+    keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
+    for r in set(range(len(rows))) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    assert len(keep) >= len(rows) - max(1, len(rows) // 100)
+    frob, elem = H.compare_out(o["out"][torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
+# ---------------------------------------------------------------- hash router
+@pytest.mark.parametrize("T,E,G,K,M", [(256, 256, 8, 8, 4), (520, 40, 8, 6, 3), (96, 16, 4, 4, 2),
+                                       (64, 9, 9, 9, 9), (8192, 1024, 64, 32, 32),
+                                       (130, 12, 2, 1, 1)])
+def test_hash_route_bit_exact(orc, T, E, G, K, M):
+    T = T - T % G
+    cfg = moe.MoeConfig(T=T, d=64, E=E, G=G, K=K, M=M, d_ff=64, n_shared=0, d_ff_shared=0,
+                        router=HASH)
+    ids = synth.token_ids(3, T, device=DEV)
+    ids[:4] = torch.tensor([0, 2**32, 2**40 + 7, 2**62], dtype=torch.int64)
+    idx = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, K, dtype=torch.float32, device=DEV)
+    moe.moe_route_hash(cfg, ids, idx, w)
+    ref_idx, ref_w = orc.hash_route(ids.cpu().numpy(), E, G, K, M)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), ref_w.view(np.uint32))
+    # no ids: the row index is the key
+    moe.moe_route_hash(cfg, None, idx, w)
+    np.testing.assert_array_equal(idx.cpu().numpy(), orc.hash_route(np.arange(T), E, G, K, M)[0])
+
+
+@pytest.mark.parametrize("name,n_sample", [("ragged", None), ("ragged2", None), ("noshared", None),
+                                           ("v3", 6)])
+def test_forward_hash(orc, name, n_sample):
+    sh = H.shape(name)
+    inp = inputs(name)
+    cfg = moe.MoeConfig.of(sh, router=HASH)
+    ws = moe.alloc_workspace(cfg)
+    o = moe.forward_outputs(cfg)
+    ids = synth.token_ids(sh.seed, sh.T, device=DEV)
+    moe.moe_forward(cfg, inp["x"], None, None, None, inp["w_gate"], inp["w_up"], inp["w_down"],
+                    inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"), o["out"],
+                    o["topk_idx"], o["topk_w"], o["counts"], o["offsets"], o["send"],
+                    o["send_tok"], ws=ws, token_ids=ids)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    ids_h = ids.cpu().numpy()
+    ref_idx_all, _ = orc.hash_route(ids_h, sh.E, sh.G, sh.K, sh.M)
+    np.testing.assert_array_equal(o["topk_idx"].cpu().numpy(), ref_idx_all)
+    np.testing.assert_array_equal(o["counts"].cpu().numpy(),
+                                  np.bincount(ref_idx_all.ravel(), minlength=sh.E))
+    rows = _rows(sh.T, n_sample)
+    ref_out, _, _, _ = H.oracle_layer_sample(orc, sh, inp, rows, router=HASH, token_ids=ids_h)
+    frob, elem = H.compare_out(o["out"][torch.as_tensor(rows, device=DEV)], ref_out)
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
+# ---------------------------------------------------------------- bias update
+def test_bias_update_bit_exact_from_forward_counts(orc):
+    """A few balancing steps: forward -> counts -> bias update -> forward ..."""
+    sh = H.RAGGED2
+    inp = synth.make_inputs(sh, DEV)
+    cfg = moe.MoeConfig.of(sh)
+    ws = moe.alloc_workspace(cfg)
+    o = moe.forward_outputs(cfg)
+    bias = inp["bias"].clone()
+    ref_bias = bias.cpu().numpy()
+    for step in range(4):
+        moe.moe_forward(cfg, inp["x"], inp["router_w"], None, bias, inp["w_gate"], inp["w_up"],
+                        inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], o["out"],
+                        counts=o["counts"], ws=ws)
+        counts = o["counts"].cpu().numpy()
+        moe.moe_bias_update(cfg, o["counts"], 1e-3, bias)
+        ref_bias = orc.bias_update(counts, sh.T, sh.K, 1e-3, ref_bias)
+        np.testing.assert_array_equal(bias.cpu().numpy().view(np.uint32), ref_bias.view(np.uint32))
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+
+
+@pytest.mark.parametrize("E,T,K", [(4, 4, 2), (3, 2, 2), (256, 8192, 8), (1024, 65536, 32),
+                                   (3, 2**26 - 2, 8)])
+def test_bias_update_bit_exact_at_and_around_the_mean(orc, E, T, K):
+    G = 1
+    cfg = moe.MoeConfig(T=T, d=64, E=E, G=G, K=min(K, E), M=1, d_ff=64, n_shared=0,
+                        d_ff_shared=0)
+    K = cfg.K
+    total = T * K
+    mean = total // E
+    rng = np.random.default_rng(E + T)
+    counts = (mean + rng.integers(-1, 2, size=E)).astype(np.int32)  # at, just above, just below
+    bias = synth.normal(1, 3, (E,), 0.01, torch.float32, DEV)
+    for gamma in (1e-3, 0.0, -2.5e-4, 1e-9):
+        b = bias.clone()
+        moe.moe_bias_update(cfg, torch.from_numpy(counts).to(DEV), gamma, b)
+        ref = orc.bias_update(counts, T, K, gamma, bias.cpu().numpy())
+        np.testing.assert_array_equal(b.cpu().numpy().view(np.uint32), ref.view(np.uint32))
