@@ -247,9 +247,9 @@ def run_ours(args, sh, world, rank, local):
     scores = torch.empty(T, E, dtype=torch.float32, device=dev)
     perm_token = torch.empty(T * K, dtype=torch.int32, device=dev)
     inv_perm = torch.empty(T, K, dtype=torch.int32, device=dev)
-    x_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
     y_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
     y_sh = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    x_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -380,6 +380,34 @@ def variants_leg(sh, inp, dev, stream, reps=20):
         return e0.elapsed_time(e1) / reps
 
     out = {}
+    # the dispatch gather fused into the expert FFN vs the two-step path
+    cfg = moe.MoeConfig.of(sh)
+    ws = moe.alloc_workspace(cfg, dev)
+    o = moe.forward_outputs(cfg, dev)
+    perm = torch.empty(T * K, dtype=torch.int32, device=dev)
+    inv = torch.empty(T, K, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * K, sh.d, dtype=torch.bfloat16, device=dev)
+    y_perm = torch.empty(T * K, sh.d, dtype=torch.bfloat16, device=dev)
+    y_sh = torch.empty(T, sh.d, dtype=torch.bfloat16, device=dev)
+    moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                  o["topk_idx"], o["topk_w"], None, ws, stream)
+
+    def two_step():
+        moe.moe_dispatch(cfg, inp["x"], o["topk_idx"], o["counts"], o["offsets"], o["send"],
+                         o["send_tok"], perm, inv, x_perm, ws, stream)
+        moe.moe_expert_ffn(cfg, x_perm, o["offsets"], inp["w_gate"], inp["w_up"], inp["w_down"],
+                           y_perm, inp["x"], inp.get("ws_gate"), inp.get("ws_up"),
+                           inp.get("ws_down"), y_sh, ws, stream)
+
+    def fused():
+        moe.moe_dispatch(cfg, inp["x"], o["topk_idx"], o["counts"], o["offsets"], o["send"],
+                         o["send_tok"], perm, inv, None, ws, stream)
+        moe.moe_expert_ffn_gather(cfg, inp["x"], perm, o["offsets"], inp["w_gate"], inp["w_up"],
+                                  inp["w_down"], y_perm, inp.get("ws_gate"), inp.get("ws_up"),
+                                  inp.get("ws_down"), y_sh, ws, stream)
+
+    out["dispatch_plus_ffn_ms"] = {"two_step_x_perm": timed(two_step), "fused_gather": timed(fused)}
+    del ws, o, x_perm, y_perm, y_sh
     names = {moe.MOE_ROUTER_SIGMOID: "sigmoid", moe.MOE_ROUTER_SQRT_SOFTPLUS: "sqrt_softplus",
              moe.MOE_ROUTER_HASH: "hash"}
     for r, name in names.items():

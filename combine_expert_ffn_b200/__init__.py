@@ -34,7 +34,7 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_read_device_status", "moe_clear_device_status", "moe_route", "moe_route_select",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_bounded_wait", "moe_dispatch_noalloc", "moe_route_hash",
-           "moe_bias_update")
+           "moe_bias_update", "moe_expert_ffn_gather")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
 
@@ -79,6 +79,8 @@ _sig = {
     "moe_forward": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _S, _P]),
     "moe_route_hash": (C.c_int, [_CP, _P, _P, _P, _P]),
+    "moe_expert_ffn_gather": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
+                                        _P]),
     "moe_bias_update": (C.c_int, [_CP, _P, C.c_float, _P, _P]),
     "moe_selftest_bounded_wait": (C.c_int, [_I64, _P, _P]),
     "moe_dispatch_noalloc": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -194,6 +196,16 @@ def moe_expert_ffn(cfg, x_perm, offsets, w_gate, w_up, w_down, y_perm, x, ws_gat
                                               _ptr(w_up), _ptr(w_down), _ptr(y_perm), _ptr(x),
                                               _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down),
                                               _ptr(y_shared), wp, wn, _stream(stream)))
+
+
+def moe_expert_ffn_gather(cfg, x, perm_token, offsets, w_gate, w_up, w_down, y_perm, ws_gate,
+                          ws_up, ws_down, y_shared, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_expert_ffn_gather",
+        _lib.moe_expert_ffn_gather(_cfg(cfg), _ptr(x), _ptr(perm_token), _ptr(offsets),
+                                   _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y_perm),
+                                   _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_shared), wp,
+                                   wn, _stream(stream)))
 
 
 def moe_combine(cfg, y_perm, inv_perm, topk_w, y_shared, out, stream=None) -> None:

@@ -1,7 +1,9 @@
 // gemm_sm100.cu -- grouped expert FFN on the 5th-generation tensor cores.
 //
 // Per routed expert e with rows R_e = [offsets[e], offsets[e+1]) of x_perm
-// and for the shared experts on all T rows of x:
+// (or, fused with the dispatch gather, rows x[perm_token[r]] read straight
+// from x by four-row TMA gathers) and for the shared experts on all T rows
+// of x:
 //   GEMM1:  h = SiLU(X W_g^T) * (X W_u^T)     (SwiGLU fused in the epilogue)
 //   GEMM2:  y = h W_d^T
 // ("shared experts (always active) + fine-grained routed experts", "MoE +
@@ -55,6 +57,7 @@ struct Cfg {
 
 struct Maps {
     CUtensorMap a_r;   // routed A  [rows_r, k_r]           box 64 x 128
+    CUtensorMap a_g;   // routed A gathered from x [T, d]   box 64 x 1 (GEMM1 with perm_token)
     CUtensorMap a_s;   // shared A  [T, k_s]                box 64 x 128
     CUtensorMap b0_r;  // routed B  gate | down  3-D        box 64 x (128 | 256) x 1
     CUtensorMap b1_r;  // routed B  up (SwiGLU only)
@@ -66,6 +69,8 @@ struct Maps {
 
 struct Params {
     const int32_t *offsets;  // [E+1]
+    const int32_t *perm_token;  // GEMM1: routed row r is x[perm_token[r]] (nullptr: A = a_r)
+    int x_rows;              // rows of x (bound of perm_token values)
     int E;
     int rows_r;              // rows of the routed A buffer (T*K)
     int T;                   // shared rows; 0 = no shared experts
@@ -193,7 +198,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         if (lane == 0) {
             tile_base[p.E] = carry;
             tma_prefetch_desc(&maps.o_r);
-            tma_prefetch_desc(&maps.a_r);
+            tma_prefetch_desc(p.perm_token != nullptr ? &maps.a_g : &maps.a_r);
             tma_prefetch_desc(&maps.b0_r);
             if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
             if (p.T > 0) {
@@ -231,26 +236,45 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t n_issued = 0;
-            for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-                const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
-                bool ok = true;
-                for (int kb = 0; kb < t.kblocks; ++kb) {
-                    if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
-                                           p.status, p.timeout_ns)) {
-                        ok = false;
-                        break;
+        // Lane 0 waits for a free stage, arms its barrier and loads the B
+        // tile; the A tile is one tiled load by lane 0, or -- for routed tiles
+        // gathered straight from x -- 32 four-row gathers, one per lane, of
+        // the rows x[perm_token[r]].
+        const bool gather = EPI == EPI_SWIGLU && p.perm_token != nullptr;
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t n_issued = 0;
+        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+            const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
+            const bool gather_tile = gather && t.e >= 0;
+            int32_t tok[4] = {0, 0, 0, 0};
+            if (gather_tile) {
+                // rows past the segment (never stored) read token 0
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = 4 * lane + i;
+                    if (r < t.rows_valid) {
+                        const int v = p.perm_token[t.row0 + r];
+                        if (v < 0 || v >= p.x_rows) record_status(p.status, MOE_ERR_DEVICE_FAULT);
+                        else tok[i] = v;
                     }
-                    const uint32_t fb = smem_u32(&full_bar[stage]);
-                    const uint32_t a_dst = smem0 + stage * STAGE_BYTES;
-                    const uint32_t b_dst = a_dst + A_BYTES;
-                    const int k = kb * BK;
+                }
+            }
+            bool ok = true;
+            for (int kb = 0; kb < t.kblocks; ++kb) {
+                if (lane == 0)
+                    ok = mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
+                                           p.status, p.timeout_ns);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                const uint32_t fb = smem_u32(&full_bar[stage]);
+                const uint32_t a_dst = smem0 + stage * STAGE_BYTES;
+                const uint32_t b_dst = a_dst + A_BYTES;
+                const int k = kb * BK;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(fb, Cfg<EPI>::TX);
                     if (t.e >= 0) {
-                        tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
+                        if (!gather_tile) tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
                         if (EPI == EPI_SWIGLU) {
                             tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
                             tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_r, fb, k, t.n0, t.e);
@@ -267,12 +291,19 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                             tma_load_3d(b_dst, &maps.b0_s, fb, k - s * p.kseg_s, t.n0, s);
                         }
                     }
-                    ++n_issued;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (!ok) break;
+                if (gather_tile) {
+                    __syncwarp();  // the barrier is armed before any gather lands
+                    tma_gather4(a_dst + lane * 4 * BK * 2, &maps.a_g, fb, k, tok[0], tok[1],
+                                tok[2], tok[3]);
+                }
+                ++n_issued;
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            // wind down: every load issued into a stage has landed
+            if (!ok) break;
+        }
+        // wind down: every load issued into a stage has landed
+        if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
                 if (n_issued > (uint32_t)s) {
                     const uint32_t uses = (n_issued - 1 - s) / STAGES + 1;
@@ -475,9 +506,16 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
 
     // GEMM1: h = SwiGLU(x_perm) per expert; h_shared = SwiGLU(x) for the shared experts
     Maps m1;
-    bool ok = map_2d(&m1.a_r, a.x_perm, rows_r, a.d, BM) &&
-              map_3d(&m1.b0_r, a.w_gate, a.E, a.d_ff, a.d, BN_ACC / 2) &&
+    const bool gather = a.perm_token != nullptr;
+    bool ok = map_3d(&m1.b0_r, a.w_gate, a.E, a.d_ff, a.d, BN_ACC / 2) &&
               map_3d(&m1.b1_r, a.w_up, a.E, a.d_ff, a.d, BN_ACC / 2);
+    if (gather) {  // routed rows straight from x: one-row boxes for four-row gathers
+        ok = ok && tensor_map_2d_bf16(&m1.a_g, a.x, a.T, a.d, BK, 1);
+        m1.a_r = m1.a_g;
+    } else {
+        ok = ok && map_2d(&m1.a_r, a.x_perm, rows_r, a.d, BM);
+        m1.a_g = m1.a_r;
+    }
     if (has_shared)
         ok = ok && map_2d(&m1.a_s, a.x, a.T, a.d, BM) &&
              map_3d(&m1.b0_s, a.ws_gate, 1, ffs, a.d, BN_ACC / 2) &&
@@ -493,6 +531,8 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     if (!ok) return cudaErrorInvalidValue;
     Params p1{};
     p1.offsets = a.offsets;
+    p1.perm_token = a.perm_token;
+    p1.x_rows = a.T;
     p1.E = a.E;
     p1.rows_r = (int)rows_r;
     p1.T = has_shared ? a.T : 0;
@@ -512,6 +552,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     Maps m2;
     ok = map_2d(&m2.a_r, a.h, rows_r, a.d_ff, BM) &&
          map_3d(&m2.b0_r, a.w_down, a.E, a.d, a.d_ff, BN_ACC);
+    m2.a_g = m2.a_r;
     if (has_shared)
         ok = ok && map_2d(&m2.a_s, a.h_shared, a.T, ffs, BM) &&
              map_3d(&m2.b0_s, a.ws_down, a.n_shared, a.d, a.d_ff_shared, BN_ACC);
@@ -526,6 +567,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
         m2.o_s = m2.o_r;
     if (!ok) return cudaErrorInvalidValue;
     Params p2 = p1;
+    p2.perm_token = nullptr;
     p2.n_out_r = a.d;
     p2.n_out_s = a.d;
     p2.k_r = a.d_ff;

@@ -48,7 +48,8 @@ cudaError_t launch_combine(const void *y_perm, const int32_t *inv_perm, const fl
 // gemm_sm100.cu
 struct FfnArgs {
     int T, d, E, K, d_ff, n_shared, d_ff_shared;
-    const void *x_perm;
+    const void *x_perm;        // [T*K, d] bf16, or unused when perm_token is set
+    const int32_t *perm_token; // [T*K] or nullptr: routed row r of GEMM1 is x[perm_token[r]]
     const int32_t *offsets;
     const void *w_gate, *w_up, *w_down;
     void *h;        // [T*K, d_ff] bf16 scratch

@@ -250,6 +250,27 @@ MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, con
                           void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Expert FFN fused with the dispatch gather: as moe_expert_ffn, but the routed
+ * rows are read straight from x -- row r of expert segment e is
+ * x[perm_token[r]] -- by four-row TMA gathers inside the gate/up GEMM, so the
+ * permuted copy x_perm is never written or read (the gather-permute step of
+ * the dispatch, "moe-node-limited-routing", "Why all to all dominates MoE step
+ * time", folded into the expert GEMM).
+ *   x           [T, d]     bf16
+ *   perm_token  [T*K]      int32 from moe_dispatch (values in [0, T))
+ *   other arguments as moe_expert_ffn (x also feeds the shared experts).
+ * Results are bit-identical to moe_dispatch(x_perm) + moe_expert_ffn.
+ * A perm_token value outside [0, T) is read as row 0 and flagged
+ * MOE_ERR_DEVICE_FAULT in the status word.
+ */
+MOE_API moe_status moe_expert_ffn_gather(const moe_config *cfg, const void *x,
+                                         const int32_t *perm_token, const int32_t *offsets,
+                                         const void *w_gate, const void *w_up, const void *w_down,
+                                         void *y_perm, const void *ws_gate, const void *ws_up,
+                                         const void *ws_down, void *y_shared, void *ws,
+                                         size_t ws_bytes, void *stream);
+
+/*
  * Combine: out[t] = y_shared[t] + sum_j topk_w[t,j] * y_perm[inv_perm[t,j]],
  * fp32 accumulation, rounded to bf16.  y_shared may be NULL (treated as 0).
  */
@@ -261,6 +282,9 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const 
  *   out [T, d] bf16 out.  topk_idx [T,K], topk_w [T,K], counts [E],
  *   offsets [E+1], send [G,G], send_tok [G,G] are optional outputs (NULL:
  *   kept in the workspace).  Intermediates live in the workspace.
+ *   The dispatch writes x_perm into the workspace and the expert FFN reads it
+ *   (moe_expert_ffn); moe_expert_ffn_gather gives the same bits without
+ *   x_perm but runs slower.
  *   The route is cfg->router's: moe_route's for SIGMOID and SQRT_SOFTPLUS
  *   (router_w required, token_ids ignored), moe_route_hash's for HASH
  *   (token_ids [T] int64 or NULL; router_w, logit_offset, bias ignored).

@@ -124,6 +124,21 @@ def test_entry_points_validate_before_cuda(moe):
     assert lib.moe_selftest_bounded_wait(10, P(fake), None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_fused_gather_validates_before_cuda(moe):
+    cfg = moe.MoeConfig.of(synth.config("tiny"))
+    ws_n = moe.moe_workspace_size(cfg)
+    lib, fake, P = moe._lib, 1 << 20, C.c_void_p
+    args = [P(fake)] * 11                      # x .. y_shared
+    assert lib.moe_expert_ffn_gather(C.byref(cfg), *args, P(fake), ws_n - 1, None) == \
+        moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    bad = list(args)
+    bad[1] = None                              # perm_token
+    assert lib.moe_expert_ffn_gather(C.byref(cfg), *bad, P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
+    bad = list(args)
+    bad[0] = P(fake + 8)                       # misaligned x
+    assert lib.moe_expert_ffn_gather(C.byref(cfg), *bad, P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
+
+
 def test_router_variants_validate_before_cuda(moe):
     sh = synth.config("tiny")
     assert moe.moe_check_config(moe.MoeConfig.of(sh, router=3)) == moe.MOE_ERR_UNSUPPORTED_SHAPE
