@@ -1,8 +1,8 @@
 // gemm_sm100.cu -- grouped expert FFN on the 5th-generation tensor cores.
 //
 // Per routed expert e with rows R_e = [offsets[e], offsets[e+1]) of x_perm
-// (or, fused with the dispatch gather, rows x[perm_token[r]] read straight
-// from x by four-row TMA gathers) and for the shared experts on all T rows
+// (or, fused with the dispatch gather, rows x[perm_token[r]] copied straight
+// from x by four gatherer warps) and for the shared experts on all T rows
 // of x:
 //   GEMM1:  h = SiLU(X W_g^T) * (X W_u^T)     (SwiGLU fused in the epilogue)
 //   GEMM2:  y = h W_d^T
@@ -41,6 +41,10 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN_ACC * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
+// Gather variant of GEMM1: four more warps copy the routed A rows
+// x[perm_token[r]] into the swizzled stage with 16-byte cp.async copies.
+constexpr int GATHER_WARPS = 4;
+constexpr int GATHER_THREADS = GATHER_WARPS * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
 constexpr int STORE_BUF = 32 * 32 * 2;     // one warp's 32 rows x 32 columns of bf16
@@ -57,7 +61,6 @@ struct Cfg {
 
 struct Maps {
     CUtensorMap a_r;   // routed A  [rows_r, k_r]           box 64 x 128
-    CUtensorMap a_g;   // routed A gathered from x [T, d]   box 64 x 1 (GEMM1 with perm_token)
     CUtensorMap a_s;   // shared A  [T, k_s]                box 64 x 128
     CUtensorMap b0_r;  // routed B  gate | down  3-D        box 64 x (128 | 256) x 1
     CUtensorMap b1_r;  // routed B  up (SwiGLU only)
@@ -69,8 +72,9 @@ struct Maps {
 
 struct Params {
     const int32_t *offsets;  // [E+1]
-    const int32_t *perm_token;  // GEMM1: routed row r is x[perm_token[r]] (nullptr: A = a_r)
-    int x_rows;              // rows of x (bound of perm_token values)
+    const int32_t *perm_token;  // gather variant: routed row r of A is x[perm_token[r]]
+    const void *x;           // gather variant: x [x_rows, k_r] bf16
+    int x_rows;
     int E;
     int rows_r;              // rows of the routed A buffer (T*K)
     int T;                   // shared rows; 0 = no shared experts
@@ -142,9 +146,10 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return g * __frcp_rn(1.0f + __expf(-g)) * u;
 }
 
-template <int EPI>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int EPI, bool GATHER>
+__global__ void __launch_bounds__(NUM_THREADS + (GATHER ? GATHER_THREADS : 0), 1)
 grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
+    static_assert(!GATHER || EPI == EPI_SWIGLU, "only GEMM1 gathers its rows");
     constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -198,7 +203,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         if (lane == 0) {
             tile_base[p.E] = carry;
             tma_prefetch_desc(&maps.o_r);
-            tma_prefetch_desc(p.perm_token != nullptr ? &maps.a_g : &maps.a_r);
+            if (!GATHER) tma_prefetch_desc(&maps.a_r);
             tma_prefetch_desc(&maps.b0_r);
             if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
             if (p.T > 0) {
@@ -210,7 +215,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     } else if (warp == 1) {
         if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
-                mbar_init(smem_u32(&full_bar[s]), 1);
+                mbar_init(smem_u32(&full_bar[s]), 1 + (GATHER ? GATHER_THREADS : 0));
                 mbar_init(smem_u32(&empty_bar[s]), 1);
             }
             for (int b = 0; b < 2; ++b) {
@@ -236,45 +241,28 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        // Lane 0 waits for a free stage, arms its barrier and loads the B
-        // tile; the A tile is one tiled load by lane 0, or -- for routed tiles
-        // gathered straight from x -- 32 four-row gathers, one per lane, of
-        // the rows x[perm_token[r]].
-        const bool gather = EPI == EPI_SWIGLU && p.perm_token != nullptr;
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t n_issued = 0;
-        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
-            const bool gather_tile = gather && t.e >= 0;
-            int32_t tok[4] = {0, 0, 0, 0};
-            if (gather_tile) {
-                // rows past the segment (never stored) read token 0
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = 4 * lane + i;
-                    if (r < t.rows_valid) {
-                        const int v = p.perm_token[t.row0 + r];
-                        if (v < 0 || v >= p.x_rows) record_status(p.status, MOE_ERR_DEVICE_FAULT);
-                        else tok[i] = v;
+        // B tiles, and A tiles except the routed ones of the gather variant
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t n_issued = 0;
+            for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
+                const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
+                const bool a_by_tma = !GATHER || t.e < 0;
+                bool ok = true;
+                for (int kb = 0; kb < t.kblocks; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
+                                           p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
                     }
-                }
-            }
-            bool ok = true;
-            for (int kb = 0; kb < t.kblocks; ++kb) {
-                if (lane == 0)
-                    ok = mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
-                                           p.status, p.timeout_ns);
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                if (!ok) break;
-                const uint32_t fb = smem_u32(&full_bar[stage]);
-                const uint32_t a_dst = smem0 + stage * STAGE_BYTES;
-                const uint32_t b_dst = a_dst + A_BYTES;
-                const int k = kb * BK;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(fb, Cfg<EPI>::TX);
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    const uint32_t a_dst = smem0 + stage * STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + A_BYTES;
+                    const int k = kb * BK;
+                    mbar_arrive_expect_tx(fb, a_by_tma ? Cfg<EPI>::TX : Cfg<EPI>::TX - A_BYTES);
                     if (t.e >= 0) {
-                        if (!gather_tile) tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
+                        if (a_by_tma) tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
                         if (EPI == EPI_SWIGLU) {
                             tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
                             tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_r, fb, k, t.n0, t.e);
@@ -291,19 +279,12 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                             tma_load_3d(b_dst, &maps.b0_s, fb, k - s * p.kseg_s, t.n0, s);
                         }
                     }
+                    ++n_issued;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (gather_tile) {
-                    __syncwarp();  // the barrier is armed before any gather lands
-                    tma_gather4(a_dst + lane * 4 * BK * 2, &maps.a_g, fb, k, tok[0], tok[1],
-                                tok[2], tok[3]);
-                }
-                ++n_issued;
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                if (!ok) break;
             }
-            if (!ok) break;
-        }
-        // wind down: every load issued into a stage has landed
-        if (lane == 0) {
+            // wind down: every load issued into a stage has landed
             for (int s = 0; s < STAGES; ++s) {
                 if (n_issued > (uint32_t)s) {
                     const uint32_t uses = (n_issued - 1 - s) / STAGES + 1;
@@ -334,6 +315,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                         break;
                     }
                     tc_fence_after();
+                    if (GATHER) fence_proxy_async();  // gathered rows: generic-proxy writes
                     const uint32_t a_addr = smem0 + stage * STAGE_BYTES;
                     const uint64_t a_desc = smem_desc_sw128(a_addr);
                     const uint64_t b_desc = smem_desc_sw128(a_addr + A_BYTES);
@@ -354,6 +336,59 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             drain_wait(smem_u32(&done_bar), 0, p.timeout_ns, p.status);
         }
         __syncwarp();
+    } else if (GATHER && warp >= NUM_THREADS / 32) {
+        // ------------------------------------------------------ A-row gatherers
+        // Thread g copies the 16-byte chunk c = g % 8 of the rows g / 8 + 16 j
+        // (j < 8) of every routed A stage: x[perm_token[row0 + r]][k + 8c ..]
+        // lands at r * 128 + ((c ^ (r % 8)) * 16), the 128-byte swizzle a TMA
+        // tile load would produce.  Every stage -- copied or not -- gets one
+        // arrival per gatherer on its full barrier, made by the copy hardware
+        // once the thread's copies have landed; the MMA thread fences the
+        // generic-proxy writes for the tensor core after its wait.
+        const int g = threadIdx.x - NUM_THREADS;
+        const int c = g & 7, r0 = g >> 3;
+        const __nv_bfloat16 *xg = static_cast<const __nv_bfloat16 *>(p.x);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+            const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
+            const bool copy = t.e >= 0;
+            const __nv_bfloat16 *src[8];
+            if (copy) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = r0 + 16 * j;
+                    int tok = 0;  // rows past the segment (never stored) read row 0
+                    if (r < t.rows_valid) {
+                        tok = p.perm_token[t.row0 + r];
+                        if (tok < 0 || tok >= p.x_rows) {
+                            record_status(p.status, MOE_ERR_DEVICE_FAULT);
+                            tok = 0;
+                        }
+                    }
+                    src[j] = xg + (size_t)tok * p.k_r + 8 * c;
+                }
+            }
+            for (int kb = 0; kb < t.kblocks; ++kb) {
+                if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
+                                       p.status, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (copy) {
+                    const uint32_t a_dst = smem0 + stage * STAGE_BYTES;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int r = r0 + 16 * j;
+                        cp_async_16(a_dst + r * (BK * 2) + ((c ^ (r & 7)) << 4), src[j] + kb * BK);
+                    }
+                }
+                cp_async_arrive_noinc(smem_u32(&full_bar[stage]));
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        cp_async_wait_all();  // no copy into this CTA's stages outlives the thread
     } else {
         // ------------------------------------------------------ epilogue
         // A full tile (128 valid rows) leaves through TMA stores: each warp
@@ -484,12 +519,13 @@ int sm_count() {
     return sms;
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 cudaError_t launch_one(const Maps &maps, const Params &p, cudaStream_t st) {
-    cudaError_t err = cudaFuncSetAttribute(grouped_ffn_gemm_kernel<EPI>,
+    cudaError_t err = cudaFuncSetAttribute(grouped_ffn_gemm_kernel<EPI, GATHER>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
     if (err != cudaSuccess) return err;
-    grouped_ffn_gemm_kernel<EPI><<<sm_count(), NUM_THREADS, SMEM_DYN, st>>>(maps, p);
+    grouped_ffn_gemm_kernel<EPI, GATHER>
+        <<<sm_count(), NUM_THREADS + (GATHER ? GATHER_THREADS : 0), SMEM_DYN, st>>>(maps, p);
     count_launch();
     return cudaGetLastError();
 }
@@ -509,13 +545,8 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     const bool gather = a.perm_token != nullptr;
     bool ok = map_3d(&m1.b0_r, a.w_gate, a.E, a.d_ff, a.d, BN_ACC / 2) &&
               map_3d(&m1.b1_r, a.w_up, a.E, a.d_ff, a.d, BN_ACC / 2);
-    if (gather) {  // routed rows straight from x: one-row boxes for four-row gathers
-        ok = ok && tensor_map_2d_bf16(&m1.a_g, a.x, a.T, a.d, BK, 1);
-        m1.a_r = m1.a_g;
-    } else {
-        ok = ok && map_2d(&m1.a_r, a.x_perm, rows_r, a.d, BM);
-        m1.a_g = m1.a_r;
-    }
+    // routed A: x_perm by tiled loads, or x rows gathered by the gatherer warps
+    ok = ok && map_2d(&m1.a_r, gather ? a.x : a.x_perm, gather ? a.T : rows_r, a.d, BM);
     if (has_shared)
         ok = ok && map_2d(&m1.a_s, a.x, a.T, a.d, BM) &&
              map_3d(&m1.b0_s, a.ws_gate, 1, ffs, a.d, BN_ACC / 2) &&
@@ -532,6 +563,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     Params p1{};
     p1.offsets = a.offsets;
     p1.perm_token = a.perm_token;
+    p1.x = a.x;
     p1.x_rows = a.T;
     p1.E = a.E;
     p1.rows_r = (int)rows_r;
@@ -545,14 +577,14 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p1.out_s = static_cast<__nv_bfloat16 *>(a.h_shared);
     p1.status = a.status;
     p1.timeout_ns = a.timeout_ns;
-    cudaError_t err = launch_one<EPI_SWIGLU>(m1, p1, st);
+    cudaError_t err = gather ? launch_one<EPI_SWIGLU, true>(m1, p1, st)
+                             : launch_one<EPI_SWIGLU, false>(m1, p1, st);
     if (err != cudaSuccess) return err;
 
     // GEMM2: y_perm = h W_d^T per expert; y_shared = h_shared Ws_d^T (k split per shared expert)
     Maps m2;
     ok = map_2d(&m2.a_r, a.h, rows_r, a.d_ff, BM) &&
          map_3d(&m2.b0_r, a.w_down, a.E, a.d, a.d_ff, BN_ACC);
-    m2.a_g = m2.a_r;
     if (has_shared)
         ok = ok && map_2d(&m2.a_s, a.h_shared, a.T, ffs, BM) &&
              map_3d(&m2.b0_s, a.ws_down, a.n_shared, a.d, a.d_ff_shared, BN_ACC);
@@ -575,7 +607,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p2.kseg_s = a.d_ff_shared;
     p2.out_r = static_cast<__nv_bfloat16 *>(a.y_perm);
     p2.out_s = static_cast<__nv_bfloat16 *>(a.y_shared);
-    return launch_one<EPI_STORE>(m2, p2, st);
+    return launch_one<EPI_STORE, false>(m2, p2, st);
 }
 
 cudaError_t launch_bounded_wait_selftest(int64_t timeout_ns, int32_t *status, cudaStream_t st) {

@@ -252,8 +252,9 @@ MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, con
 /*
  * Expert FFN fused with the dispatch gather: as moe_expert_ffn, but the routed
  * rows are read straight from x -- row r of expert segment e is
- * x[perm_token[r]] -- by four-row TMA gathers inside the gate/up GEMM, so the
- * permuted copy x_perm is never written or read (the gather-permute step of
+ * x[perm_token[r]] -- by gatherer warps of the gate/up GEMM (16-byte
+ * asynchronous copies into the swizzled operand stage), so the permuted copy
+ * x_perm is never written or read (the gather-permute step of
  * the dispatch, "moe-node-limited-routing", "Why all to all dominates MoE step
  * time", folded into the expert GEMM).
  *   x           [T, d]     bf16
