@@ -48,8 +48,14 @@ def lib():
                                            P, P, P, P, P, P, P, P, P, P, i32, P, P, P, P]
         _lib.oracle_router_affinity.argtypes = [i32, P, i32, i32, P, P, P, i32, P]
         _lib.oracle_layer_rows_ex.argtypes = [i32, P, i32, i32, i32, i32, i32, i32, i32, i32,
-                                              P, P, P, P, i32, P, P, P, P, P, P, P, i32, P, P,
-                                              P, P]
+                                              P, P, P, P, i32, P, i32, P, P, P, P, P, P, i32, P,
+                                              P, P, P]
+        _lib.oracle_e4m3_decode.argtypes = [C.c_uint8]
+        _lib.oracle_e4m3_decode.restype = C.c_double
+        _lib.oracle_e4m3_encode.argtypes = [C.c_float]
+        _lib.oracle_e4m3_encode.restype = C.c_uint8
+        _lib.oracle_fp8_quantize_row.argtypes = [i32, P, P, P]
+        _lib.oracle_fp8_dequantize_row.argtypes = [i32, P, P, P]
         _lib.oracle_hash_route.argtypes = [i32, P, i32, i32, i32, i32, P, P]
         _lib.oracle_lowbias32.argtypes = [C.c_uint32]
         _lib.oracle_lowbias32.restype = C.c_uint32
@@ -57,7 +63,8 @@ def lib():
         for f in ("oracle_router_scores", "oracle_select", "oracle_dispatch",
                   "oracle_ffn_row", "oracle_shared_row", "oracle_combine",
                   "oracle_layer_rows", "oracle_router_affinity", "oracle_layer_rows_ex",
-                  "oracle_hash_route", "oracle_bias_update"):
+                  "oracle_hash_route", "oracle_bias_update", "oracle_fp8_quantize_row",
+                  "oracle_fp8_dequantize_row"):
             getattr(_lib, f).restype = C.c_int
     return _lib
 
@@ -195,14 +202,50 @@ def combine(y_perm, inv_perm, topk_w, y_shared=None):
     return out
 
 
+def e4m3_decode(code):
+    return float(lib().oracle_e4m3_decode(int(code) & 0xFF))
+
+
+def e4m3_encode(v):
+    return int(lib().oracle_e4m3_encode(C.c_float(float(v))))
+
+
+def fp8_quantize(x):
+    """FP8 payload of bf16 rows x [n, d]: (q uint8 [n, d], scale fp32 [n, d/128])."""
+    x = _np(x, np.uint16)
+    x2 = x.reshape(-1, x.shape[-1])
+    n, d = x2.shape
+    q = np.empty((n, d), np.uint8)
+    sc = np.empty((n, d // 128), np.float32)
+    for r in range(n):
+        _check(lib().oracle_fp8_quantize_row(d, _p(x2[r]), _p(q[r]), _p(sc[r])),
+               "oracle_fp8_quantize_row")
+    return q.reshape(x.shape), sc.reshape(x.shape[:-1] + (d // 128,))
+
+
+def fp8_dequantize(q, scale):
+    """bf16 bits (uint16) the expert GEMM sees for an FP8 payload."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sc = np.ascontiguousarray(scale, dtype=np.float32)
+    q2 = q.reshape(-1, q.shape[-1])
+    s2 = sc.reshape(-1, sc.shape[-1])
+    out = np.empty(q2.shape, np.uint16)
+    for r in range(q2.shape[0]):
+        _check(lib().oracle_fp8_dequantize_row(q2.shape[1], _p(q2[r]), _p(s2[r]), _p(out[r])),
+               "oracle_fp8_dequantize_row")
+    return out.reshape(q.shape)
+
+
 def layer_rows(rows, shape, x, router_w, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
-               logit_offset=None, round_h=False, router=ROUTER_SIGMOID, token_ids=None):
+               logit_offset=None, round_h=False, router=ROUTER_SIGMOID, token_ids=None,
+               payload=0):
     """The whole layer for the token rows ``rows``.
 
     ``w_gate``/``w_up``/``w_down`` are sequences of per-expert host matrices
     (entries may be None for experts no listed token selects).
     ``router`` is ROUTER_SIGMOID, ROUTER_SQRT_SOFTPLUS or ROUTER_HASH (the
-    last keyed by ``token_ids[row]``, or the row index when None).
+    last keyed by ``token_ids[row]``, or the row index when None); ``payload``
+    1 feeds the routed experts the FP8 round trip of x.
     Returns (out float64 [n,d], topk_idx [n,K], topk_w [n,K], scores [n,E]).
     """
     r = _np(np.asarray(rows, dtype=np.int64), np.int64)
@@ -233,6 +276,7 @@ def layer_rows(rows, shape, x, router_w, bias, w_gate, w_up, w_down, ws_gate, ws
     rc = lib().oracle_layer_rows_ex(n, _p(r), shape.d, shape.E, shape.G, shape.K, shape.M,
                                     shape.d_ff, shape.n_shared, shape.d_ff_shared,
                                     _p(x), _p(e), _p(off), _p(b), int(router), _p(tid),
+                                    int(payload),
                                     C.cast(g, C.c_void_p), C.cast(u, C.c_void_p),
                                     C.cast(dn, C.c_void_p), _p(sg), _p(su), _p(sd),
                                     int(round_h), _p(out), _p(idx), _p(w), _p(sc))

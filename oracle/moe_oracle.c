@@ -10,8 +10,8 @@
  * What it computes, step by step, and where each step comes from:
  *   1. router affinity  s_i = sigmoid(x . e_i (+ o_i))   -- affinities feed
  *      top-k gating ["MoE + Expert-Parallel Overlap (Exp08)", Implemented];
- *      the sigmoid form is DeepSeek-V3's (that page gives the V4
- *      Sqrt(Softplus) form, which this layer does not use).  o_i is an
+ *      the sigmoid form is DeepSeek-V3's; that page's V4 form
+ *      sqrt(softplus(.)) is the variant "affinity kind 1".  o_i is an
  *      optional per-expert logit offset (the skewed-load workload).
  *   2. selection bias  b_i = s_i + bias_i  (auxiliary-loss-free balancing:
  *      "per-expert bias updates", Exp08 Implemented) -- used to choose
@@ -34,6 +34,10 @@
  *      experts are always on with weight 1 ("shared experts (always active) +
  *      fine-grained routed experts", Exp08 Implemented).
  *   7. combine: out_t = sum_shared FFN_s(x_t) + sum_j w_j FFN_{e_j}(x_t).
+ * Variants, each behind its own function or flag: the hash router, the
+ * per-expert bias update, and the FP8 dispatch payload (the routed copies of
+ * x travel as FP8 E4M3 with one fp32 scale per 128 values; "Compression has a
+ * numerical price", shivam2003 section 4).
  *
  * Arithmetic: dot products accumulate in double from the exact bf16/fp32
  * inputs; sigmoid and SiLU use libm exp() in double.  The selection steps
@@ -374,11 +378,16 @@ int oracle_hash_route(int n_rows, const int64_t *token_ids, int E, int G, int K,
  *   router 1: sqrt(softplus) affinities + the same selection (V4)
  *   router 2: hash router keyed by token_ids[rows[r]] (or rows[r] when
  *             token_ids is NULL); e, off, bias unused, scores_out untouched. */
+int oracle_fp8_quantize_row(int d, const uint16_t *x, uint8_t *q, float *scale);
+int oracle_fp8_dequantize_row(int d, const uint8_t *q, const float *scale, uint16_t *x_hat);
+
+/* payload 0: the routed experts read x; payload 1: they read the FP8 round
+ * trip x_hat of the FP8 dispatch payload (shared experts always read x). */
 int oracle_layer_rows_ex(int n_rows, const int64_t *rows,
                          int d, int E, int G, int K, int M, int d_ff,
                          int n_shared, int d_ff_s,
                          const uint16_t *x, const float *e, const float *off,
-                         const float *bias, int router, const int64_t *token_ids,
+                         const float *bias, int router, const int64_t *token_ids, int payload,
                          const uint16_t *const *Wg, const uint16_t *const *Wu,
                          const uint16_t *const *Wd,
                          const uint16_t *Wsg, const uint16_t *Wsu, const uint16_t *Wsd,
@@ -386,12 +395,16 @@ int oracle_layer_rows_ex(int n_rows, const int64_t *rows,
                          float *scores_out)
 {
     if (n_rows < 0 || !rows || !x || !Wg || !Wu || !Wd || !out || !topk_idx || !topk_w ||
-        router < 0 || router > 2 || (router < 2 && (!e || !bias)))
+        router < 0 || router > 2 || (router < 2 && (!e || !bias)) || payload < 0 ||
+        payload > 1 || (payload == 1 && d % 128))
         return ORC_EBADARG;
     int rc = ORC_OK;
     float *scores = malloc(sizeof(float) * (size_t)E * (n_rows > 0 ? n_rows : 1));
     double *y = malloc(sizeof(double) * d);
-    if (!scores || !y) {
+    uint16_t *xq = malloc(sizeof(uint16_t) * d);
+    uint8_t *q = malloc((size_t)d);
+    float *qs = malloc(sizeof(float) * (size_t)(d / 128 + 1));
+    if (!scores || !y || !xq || !q || !qs) {
         rc = ORC_ENOMEM;
         goto done;
     }
@@ -414,13 +427,19 @@ int oracle_layer_rows_ex(int n_rows, const int64_t *rows,
         rc = oracle_shared_row(d, n_shared, d_ff_s, xr, Wsg, Wsu, Wsd, round_h, o);
         if (rc)
             goto done;
+        const uint16_t *xe = xr;  /* the routed experts' input row */
+        if (payload == 1) {
+            oracle_fp8_quantize_row(d, xr, q, qs);
+            oracle_fp8_dequantize_row(d, q, qs, xq);
+            xe = xq;
+        }
         for (int j = 0; j < K; ++j) {
             int ex = topk_idx[(int64_t)r * K + j];
             if (!Wg[ex] || !Wu[ex] || !Wd[ex]) {
                 rc = ORC_EBADARG;
                 goto done;
             }
-            rc = oracle_ffn_row(d, d_ff, xr, Wg[ex], Wu[ex], Wd[ex], round_h, y);
+            rc = oracle_ffn_row(d, d_ff, xe, Wg[ex], Wu[ex], Wd[ex], round_h, y);
             if (rc)
                 goto done;
             double w = (double)topk_w[(int64_t)r * K + j];
@@ -433,6 +452,9 @@ int oracle_layer_rows_ex(int n_rows, const int64_t *rows,
 done:
     free(scores);
     free(y);
+    free(xq);
+    free(q);
+    free(qs);
     return rc;
 }
 
@@ -448,7 +470,7 @@ int oracle_layer_rows(int n_rows, const int64_t *rows,
                       float *scores_out)
 {
     return oracle_layer_rows_ex(n_rows, rows, d, E, G, K, M, d_ff, n_shared, d_ff_s, x, e, off,
-                                bias, 0, NULL, Wg, Wu, Wd, Wsg, Wsu, Wsd, round_h, out, topk_idx,
+                                bias, 0, NULL, 0, Wg, Wu, Wd, Wsg, Wsu, Wsd, round_h, out, topk_idx,
                                 topk_w, scores_out);
 }
 
@@ -539,6 +561,98 @@ int oracle_bias_update(int E, int T, int K, const int32_t *counts, float gamma, 
         const int64_t c = (int64_t)counts[i] * E;
         const float step = c < total ? gamma : (c > total ? -gamma : 0.0f);
         bias[i] = bias[i] + step;
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ FP8 payload */
+/* Lower-precision dispatch payload ("sending fewer bytes through
+ * lower-precision activations ... quantization and dequantization add kernels
+ * and error", shivam2003 "DeepSeek 8.7", section 4).  The pages fix neither
+ * the format nor the scaling, so the reading is DeepSeek-V3's published
+ * recipe: OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * no infinities, S.1111.111 = NaN, largest finite 448) with one fp32 scale per
+ * token and block of 128 channels:
+ *   amax = max |x_i| over the block,  s = amax / 448  (fp32),
+ *   q_i  = E4M3(x_i / s)   (fp32 division; nearest, ties to even mantissa;
+ *                           |v| >= 448 saturates to 448; amax = 0 gives q = 0)
+ * The expert GEMM consumes  x_hat_i = bf16(float(E4M3^-1(q_i)) * s)  (one fp32
+ * multiply, then bf16 nearest-even).  Router and shared experts keep x. */
+double oracle_e4m3_decode(uint8_t q)
+{
+    const int sgn = q >> 7, e = (q >> 3) & 15, m = q & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);          /* subnormal: m/8 * 2^-6 */
+    else
+        v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+    return sgn ? -v : v;
+}
+
+/* Nearest E4M3 code to a finite float by direct search over the 127
+ * non-negative finite codes (ties to the even code), saturating at 448. */
+uint8_t oracle_e4m3_encode(float f)
+{
+    const uint8_t sgn = signbit(f) ? 0x80 : 0x00;
+    const double a = fabs((double)f);
+    if (a >= 448.0)
+        return sgn | 0x7E;
+    int best = 0;
+    double best_err = a;
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double err = fabs(oracle_e4m3_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return sgn | (uint8_t)best;
+}
+
+static float bf16_round_float(float v)
+{
+    uint32_t bits;
+    memcpy(&bits, &v, 4);
+    bits += 0x7FFFu + ((bits >> 16) & 1u);
+    bits &= 0xFFFF0000u;
+    memcpy(&v, &bits, 4);
+    return v;
+}
+
+/* Quantize one bf16 row of d values (d % 128 == 0): q[d] codes, scale[d/128]. */
+int oracle_fp8_quantize_row(int d, const uint16_t *x, uint8_t *q, float *scale)
+{
+    if (d <= 0 || d % 128 || !x || !q || !scale)
+        return ORC_EBADARG;
+    for (int b = 0; b < d / 128; ++b) {
+        float amax = 0.0f;
+        for (int i = 0; i < 128; ++i) {
+            const float v = fabsf((float)bf16_value(x[b * 128 + i]));
+            if (v > amax)
+                amax = v;
+        }
+        const float sc = amax / 448.0f;
+        scale[b] = sc;
+        for (int i = 0; i < 128; ++i) {
+            const float v = (float)bf16_value(x[b * 128 + i]);
+            q[b * 128 + i] = amax == 0.0f ? 0 : oracle_e4m3_encode(v / sc);
+        }
+    }
+    return ORC_OK;
+}
+
+/* The bf16 row the expert GEMM sees: x_hat_i = bf16(decode(q_i) * s). */
+int oracle_fp8_dequantize_row(int d, const uint8_t *q, const float *scale, uint16_t *x_hat)
+{
+    if (d <= 0 || d % 128 || !q || !scale || !x_hat)
+        return ORC_EBADARG;
+    for (int i = 0; i < d; ++i) {
+        const float v = bf16_round_float((float)oracle_e4m3_decode(q[i]) * scale[i / 128]);
+        uint32_t bits;
+        memcpy(&bits, &v, 4);
+        x_hat[i] = (uint16_t)(bits >> 16);
     }
     return ORC_OK;
 }
