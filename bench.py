@@ -406,8 +406,34 @@ def variants_leg(sh, inp, dev, stream, reps=20):
                                   inp["w_down"], y_perm, inp.get("ws_gate"), inp.get("ws_up"),
                                   inp.get("ws_down"), y_sh, ws, stream)
 
-    out["dispatch_plus_ffn_ms"] = {"two_step_x_perm": timed(two_step), "fused_gather": timed(fused)}
+    res = {"two_step_x_perm": timed(two_step), "fused_gather": timed(fused)}
+    if sh.d % 128 == 0:  # the FP8 payload: 1-byte codes + 1x128 scales
+        cfg8 = moe.MoeConfig.of(sh, payload=moe.MOE_PAYLOAD_FP8)
+        xq = torch.empty(T * K, sh.d, dtype=torch.uint8, device=dev)
+        xs = torch.empty(T * K, sh.d // 128, dtype=torch.float32, device=dev)
+
+        def fp8_payload():
+            moe.moe_dispatch_fp8(cfg8, inp["x"], o["topk_idx"], o["counts"], o["offsets"],
+                                 o["send"], o["send_tok"], perm, inv, xq, xs, ws, stream)
+            moe.moe_expert_ffn_fp8(cfg8, xq, xs, o["offsets"], inp["w_gate"], inp["w_up"],
+                                   inp["w_down"], y_perm, inp["x"], inp.get("ws_gate"),
+                                   inp.get("ws_up"), inp.get("ws_down"), y_sh, ws, stream)
+
+        res["fp8_payload"] = timed(fp8_payload)
+        del xq, xs
+    out["dispatch_plus_ffn_ms"] = res
     del ws, o, x_perm, y_perm, y_sh
+    if sh.d % 128 == 0:
+        cfg8 = moe.MoeConfig.of(sh, payload=moe.MOE_PAYLOAD_FP8)
+        ws8 = moe.alloc_workspace(cfg8, dev)
+        o8 = moe.forward_outputs(cfg8, dev)
+        ms = timed(lambda: moe.moe_forward(cfg8, inp["x"], inp["router_w"],
+                                           inp.get("logit_offset"), inp["bias"], inp["w_gate"],
+                                           inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                                           inp.get("ws_up"), inp.get("ws_down"), o8["out"],
+                                           ws=ws8, stream=stream))
+        out["fp8_payload_forward"] = {"forward_ms": ms, "forward_tokens_per_s": T / (ms / 1e3)}
+        del ws8, o8
     names = {moe.MOE_ROUTER_SIGMOID: "sigmoid", moe.MOE_ROUTER_SQRT_SOFTPLUS: "sqrt_softplus",
              moe.MOE_ROUTER_HASH: "hash"}
     for r, name in names.items():

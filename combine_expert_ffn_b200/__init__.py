@@ -34,23 +34,30 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_read_device_status", "moe_clear_device_status", "moe_route", "moe_route_select",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_bounded_wait", "moe_dispatch_noalloc", "moe_route_hash",
-           "moe_bias_update", "moe_expert_ffn_gather")
+           "moe_bias_update", "moe_expert_ffn_gather", "moe_dispatch_fp8",
+           "moe_expert_ffn_fp8")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
+MOE_PAYLOAD_BF16, MOE_PAYLOAD_FP8 = 0, 1
 
 
 class MoeConfig(C.Structure):
     """Mirror of ``moe_config``."""
     _fields_ = [(n, C.c_int32) for n in
-                ("T", "d", "E", "G", "K", "M", "d_ff", "n_shared", "d_ff_shared", "router")]
+                ("T", "d", "E", "G", "K", "M", "d_ff", "n_shared", "d_ff_shared", "router",
+                 "payload")]
 
     @classmethod
-    def of(cls, shape, router=None) -> "MoeConfig":
+    def of(cls, shape, router=None, payload=None) -> "MoeConfig":
         """From any object with the nine size attributes (e.g. ``synth.MoeShape``);
-        the router is ``router``, else the object's ``router``, else the sigmoid."""
+        router and payload from the arguments, else the object's, else the defaults
+        (sigmoid router, bf16 payload)."""
         if router is None:
             router = getattr(shape, "router", MOE_ROUTER_SIGMOID)
-        return cls(*(int(getattr(shape, n)) for n, _ in cls._fields_[:-1]), int(router))
+        if payload is None:
+            payload = getattr(shape, "payload", MOE_PAYLOAD_BF16)
+        return cls(*(int(getattr(shape, n)) for n, _ in cls._fields_[:-2]), int(router),
+                   int(payload))
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -79,6 +86,9 @@ _sig = {
     "moe_forward": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _S, _P]),
     "moe_route_hash": (C.c_int, [_CP, _P, _P, _P, _P]),
+    "moe_dispatch_fp8": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "moe_expert_ffn_fp8": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
+                                     _P]),
     "moe_expert_ffn_gather": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
                                         _P]),
     "moe_bias_update": (C.c_int, [_CP, _P, C.c_float, _P, _P]),
@@ -206,6 +216,25 @@ def moe_expert_ffn_gather(cfg, x, perm_token, offsets, w_gate, w_up, w_down, y_p
                                    _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y_perm),
                                    _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_shared), wp,
                                    wn, _stream(stream)))
+
+
+def moe_dispatch_fp8(cfg, x, topk_idx, counts, offsets, send, send_tok, perm_token, inv_perm,
+                     x_perm_q, x_scale, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_dispatch_fp8",
+        _lib.moe_dispatch_fp8(_cfg(cfg), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                              _ptr(send), _ptr(send_tok), _ptr(perm_token), _ptr(inv_perm),
+                              _ptr(x_perm_q), _ptr(x_scale), wp, wn, _stream(stream)))
+
+
+def moe_expert_ffn_fp8(cfg, x_perm_q, x_scale, offsets, w_gate, w_up, w_down, y_perm, x, ws_gate,
+                       ws_up, ws_down, y_shared, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_expert_ffn_fp8",
+        _lib.moe_expert_ffn_fp8(_cfg(cfg), _ptr(x_perm_q), _ptr(x_scale), _ptr(offsets),
+                                _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y_perm), _ptr(x),
+                                _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_shared), wp, wn,
+                                _stream(stream)))
 
 
 def moe_combine(cfg, y_perm, inv_perm, topk_w, y_shared, out, stream=None) -> None:

@@ -105,6 +105,9 @@ moe_status moe_check_config(const moe_config *c) {
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->router < MOE_ROUTER_SIGMOID || c->router > MOE_ROUTER_HASH)
         return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->payload < MOE_PAYLOAD_BF16 || c->payload > MOE_PAYLOAD_FP8)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->payload == MOE_PAYLOAD_FP8 && c->d % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->E % c->G || c->K % c->M || c->M > c->G || c->K / c->M > c->E / c->G)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->K > 32 || c->E > 1024 || c->G > 64) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -225,6 +228,66 @@ moe_status moe_dispatch(const moe_config *c, const void *x, const int32_t *topk_
     return cuda_status(launch_dispatch(x, topk_idx, c->T, c->d, c->E, c->G, c->K, counts, offsets,
                                        send, send_tok, perm_token, inv_perm, x_perm, dw,
                                        at<int32_t>(ws, L.status), as_stream(stream)));
+}
+
+moe_status moe_dispatch_fp8(const moe_config *c, const void *x, const int32_t *topk_idx,
+                            int32_t *counts, int32_t *offsets, int32_t *send, int32_t *send_tok,
+                            int32_t *perm_token, int32_t *inv_perm, uint8_t *x_perm_q,
+                            float *x_scale, void *ws, size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->d % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!counts || !offsets || !send || !ws) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0 && (!x || !topk_idx || !perm_token || !inv_perm || !x_perm_q || !x_scale))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm_q) || !aligned16(x_scale)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout(*c);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    cudaStream_t s = as_stream(stream);
+    DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),
+                  at<int32_t>(ws, L.send_part), at<int32_t>(ws, L.sendtok_part)};
+    if (launch_dispatch(x, topk_idx, c->T, c->d, c->E, c->G, c->K, counts, offsets, send, send_tok,
+                        perm_token, inv_perm, nullptr, dw, at<int32_t>(ws, L.status), s))
+        return MOE_ERR_CUDA;
+    return cuda_status(launch_gather_fp8(x, inv_perm, c->T, c->d, c->K, x_perm_q, x_scale, s));
+}
+
+moe_status moe_expert_ffn_fp8(const moe_config *c, const uint8_t *x_perm_q, const float *x_scale,
+                              const int32_t *offsets, const void *w_gate, const void *w_up,
+                              const void *w_down, void *y_perm, const void *x, const void *ws_gate,
+                              const void *ws_up, const void *ws_down, void *y_shared, void *ws,
+                              size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->d % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0) {
+        if (!x_perm_q || !x_scale || !offsets || !w_gate || !w_up || !w_down || !y_perm || !x)
+            return MOE_ERR_INVALID_ARG;
+        if (c->n_shared > 0 && (!ws_gate || !ws_up || !ws_down || !y_shared))
+            return MOE_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {x_perm_q, x_scale, w_gate, w_up, w_down, y_perm, x, ws_gate, ws_up,
+                          ws_down, y_shared};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout(*c);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    FfnArgs a{};
+    a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
+    a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
+    a.x_perm_q = x_perm_q; a.x_scale = x_scale; a.offsets = offsets;
+    a.w_gate = w_gate; a.w_up = w_up; a.w_down = w_down;
+    a.h = at<void>(ws, L.h); a.y_perm = y_perm;
+    a.x = x; a.ws_gate = ws_gate; a.ws_up = ws_up; a.ws_down = ws_down;
+    a.h_shared = at<void>(ws, L.h_sh); a.y_shared = y_shared;
+    a.status = at<int32_t>(ws, L.status);
+    a.timeout_ns = kWaitTimeoutNs;
+    return cuda_status(launch_expert_ffn(a, as_stream(stream)));
 }
 
 moe_status moe_expert_ffn(const moe_config *c, const void *x_perm, const int32_t *offsets,
@@ -360,14 +423,22 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
     // but measured about 13% slower for dispatch + expert FFN at V3 sizes: its
     // 16-byte row copies feed the tensor core more slowly than whole-tile TMA
     // loads of the contiguous x_perm rows.)
+    // With the FP8 payload the x_perm region holds the codes [T*K, d] and, after
+    // them, the scales [T*K, d/128] (together at most half of its 2*T*K*d bytes + 16).
     void *x_perm = at<void>(ws, L.x_perm);
+    const bool fp8 = c->payload == MOE_PAYLOAD_FP8;
+    uint8_t *x_perm_q = static_cast<uint8_t *>(x_perm);
+    float *x_scale = reinterpret_cast<float *>(x_perm_q + (size_t)c->T * c->K * c->d);
     if (launch_dispatch(x, topk_idx, c->T, c->d, c->E, c->G, c->K, counts, offsets, send, send_tok,
-                        perm_token, inv_perm, x_perm, dw, status, s))
+                        perm_token, inv_perm, fp8 ? nullptr : x_perm, dw, status, s))
+        return MOE_ERR_CUDA;
+    if (fp8 && launch_gather_fp8(x, inv_perm, c->T, c->d, c->K, x_perm_q, x_scale, s))
         return MOE_ERR_CUDA;
     FfnArgs a{};
     a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
     a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
-    a.x_perm = x_perm; a.perm_token = nullptr; a.offsets = offsets;
+    a.x_perm = fp8 ? nullptr : x_perm; a.perm_token = nullptr; a.offsets = offsets;
+    a.x_perm_q = fp8 ? x_perm_q : nullptr; a.x_scale = fp8 ? x_scale : nullptr;
     a.w_gate = w_gate; a.w_up = w_up; a.w_down = w_down;
     a.h = at<void>(ws, L.h); a.y_perm = y_perm;
     a.x = x; a.ws_gate = ws_gate; a.ws_up = ws_up; a.ws_down = ws_down;

@@ -16,6 +16,8 @@
 //             offsets = exclusive scan of counts (recomputed per block)
 //   gather  : x_perm[row] = x[t], reading each x row once and writing it K
 //             times with 16-byte vector accesses
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 
 namespace moe {
@@ -208,6 +210,77 @@ dispatch_gather_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ 
             if (row >= 0 && row < n_rows) x_perm[(int64_t)row * chunks + c] = v;
         }
     }
+}
+
+// FP8 payload gather.  One 16-lane group per (token, 128-channel block);
+// lane l of the group holds channels 8l .. 8l+7.  s = amax / 448 in fp32,
+// q = E4M3(x / s) (fp32 division, nearest-even, saturating), all-zero blocks
+// give s = 0 and q = 0.  Each token's codes and scales are written to its K
+// permuted rows.
+__global__ void __launch_bounds__(256)
+dispatch_gather_fp8_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ inv_perm,
+                           int T, int chunks, int K, int64_t n_rows, uint2 *__restrict__ xq,
+                           float *__restrict__ xs) {
+    const int64_t total = (int64_t)T * chunks;  // a multiple of 16: groups never straddle it
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + (threadIdx.x & ~31); i0 < total;
+         i0 += stride) {
+        const int64_t i = i0 + lane;
+        const bool in = i < total;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (in) v = __ldg(x + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            f[2 * j] = bf16_lo(w[j]);
+            f[2 * j + 1] = bf16_hi(w[j]);
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        if (!in) continue;
+        const float sc = __fdiv_rn(amax, 448.0f);
+        uint32_t q[2] = {0u, 0u};
+        if (amax > 0.f) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(f[2 * j], sc), __fdiv_rn(f[2 * j + 1], sc)),
+                    __NV_SATFINITE, __NV_E4M3);
+                q[j >> 1] |= (uint32_t)b << (16 * (j & 1));
+            }
+        }
+        const uint2 packed = make_uint2(q[0], q[1]);
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        for (int j = 0; j < K; ++j) {
+            const int row = __ldg(inv_perm + t * K + j);
+            if (row < 0 || row >= n_rows) continue;
+            xq[(int64_t)row * chunks + c] = packed;
+            if ((c & 15) == 0) xs[(int64_t)row * (chunks >> 4) + (c >> 4)] = sc;
+        }
+    }
+}
+
+cudaError_t launch_gather_fp8(const void *x, const int32_t *inv_perm, int T, int d, int K,
+                              uint8_t *x_perm_q, float *x_scale, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    const int64_t total = (int64_t)T * chunks;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (total + 255) / 256;
+    const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+    dispatch_gather_fp8_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4 *>(x), inv_perm, T,
+                                                     chunks, K, (int64_t)T * K,
+                                                     reinterpret_cast<uint2 *>(x_perm_q), x_scale);
+    count_launch();
+    return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d, int E, int G,

@@ -27,6 +27,9 @@
 // those rows are computed and never stored.  Every wait is bounded; on
 // running out the kernel records MOE_ERR_DEVICE_TIMEOUT, drains its own TMA
 // loads and MMAs, frees TMEM and returns.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 
 
@@ -41,10 +44,13 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN_ACC * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
-// Gather variant of GEMM1: four more warps copy the routed A rows
-// x[perm_token[r]] into the swizzled stage with 16-byte cp.async copies.
+// Variants of GEMM1's routed A operand: TMA tiles of x_perm; rows gathered
+// from x by four extra warps (16-byte cp.async copies); or the FP8 payload,
+// TMA-loaded as bytes and widened to bf16 in place by four extra warps.
+enum { A_TMA = 0, A_GATHER = 1, A_FP8 = 2 };
 constexpr int GATHER_WARPS = 4;
 constexpr int GATHER_THREADS = GATHER_WARPS * 32;
+constexpr int FP8_STAGE_OFF = A_BYTES / 2;  // FP8 bytes land in the upper half of the A stage
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
 constexpr int STORE_BUF = 32 * 32 * 2;     // one warp's 32 rows x 32 columns of bf16
@@ -68,6 +74,7 @@ struct Maps {
     CUtensorMap b1_s;  // shared B  up
     CUtensorMap o_r;   // routed output [rows_r, n_out_r]    box 32 x 32, for full tiles
     CUtensorMap o_s;   // shared output [T, n_out_s]         box 32 x 32
+    CUtensorMap a_q;   // routed FP8 payload [rows_r, k_r] bytes, box 64 x 128 (A_FP8)
 };
 
 struct Params {
@@ -75,6 +82,7 @@ struct Params {
     const int32_t *perm_token;  // gather variant: routed row r of A is x[perm_token[r]]
     const void *x;           // gather variant: x [x_rows, k_r] bf16
     int x_rows;
+    const float *x_scale;    // FP8 variant: [rows_r, k_r / 128] payload scales
     int E;
     int rows_r;              // rows of the routed A buffer (T*K)
     int T;                   // shared rows; 0 = no shared experts
@@ -146,10 +154,16 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return g * __frcp_rn(1.0f + __expf(-g)) * u;
 }
 
-template <int EPI, bool GATHER>
-__global__ void __launch_bounds__(NUM_THREADS + (GATHER ? GATHER_THREADS : 0), 1)
+__device__ __forceinline__ void converters_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(GATHER_THREADS) : "memory");
+}
+
+template <int EPI, int AMODE>
+__global__ void __launch_bounds__(NUM_THREADS + (AMODE != A_TMA ? GATHER_THREADS : 0), 1)
 grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
-    static_assert(!GATHER || EPI == EPI_SWIGLU, "only GEMM1 gathers its rows");
+    static_assert(AMODE == A_TMA || EPI == EPI_SWIGLU, "only GEMM1 has A-operand variants");
+    constexpr bool GATHER = AMODE == A_GATHER;
+    constexpr bool EXTRA = AMODE != A_TMA;  // extra warps write A stages
     constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -157,6 +171,8 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     __shared__ __align__(8) uint64_t tfull_bar[2];
     __shared__ __align__(8) uint64_t tempty_bar[2];
     __shared__ __align__(8) uint64_t done_bar;
+    __shared__ __align__(8) uint64_t qfull_bar[STAGES];  // A_FP8: payload bytes of a stage landed
+    __shared__ int conv_ok_s;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_base[MAX_E + 1];
@@ -203,7 +219,8 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         if (lane == 0) {
             tile_base[p.E] = carry;
             tma_prefetch_desc(&maps.o_r);
-            if (!GATHER) tma_prefetch_desc(&maps.a_r);
+            if (AMODE == A_TMA) tma_prefetch_desc(&maps.a_r);
+            if (AMODE == A_FP8) tma_prefetch_desc(&maps.a_q);
             tma_prefetch_desc(&maps.b0_r);
             if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
             if (p.T > 0) {
@@ -215,7 +232,8 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     } else if (warp == 1) {
         if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
-                mbar_init(smem_u32(&full_bar[s]), 1 + (GATHER ? GATHER_THREADS : 0));
+                mbar_init(smem_u32(&full_bar[s]), 1 + (EXTRA ? GATHER_THREADS : 0));
+                mbar_init(smem_u32(&qfull_bar[s]), 1);
                 mbar_init(smem_u32(&empty_bar[s]), 1);
             }
             for (int b = 0; b < 2; ++b) {
@@ -248,7 +266,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             uint32_t n_issued = 0;
             for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
                 const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
-                const bool a_by_tma = !GATHER || t.e < 0;
+                const bool a_by_tma = AMODE == A_TMA || t.e < 0;
                 bool ok = true;
                 for (int kb = 0; kb < t.kblocks; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
@@ -261,6 +279,15 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                     const uint32_t b_dst = a_dst + A_BYTES;
                     const int k = kb * BK;
                     mbar_arrive_expect_tx(fb, a_by_tma ? Cfg<EPI>::TX : Cfg<EPI>::TX - A_BYTES);
+                    if (AMODE == A_FP8) {  // converters wait for this barrier every stage
+                        const uint32_t qb = smem_u32(&qfull_bar[stage]);
+                        if (a_by_tma) {
+                            mbar_arrive(qb);
+                        } else {
+                            mbar_arrive_expect_tx(qb, A_BYTES / 2);
+                            tma_load_2d(a_dst + FP8_STAGE_OFF, &maps.a_q, qb, k, t.row0);
+                        }
+                    }
                     if (t.e >= 0) {
                         if (a_by_tma) tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
                         if (EPI == EPI_SWIGLU) {
@@ -315,7 +342,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                         break;
                     }
                     tc_fence_after();
-                    if (GATHER) fence_proxy_async();  // gathered rows: generic-proxy writes
+                    if (EXTRA) fence_proxy_async();  // A rows written through the generic proxy
                     const uint32_t a_addr = smem0 + stage * STAGE_BYTES;
                     const uint64_t a_desc = smem_desc_sw128(a_addr);
                     const uint64_t b_desc = smem_desc_sw128(a_addr + A_BYTES);
@@ -336,6 +363,80 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             drain_wait(smem_u32(&done_bar), 0, p.timeout_ns, p.status);
         }
         __syncwarp();
+    } else if (AMODE == A_FP8 && warp >= NUM_THREADS / 32) {
+        // ------------------------------------------------------ FP8 converters
+        // Thread g widens the 8-byte chunk c = g % 8 of the rows g / 8 + 16 j
+        // (j < 8): x_hat = bf16(E4M3^-1(q) * s), s the row's scale of the
+        // 128-channel block, into the 128-byte-swizzled bf16 stage.  The
+        // payload sits in the upper half of that stage, so every converter
+        // reads its bytes before any writes (named barrier).  Thread 0 alone
+        // waits (bounded) for the payload and shares the outcome.
+        const int g = threadIdx.x - NUM_THREADS;
+        const int c = g & 7, r0 = g >> 3;
+        const int nsb = p.k_r / 128;  // scales per row
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+            const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
+            const bool conv = t.e >= 0;
+            float s_cur[8], s_next[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = r0 + 16 * j;
+                s_cur[j] = 0.f;
+                s_next[j] = conv && r < t.rows_valid ? p.x_scale[(size_t)(t.row0 + r) * nsb] : 0.f;
+            }
+            for (int kb = 0; kb < t.kblocks; ++kb) {
+                if (conv && (kb & 1) == 0) {  // a new 128-channel block: its scales were loaded ahead
+                    const int nb = kb / 2 + 1;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int r = r0 + 16 * j;
+                        s_cur[j] = s_next[j];
+                        s_next[j] = nb < nsb && r < t.rows_valid
+                                        ? p.x_scale[(size_t)(t.row0 + r) * nsb + nb] : 0.f;
+                    }
+                }
+                if (g == 0)
+                    conv_ok_s = mbar_wait_bounded(smem_u32(&qfull_bar[stage]), phase, abort_flag,
+                                                  p.status, p.timeout_ns);
+                converters_sync();
+                ok = *reinterpret_cast<volatile int *>(&conv_ok_s) != 0;
+                if (!ok) break;  // every converter read the same flag
+                uint8_t *st = smem + stage * STAGE_BYTES;
+                uint2 raw[8];
+                if (conv) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        raw[j] = *reinterpret_cast<const uint2 *>(st + FP8_STAGE_OFF +
+                                                                  (r0 + 16 * j) * 64 + c * 8);
+                }
+                // every payload byte is in registers, and every converter has read
+                // the flag before thread 0 may write the next one
+                converters_sync();
+                if (conv) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int r = r0 + 16 * j;
+                        const uint32_t w2[2] = {raw[j].x, raw[j].y};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                                (__nv_fp8x2_storage_t)(w2[h >> 1] >> (16 * (h & 1))), __NV_E4M3);
+                            const float2 f = __half22float2(__half2(hr));
+                            o[h] = pack_bf16x2(__fmul_rn(f.x, s_cur[j]), __fmul_rn(f.y, s_cur[j]));
+                        }
+                        *reinterpret_cast<uint4 *>(st + r * (BK * 2) + ((c ^ (r & 7)) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                    fence_proxy_async();
+                }
+                mbar_arrive(smem_u32(&full_bar[stage]));
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
     } else if (GATHER && warp >= NUM_THREADS / 32) {
         // ------------------------------------------------------ A-row gatherers
         // Thread g copies the 16-byte chunk c = g % 8 of the rows g / 8 + 16 j
@@ -519,13 +620,13 @@ int sm_count() {
     return sms;
 }
 
-template <int EPI, bool GATHER>
+template <int EPI, int AMODE>
 cudaError_t launch_one(const Maps &maps, const Params &p, cudaStream_t st) {
-    cudaError_t err = cudaFuncSetAttribute(grouped_ffn_gemm_kernel<EPI, GATHER>,
+    cudaError_t err = cudaFuncSetAttribute(grouped_ffn_gemm_kernel<EPI, AMODE>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
     if (err != cudaSuccess) return err;
-    grouped_ffn_gemm_kernel<EPI, GATHER>
-        <<<sm_count(), NUM_THREADS + (GATHER ? GATHER_THREADS : 0), SMEM_DYN, st>>>(maps, p);
+    grouped_ffn_gemm_kernel<EPI, AMODE>
+        <<<sm_count(), NUM_THREADS + (AMODE != A_TMA ? GATHER_THREADS : 0), SMEM_DYN, st>>>(maps, p);
     count_launch();
     return cudaGetLastError();
 }
@@ -545,8 +646,15 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     const bool gather = a.perm_token != nullptr;
     bool ok = map_3d(&m1.b0_r, a.w_gate, a.E, a.d_ff, a.d, BN_ACC / 2) &&
               map_3d(&m1.b1_r, a.w_up, a.E, a.d_ff, a.d, BN_ACC / 2);
-    // routed A: x_perm by tiled loads, or x rows gathered by the gatherer warps
-    ok = ok && map_2d(&m1.a_r, gather ? a.x : a.x_perm, gather ? a.T : rows_r, a.d, BM);
+    // routed A: x_perm by tiled loads, x rows gathered by the gatherer warps, or the
+    // FP8 payload by byte tiles (a_r then only stands in for the unused map)
+    const bool fp8 = a.x_perm_q != nullptr;
+    if (fp8)
+        ok = ok && tensor_map_2d_u8(&m1.a_q, a.x_perm_q, rows_r, a.d, BK, BM) &&
+             map_2d(&m1.a_r, a.x, a.T, a.d, BM);
+    else
+        ok = ok && map_2d(&m1.a_r, gather ? a.x : a.x_perm, gather ? a.T : rows_r, a.d, BM);
+    if (!fp8) m1.a_q = m1.a_r;
     if (has_shared)
         ok = ok && map_2d(&m1.a_s, a.x, a.T, a.d, BM) &&
              map_3d(&m1.b0_s, a.ws_gate, 1, ffs, a.d, BN_ACC / 2) &&
@@ -565,6 +673,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p1.perm_token = a.perm_token;
     p1.x = a.x;
     p1.x_rows = a.T;
+    p1.x_scale = a.x_scale;
     p1.E = a.E;
     p1.rows_r = (int)rows_r;
     p1.T = has_shared ? a.T : 0;
@@ -577,8 +686,9 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p1.out_s = static_cast<__nv_bfloat16 *>(a.h_shared);
     p1.status = a.status;
     p1.timeout_ns = a.timeout_ns;
-    cudaError_t err = gather ? launch_one<EPI_SWIGLU, true>(m1, p1, st)
-                             : launch_one<EPI_SWIGLU, false>(m1, p1, st);
+    cudaError_t err = fp8      ? launch_one<EPI_SWIGLU, A_FP8>(m1, p1, st)
+                      : gather ? launch_one<EPI_SWIGLU, A_GATHER>(m1, p1, st)
+                               : launch_one<EPI_SWIGLU, A_TMA>(m1, p1, st);
     if (err != cudaSuccess) return err;
 
     // GEMM2: y_perm = h W_d^T per expert; y_shared = h_shared Ws_d^T (k split per shared expert)
@@ -591,6 +701,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     else
         m2.a_s = m2.a_r, m2.b0_s = m2.b0_r;
     m2.b1_r = m2.b0_r;
+    m2.a_q = m2.a_r;
     m2.b1_s = m2.b0_s;
     ok = ok && tensor_map_2d_bf16(&m2.o_r, a.y_perm, rows_r, a.d, 32, 32, 0);
     if (has_shared)
@@ -600,6 +711,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     if (!ok) return cudaErrorInvalidValue;
     Params p2 = p1;
     p2.perm_token = nullptr;
+    p2.x_scale = nullptr;
     p2.n_out_r = a.d;
     p2.n_out_s = a.d;
     p2.k_r = a.d_ff;
@@ -607,7 +719,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p2.kseg_s = a.d_ff_shared;
     p2.out_r = static_cast<__nv_bfloat16 *>(a.y_perm);
     p2.out_s = static_cast<__nv_bfloat16 *>(a.y_shared);
-    return launch_one<EPI_STORE, false>(m2, p2, st);
+    return launch_one<EPI_STORE, A_TMA>(m2, p2, st);
 }
 
 cudaError_t launch_bounded_wait_selftest(int64_t timeout_ns, int32_t *status, cudaStream_t st) {

@@ -21,6 +21,9 @@ bool tensor_map_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_
 bool tensor_map_3d_bf16(CUtensorMap *m, const void *base, uint64_t n_mat, uint64_t rows,
                         uint64_t cols, uint32_t box_cols, uint32_t box_rows,
                         uint32_t swizzle_bytes = 128);
+// byte tiles (FP8 payload), row-major box without swizzle
+bool tensor_map_2d_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                      uint32_t box_cols, uint32_t box_rows);
 
 // route.cu
 cudaError_t launch_route_select(const float *scores, const float *bias, int T, int E, int G,
@@ -40,6 +43,11 @@ cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d
                             int32_t *send_tok, int32_t *perm_token, int32_t *inv_perm,
                             void *x_perm, const DispatchWs &ws, int32_t *status, cudaStream_t st);
 
+// dispatch.cu, FP8 payload: x_perm_q[row] = E4M3(x[token] / s) and x_scale[row][b] = s
+// (one scale per 128 channels, s = amax / 448); d % 128 == 0
+cudaError_t launch_gather_fp8(const void *x, const int32_t *inv_perm, int T, int d, int K,
+                              uint8_t *x_perm_q, float *x_scale, cudaStream_t st);
+
 // combine.cu
 cudaError_t launch_combine(const void *y_perm, const int32_t *inv_perm, const float *topk_w,
                            const void *y_shared, int T, int d, int K, int64_t n_rows, void *out,
@@ -48,8 +56,10 @@ cudaError_t launch_combine(const void *y_perm, const int32_t *inv_perm, const fl
 // gemm_sm100.cu
 struct FfnArgs {
     int T, d, E, K, d_ff, n_shared, d_ff_shared;
-    const void *x_perm;        // [T*K, d] bf16, or unused when perm_token is set
+    const void *x_perm;        // [T*K, d] bf16, or unused when perm_token / x_perm_q is set
     const int32_t *perm_token; // [T*K] or nullptr: routed row r of GEMM1 is x[perm_token[r]]
+    const uint8_t *x_perm_q;   // [T*K, d] FP8 E4M3 payload or nullptr (with x_scale)
+    const float *x_scale;      // [T*K, d/128]
     const int32_t *offsets;
     const void *w_gate, *w_up, *w_down;
     void *h;        // [T*K, d_ff] bf16 scratch

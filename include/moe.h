@@ -71,7 +71,14 @@ typedef enum moe_router {
     MOE_ROUTER_HASH = 2           /* experts from a hash of the token id       */
 } moe_router;
 
-/* Layer sizes and router.  A zero-initialised `router` is the sigmoid. */
+/* Element type of the dispatched (routed) copies of x (moe_config.payload). */
+typedef enum moe_payload {
+    MOE_PAYLOAD_BF16 = 0, /* x_perm in bf16; the default                       */
+    MOE_PAYLOAD_FP8 = 1   /* FP8 E4M3 codes + one fp32 scale per 128 channels   */
+} moe_payload;
+
+/* Layer sizes, router and payload.  Zero-initialised `router` and `payload`
+ * are the sigmoid router and the bf16 payload. */
 typedef struct moe_config {
     int32_t T;           /* tokens in the batch                               */
     int32_t d;           /* hidden size                                       */
@@ -83,6 +90,7 @@ typedef struct moe_config {
     int32_t n_shared;    /* always-on shared experts (0 allowed)              */
     int32_t d_ff_shared; /* shared expert intermediate size                   */
     int32_t router;      /* moe_router; other values: UNSUPPORTED_SHAPE       */
+    int32_t payload;     /* moe_payload; FP8 needs d % 128 == 0               */
 } moe_config;
 
 typedef enum moe_status {
@@ -229,6 +237,39 @@ MOE_API moe_status moe_dispatch_noalloc(const moe_config *cfg, const void *x,
                                         int32_t *device_status, void *stream);
 
 /*
+ * FP8 dispatch payload ("sending fewer bytes through lower-precision
+ * activations", "DeepSeek 8.7 - communication", section 4; the format is the
+ * library's reading, DeepSeek-V3's recipe): the dispatch of moe_dispatch, but
+ * the permuted copies of x are written as OCP FP8 E4M3 codes with one fp32
+ * scale per token and 128-channel block:
+ *   s = amax / 448 over the block (fp32),  q = E4M3(x / s) (fp32 division,
+ *   nearest-even, saturating to +-448);  an all-zero block has s = 0, q = 0.
+ *   x_perm_q  [T*K, d]      uint8 out (codes)
+ *   x_scale   [T*K, d/128]  fp32 out
+ *   other arguments as moe_dispatch.  Needs d % 128 == 0 (else
+ *   MOE_ERR_UNSUPPORTED_SHAPE); half the bytes of a bf16 x_perm plus 1/64.
+ */
+MOE_API moe_status moe_dispatch_fp8(const moe_config *cfg, const void *x, const int32_t *topk_idx,
+                                    int32_t *counts, int32_t *offsets, int32_t *send,
+                                    int32_t *send_tok, int32_t *perm_token, int32_t *inv_perm,
+                                    uint8_t *x_perm_q, float *x_scale, void *ws, size_t ws_bytes,
+                                    void *stream);
+
+/*
+ * Expert FFN on the FP8 payload: as moe_expert_ffn, with the routed rows given
+ * as x_perm_q / x_scale (moe_dispatch_fp8).  The gate/up GEMM widens each row
+ * to x_hat = bf16(float(E4M3^-1(q)) * s) (one fp32 multiply, bf16 nearest-even)
+ * in shared memory before the tensor cores read it, so the results equal
+ * moe_expert_ffn on x_perm = x_hat bit for bit.  The shared experts read x.
+ */
+MOE_API moe_status moe_expert_ffn_fp8(const moe_config *cfg, const uint8_t *x_perm_q,
+                                      const float *x_scale, const int32_t *offsets,
+                                      const void *w_gate, const void *w_up, const void *w_down,
+                                      void *y_perm, const void *x, const void *ws_gate,
+                                      const void *ws_up, const void *ws_down, void *y_shared,
+                                      void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Expert FFN: grouped SwiGLU over the expert segments plus the shared experts.
  *   x_perm    [T*K, d]             bf16 expert-contiguous rows
  *   offsets   [E+1]                int32 segment starts (offsets[E] == T*K)
@@ -285,7 +326,9 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const 
  *   kept in the workspace).  Intermediates live in the workspace.
  *   The dispatch writes x_perm into the workspace and the expert FFN reads it
  *   (moe_expert_ffn); moe_expert_ffn_gather gives the same bits without
- *   x_perm but runs slower.
+ *   x_perm but runs slower.  With cfg->payload == MOE_PAYLOAD_FP8 the copies
+ *   travel as FP8 (moe_dispatch_fp8 + moe_expert_ffn_fp8); the router and the
+ *   shared experts still read x.
  *   The route is cfg->router's: moe_route's for SIGMOID and SQRT_SOFTPLUS
  *   (router_w required, token_ids ignored), moe_route_hash's for HASH
  *   (token_ids [T] int64 or NULL; router_w, logit_offset, bias ignored).

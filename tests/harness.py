@@ -65,12 +65,13 @@ def expert_mats_host(inp: dict, experts, E: int):
 
 
 def oracle_layer_sample(orc, sh: synth.MoeShape, inp: dict, rows, router: int = 0,
-                        token_ids=None):
+                        token_ids=None, payload: int = 0):
     """Oracle layer output for the token rows `rows` of device inputs `inp`.
 
     Only the x rows and the experts those tokens choose (by the oracle's own
     routing) are copied to the host.  `router`: 0 sigmoid, 1 sqrt(softplus),
-    2 hash keyed by `token_ids` (host int64 [T] or None for the row index).
+    2 hash keyed by `token_ids` (host int64 [T] or None for the row index);
+    `payload` 1 feeds the routed experts the FP8 round trip of x.
     """
     rows = np.asarray(rows, dtype=np.int64)
     x_h = inp["x"].cpu()
@@ -89,7 +90,7 @@ def oracle_layer_sample(orc, sh: synth.MoeShape, inp: dict, rows, router: int = 
     Su = inp["ws_up"].cpu() if ns else torch.zeros(1, 64, sh.d, dtype=torch.bfloat16)
     Sd = inp["ws_down"].cpu() if ns else torch.zeros(1, sh.d, 64, dtype=torch.bfloat16)
     return orc.layer_rows(rows, sh, x_h, e_h, b_h, g, u, d, Sg, Su, Sd, logit_offset=off_h,
-                          router=router, token_ids=token_ids)
+                          router=router, token_ids=token_ids, payload=payload)
 
 
 def near_tie_certified(sh: synth.MoeShape, s_orc: np.ndarray, bias: np.ndarray,

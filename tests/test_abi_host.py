@@ -139,6 +139,29 @@ def test_fused_gather_validates_before_cuda(moe):
     assert lib.moe_expert_ffn_gather(C.byref(cfg), *bad, P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_fp8_payload_validates_before_cuda(moe):
+    tiny = synth.config("tiny")
+    assert moe.moe_check_config(moe.MoeConfig.of(tiny, payload=1)) == moe.MOE_OK
+    assert moe.moe_check_config(moe.MoeConfig.of(tiny, payload=2)) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert moe.moe_check_config(moe.MoeConfig.of(tiny.replace(d=192), payload=1)) == \
+        moe.MOE_ERR_UNSUPPORTED_SHAPE
+    lib, fake, P = moe._lib, 1 << 20, C.c_void_p
+    odd = moe.MoeConfig.of(tiny.replace(d=192))          # bf16 payload: fine, but no FP8 entry
+    ws_n = moe.moe_workspace_size(odd)
+    args = [P(fake)] * 10
+    assert lib.moe_dispatch_fp8(C.byref(odd), *args, P(fake), ws_n, None) == \
+        moe.MOE_ERR_UNSUPPORTED_SHAPE
+    cfg = moe.MoeConfig.of(tiny)
+    ws_n = moe.moe_workspace_size(cfg)
+    bad = list(args)
+    bad[9] = None                                         # x_scale
+    assert lib.moe_dispatch_fp8(C.byref(cfg), *bad, P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
+    fargs = [P(fake)] * 12
+    fargs[1] = P(fake + 4)                                # misaligned scales
+    assert lib.moe_expert_ffn_fp8(C.byref(cfg), *fargs, P(fake), ws_n, None) == \
+        moe.MOE_ERR_INVALID_ARG
+
+
 def test_router_variants_validate_before_cuda(moe):
     sh = synth.config("tiny")
     assert moe.moe_check_config(moe.MoeConfig.of(sh, router=3)) == moe.MOE_ERR_UNSUPPORTED_SHAPE

@@ -1,0 +1,173 @@
+"""Parity of the FP8 dispatch payload (moe_dispatch_fp8, moe_expert_ffn_fp8,
+moe_forward with payload = FP8) against the oracle.
+
+Bars: the codes and scales bit-exact (the quantization is integer work once
+the fp32 division is fixed); the FP8 expert FFN bit-identical to the bf16
+expert FFN run on the widened rows x_hat = bf16(decode(q) * s); the layer
+within the output bars of the oracle's FP8-payload layer.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import combine_expert_ffn_b200 as moe
+else:  # collected on CPU-only machines, skipped by the marker filter
+    moe = None
+
+DEV = "cuda"
+FP8 = 1
+FP8_RAGGED = synth.MoeShape("fp8_ragged", T=264, d=384, E=12, G=4, K=4, M=2, d_ff=192,
+                            n_shared=1, d_ff_shared=128, x_sigma=1.0, e_sigma=384 ** -0.5,
+                            bias_sigma=0.1, seed=8)
+
+
+@pytest.fixture(autouse=True)
+def _free_gpu():
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def _shape(name):
+    return FP8_RAGGED if name == "fp8_ragged" else H.shape(name)
+
+
+def _i32(*s):
+    return torch.empty(*s, dtype=torch.int32, device=DEV)
+
+
+def _route_and_dispatch_fp8(sh, inp, ws):
+    cfg = moe.MoeConfig.of(sh, payload=FP8)
+    idx, w = _i32(sh.T, sh.K), torch.empty(sh.T, sh.K, dtype=torch.float32, device=DEV)
+    moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"], idx, w,
+                  ws=ws)
+    n = sh.T * sh.K
+    o = {"counts": _i32(sh.E), "offsets": _i32(sh.E + 1), "send": _i32(sh.G, sh.G),
+         "send_tok": _i32(sh.G, sh.G), "perm": _i32(n), "inv": _i32(sh.T, sh.K),
+         "q": torch.empty(n, sh.d, dtype=torch.uint8, device=DEV),
+         "s": torch.empty(n, sh.d // 128, dtype=torch.float32, device=DEV), "idx": idx, "w": w}
+    moe.moe_dispatch_fp8(cfg, inp["x"], idx, o["counts"], o["offsets"], o["send"], o["send_tok"],
+                         o["perm"], o["inv"], o["q"], o["s"], ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    return cfg, o
+
+
+def _widen(q, s):
+    """x_hat = bf16(float(E4M3^-1(q)) * s) with torch's own float8 type."""
+    return (q.view(torch.float8_e4m3fn).float() * s.repeat_interleave(128, dim=1)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("name,n_sample", [("tiny", None), ("fp8_ragged", None), ("noshared", None),
+                                           ("mid", 96), ("v3", 24)])
+def test_dispatch_fp8_codes_and_scales_bit_exact(orc, name, n_sample):
+    sh = _shape(name)
+    inp = synth.make_inputs(sh, DEV, weights=False)
+    ws = moe.alloc_workspace(moe.MoeConfig.of(sh, payload=FP8))
+    cfg, o = _route_and_dispatch_fp8(sh, inp, ws)
+    n = sh.T * sh.K
+    rows = np.arange(n) if n_sample is None else np.unique(np.linspace(0, n - 1, n_sample).astype(np.int64))
+    perm = o["perm"].cpu().numpy()
+    xr = inp["x"][torch.as_tensor(perm[rows], device=DEV)].cpu()
+    ref_q, ref_s = orc.fp8_quantize(xr)
+    np.testing.assert_array_equal(o["q"].cpu().numpy()[rows], ref_q)
+    np.testing.assert_array_equal(o["s"].cpu().numpy()[rows].view(np.uint32), ref_s.view(np.uint32))
+    # the plan is the bf16 dispatch's
+    ref = orc.dispatch(o["idx"].cpu().numpy(), sh.E, sh.G)
+    np.testing.assert_array_equal(perm, ref["perm_token"])
+    np.testing.assert_array_equal(o["counts"].cpu().numpy(), ref["counts"])
+
+
+def test_dispatch_fp8_zero_blocks_and_wide_range(orc):
+    """Blocks of zeros, blocks with one huge value among tiny ones (subnormal codes)."""
+    sh = FP8_RAGGED.replace(T=64)
+    inp = synth.make_inputs(sh, DEV, weights=False)
+    x = inp["x"].float()
+    x[3] = 0
+    x[5, :128] = 0
+    x[7, 128:256] *= 1e-4
+    x[7, 130] = 300.0
+    x[9, 256:] = -1e-30
+    inp["x"] = x.to(torch.bfloat16)
+    ws = moe.alloc_workspace(moe.MoeConfig.of(sh, payload=FP8))
+    cfg, o = _route_and_dispatch_fp8(sh, inp, ws)
+    perm = o["perm"].cpu().numpy()
+    ref_q, ref_s = orc.fp8_quantize(inp["x"][torch.as_tensor(perm, device=DEV)].cpu())
+    np.testing.assert_array_equal(o["q"].cpu().numpy(), ref_q)
+    np.testing.assert_array_equal(o["s"].cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+    assert (ref_s == 0).any() and ((ref_q & 0x78) == 0).sum() > 0   # zero scales and subnormal codes
+
+
+@pytest.mark.parametrize("name", ["tiny", "fp8_ragged", "noshared", "mid", "v3"])
+def test_expert_ffn_fp8_equals_bf16_ffn_on_widened_rows(orc, name):
+    sh = _shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    ws = moe.alloc_workspace(moe.MoeConfig.of(sh, payload=FP8))
+    cfg, o = _route_and_dispatch_fp8(sh, inp, ws)
+    n = sh.T * sh.K
+    ns = sh.n_shared
+    y8 = torch.full((n, sh.d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ys8 = torch.full((sh.T, sh.d), float("nan"), dtype=torch.bfloat16, device=DEV) if ns else None
+    moe.moe_expert_ffn_fp8(cfg, o["q"], o["s"], o["offsets"], inp["w_gate"], inp["w_up"],
+                           inp["w_down"], y8, inp["x"], inp.get("ws_gate"), inp.get("ws_up"),
+                           inp.get("ws_down"), ys8, ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    x_hat = _widen(o["q"], o["s"])
+    y16 = torch.full_like(y8, float("nan"))
+    ys16 = torch.full_like(ys8, float("nan")) if ns else None
+    moe.moe_expert_ffn(cfg, x_hat, o["offsets"], inp["w_gate"], inp["w_up"], inp["w_down"], y16,
+                       inp["x"] if ns else None, inp.get("ws_gate"), inp.get("ws_up"),
+                       inp.get("ws_down"), ys16, ws)
+    assert torch.equal(y8.view(torch.int16), y16.view(torch.int16))
+    if ns:
+        assert torch.equal(ys8.view(torch.int16), ys16.view(torch.int16))
+    # the widening itself against the oracle on a few rows
+    rows = np.unique(np.linspace(0, n - 1, 16).astype(np.int64))
+    ref = orc.fp8_dequantize(o["q"].cpu().numpy()[rows], o["s"].cpu().numpy()[rows])
+    got = x_hat.cpu()[torch.as_tensor(rows)].view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("name,n_sample", [("fp8_ragged", None), ("noshared", None), ("v3", 6)])
+def test_forward_fp8_payload_matches_oracle(orc, name, n_sample):
+    sh = _shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    cfg = moe.MoeConfig.of(sh, payload=FP8)
+    ws = moe.alloc_workspace(cfg)
+    o = moe.forward_outputs(cfg)
+    moe.moe_forward(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                    inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                    inp.get("ws_up"), inp.get("ws_down"), o["out"], o["topk_idx"], o["topk_w"],
+                    o["counts"], o["offsets"], o["send"], o["send_tok"], ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    rows = np.arange(sh.T) if n_sample is None else \
+        np.unique(np.linspace(0, sh.T - 1, n_sample).astype(np.int64))
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows, payload=FP8)
+    gi = o["topk_idx"].cpu().numpy()[rows]
+    keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
+    for r in set(range(len(rows))) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    assert len(keep) >= len(rows) - max(1, len(rows) // 100)
+    frob, elem = H.compare_out(o["out"][torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+    # against the bf16-payload layer the difference is the price of the compression
+    cfg16 = moe.MoeConfig.of(sh)
+    o16 = moe.forward_outputs(cfg16)
+    moe.moe_forward(cfg16, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                    inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                    inp.get("ws_up"), inp.get("ws_down"), o16["out"], ws=ws)
+    a, b = o["out"].float(), o16["out"].float()
+    rel = float((a - b).norm() / b.norm())
+    assert 1e-3 < rel < 0.1, rel
+
+
+def test_fp8_payload_needs_d_multiple_of_128():
+    sh = H.RAGGED  # d = 320
+    assert moe.moe_check_config(moe.MoeConfig.of(sh, payload=FP8)) == moe.MOE_ERR_UNSUPPORTED_SHAPE
