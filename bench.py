@@ -8,8 +8,9 @@ combine) over one batch of seeded synthetic tokens of the named workload,
 inputs resident in HBM.  The stages are issued as the four ABI calls that
 moe_forward makes, with CUDA events between them on the launching stream, so
 the timed region also yields each stage's device time.  `e2e` times the
-public moe_forward call on pinned HOST buffers with the host->device copy of
-x and the device->host copy of the output inside the timed region.
+public moe_forward call on pinned HOST buffers with every step's host->device
+copy of x and device->host copy of the output inside the timed region, the
+copies of neighbouring steps overlapping the compute as in a serving loop.
 
 Multi-GPU: the layer does not shard (one GPU per layer instance), so N > 1
 runs N independent replicas, one per rank, each on its own batch; the job's
@@ -323,37 +324,57 @@ def run_ours(args, sh, world, rank, local):
 
 
 def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world):
-    """moe_forward on pinned host buffers: H2D of x and D2H of out inside the timed region."""
+    """moe_forward on pinned host buffers, every step's H2D of x and D2H of out
+    inside the timed region.  Steps are pipelined the way a serving loop runs
+    them: x of step i+1 goes up on a copy stream and out of step i-1 comes
+    down on another while step i computes (two device buffers each; events
+    order every reuse)."""
     import combine_expert_ffn_b200 as moe
     T, d = sh.T, sh.d
+    NB = 2
     x_host = inp["x"].cpu().pin_memory()
-    out_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
-    out_dev = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    out_host = [torch.empty(T, d, dtype=torch.bfloat16).pin_memory() for _ in range(NB)]
+    x_dev = [torch.empty_like(inp["x"]) for _ in range(NB)]
+    out_dev = [torch.empty(T, d, dtype=torch.bfloat16, device=dev) for _ in range(NB)]
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    up_done = [torch.cuda.Event() for _ in range(NB)]
+    fwd_done = [torch.cuda.Event() for _ in range(NB)]
+    down_done = [torch.cuda.Event() for _ in range(NB)]
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.moe_forward(cfg, x_dev, inp["router_w"], inp.get("logit_offset"), inp["bias"],
-                        inp["w_gate"], inp["w_up"], inp["w_down"], inp["ws_gate"], inp["ws_up"],
-                        inp["ws_down"], out_dev, ws=ws, stream=stream)
-        out_host.copy_(out_dev, non_blocking=True)
+    def run(n):
+        for i in range(n):
+            b = i % NB
+            if i >= NB:
+                s_up.wait_event(fwd_done[b])       # step i-NB has read x_dev[b]
+            with torch.cuda.stream(s_up):
+                x_dev[b].copy_(x_host, non_blocking=True)
+            up_done[b].record(s_up)
+            stream.wait_event(up_done[b])
+            if i >= NB:
+                stream.wait_event(down_done[b])    # step i-NB's out_dev[b] is on the host
+            moe.moe_forward(cfg, x_dev[b], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                            inp["w_gate"], inp["w_up"], inp["w_down"], inp["ws_gate"],
+                            inp["ws_up"], inp["ws_down"], out_dev[b], ws=ws, stream=stream)
+            fwd_done[b].record(stream)
+            s_down.wait_event(fwd_done[b])
+            with torch.cuda.stream(s_down):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+            down_done[b].record(s_down)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    run(args.warmup)
     barrier(world)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_up)
+    run(args.steps)
+    e1.record(s_down)                              # after the last step's D2H
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = job_tokens_per_s(T, world, args.steps, e2e_ms)
-    if not torch.equal(out_host, o["out"].cpu()) and world == 1:
+    if not torch.equal(out_host[(args.steps - 1) % NB], o["out"].cpu()) and world == 1:
         raise RuntimeError("moe_forward and the staged calls disagree")
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
-            "d2h_bytes_per_step": T * d * 2}
+            "d2h_bytes_per_step": T * d * 2, "pipelined": "H2D, forward and D2H of consecutive steps on three streams"}
 
 
 def variants_leg(sh, inp, dev, stream, reps=20):
@@ -496,8 +517,11 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
                      "traffic": traffic},
         "stages": {
             "ms": stage_ms,
-            "route": {"bound": "alu", "achieved": route_tflops, "unit": "TFLOP/s (fp32 FMA)",
-                      "peak": fp32_peak, "frac": route_tflops / fp32_peak},
+            "route": {"bound": "tensor", "achieved": route_tflops, "unit": "TFLOP/s",
+                      "peak": peaks["bf16_tflops"], "frac": route_tflops / peaks["bf16_tflops"],
+                      "note": "algorithmic 2*E*d per token; the kernel issues 3 bf16 MMAs per "
+                              "product (fp32 weights split into exact bf16 parts); "
+                              "fp32 CUDA-core peak at the sampled clock: %.1f TFLOP/s" % fp32_peak},
             "dispatch": {"bound": "hbm", "achieved": disp_gbs, "unit": "GB/s", "peak": hbm,
                          "frac": disp_gbs / hbm},
             "combine": {"bound": "hbm", "achieved": comb_gbs, "unit": "GB/s", "peak": hbm,
