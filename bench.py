@@ -66,6 +66,8 @@ def algorithmic(sh):
         "route_flop": 2.0 * E * d,
         # dispatch: read x once, write K copies (bf16) + 3 int32 index words per copy
         "dispatch_bytes": 2.0 * d * (1 + K) + 4.0 * 3 * K,
+        # its gather-permute part: read x once, read K row indices, write K copies
+        "permute_bytes": 2.0 * d * (1 + K) + 4.0 * K,
         # expert FFN: 6 d d_ff per token-expert (gate, up, down), routed + shared
         "ffn_flop": 6.0 * d * (ff * K + shared_ff),
         # combine: read K y rows + y_shared + K (idx, w), write out
@@ -260,18 +262,23 @@ def run_ours(args, sh, world, rank, local):
                       o["topk_idx"], o["topk_w"], scores, ws, stream)
         if ev is not None:
             ev[1].record(stream)
+        # the dispatch as its two parts: the plan (counting sort of the copies), then
+        # the gather-permute of the x rows (together: moe_dispatch with x_perm)
         moe.moe_dispatch(cfg, inp["x"], o["topk_idx"], o["counts"], o["offsets"], o["send"],
-                         o["send_tok"], perm_token, inv_perm, x_perm, ws, stream)
+                         o["send_tok"], perm_token, inv_perm, None, ws, stream)
         if ev is not None:
             ev[2].record(stream)
+        moe.moe_permute(cfg, inp["x"], inv_perm, x_perm, stream)
+        if ev is not None:
+            ev[3].record(stream)
         moe.moe_expert_ffn(cfg, x_perm, o["offsets"], inp["w_gate"], inp["w_up"], inp["w_down"],
                            y_perm, inp["x"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], y_sh,
                            ws, stream)
         if ev is not None:
-            ev[3].record(stream)
+            ev[4].record(stream)
         moe.moe_combine(cfg, y_perm, inv_perm, o["topk_w"], y_sh, o["out"], stream)
         if ev is not None:
-            ev[4].record(stream)
+            ev[5].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -279,7 +286,7 @@ def run_ours(args, sh, world, rank, local):
     if moe.moe_read_device_status(ws) != moe.MOE_OK:
         raise RuntimeError("device status after warm-up: %d" % moe.moe_read_device_status(ws))
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize(dev)
@@ -297,11 +304,12 @@ def run_ours(args, sh, world, rank, local):
     clk = clocks.stop()
     barrier(world)
     ms_total = max_over_ranks(start.elapsed_time(end), world)
-    stage_ms = {k: 0.0 for k in ("route", "dispatch", "expert_ffn", "combine")}
+    stage_ms = {k: 0.0 for k in ("route", "dispatch_plan", "permute", "expert_ffn", "combine")}
     for ev in evs:
         for j, k in enumerate(stage_ms):
             stage_ms[k] += ev[j].elapsed_time(ev[j + 1])
     stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
+    stage_ms["dispatch"] = stage_ms["dispatch_plan"] + stage_ms["permute"]
     status = moe.moe_read_device_status(ws)
     if status != moe.MOE_OK:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -311,6 +319,14 @@ def run_ours(args, sh, world, rank, local):
     if rank != 0:
         return 0
     line = report(args, sh, world, ms_total, stage_ms, launches, clk, e2e)
+    # the routing of the timed batch: expert loads and the group-to-group send matrices
+    counts = o["counts"].cpu()
+    line["routing"] = {
+        "max_over_mean_expert_load": float(counts.max()) / (T * K / E),
+        "min_over_mean_expert_load": float(counts.min()) / (T * K / E),
+        "send": o["send"].cpu().tolist(),
+        "send_tok": o["send_tok"].cpu().tolist(),
+    }
     if not args.no_variants:
         line["variants"] = variants_leg(sh, inp, dev, stream)
     if world == 1 and not args.no_cpu_baseline:
@@ -498,6 +514,7 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
     route_tflops = alg["route_flop"] * T / (stage_ms["route"] / 1e3) / 1e12
     fp32_peak = FP32_LANES * clock_for_alu * 1e6 / 1e12
     disp_gbs = alg["dispatch_bytes"] * T / (stage_ms["dispatch"] / 1e3) / 1e9
+    perm_gbs = alg["permute_bytes"] * T / (stage_ms["permute"] / 1e3) / 1e9
     comb_gbs = alg["combine_bytes"] * T / (stage_ms["combine"] / 1e3) / 1e9
     traffic = traffic_from_profile(sh)
 
@@ -523,7 +540,9 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
                               "product (fp32 weights split into exact bf16 parts); "
                               "fp32 CUDA-core peak at the sampled clock: %.1f TFLOP/s" % fp32_peak},
             "dispatch": {"bound": "hbm", "achieved": disp_gbs, "unit": "GB/s", "peak": hbm,
-                         "frac": disp_gbs / hbm},
+                         "frac": disp_gbs / hbm, "note": "plan + permute"},
+            "permute": {"bound": "hbm", "achieved": perm_gbs, "unit": "GB/s", "peak": hbm,
+                        "frac": perm_gbs / hbm},
             "combine": {"bound": "hbm", "achieved": comb_gbs, "unit": "GB/s", "peak": hbm,
                         "frac": comb_gbs / hbm},
         },

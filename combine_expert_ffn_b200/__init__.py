@@ -35,7 +35,7 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_bounded_wait", "moe_dispatch_noalloc", "moe_route_hash",
            "moe_bias_update", "moe_expert_ffn_gather", "moe_dispatch_fp8",
-           "moe_expert_ffn_fp8")
+           "moe_expert_ffn_fp8", "moe_permute")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
 MOE_PAYLOAD_BF16, MOE_PAYLOAD_FP8 = 0, 1
@@ -86,6 +86,7 @@ _sig = {
     "moe_forward": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                               _P, _P, _P, _P, _P, _S, _P]),
     "moe_route_hash": (C.c_int, [_CP, _P, _P, _P, _P]),
+    "moe_permute": (C.c_int, [_CP, _P, _P, _P, _P]),
     "moe_dispatch_fp8": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_expert_ffn_fp8": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
                                      _P]),
@@ -216,6 +217,11 @@ def moe_expert_ffn_gather(cfg, x, perm_token, offsets, w_gate, w_up, w_down, y_p
                                    _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y_perm),
                                    _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_shared), wp,
                                    wn, _stream(stream)))
+
+
+def moe_permute(cfg, x, inv_perm, x_perm, stream=None) -> None:
+    _ok("moe_permute", _lib.moe_permute(_cfg(cfg), _ptr(x), _ptr(inv_perm), _ptr(x_perm),
+                                        _stream(stream)))
 
 
 def moe_dispatch_fp8(cfg, x, topk_idx, counts, offsets, send, send_tok, perm_token, inv_perm,

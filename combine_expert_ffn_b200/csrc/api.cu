@@ -230,6 +230,16 @@ moe_status moe_dispatch(const moe_config *c, const void *x, const int32_t *topk_
                                        at<int32_t>(ws, L.status), as_stream(stream)));
 }
 
+moe_status moe_permute(const moe_config *c, const void *x, const int32_t *inv_perm, void *x_perm,
+                       void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->T > 0 && (!x || !inv_perm || !x_perm)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_permute(x, inv_perm, c->T, c->d, c->K, x_perm, as_stream(stream)));
+}
+
 moe_status moe_dispatch_fp8(const moe_config *c, const void *x, const int32_t *topk_idx,
                             int32_t *counts, int32_t *offsets, int32_t *send, int32_t *send_tok,
                             int32_t *perm_token, int32_t *inv_perm, uint8_t *x_perm_q,

@@ -283,6 +283,23 @@ cudaError_t launch_gather_fp8(const void *x, const int32_t *inv_perm, int T, int
     return cudaGetLastError();
 }
 
+cudaError_t launch_permute(const void *x, const int32_t *inv_perm, int T, int d, int K,
+                           void *x_perm, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    const int64_t total = (int64_t)T * chunks;
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (total + 255) / 256;
+    const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+    dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4 *>(x), inv_perm, T, chunks,
+                                                 K, (int64_t)T * K, static_cast<uint4 *>(x_perm));
+    count_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d, int E, int G,
                             int K, int32_t *counts, int32_t *offsets, int32_t *send,
                             int32_t *send_tok, int32_t *perm_token, int32_t *inv_perm,
@@ -320,21 +337,7 @@ cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d
                                                              offsets, perm_token, inv_perm);
     count_launch();
     if ((err = cudaGetLastError())) return err;
-    if (x_perm) {
-        const int chunks = d / 8;
-        const int64_t total = (int64_t)T * chunks;
-        int sms = 148;
-        int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int64_t want = (total + 255) / 256;
-        const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
-        dispatch_gather_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4 *>(x), inv_perm, T,
-                                                     chunks, K, (int64_t)T * K,
-                                                     static_cast<uint4 *>(x_perm));
-        count_launch();
-        if ((err = cudaGetLastError())) return err;
-    }
+    if (x_perm) return launch_permute(x, inv_perm, T, d, K, x_perm, st);
     return cudaSuccess;
 }
 

@@ -43,6 +43,9 @@ cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d
                             int32_t *send_tok, int32_t *perm_token, int32_t *inv_perm,
                             void *x_perm, const DispatchWs &ws, int32_t *status, cudaStream_t st);
 
+// dispatch.cu: the gather-permute alone, x_perm[inv_perm[t][j]] = x[t]
+cudaError_t launch_permute(const void *x, const int32_t *inv_perm, int T, int d, int K,
+                           void *x_perm, cudaStream_t st);
 // dispatch.cu, FP8 payload: x_perm_q[row] = E4M3(x[token] / s) and x_scale[row][b] = s
 // (one scale per 128 channels, s = amax / 448); d % 128 == 0
 cudaError_t launch_gather_fp8(const void *x, const int32_t *inv_perm, int T, int d, int K,

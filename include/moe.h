@@ -206,6 +206,19 @@ MOE_API moe_status moe_dispatch(const moe_config *cfg, const void *x, const int3
                         void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The gather-permute step of moe_dispatch alone: x_perm[inv_perm[t][j]] = x[t]
+ * for every copy (t, j), 16-byte vector copies reading each x row once.
+ *   x         [T, d]     bf16
+ *   inv_perm  [T, K]     int32 from moe_dispatch (rows outside [0, T*K) are
+ *                        skipped)
+ *   x_perm    [T*K, d]   bf16 out
+ * moe_dispatch(x_perm = NULL) followed by moe_permute equals moe_dispatch
+ * with x_perm, bit for bit.
+ */
+MOE_API moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *inv_perm,
+                               void *x_perm, void *stream);
+
+/*
  * moe_dispatch for callers that cannot allocate device memory.  No passage of
  * the pages has a counterpart: this entry point exists for deployment only.
  * Callers such as a serving runtime that owns the whole HBM budget through

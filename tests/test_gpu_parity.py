@@ -165,6 +165,21 @@ def test_dispatch_bit_exact(orc, name, zipf):
     assert torch.equal(x_perm.view(torch.int16), x.view(torch.int16)[pt])
 
 
+@pytest.mark.parametrize("name", ["ragged", "v3"])
+def test_permute_alone_equals_dispatch_gather(name):
+    """moe_dispatch(x_perm=NULL) + moe_permute == moe_dispatch(x_perm), bit for bit."""
+    sh = H.shape(name)
+    topk = synth.random_routing(sh.seed, sh.T, sh.E, sh.K, 0.0, DEV)
+    x = synth.normal(sh.seed, synth.TENSOR_IDS["x"], (sh.T, sh.d), 1.0, torch.bfloat16, DEV)
+    out, x_perm, status = _dispatch_gpu(sh, x, topk)
+    assert status == moe.MOE_OK
+    out2, none, status = _dispatch_gpu(sh, x, topk, with_x=False)
+    assert status == moe.MOE_OK and none is None
+    x_perm2 = torch.zeros_like(x_perm)
+    moe.moe_permute(moe.MoeConfig.of(sh), x, out2["inv_perm"], x_perm2)
+    assert torch.equal(x_perm.view(torch.int16), x_perm2.view(torch.int16))
+
+
 def test_dispatch_edge_cases(orc):
     # all tokens to the same K experts (one group), T not a multiple of 256
     sh = H.RAGGED.replace(T=300, G=4)
