@@ -318,9 +318,10 @@ def run_ours(args, sh, world, rank, local):
     e2e = e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world) if not args.no_e2e else None
     if rank != 0:
         return 0
-    line = report(args, sh, world, ms_total, stage_ms, launches, clk, e2e)
-    # the routing of the timed batch: expert loads and the group-to-group send matrices
     counts = o["counts"].cpu()
+    line = report(args, sh, world, ms_total, stage_ms, launches, clk, e2e,
+                  touched_experts=int((counts > 0).sum()))
+    # the routing of the timed batch: expert loads and the group-to-group send matrices
     line["routing"] = {
         "max_over_mean_expert_load": float(counts.max()) / (T * K / E),
         "min_over_mean_expert_load": float(counts.min()) / (T * K / E),
@@ -500,7 +501,7 @@ def variants_leg(sh, inp, dev, stream, reps=20):
     return out
 
 
-def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
+def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e, touched_experts=None):
     T = sh.T
     ms_step = ms_total / args.steps
     value = job_tokens_per_s(T, world, args.steps, ms_total)
@@ -517,6 +518,13 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
     perm_gbs = alg["permute_bytes"] * T / (stage_ms["permute"] / 1e3) / 1e9
     comb_gbs = alg["combine_bytes"] * T / (stage_ms["combine"] / 1e3) / 1e9
     traffic = traffic_from_profile(sh)
+    # expert weights the step reads: every routed expert that got a row, plus the shared ones
+    touched = sh.E if touched_experts is None else touched_experts
+    w_bytes = 2.0 * 3 * sh.d * (touched * sh.d_ff + sh.n_shared * sh.d_ff_shared)
+    w_gbs = w_bytes / ffn_s / 1e9
+    # below the ridge (FLOPs per weight byte < tensor peak / HBM bandwidth) the expert FFN is
+    # bound by streaming its weights, and that is the roofline reported
+    weight_bound = alg["ffn_flop"] * T / w_bytes < tensor_peak * 1e12 / (hbm * 1e9)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -526,12 +534,21 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e):
         "config": {"workload": sh.name, **sh.as_dict(), "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
                          % ((3 * sh.E * sh.d * sh.d_ff + 3 * sh.n_shared * sh.d * sh.d_ff_shared) * 2 / 1e9)},
-        "roofline": {"bound": "tensor", "kernel": "expert FFN: grouped_ffn_gemm_kernel<SwiGLU> + <store> (2 launches)",
-                     "achieved": ffn_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
-                     "frac": ffn_tflops / tensor_peak,
-                     "peak_kind": f"{peaks['source']} bf16 sustained (burst {peaks['bf16_tflops']})",
-                     "frac_of_burst": ffn_tflops / peaks["bf16_tflops"],
-                     "traffic": traffic},
+        "roofline": ({"bound": "tensor", "kernel": "expert FFN: grouped_ffn_gemm_kernel<SwiGLU> + <store> (2 launches)",
+                      "achieved": ffn_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+                      "frac": ffn_tflops / tensor_peak,
+                      "peak_kind": f"{peaks['source']} bf16 sustained (burst {peaks['bf16_tflops']})",
+                      "frac_of_burst": ffn_tflops / peaks["bf16_tflops"],
+                      "traffic": traffic}
+                     if not weight_bound else
+                     {"bound": "hbm", "kernel": "expert FFN: grouped_ffn_gemm_kernel<SwiGLU> + <store> (2 launches)",
+                      "achieved": w_gbs, "peak": hbm, "unit": "GB/s", "frac": w_gbs / hbm,
+                      "peak_kind": f"{peaks['source']} HBM copy",
+                      "basis": "bytes of the expert weights touched (%d of %d routed experts + shared) per launch pair"
+                               % (touched, sh.E),
+                      "tensor_tflops": ffn_tflops, "traffic": traffic}),
+        "expert_weights": {"touched_experts": touched, "bytes": w_bytes, "achieved_gbs": w_gbs,
+                           "frac_of_hbm": w_gbs / hbm},
         "stages": {
             "ms": stage_ms,
             "route": {"bound": "tensor", "achieved": route_tflops, "unit": "TFLOP/s",
