@@ -22,7 +22,7 @@ constexpr int64_t kWaitTimeoutNs = 2000000000LL;  // 2 s per device wait
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-    size_t status, scores, e_split, hist_t, base_t, send_part, sendtok_part;
+    size_t status, scores, e_split, router_part, hist_t, base_t, send_part, sendtok_part;
     size_t topk_idx, topk_w, counts, offsets, send, send_tok, perm_token, inv_perm;
     size_t x_perm, h, y_perm, h_sh, y_sh;
     size_t total;
@@ -41,6 +41,10 @@ Layout layout(const moe_config &c) {
     L.status = take(256);
     L.scores = take(4 * T * E);
     L.e_split = take(2 * 3 * E * (size_t)c.d);
+    // router partial logits: splits * T * E <= splits * tiles * 128 * 128 <= 148 * 128 * 128
+    // floats (router_splits keeps splits * tiles <= 148), reserved whole so that the
+    // workspace stays monotone in T
+    L.router_part = take(c.T > 0 ? 4 * (size_t)148 * 128 * 128 : 0);
     L.hist_t = take(4 * E * nblk);
     L.base_t = take(4 * E * nblk);
     L.send_part = take(4 * nblk * G * G);
@@ -184,8 +188,8 @@ moe_status moe_route(const moe_config *c, const void *x, const float *router_w,
     if ((st = check_device())) return st;
     cudaStream_t s = as_stream(stream);
     if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, c->router,
-                                at<void>(ws, L.e_split), scores, at<int32_t>(ws, L.status),
-                                kWaitTimeoutNs, s))
+                                at<void>(ws, L.e_split), at<float>(ws, L.router_part), scores,
+                                at<int32_t>(ws, L.status), kWaitTimeoutNs, s))
         return MOE_ERR_CUDA;
     return cuda_status(
         launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s));
@@ -421,7 +425,8 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
             return MOE_ERR_CUDA;
     } else {
         if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, c->router,
-                                    at<void>(ws, L.e_split), scores, status, kWaitTimeoutNs, s))
+                                    at<void>(ws, L.e_split), at<float>(ws, L.router_part), scores,
+                                    status, kWaitTimeoutNs, s))
             return MOE_ERR_CUDA;
         if (launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
             return MOE_ERR_CUDA;

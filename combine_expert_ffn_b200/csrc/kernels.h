@@ -78,9 +78,20 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st);
 // router_tc.cu: router affinities on the tensor cores; e (fp32 [E, d]) is
 // split into three bf16 parts in e_split ([3, E, d] bf16 scratch);
 // scores = f(x.e + off), f = sigmoid (affinity 0) or sqrt(softplus) (1).
+// Work is split over d into router_splits(T, E, d) ranges when the batch has
+// too few 128 x 128 tiles to fill the SMs; partial ([splits, T, E] fp32
+// scratch, needed when splits > 1) holds their logits.
+inline int router_splits(int T, int E, int d) {
+    const int tiles = ((T + 127) / 128) * ((E + 127) / 128);
+    const int kmax = d / 64 / 4;  // at least four k blocks per range
+    int s = tiles > 0 ? 148 / tiles : 1;
+    if (s > kmax) s = kmax;
+    return s < 1 ? 1 : s;
+}
 cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *off, int T, int d,
-                                    int E, int affinity, void *e_split, float *scores,
-                                    int32_t *status, int64_t timeout_ns, cudaStream_t st);
+                                    int E, int affinity, void *e_split, float *partial,
+                                    float *scores, int32_t *status, int64_t timeout_ns,
+                                    cudaStream_t st);
 
 // route_variants.cu: the hash router (token ids -> K experts in M groups,
 // gates 1/K; token_ids NULL = row index) and the per-expert bias update.

@@ -1,7 +1,7 @@
-// route.cu -- node-limited top-K selection (the affinities s_i = sigmoid(x .
-// e_i + o_i) come from the tensor-core router GEMM in gemm_sm100.cu; top-k
-// gating over expert affinities, "MoE + Expert-Parallel Overlap (Exp08)",
-// Implemented; the sigmoid form is DeepSeek-V3's).
+// route.cu -- node-limited top-K selection (the affinities s_i = f(x . e_i +
+// o_i) come from the tensor-core router in router_tc.cu; top-k gating over
+// expert affinities, "MoE + Expert-Parallel Overlap (Exp08)", Implemented; f is
+// DeepSeek-V3's sigmoid or the V4 sqrt(softplus)).
 // Selection: b_i = s_i + bias_i chooses, s_i weights; experts lie in at most M
 // of the G contiguous groups ("moe-node-limited-routing", opening definition);
 // a group scores the sum of its top-(K/M) b; ties go to the lower index.

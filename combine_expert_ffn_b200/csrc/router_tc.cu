@@ -15,6 +15,11 @@
 // partial sum into IEEE fp32 registers.  Affinities then agree with the
 // double-precision definition to a few 1e-7 at V3 scale.
 //
+// Small batches leave most SMs idle (a decode batch of 128 tokens and 256
+// experts is 2 tiles), so the reduction over d is split into `splits` ranges
+// of k blocks (router_splits): each work item writes its partial logits, and
+// router_finish_kernel adds them in split order and applies the affinity.
+//
 // Persistent kernel, one CTA per SM, tile = 128 tokens x 128 experts:
 //   warp 0      TMA: x tile (128 x 64) + the three weight parts (3 x 128 x 64)
 //               per stage, 3 stages of 64 KB
@@ -46,6 +51,8 @@ struct Maps {
 struct Params {
     int T, E, d;
     int affinity;  // 0: sigmoid, 1: sqrt(softplus)
+    int splits;    // k ranges per tile; > 1: partial logits go to `partial`
+    float *partial;  // [splits, T, E] fp32 (splits > 1)
     const float *off;
     float *scores;
     int32_t *status;
@@ -113,8 +120,9 @@ router_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
     const uint32_t tmem_base = tmem_base_s;
 
     const int mt = (p.T + BM - 1) / BM, nt = (p.E + BN - 1) / BN;
-    const int total = mt * nt;
+    const int total = mt * nt * p.splits;     // work items: (tile, split), split fastest
     const int kblocks = p.d / BK;
+    const int kper = (kblocks + p.splits - 1) / p.splits;
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
@@ -123,8 +131,10 @@ router_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
             uint32_t phase = 0, n_issued = 0;
             bool ok = true;
             for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-                const int m0 = (idx / nt) * BM, n0 = (idx % nt) * BN;
-                for (int kb = 0; kb < kblocks; ++kb) {
+                const int tile = idx / p.splits, sp = idx - tile * p.splits;
+                const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
+                const int kb1 = min(kblocks, (sp + 1) * kper);
+                for (int kb = sp * kper; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
                                            p.status, p.timeout_ns)) {
                         ok = false;
@@ -155,7 +165,9 @@ router_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
             constexpr uint32_t idesc = idesc_bf16_f32<BM, BN>();
             bool ok = true;
             for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-                for (int kb = 0; kb < kblocks; ++kb) {
+                const int sp = idx % p.splits;
+                const int kb1 = min(kblocks, (sp + 1) * kper);
+                for (int kb = sp * kper; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&cempty_bar[buf]), bphase ^ 1u, abort_flag,
                                            p.status, p.timeout_ns) ||
                         !mbar_wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.status,
@@ -195,11 +207,13 @@ router_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
         uint32_t bphase = 0;
         bool ok = true;
         for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-            const int m0 = (idx / nt) * BM, n0 = (idx % nt) * BN;
+            const int tile = idx / p.splits, sp = idx - tile * p.splits;
+            const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
+            const int kb1 = min(kblocks, (sp + 1) * kper);
             float acc[BN];
 #pragma unroll
             for (int c = 0; c < BN; ++c) acc[c] = 0.f;
-            for (int kb = 0; kb < kblocks; ++kb) {
+            for (int kb = sp * kper; kb < kb1; ++kb) {
                 if (!mbar_wait_bounded(smem_u32(&cfull_bar[buf]), bphase, abort_flag, p.status,
                                        p.timeout_ns)) {
                     ok = false;
@@ -221,7 +235,12 @@ router_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
             }
             if (!ok) break;
             const int t = m0 + row;
-            if (t < p.T) {
+            if (t < p.T && p.splits > 1) {  // partial logits of this k range
+                float *out = p.partial + ((size_t)sp * p.T + t) * p.E;
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (n0 + c < p.E) out[n0 + c] = acc[c];
+            } else if (t < p.T) {
                 float *out = p.scores + (size_t)t * p.E;
 #pragma unroll
                 for (int c = 0; c < BN; ++c) {
@@ -261,11 +280,26 @@ __global__ void router_split_kernel(const float *__restrict__ e, int64_t n,
     }
 }
 
+// scores[t][e] = f(sum over splits, in split order, of partial[s][t][e] + off[e])
+__global__ void router_finish_kernel(const float *__restrict__ partial, int splits, int T, int E,
+                                     const float *__restrict__ off, int affinity,
+                                     float *__restrict__ scores) {
+    const int64_t n = (int64_t)T * E;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float L = partial[i];
+        for (int s = 1; s < splits; ++s) L = __fadd_rn(L, partial[(size_t)s * n + i]);
+        if (off) L += off[i % E];
+        scores[i] = affinity == 1 ? sqrt_softplus(L) : 1.0f / (1.0f + expf(-L));
+    }
+}
+
 }  // namespace router
 
 cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *off, int T, int d,
-                                    int E, int affinity, void *e_split, float *scores,
-                                    int32_t *status, int64_t timeout_ns, cudaStream_t st) {
+                                    int E, int affinity, void *e_split, float *partial,
+                                    float *scores, int32_t *status, int64_t timeout_ns,
+                                    cudaStream_t st) {
     using namespace router;
     if (T == 0) return cudaSuccess;
     int dev = 0, sms = 148;
@@ -281,11 +315,18 @@ cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *
     if (!tensor_map_2d_bf16(&m.x, x, T, d, BK, BM) ||
         !tensor_map_3d_bf16(&m.parts, e_split, 3, E, d, BK, BN))
         return cudaErrorInvalidValue;
-    Params p{T, E, d, affinity, off, scores, status, timeout_ns};
+    const int splits = router_splits(T, E, d);
+    if (splits > 1 && !partial) return cudaErrorInvalidValue;
+    Params p{T, E, d, affinity, splits, partial, off, scores, status, timeout_ns};
     err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
     if (err != cudaSuccess) return err;
-    const int tiles = ((T + BM - 1) / BM) * ((E + BN - 1) / BN);
-    router_tc_kernel<<<std::min(tiles, sms), NUM_THREADS, SMEM_DYN, st>>>(m, p);
+    const int items = ((T + BM - 1) / BM) * ((E + BN - 1) / BN) * splits;
+    router_tc_kernel<<<std::min(items, sms), NUM_THREADS, SMEM_DYN, st>>>(m, p);
+    count_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess || splits == 1) return err;
+    const int64_t n_out = (int64_t)T * E;
+    router_finish_kernel<<<(int)std::min<int64_t>((n_out + 255) / 256, (int64_t)sms * 8), 256, 0,
+                           st>>>(partial, splits, T, E, off, affinity, scores);
     count_launch();
     return cudaGetLastError();
 }

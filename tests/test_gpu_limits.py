@@ -112,3 +112,36 @@ def test_forward_degenerate_and_max_layers(orc, sh):
     assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
     if sh.K == sh.E:
         assert (np.sort(gi, axis=1) == np.arange(sh.E)).all()
+
+
+# Router work split over d (small batches): decode has 2 tiles and 28 k ranges;
+# T=640, E=128, d=7040 has 5 tiles and 27 ranges of 5 k blocks, the last five of
+# them empty (their partial logits are zeros).
+SPLIT_ROUTES = [
+    ("decode", None),
+    ("split_empty", _shape("split_empty", T=640, d=7040, E=128, G=8, K=8, M=4, d_ff=64,
+                           n_shared=0, d_ff_shared=0, x_sigma=1.0, e_sigma=7040 ** -0.5)),
+]
+
+
+@pytest.mark.parametrize("name,sh", SPLIT_ROUTES, ids=[n for n, _ in SPLIT_ROUTES])
+@pytest.mark.parametrize("router", [0, 1])
+def test_router_split_over_d(orc, name, sh, router):
+    sh = H.shape(name) if sh is None else sh
+    inp = synth.make_inputs(sh, DEV, weights=False)
+    cfg = moe.MoeConfig.of(sh, router=router)
+    idx = torch.empty(sh.T, sh.K, dtype=torch.int32, device=DEV)
+    w = torch.empty(sh.T, sh.K, dtype=torch.float32, device=DEV)
+    s = torch.empty(sh.T, sh.E, dtype=torch.float32, device=DEV)
+    ws = moe.alloc_workspace(cfg)
+    moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"], idx, w,
+                  scores=s, ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    rows = np.unique(np.linspace(0, sh.T - 1, 48).astype(np.int64))
+    ref = orc.router_scores(inp["x"].cpu(), inp["router_w"].cpu(), H.host(inp.get("logit_offset")),
+                            rows=rows, affinity=router)
+    gs = s.cpu().numpy()
+    assert np.abs(gs[rows] - ref).max() <= H.TOL_AFFINITY
+    sel_idx, sel_w = orc.select(gs, inp["bias"].cpu(), sh.G, sh.K, sh.M)
+    np.testing.assert_array_equal(idx.cpu().numpy(), sel_idx)
+    np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), sel_w.view(np.uint32))
