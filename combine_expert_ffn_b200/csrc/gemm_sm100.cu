@@ -50,6 +50,13 @@ constexpr int NUM_THREADS = 192;
 enum { A_TMA = 0, A_GATHER = 1, A_FP8 = 2 };
 constexpr int GATHER_WARPS = 4;
 constexpr int GATHER_THREADS = GATHER_WARPS * 32;
+// The FP8 variant runs two such groups of converter warps on alternate stages,
+// so that one group's barriers and widening overlap the other's.
+constexpr int CONV_GROUPS = 2;
+template <int AMODE>
+constexpr int extra_threads() {
+    return AMODE == A_FP8 ? CONV_GROUPS * GATHER_THREADS : AMODE == A_GATHER ? GATHER_THREADS : 0;
+}
 constexpr int FP8_STAGE_OFF = A_BYTES / 2;  // FP8 bytes land in the upper half of the A stage
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
@@ -154,12 +161,13 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return g * __frcp_rn(1.0f + __expf(-g)) * u;
 }
 
-__device__ __forceinline__ void converters_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(GATHER_THREADS) : "memory");
+// Named barrier of converter group grp (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void converters_sync(int grp) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "n"(GATHER_THREADS) : "memory");
 }
 
 template <int EPI, int AMODE>
-__global__ void __launch_bounds__(NUM_THREADS + (AMODE != A_TMA ? GATHER_THREADS : 0), 1)
+__global__ void __launch_bounds__(NUM_THREADS + extra_threads<AMODE>(), 1)
 grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     static_assert(AMODE == A_TMA || EPI == EPI_SWIGLU, "only GEMM1 has A-operand variants");
     constexpr bool GATHER = AMODE == A_GATHER;
@@ -172,7 +180,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     __shared__ __align__(8) uint64_t tempty_bar[2];
     __shared__ __align__(8) uint64_t done_bar;
     __shared__ __align__(8) uint64_t qfull_bar[STAGES];  // A_FP8: payload bytes of a stage landed
-    __shared__ int conv_ok_s;
+    __shared__ int conv_ok_s[CONV_GROUPS];
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ int tile_base[MAX_E + 1];
@@ -365,17 +373,20 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         __syncwarp();
     } else if (AMODE == A_FP8 && warp >= NUM_THREADS / 32) {
         // ------------------------------------------------------ FP8 converters
-        // Thread g widens the 8-byte chunk c = g % 8 of the rows g / 8 + 16 j
-        // (j < 8): x_hat = bf16(E4M3^-1(q) * s), s the row's scale of the
-        // 128-channel block, into the 128-byte-swizzled bf16 stage.  The
-        // payload sits in the upper half of that stage, so every converter
-        // reads its bytes before any writes (named barrier).  Thread 0 alone
-        // waits (bounded) for the payload and shares the outcome.
-        const int g = threadIdx.x - NUM_THREADS;
+        // Two groups of four warps take alternate stages.  In its stages,
+        // thread g of a group widens the 8-byte chunk c = g % 8 of the rows
+        // g / 8 + 16 j (j < 8): x_hat = bf16(E4M3^-1(q) * s), s the row's scale
+        // of the 128-channel block, into the 128-byte-swizzled bf16 stage.  The
+        // payload sits in the upper half of that stage, so every converter of
+        // the group reads its bytes before any writes (named barrier).  Thread 0
+        // of the group alone waits (bounded) for the payload and shares the
+        // outcome.
+        const int grp = (warp - NUM_THREADS / 32) / GATHER_WARPS;
+        const int g = threadIdx.x - NUM_THREADS - grp * GATHER_THREADS;
         const int c = g & 7, r0 = g >> 3;
         const int nsb = p.k_r / 128;  // scales per row
         int stage = 0;
-        uint32_t phase = 0;
+        uint32_t phase = 0, n_use = 0;
         bool ok = true;
         for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
             const Tile t = decode_tile<EPI>(idx, tile_base, seg, segc, p, ntr, mt_s, nt_s);
@@ -387,8 +398,12 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                 s_cur[j] = 0.f;
                 s_next[j] = conv && r < t.rows_valid ? p.x_scale[(size_t)(t.row0 + r) * nsb] : 0.f;
             }
-            for (int kb = 0; kb < t.kblocks; ++kb) {
-                if (conv && (kb & 1) == 0) {  // a new 128-channel block: its scales were loaded ahead
+            for (int kb = 0; kb < t.kblocks; ++kb, ++n_use) {
+                if ((int)(n_use % CONV_GROUPS) != grp) {  // the other group's stage
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    continue;
+                }
+                if (conv) {  // this group's stages step one 128-channel block each
                     const int nb = kb / 2 + 1;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -399,11 +414,11 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                     }
                 }
                 if (g == 0)
-                    conv_ok_s = mbar_wait_bounded(smem_u32(&qfull_bar[stage]), phase, abort_flag,
-                                                  p.status, p.timeout_ns);
-                converters_sync();
-                ok = *reinterpret_cast<volatile int *>(&conv_ok_s) != 0;
-                if (!ok) break;  // every converter read the same flag
+                    conv_ok_s[grp] = mbar_wait_bounded(smem_u32(&qfull_bar[stage]), phase,
+                                                       abort_flag, p.status, p.timeout_ns);
+                converters_sync(grp);
+                ok = *reinterpret_cast<volatile int *>(&conv_ok_s[grp]) != 0;
+                if (!ok) break;  // every converter of the group read the same flag
                 uint8_t *st = smem + stage * STAGE_BYTES;
                 uint2 raw[8];
                 if (conv) {
@@ -412,9 +427,9 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                         raw[j] = *reinterpret_cast<const uint2 *>(st + FP8_STAGE_OFF +
                                                                   (r0 + 16 * j) * 64 + c * 8);
                 }
-                // every payload byte is in registers, and every converter has read
-                // the flag before thread 0 may write the next one
-                converters_sync();
+                // every payload byte is in registers, and every converter of the
+                // group has read the flag before thread 0 may write the next one
+                converters_sync(grp);
                 if (conv) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -626,7 +641,7 @@ cudaError_t launch_one(const Maps &maps, const Params &p, cudaStream_t st) {
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
     if (err != cudaSuccess) return err;
     grouped_ffn_gemm_kernel<EPI, AMODE>
-        <<<sm_count(), NUM_THREADS + (AMODE != A_TMA ? GATHER_THREADS : 0), SMEM_DYN, st>>>(maps, p);
+        <<<sm_count(), NUM_THREADS + extra_threads<AMODE>(), SMEM_DYN, st>>>(maps, p);
     count_launch();
     return cudaGetLastError();
 }
