@@ -168,6 +168,33 @@ def test_forward_fp8_payload_matches_oracle(orc, name, n_sample):
     assert 1e-3 < rel < 0.1, rel
 
 
+@pytest.mark.parametrize("router", [1, 2])
+def test_forward_fp8_payload_with_router_variants(orc, router):
+    """The payload and router options combine: sqrt(softplus) or hash routing
+    with the FP8 dispatch payload."""
+    sh = FP8_RAGGED
+    inp = synth.make_inputs(sh, DEV)
+    cfg = moe.MoeConfig.of(sh, router=router, payload=FP8)
+    ws = moe.alloc_workspace(cfg)
+    o = moe.forward_outputs(cfg)
+    ids = synth.token_ids(sh.seed, sh.T, device=DEV)
+    moe.moe_forward(cfg, inp["x"], inp["router_w"], None, inp["bias"], inp["w_gate"],
+                    inp["w_up"], inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"],
+                    o["out"], o["topk_idx"], ws=ws, token_ids=ids)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    rows = np.arange(sh.T)
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows, router=router,
+                                                      token_ids=ids.cpu().numpy(), payload=FP8)
+    gi = o["topk_idx"].cpu().numpy()
+    keep = [r for r in rows if np.array_equal(gi[r], ref_idx[r])]
+    if router == 2:
+        assert len(keep) == len(rows)                          # hash routes are exact
+    for r in set(rows.tolist()) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    frob, elem = H.compare_out(o["out"][torch.as_tensor(keep, device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
 def test_fp8_payload_needs_d_multiple_of_128():
     sh = H.RAGGED  # d = 320
     assert moe.moe_check_config(moe.MoeConfig.of(sh, payload=FP8)) == moe.MOE_ERR_UNSUPPORTED_SHAPE

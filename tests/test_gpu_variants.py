@@ -210,3 +210,31 @@ def test_bias_update_bit_exact_at_and_around_the_mean(orc, E, T, K):
         moe.moe_bias_update(cfg, torch.from_numpy(counts).to(DEV), gamma, b)
         ref = orc.bias_update(counts, T, K, gamma, bias.cpu().numpy())
         np.testing.assert_array_equal(b.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def test_bias_updates_balance_a_skewed_router():
+    """The purpose of the bias update: repeated forward -> counts -> update steps
+    on a router with a strong per-expert preference (Zipf logit offsets) pull the
+    expert loads toward the mean, without any auxiliary loss."""
+    sh = synth.MoeShape("skew_small", T=2048, d=256, E=32, G=4, K=4, M=2, d_ff=64, n_shared=0,
+                        d_ff_shared=0, x_sigma=1.0, e_sigma=256 ** -0.5, bias_sigma=0.0,
+                        zipf_s=1.2, seed=21)
+    inp = synth.make_inputs(sh, DEV)
+    cfg = moe.MoeConfig.of(sh)
+    ws = moe.alloc_workspace(cfg)
+    idx = torch.empty(sh.T, sh.K, dtype=torch.int32, device=DEV)
+    w = torch.empty(sh.T, sh.K, dtype=torch.float32, device=DEV)
+    i32 = lambda *s: torch.empty(*s, dtype=torch.int32, device=DEV)  # noqa: E731
+    counts, offsets, send, send_tok = i32(sh.E), i32(sh.E + 1), i32(sh.G, sh.G), i32(sh.G, sh.G)
+    perm, inv = i32(sh.T * sh.K), i32(sh.T, sh.K)
+    bias = torch.zeros(sh.E, dtype=torch.float32, device=DEV)
+    mean = sh.T * sh.K / sh.E
+    imbalance = []
+    for step in range(60):
+        moe.moe_route(cfg, inp["x"], inp["router_w"], inp["logit_offset"], bias, idx, w, ws=ws)
+        moe.moe_dispatch(cfg, inp["x"], idx, counts, offsets, send, send_tok, perm, inv, None, ws)
+        imbalance.append(float(counts.max()) / mean)
+        moe.moe_bias_update(cfg, counts, 0.02, bias)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    assert imbalance[0] > 3.0                     # the offsets make the first routing lopsided
+    assert min(imbalance[-10:]) < 0.5 * imbalance[0]
