@@ -1,9 +1,7 @@
 // gemm_sm100.cu -- grouped expert FFN on the 5th-generation tensor cores.
 //
 // Per routed expert e with rows R_e = [offsets[e], offsets[e+1]) of x_perm
-// (or, fused with the dispatch gather, rows x[perm_token[r]] copied straight
-// from x by four gatherer warps) and for the shared experts on all T rows
-// of x:
+// and for the shared experts on all T rows of x:
 //   GEMM1:  h = SiLU(X W_g^T) * (X W_u^T)     (SwiGLU fused in the epilogue)
 //   GEMM2:  y = h W_d^T
 // ("shared experts (always active) + fine-grained routed experts", "MoE +
@@ -16,10 +14,14 @@
 //   warp 1      TMEM owner (512 columns = two 128 x 256 fp32 accumulators)
 //               and single-thread tcgen05.mma issuer (M=128, N=256, K=16)
 //   warps 2..5  epilogue: tcgen05.ld -> SwiGLU or plain -> bf16 -> global
+// GEMM1 has two more A-operand variants with extra warps: rows gathered from
+// x (x[perm_token[r]], 4 warps of 16-byte cp.async copies) and the FP8
+// payload widened to bf16 in shared memory (2 groups of 4 converter warps).
 // The accumulator is double-buffered so the epilogue of tile i overlaps the
 // mainloop of tile i+1.  (Token rows on the MMA's M side and weight rows on N:
 // measured on B200, weights-stationary tiles with tokens on N -- 1-CTA or CTA
-// pair -- lost 20-45% to TMA issue throughput despite doing less MMA work.)  Tiles: for every expert, ceil(R_e/128) row tiles x
+// pair -- lost 20-45% to TMA issue throughput despite doing less MMA work.)
+// Tiles: for every expert, ceil(R_e/128) row tiles x
 // the output column tiles; row tiles of one expert are adjacent in the tile
 // order so the expert's weight tiles are read from HBM about once and served
 // from L2 to its other row tiles.  Row tiles may run past the segment end
@@ -46,7 +48,7 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 // Variants of GEMM1's routed A operand: TMA tiles of x_perm; rows gathered
 // from x by four extra warps (16-byte cp.async copies); or the FP8 payload,
-// TMA-loaded as bytes and widened to bf16 in place by four extra warps.
+// TMA-loaded as bytes and widened to bf16 in place by converter warps.
 enum { A_TMA = 0, A_GATHER = 1, A_FP8 = 2 };
 constexpr int GATHER_WARPS = 4;
 constexpr int GATHER_THREADS = GATHER_WARPS * 32;
