@@ -460,6 +460,19 @@ def variants_leg(sh, inp, dev, stream, reps=20):
         res["fp8_payload"] = timed(fp8_payload)
         del xq, xs
     out["dispatch_plus_ffn_ms"] = res
+    # moe_forward replayed from a CUDA graph (launch overheads gone)
+    g = torch.cuda.CUDAGraph()
+    s_cap = torch.cuda.Stream(dev)
+    s_cap.wait_stream(stream)
+    with torch.cuda.stream(s_cap):
+        with torch.cuda.graph(g, stream=s_cap):
+            moe.moe_forward(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                            inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                            inp.get("ws_up"), inp.get("ws_down"), o["out"], ws=ws, stream=s_cap)
+    stream.wait_stream(s_cap)
+    gms = timed(g.replay)
+    out["graph_forward"] = {"forward_ms": gms, "forward_tokens_per_s": T / (gms / 1e3)}
+    del g
     del ws, o, x_perm, y_perm, y_sh
     if sh.d % 128 == 0:
         cfg8 = moe.MoeConfig.of(sh, payload=moe.MOE_PAYLOAD_FP8)
