@@ -55,6 +55,7 @@ def lib():
         _lib.oracle_e4m3_encode.argtypes = [C.c_float]
         _lib.oracle_e4m3_encode.restype = C.c_uint8
         _lib.oracle_fp8_quantize_row.argtypes = [i32, P, P, P]
+        _lib.oracle_ep_plan.argtypes = [i32, i32, P, P, P]
         _lib.oracle_fp8_dequantize_row.argtypes = [i32, P, P, P]
         _lib.oracle_hash_route.argtypes = [i32, P, i32, i32, i32, i32, P, P]
         _lib.oracle_lowbias32.argtypes = [C.c_uint32]
@@ -64,7 +65,7 @@ def lib():
                   "oracle_ffn_row", "oracle_shared_row", "oracle_combine",
                   "oracle_layer_rows", "oracle_router_affinity", "oracle_layer_rows_ex",
                   "oracle_hash_route", "oracle_bias_update", "oracle_fp8_quantize_row",
-                  "oracle_fp8_dequantize_row"):
+                  "oracle_fp8_dequantize_row", "oracle_ep_plan"):
             getattr(_lib, f).restype = C.c_int
     return _lib
 
@@ -208,6 +209,17 @@ def e4m3_decode(code):
 
 def e4m3_encode(v):
     return int(lib().oracle_e4m3_encode(C.c_float(float(v))))
+
+
+def ep_plan(counts_all):
+    """Expert-parallel row placement from counts_all [world, E]: returns
+    (base [world, E], local_offsets [world, E/world + 1]) int32."""
+    c = _np(np.asarray(counts_all, dtype=np.int32), np.int32)
+    world, E = c.shape
+    base = np.empty((world, E), np.int32)
+    loff = np.empty((world, E // world + 1), np.int32)
+    _check(lib().oracle_ep_plan(world, E, _p(c), _p(base), _p(loff)), "oracle_ep_plan")
+    return base, loff
 
 
 def fp8_quantize(x):

@@ -656,3 +656,36 @@ int oracle_fp8_dequantize_row(int d, const uint8_t *q, const float *scale, uint1
     }
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ expert parallelism */
+/* Row placement of the dispatch all-to-all when the experts are split over
+ * `world` ranks in contiguous blocks of El = E / world ("four experts per
+ * GPU", deepnotes "The real cluster, and the mesh DeepSeek actually
+ * disclosed"; the all-to-all of "moe-node-limited-routing", "Why all to all
+ * dominates MoE step time").  Reading of the receive layout at owner o: its
+ * experts in order; inside an expert, the copies of rank 0, then rank 1, ...,
+ * each rank's in its token order.
+ *   counts_all [world, E]: copies of rank r's tokens to expert e
+ *   base [world, E] out:   first row of rank r's copies for e at owner(e)
+ *   local_offsets [world, El + 1] out: segment starts of owner o's experts
+ *                          (last entry: rows o receives)                    */
+int oracle_ep_plan(int world, int E, const int32_t *counts_all, int32_t *base,
+                   int32_t *local_offsets)
+{
+    if (world <= 0 || E <= 0 || E % world || !counts_all || !base || !local_offsets)
+        return ORC_EBADARG;
+    const int El = E / world;
+    for (int o = 0; o < world; ++o) {
+        int64_t row = 0;
+        for (int i = 0; i < El; ++i) {
+            const int e = o * El + i;
+            local_offsets[o * (El + 1) + i] = (int32_t)row;
+            for (int r = 0; r < world; ++r) {
+                base[r * E + e] = (int32_t)row;
+                row += counts_all[r * E + e];
+            }
+        }
+        local_offsets[o * (El + 1) + El] = (int32_t)row;
+    }
+    return ORC_OK;
+}
