@@ -35,7 +35,9 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_bounded_wait", "moe_dispatch_noalloc", "moe_route_hash",
            "moe_bias_update", "moe_expert_ffn_gather", "moe_dispatch_fp8",
-           "moe_expert_ffn_fp8", "moe_permute")
+           "moe_expert_ffn_fp8", "moe_permute", "moe_ep_workspace_size", "moe_ep_plan",
+           "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ipc_get_handle",
+           "moe_ipc_open_handle", "moe_ipc_close_handle")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
 MOE_PAYLOAD_BF16, MOE_PAYLOAD_FP8 = 0, 1
@@ -87,6 +89,15 @@ _sig = {
                               _P, _P, _P, _P, _P, _S, _P]),
     "moe_route_hash": (C.c_int, [_CP, _P, _P, _P, _P]),
     "moe_permute": (C.c_int, [_CP, _P, _P, _P, _P]),
+    "moe_ep_workspace_size": (_S, [_CP, C.c_int32]),
+    "moe_ep_plan": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P, _P]),
+    "moe_ep_dispatch": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_expert_ffn": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P,
+                                    _P, _P, _P, _P, _S, _P]),
+    "moe_ep_combine": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ipc_get_handle": (C.c_int, [_P, _P]),
+    "moe_ipc_open_handle": (C.c_int, [_P, _P]),
+    "moe_ipc_close_handle": (C.c_int, [_P]),
     "moe_dispatch_fp8": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_expert_ffn_fp8": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S,
                                      _P]),
@@ -222,6 +233,60 @@ def moe_expert_ffn_gather(cfg, x, perm_token, offsets, w_gate, w_up, w_down, y_p
 def moe_permute(cfg, x, inv_perm, x_perm, stream=None) -> None:
     _ok("moe_permute", _lib.moe_permute(_cfg(cfg), _ptr(x), _ptr(inv_perm), _ptr(x_perm),
                                         _stream(stream)))
+
+
+# ----------------------------------------------------------------- expert parallelism
+def moe_ep_workspace_size(cfg, world) -> int:
+    return _lib.moe_ep_workspace_size(_cfg(cfg), int(world))
+
+
+def moe_ep_plan(cfg, world, rank, counts_all, base, local_offsets, stream=None) -> None:
+    _ok("moe_ep_plan", _lib.moe_ep_plan(_cfg(cfg), int(world), int(rank), _ptr(counts_all),
+                                        _ptr(base), _ptr(local_offsets), _stream(stream)))
+
+
+def moe_ep_dispatch(cfg, world, x, topk_idx, offsets, inv_perm, base, recv_x_ptrs,
+                    device_status=None, stream=None) -> None:
+    """recv_x_ptrs: device int64 tensor of `world` device pointers."""
+    _ok("moe_ep_dispatch",
+        _lib.moe_ep_dispatch(_cfg(cfg), int(world), _ptr(x), _ptr(topk_idx), _ptr(offsets),
+                             _ptr(inv_perm), _ptr(base), _ptr(recv_x_ptrs), _ptr(device_status),
+                             _stream(stream)))
+
+
+def moe_ep_expert_ffn(cfg, world, rank, recv_x, local_offsets, w_gate, w_up, w_down, recv_y, x,
+                      ws_gate, ws_up, ws_down, y_shared, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_ep_expert_ffn",
+        _lib.moe_ep_expert_ffn(_cfg(cfg), int(world), int(rank), _ptr(recv_x),
+                               _ptr(local_offsets), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                               _ptr(recv_y), _ptr(x), _ptr(ws_gate), _ptr(ws_up),
+                               _ptr(ws_down), _ptr(y_shared), wp, wn, _stream(stream)))
+
+
+def moe_ep_combine(cfg, world, topk_idx, topk_w, offsets, inv_perm, base, recv_y_ptrs, y_shared,
+                   out, device_status=None, stream=None) -> None:
+    _ok("moe_ep_combine",
+        _lib.moe_ep_combine(_cfg(cfg), int(world), _ptr(topk_idx), _ptr(topk_w), _ptr(offsets),
+                            _ptr(inv_perm), _ptr(base), _ptr(recv_y_ptrs), _ptr(y_shared),
+                            _ptr(out), _ptr(device_status), _stream(stream)))
+
+
+def moe_ipc_get_handle(t) -> bytes:
+    h = (C.c_char * 64)()
+    _ok("moe_ipc_get_handle", _lib.moe_ipc_get_handle(_ptr(t), C.cast(h, C.c_void_p)))
+    return bytes(h)
+
+
+def moe_ipc_open_handle(handle: bytes) -> int:
+    buf = (C.c_char * 64).from_buffer_copy(handle)
+    p = C.c_void_p()
+    _ok("moe_ipc_open_handle", _lib.moe_ipc_open_handle(C.cast(buf, C.c_void_p), C.byref(p)))
+    return p.value
+
+
+def moe_ipc_close_handle(ptr: int) -> None:
+    _ok("moe_ipc_close_handle", _lib.moe_ipc_close_handle(C.c_void_p(ptr)))
 
 
 def moe_dispatch_fp8(cfg, x, topk_idx, counts, offsets, send, send_tok, perm_token, inv_perm,

@@ -465,6 +465,135 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
                                       (int64_t)c->T * c->K, out, s));
 }
 
+// ----------------------------------------------------------------- expert parallelism
+namespace {
+bool ep_args_ok(const moe_config *c, int32_t world) {
+    return world >= 1 && world <= 64 && c->E % world == 0;
+}
+moe_config ep_global(const moe_config *c, int32_t world) {
+    moe_config g = *c;
+    g.T = c->T * world;
+    return g;
+}
+}  // namespace
+
+size_t moe_ep_workspace_size(const moe_config *c, int32_t world) {
+    if (moe_check_config(c) != MOE_OK || !ep_args_ok(c, world)) return 0;
+    const moe_config g = ep_global(c, world);
+    return moe_workspace_size(&g);
+}
+
+moe_status moe_ep_plan(const moe_config *c, int32_t world, int32_t rank, const int32_t *counts_all,
+                       int32_t *base, int32_t *local_offsets, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world) || rank < 0 || rank >= world) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!counts_all || !base || !local_offsets) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_ep_plan(counts_all, world, c->E, rank, base, local_offsets,
+                                      as_stream(stream)));
+}
+
+moe_status moe_ep_dispatch(const moe_config *c, int32_t world, const void *x,
+                           const int32_t *topk_idx, const int32_t *offsets, const int32_t *inv_perm,
+                           const int32_t *base, void *const *recv_x, int32_t *device_status,
+                           void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!x || !topk_idx || !offsets || !inv_perm || !base || !recv_x))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t cap = (int64_t)world * c->T * c->K;
+    return cuda_status(launch_ep_dispatch(x, topk_idx, offsets, inv_perm, base, recv_x, cap, c->T,
+                                          c->d, c->E, c->K, world, device_status,
+                                          as_stream(stream)));
+}
+
+moe_status moe_ep_expert_ffn(const moe_config *c, int32_t world, int32_t rank, const void *recv_x,
+                             const int32_t *local_offsets, const void *w_gate, const void *w_up,
+                             const void *w_down, void *recv_y, const void *x, const void *ws_gate,
+                             const void *ws_up, const void *ws_down, void *y_shared, void *ws,
+                             size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world) || rank < 0 || rank >= world) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0) {
+        if (!recv_x || !local_offsets || !w_gate || !w_up || !w_down || !recv_y)
+            return MOE_ERR_INVALID_ARG;
+        if (c->n_shared > 0 && (!x || !ws_gate || !ws_up || !ws_down || !y_shared))
+            return MOE_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {recv_x, w_gate, w_up, w_down, recv_y, x, ws_gate, ws_up, ws_down, y_shared};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const moe_config g = ep_global(c, world);
+    const Layout L = layout(g);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    // the local experts over the received rows: world * T * K rows of capacity
+    // (every copy of every rank could come here), this rank's T tokens for the
+    // shared experts
+    FfnArgs a{};
+    a.T = c->T; a.d = c->d; a.E = c->E / world; a.K = c->K * world; a.d_ff = c->d_ff;
+    a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
+    a.x_perm = recv_x; a.perm_token = nullptr; a.offsets = local_offsets;
+    a.w_gate = w_gate; a.w_up = w_up; a.w_down = w_down;
+    a.h = at<void>(ws, L.h); a.y_perm = recv_y;
+    a.x = x; a.ws_gate = ws_gate; a.ws_up = ws_up; a.ws_down = ws_down;
+    a.h_shared = at<void>(ws, L.h_sh); a.y_shared = y_shared;
+    a.status = at<int32_t>(ws, L.status);
+    a.timeout_ns = kWaitTimeoutNs;
+    return cuda_status(launch_expert_ffn(a, as_stream(stream)));
+}
+
+moe_status moe_ep_combine(const moe_config *c, int32_t world, const int32_t *topk_idx,
+                          const float *topk_w, const int32_t *offsets, const int32_t *inv_perm,
+                          const int32_t *base, const void *const *recv_y, const void *y_shared,
+                          void *out, int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!topk_idx || !topk_w || !offsets || !inv_perm || !base || !recv_y || !out))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_shared) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t cap = (int64_t)world * c->T * c->K;
+    return cuda_status(launch_ep_combine(topk_idx, topk_w, offsets, inv_perm, base, recv_y, cap,
+                                         y_shared, c->T, c->d, c->E, c->K, world, out,
+                                         device_status, as_stream(stream)));
+}
+
+moe_status moe_ipc_get_handle(const void *dev_ptr, void *handle) {
+    if (!dev_ptr || !handle) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_device();
+    if (st) return st;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, const_cast<void *>(dev_ptr)) != cudaSuccess) return MOE_ERR_CUDA;
+    static_assert(sizeof(h) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+    std::memcpy(handle, &h, sizeof(h));
+    return MOE_OK;
+}
+
+moe_status moe_ipc_open_handle(const void *handle, void **dev_ptr) {
+    if (!handle || !dev_ptr) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_device();
+    if (st) return st;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    return cuda_status(cudaIpcOpenMemHandle(dev_ptr, h, cudaIpcMemLazyEnablePeerAccess));
+}
+
+moe_status moe_ipc_close_handle(void *dev_ptr) {
+    if (!dev_ptr) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_device();
+    if (st) return st;
+    return cuda_status(cudaIpcCloseMemHandle(dev_ptr));
+}
+
 moe_status moe_selftest_bounded_wait(int64_t timeout_ns, void *ws, void *stream) {
     if (!ws || timeout_ns < 1000 || timeout_ns > 10000000000LL) return MOE_ERR_INVALID_ARG;
     moe_status st = check_device();

@@ -1,0 +1,197 @@
+// ep.cu -- expert parallelism: the dispatch and combine all-to-alls fused
+// with their gather and reduce, over peer memory.
+//
+// The pages' layout: experts are partitioned over the ranks (contiguous blocks
+// of E / world per rank, "four experts per GPU", deepnotes "The real cluster,
+// and the mesh DeepSeek actually disclosed"), each rank routes its own tokens,
+// and the dispatch all-to-all sends every token copy to the rank owning its
+// expert; the combine all-to-all brings the expert outputs back
+// ("moe-node-limited-routing", "Why all to all dominates MoE step time").
+//
+// Receive layout at owner o: its experts' segments in expert order; inside a
+// segment, the copies from source rank 0, then 1, ... , each source's in its
+// token order.  With the batch split into equal contiguous rank chunks this
+// is exactly the single-GPU x_perm restricted to o's experts, so every row
+// meets the same expert GEMM arithmetic and the layer's output is the same.
+//
+// Per rank, with counts_all[r][e] the copies of rank r to expert e:
+//   base[e]          = first row of this rank's copies for e at owner(e)
+//                    = seg_start(e) + sum_{r < me} counts_all[r][e]
+//   local_offsets[i] = seg_start(me * El + i) at this rank as owner
+// dispatch: x row of copy (t, j) -> recv_x[owner(e)][base[e] + rank of t
+//           among this rank's tokens choosing e]; one load, K peer stores
+// combine:  out[t] = y_shared[t] + sum_j w_j recv_y[owner(e_j)][same row],
+//           fp32 multiply-adds in slot order (as the single-GPU combine)
+// recv_x / recv_y are device arrays of `world` device pointers: this GPU's
+// buffers and peers' buffers mapped into its address space; the kernels use
+// plain loads and stores through them.
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+__global__ void ep_plan_kernel(const int32_t *__restrict__ counts_all, int world, int E, int me,
+                               int32_t *__restrict__ base, int32_t *__restrict__ local_offsets) {
+    // one block; thread e owns expert e (E <= 1024)
+    __shared__ int32_t col[1024];   // sum over ranks of counts_all[.][e]
+    __shared__ int32_t start[1024]; // seg_start(e) within owner(e)'s buffer
+    const int e = threadIdx.x;
+    const int El = E / world;
+    if (e < E) {
+        int s = 0;
+        for (int r = 0; r < world; ++r) s += counts_all[r * E + e];
+        col[e] = s;
+    }
+    __syncthreads();
+    if (e < E) {
+        const int first = (e / El) * El;  // first expert of owner(e)
+        int st = 0;
+        for (int q = first; q < e; ++q) st += col[q];
+        start[e] = st;
+        int b = st;
+        for (int r = 0; r < me; ++r) b += counts_all[r * E + e];
+        base[e] = b;
+    }
+    __syncthreads();
+    if (e <= El) local_offsets[e] = e < El ? start[me * El + e] : start[me * El + El - 1] +
+                                                                  col[me * El + El - 1];
+}
+
+__global__ void __launch_bounds__(256)
+ep_dispatch_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
+                   const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
+                   const int32_t *__restrict__ base, uint4 *const *__restrict__ recv_x,
+                   int64_t recv_rows, int T, int chunks, int E, int K, int El,
+                   int32_t *status) {
+    const int64_t total = (int64_t)T * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        const uint4 v = __ldg(x + i);
+        for (int j = 0; j < K; ++j) {
+            const int e = __ldg(topk_idx + t * K + j);
+            if (e < 0 || e >= E) continue;  // flagged by the local dispatch plan
+            const int64_t row = (int64_t)__ldg(base + e) + __ldg(inv_perm + t * K + j) -
+                                __ldg(offsets + e);
+            if (row < 0 || row >= recv_rows) {
+                if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                continue;
+            }
+            recv_x[e / El][row * chunks + c] = v;
+        }
+    }
+}
+
+__device__ __forceinline__ void ep_acc_row(float (&acc)[8], float wj, const uint4 &v) {
+    acc[0] = fmaf(wj, bf16_lo(v.x), acc[0]); acc[1] = fmaf(wj, bf16_hi(v.x), acc[1]);
+    acc[2] = fmaf(wj, bf16_lo(v.y), acc[2]); acc[3] = fmaf(wj, bf16_hi(v.y), acc[3]);
+    acc[4] = fmaf(wj, bf16_lo(v.z), acc[4]); acc[5] = fmaf(wj, bf16_hi(v.z), acc[5]);
+    acc[6] = fmaf(wj, bf16_lo(v.w), acc[6]); acc[7] = fmaf(wj, bf16_hi(v.w), acc[7]);
+}
+
+__global__ void __launch_bounds__(256)
+ep_combine_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
+                  const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
+                  const int32_t *__restrict__ base, const uint4 *const *__restrict__ recv_y,
+                  int64_t recv_rows, const uint4 *__restrict__ y_shared, int T, int chunks,
+                  int E, int K, int El, uint4 *__restrict__ out, int32_t *status) {
+    const int64_t total = (int64_t)T * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        float acc[8];
+        if (y_shared) {
+            const uint4 v = __ldg(y_shared + i);
+            acc[0] = bf16_lo(v.x); acc[1] = bf16_hi(v.x);
+            acc[2] = bf16_lo(v.y); acc[3] = bf16_hi(v.y);
+            acc[4] = bf16_lo(v.z); acc[5] = bf16_hi(v.z);
+            acc[6] = bf16_lo(v.w); acc[7] = bf16_hi(v.w);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        }
+        // slots in batches of 8: every peer load of a batch is in flight before
+        // its multiply-adds, which run in slot order
+        for (int j0 = 0; j0 < K; j0 += 8) {
+            uint4 rows[8];
+            float w[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int j = j0 + q;
+                rows[q] = make_uint4(0u, 0u, 0u, 0u);
+                w[q] = 0.f;
+                if (j >= K) continue;
+                w[q] = __ldg(topk_w + t * K + j);
+                const int e = __ldg(topk_idx + t * K + j);
+                if (e < 0 || e >= E) continue;
+                const int64_t row = (int64_t)__ldg(base + e) + __ldg(inv_perm + t * K + j) -
+                                    __ldg(offsets + e);
+                if (row < 0 || row >= recv_rows) {
+                    if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                    continue;
+                }
+                rows[q] = recv_y[e / El][row * chunks + c];
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (j0 + q < K) ep_acc_row(acc, w[q], rows[q]);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        out[i] = o;
+    }
+}
+
+int grid_for(int64_t total) {
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (total + 255) / 256;
+    return (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+}
+
+}  // namespace
+
+cudaError_t launch_ep_plan(const int32_t *counts_all, int world, int E, int me, int32_t *base,
+                           int32_t *local_offsets, cudaStream_t st) {
+    ep_plan_kernel<<<1, 1024, 0, st>>>(counts_all, world, E, me, base, local_offsets);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_dispatch(const void *x, const int32_t *topk_idx, const int32_t *offsets,
+                               const int32_t *inv_perm, const int32_t *base, void *const *recv_x,
+                               int64_t recv_rows, int T, int d, int E, int K, int world,
+                               int32_t *status, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_dispatch_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
+        static_cast<const uint4 *>(x), topk_idx, offsets, inv_perm, base,
+        reinterpret_cast<uint4 *const *>(recv_x), recv_rows, T, chunks, E, K, E / world, status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_combine(const int32_t *topk_idx, const float *topk_w, const int32_t *offsets,
+                              const int32_t *inv_perm, const int32_t *base,
+                              const void *const *recv_y, int64_t recv_rows, const void *y_shared,
+                              int T, int d, int E, int K, int world, void *out, int32_t *status,
+                              cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_combine_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
+        topk_idx, topk_w, offsets, inv_perm, base,
+        reinterpret_cast<const uint4 *const *>(recv_y), recv_rows,
+        static_cast<const uint4 *>(y_shared), T, chunks, E, K, E / world,
+        static_cast<uint4 *>(out), status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -51,6 +51,19 @@ cudaError_t launch_permute(const void *x, const int32_t *inv_perm, int T, int d,
 cudaError_t launch_gather_fp8(const void *x, const int32_t *inv_perm, int T, int d, int K,
                               uint8_t *x_perm_q, float *x_scale, cudaStream_t st);
 
+// ep.cu: expert parallelism over `world` ranks (E / world experts each)
+cudaError_t launch_ep_plan(const int32_t *counts_all, int world, int E, int me, int32_t *base,
+                           int32_t *local_offsets, cudaStream_t st);
+cudaError_t launch_ep_dispatch(const void *x, const int32_t *topk_idx, const int32_t *offsets,
+                               const int32_t *inv_perm, const int32_t *base, void *const *recv_x,
+                               int64_t recv_rows, int T, int d, int E, int K, int world,
+                               int32_t *status, cudaStream_t st);
+cudaError_t launch_ep_combine(const int32_t *topk_idx, const float *topk_w, const int32_t *offsets,
+                              const int32_t *inv_perm, const int32_t *base,
+                              const void *const *recv_y, int64_t recv_rows, const void *y_shared,
+                              int T, int d, int E, int K, int world, void *out, int32_t *status,
+                              cudaStream_t st);
+
 // combine.cu
 cudaError_t launch_combine(const void *y_perm, const int32_t *inv_perm, const float *topk_w,
                            const void *y_shared, int T, int d, int K, int64_t n_rows, void *out,

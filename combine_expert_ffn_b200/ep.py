@@ -1,0 +1,190 @@
+"""Expert parallelism over ranks: the host-side steps around the EP entry
+points of libmoe (argument marshalling and the collectives that order them).
+
+A rank owns E / world experts and routes its own tokens.  One step:
+
+    moe_route, moe_dispatch(x_perm=None)     local routing and dispatch plan
+    all-gather of the per-expert counts       counts_all [world, E]
+    moe_ep_plan                               where this rank's copies go
+    moe_ep_dispatch                           gather + peer stores
+    barrier                                   every rank's stores are done
+    moe_ep_expert_ffn                         this rank's experts, shared experts
+    barrier                                   every rank's outputs are done
+    moe_ep_combine                            peer loads + gate-weighted sum
+
+`EPLayer` runs that step in a process group of one process per GPU, with the
+receive buffers mapped into every rank by CUDA IPC and the barriers as
+stream-ordered all-reduces.  `emulate_forward` runs all ranks of one step on a
+single GPU, one after the other (no rank waits on another inside a kernel),
+with the same kernels and plain same-device pointers in the tables.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (MoeConfig, alloc_workspace, moe_dispatch, moe_ep_combine, moe_ep_dispatch,
+               moe_ep_expert_ffn, moe_ep_plan, moe_ep_workspace_size, moe_ipc_close_handle,
+               moe_ipc_get_handle, moe_ipc_open_handle, moe_route, moe_route_hash,
+               MOE_ROUTER_HASH)
+
+
+def _i32(n, device):
+    return torch.empty(n, dtype=torch.int32, device=device)
+
+
+class _RankState:
+    """Per-rank buffers of one EP step."""
+
+    def __init__(self, cfg: MoeConfig, world: int, device):
+        T, K, E, G, d = cfg.T, cfg.K, cfg.E, cfg.G, cfg.d
+        self.cfg = cfg
+        self.topk_idx = torch.empty(T, K, dtype=torch.int32, device=device)
+        self.topk_w = torch.empty(T, K, dtype=torch.float32, device=device)
+        self.counts, self.offsets = _i32(E, device), _i32(E + 1, device)
+        self.send = torch.empty(G, G, dtype=torch.int32, device=device)
+        self.send_tok = torch.empty(G, G, dtype=torch.int32, device=device)
+        self.perm, self.inv = _i32(T * K, device), torch.empty(T, K, dtype=torch.int32, device=device)
+        self.base, self.local_offsets = _i32(E, device), _i32(E // world + 1, device)
+        cap = world * T * K
+        self.recv_x = torch.empty(cap, d, dtype=torch.bfloat16, device=device)
+        self.recv_y = torch.empty(cap, d, dtype=torch.bfloat16, device=device)
+        self.y_shared = torch.empty(T, d, dtype=torch.bfloat16, device=device)
+        self.out = torch.empty(T, d, dtype=torch.bfloat16, device=device)
+        n = moe_ep_workspace_size(cfg, world)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=device)
+        self.ws[:256].zero_()
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def route_and_plan_local(self, x, router_w, logit_offset, bias, token_ids, stream):
+        cfg = self.cfg
+        if cfg.router == MOE_ROUTER_HASH:
+            moe_route_hash(cfg, token_ids, self.topk_idx, self.topk_w, stream)
+        else:
+            moe_route(cfg, x, router_w, logit_offset, bias, self.topk_idx, self.topk_w, None,
+                      self.ws, stream)
+        moe_dispatch(cfg, x, self.topk_idx, self.counts, self.offsets, self.send, self.send_tok,
+                     self.perm, self.inv, None, self.ws, stream)
+
+
+def gather_counts(counts, group=None):
+    """counts_all [world, E]: every rank's per-expert copy counts, in rank order."""
+    import torch.distributed as dist
+    parts = [torch.empty_like(counts) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, counts, group=group)
+    return torch.stack(parts)
+
+
+def _local_weights(w, rank, world):
+    El = w.shape[0] // world
+    return w[rank * El:(rank + 1) * El]
+
+
+def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, stream=None):
+    """All `world` ranks of one EP step on this GPU.  The batch is split into
+    equal contiguous chunks (T % world == 0 and (T / world) % G == 0); returns
+    (out [T, d], per-rank states)."""
+    device = inp["x"].device
+    base_cfg = MoeConfig.of(shape, router=router)
+    T = base_cfg.T
+    if T % world or base_cfg.E % world:
+        raise ValueError("T and E must be multiples of world")
+    Tr = T // world
+    cfg = MoeConfig.of(shape.replace(T=Tr), router=router)
+    ranks = [_RankState(cfg, world, device) for _ in range(world)]
+    x = inp["x"]
+    xs = [x[r * Tr:(r + 1) * Tr] for r in range(world)]
+    ids = [None if token_ids is None else token_ids[r * Tr:(r + 1) * Tr] for r in range(world)]
+    for r, st in enumerate(ranks):
+        st.route_and_plan_local(xs[r], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                                ids[r], stream)
+    counts_all = torch.stack([st.counts for st in ranks])        # the all-gather
+    recv_x_ptrs = torch.tensor([st.recv_x.data_ptr() for st in ranks], dtype=torch.int64,
+                               device=device)
+    recv_y_ptrs = torch.tensor([st.recv_y.data_ptr() for st in ranks], dtype=torch.int64,
+                               device=device)
+    for r, st in enumerate(ranks):
+        moe_ep_plan(cfg, world, r, counts_all, st.base, st.local_offsets, stream)
+    for r, st in enumerate(ranks):
+        moe_ep_dispatch(cfg, world, xs[r], st.topk_idx, st.offsets, st.inv, st.base,
+                        recv_x_ptrs, st.status, stream)
+    for r, st in enumerate(ranks):                                 # (barrier)
+        moe_ep_expert_ffn(cfg, world, r, st.recv_x, st.local_offsets,
+                          _local_weights(inp["w_gate"], r, world),
+                          _local_weights(inp["w_up"], r, world),
+                          _local_weights(inp["w_down"], r, world), st.recv_y, xs[r],
+                          inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"),
+                          st.y_shared if cfg.n_shared else None, st.ws, stream)
+    for r, st in enumerate(ranks):                                 # (barrier)
+        moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,
+                       recv_y_ptrs, st.y_shared if cfg.n_shared else None, st.out, st.status,
+                       stream)
+    return torch.cat([st.out for st in ranks]), ranks
+
+
+class EPLayer:
+    """One rank of an expert-parallel MoE layer in a process group with one
+    process per GPU (NCCL backend).  Holds this rank's experts
+    (w_gate / w_up / w_down [E/world, ...]), the replicated router and shared
+    experts, and the receive buffers, mapped into every rank by CUDA IPC.
+
+    Not run on more than one GPU here: every GPU run of this build had one GPU.
+    """
+
+    def __init__(self, shape_local, group, router_w, bias, w_gate_local, w_up_local,
+                 w_down_local, ws_gate=None, ws_up=None, ws_down=None, logit_offset=None,
+                 router=None):
+        import torch.distributed as dist
+        self.dist = dist
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.device = w_gate_local.device
+        self.cfg = MoeConfig.of(shape_local, router=router)
+        self.st = _RankState(self.cfg, self.world, self.device)
+        self.router_w, self.bias, self.logit_offset = router_w, bias, logit_offset
+        self.w = (w_gate_local, w_up_local, w_down_local)
+        self.ws_shared = (ws_gate, ws_up, ws_down)
+        self._opened = []
+        self.recv_x_ptrs = self._map_peers(self.st.recv_x)
+        self.recv_y_ptrs = self._map_peers(self.st.recv_y)
+        self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
+
+    def _map_peers(self, buf):
+        handles = [None] * self.world
+        self.dist.all_gather_object(handles, moe_ipc_get_handle(buf), group=self.group)
+        ptrs = []
+        for r, h in enumerate(handles):
+            if r == self.rank:
+                ptrs.append(buf.data_ptr())
+            else:
+                p = moe_ipc_open_handle(h)
+                self._opened.append(p)
+                ptrs.append(p)
+        return torch.tensor(ptrs, dtype=torch.int64, device=self.device)
+
+    def _barrier(self):
+        # stream-ordered: completes on every rank only after every rank's
+        # preceding kernels on its stream have completed
+        self.dist.all_reduce(self._flag, group=self.group)
+
+    def forward(self, x, token_ids=None, stream=None):
+        st, cfg, world, r = self.st, self.cfg, self.world, self.rank
+        st.route_and_plan_local(x, self.router_w, self.logit_offset, self.bias, token_ids, stream)
+        counts_all = gather_counts(st.counts, self.group)
+        moe_ep_plan(cfg, world, r, counts_all, st.base, st.local_offsets, stream)
+        self._barrier()                       # every rank's recv_x is free again
+        moe_ep_dispatch(cfg, world, x, st.topk_idx, st.offsets, st.inv, st.base,
+                        self.recv_x_ptrs, st.status, stream)
+        self._barrier()
+        moe_ep_expert_ffn(cfg, world, r, st.recv_x, st.local_offsets, *self.w, st.recv_y, x,
+                          *self.ws_shared, st.y_shared if cfg.n_shared else None, st.ws, stream)
+        self._barrier()
+        moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,
+                       self.recv_y_ptrs, st.y_shared if cfg.n_shared else None, st.out,
+                       st.status, stream)
+        return st.out
+
+    def close(self):
+        for p in self._opened:
+            moe_ipc_close_handle(p)
+        self._opened = []

@@ -355,6 +355,81 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Expert parallelism over `world` ranks, one GPU each (the dispatch and
+ * combine all-to-alls of "moe-node-limited-routing", "Why all to all
+ * dominates MoE step time", and the expert placement of deepnotes "The real
+ * cluster, and the mesh DeepSeek actually disclosed").  Rank r owns experts
+ * [r*E/world, (r+1)*E/world) and routes its own T tokens (cfg is the
+ * per-rank configuration, cfg->T its token count; E % world == 0, world <= 64).
+ * A rank's step: moe_route and moe_dispatch(x_perm = NULL) on its tokens; an
+ * all-gather of the dispatch counts into counts_all [world, E] (the caller's
+ * collective); moe_ep_plan; moe_ep_dispatch; a barrier (every rank's stores
+ * done); moe_ep_expert_ffn; a barrier; moe_ep_combine.
+ * Receive buffers: recv_x and recv_y of every rank hold world * T * K rows of
+ * d bf16 (every copy of every rank could go to one owner).  The kernels reach
+ * the other ranks' buffers through device arrays of `world` device pointers
+ * (this rank's own and peers' buffers mapped with moe_ipc_open_handle), with
+ * plain peer stores (dispatch) and peer loads (combine): the transfer is the
+ * gather / reduce itself, with no staging copy.
+ * Row layout at owner o: its experts in order; inside an expert's segment the
+ * copies of rank 0, then rank 1, ..., each in its token order.  With a batch
+ * split into equal contiguous rank chunks this is the single-GPU x_perm
+ * restricted to o's experts, so the layer equals moe_forward bit for bit.
+ */
+/* Workspace bytes for moe_ep_expert_ffn: moe_workspace_size of the global
+ * batch (cfg with T * world); 0 if unsupported. */
+MOE_API size_t moe_ep_workspace_size(const moe_config *cfg, int32_t world);
+
+/* From counts_all [world, E] int32 (counts_all[r][e] = copies of rank r's
+ * tokens to expert e): base [E] int32 out, the first row of this rank's copies
+ * for expert e in owner(e)'s receive buffer; local_offsets [E/world + 1]
+ * int32 out, the segment starts of this rank's experts in its own receive
+ * buffer (the last entry = rows received). */
+MOE_API moe_status moe_ep_plan(const moe_config *cfg, int32_t world, int32_t rank,
+                               const int32_t *counts_all, int32_t *base, int32_t *local_offsets,
+                               void *stream);
+
+/* Dispatch fused with its all-to-all: x [T, d] bf16, topk_idx [T, K],
+ * offsets [E+1] and inv_perm [T, K] from this rank's moe_dispatch, base from
+ * moe_ep_plan; recv_x: device array of `world` device pointers to the ranks'
+ * receive buffers.  Copy (t, j) of expert e lands in row base[e] + (inv_perm
+ * [t][j] - offsets[e]) of recv_x[e / (E/world)].  Rows outside the buffer are
+ * skipped and flagged MOE_ERR_DEVICE_FAULT in *device_status (may be NULL). */
+MOE_API moe_status moe_ep_dispatch(const moe_config *cfg, int32_t world, const void *x,
+                                   const int32_t *topk_idx, const int32_t *offsets,
+                                   const int32_t *inv_perm, const int32_t *base,
+                                   void *const *recv_x, int32_t *device_status, void *stream);
+
+/* The expert FFN of this rank: its E/world experts (w_gate / w_up
+ * [E/world, d_ff, d], w_down [E/world, d, d_ff]) over recv_x with
+ * local_offsets, into recv_y (same capacity); the shared experts on this
+ * rank's x [T, d] into y_shared [T, d].  ws: moe_ep_workspace_size bytes. */
+MOE_API moe_status moe_ep_expert_ffn(const moe_config *cfg, int32_t world, int32_t rank,
+                                     const void *recv_x, const int32_t *local_offsets,
+                                     const void *w_gate, const void *w_up, const void *w_down,
+                                     void *recv_y, const void *x, const void *ws_gate,
+                                     const void *ws_up, const void *ws_down, void *y_shared,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* Combine fused with its all-to-all: out[t] = y_shared[t] + sum_j topk_w[t][j]
+ * * (row of copy (t, j) in recv_y[owner]), fp32 multiply-adds in slot order,
+ * bf16 out [T, d].  recv_y: device array of `world` device pointers. */
+MOE_API moe_status moe_ep_combine(const moe_config *cfg, int32_t world, const int32_t *topk_idx,
+                                  const float *topk_w, const int32_t *offsets,
+                                  const int32_t *inv_perm, const int32_t *base,
+                                  const void *const *recv_y, const void *y_shared, void *out,
+                                  int32_t *device_status, void *stream);
+
+/* CUDA IPC of a device allocation for the peer pointer tables: the handle is
+ * MOE_IPC_HANDLE_BYTES opaque bytes to send to the other ranks; open maps a
+ * peer's allocation into this GPU's address space (peer access enabled),
+ * close unmaps it. */
+#define MOE_IPC_HANDLE_BYTES 64
+MOE_API moe_status moe_ipc_get_handle(const void *dev_ptr, void *handle);
+MOE_API moe_status moe_ipc_open_handle(const void *handle, void **dev_ptr);
+MOE_API moe_status moe_ipc_close_handle(void *dev_ptr);
+
+/*
  * Self-test of the bounded device waits: launches one kernel that waits on
  * an mbarrier no thread ever arrives on, with a limit of `timeout_ns`
  * nanoseconds (1e3 .. 1e10).  The kernel must give up, record
