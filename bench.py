@@ -330,6 +330,8 @@ def run_ours(args, sh, world, rank, local):
     }
     if not args.no_variants:
         line["variants"] = variants_leg(sh, inp, dev, stream)
+    if args.ep_world > 1:
+        line["expert_parallel"] = ep_leg(sh, inp, dev, stream, args.ep_world)
     if world == 1 and not args.no_cpu_baseline:
         n = args.cpu_tokens
         v, dt = oracle_tokens_per_s(sh, inp, n)
@@ -514,6 +516,98 @@ def variants_leg(sh, inp, dev, stream, reps=20):
     return out
 
 
+# measured peer copy over NVLink 5, one direction per GPU (GB/s)
+NVLINK_GBS = 770.0
+
+
+def ep_leg(sh, inp, dev, stream, world, reps=20):
+    """Expert parallelism over `world` ranks, emulated on this GPU: every rank
+    of the step runs in sequence with same-device pointer tables (peer stores
+    and loads become local HBM traffic).  Reports each stage's device time
+    (every rank's launches of the stage replayed from one CUDA graph) summed
+    over the ranks and per rank, the fused dispatch and combine
+    against the HBM peak, and the bytes of those two exchanges that would
+    cross NVLink on `world` GPUs with their time at the measured peer-copy
+    bandwidth (the larger of a rank's outgoing and incoming bytes).  Not part
+    of the headline step."""
+    import combine_expert_ffn_b200 as moe
+    from combine_expert_ffn_b200 import ep
+    if sh.T % world or sh.E % world or (sh.T // world) % sh.G:
+        return {"world": world, "skipped": "T, E or T/world not divisible"}
+    em = ep.EmulatedEP(sh, inp, world, stream=stream)
+    em.forward()
+    torch.cuda.synchronize(dev)
+    for st in em.ranks:
+        if int(st.status.item()) != moe.MOE_OK or moe.moe_read_device_status(st.ws) != moe.MOE_OK:
+            raise RuntimeError("device status after the emulated EP step")
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    def graphed(stage):
+        # one stage of all ranks captured once and replayed: the host's
+        # per-call overhead would otherwise exceed the short kernels' time
+        g = torch.cuda.CUDAGraph()
+        s_cap = torch.cuda.Stream(dev)
+        s_cap.wait_stream(stream)
+        em.stream = s_cap
+        with torch.cuda.stream(s_cap):
+            with torch.cuda.graph(g, stream=s_cap):
+                getattr(em, stage)()
+        em.stream = stream
+        stream.wait_stream(s_cap)
+        return g
+
+    stages = ("route_and_plan_local", "exchange_counts", "plan", "dispatch", "expert_ffn",
+              "combine")
+    graphs = {k: graphed(k) for k in stages}
+    # the HBM-bound exchange stages first, the expert GEMMs (which pull the SM
+    # clock down to the power cap) last
+    timing_order = ("exchange_counts", "plan", "dispatch", "combine", "route_and_plan_local",
+                    "expert_ffn")
+    t_ms = {k: timed(graphs[k].replay) for k in timing_order}
+    all_ranks = {k: t_ms[k] for k in stages}
+    for st in em.ranks:
+        if int(st.status.item()) != moe.MOE_OK or moe.moe_read_device_status(st.ws) != moe.MOE_OK:
+            raise RuntimeError("device status after the emulated EP stages")
+    del graphs
+    Tr, d, K, E = sh.T // world, sh.d, sh.K, sh.E
+    El = E // world
+    hbm = load_peaks()["hbm_gbs"]
+    disp_bytes = (2.0 * d * (1 + K) + 8.0 * K) * Tr      # x row, K copies, idx + inv
+    comb_bytes = (2.0 * d * (K + 1 + (1 if sh.n_shared else 0)) + 12.0 * K) * Tr
+    per_rank = {k: v / world for k, v in all_ranks.items()}
+    ca = em.counts_all.cpu().to(torch.int64)
+    owner = torch.arange(E) // El
+    out_copies = [int(ca[r][owner != r].sum()) for r in range(world)]
+    in_copies = [int(ca[:, owner == o].sum() - ca[o, owner == o].sum()) for o in range(world)]
+    link_bytes = 2.0 * d * max(max(out_copies), max(in_copies))
+    res = {
+        "world": world, "tokens_per_rank": Tr,
+        "stage_ms_all_ranks": all_ranks, "stage_ms_per_rank": per_rank,
+        "dispatch": {"bytes_per_rank": disp_bytes,
+                     "achieved_gbs": disp_bytes / (per_rank["dispatch"] / 1e3) / 1e9,
+                     "frac_of_hbm": disp_bytes / (per_rank["dispatch"] / 1e3) / 1e9 / hbm},
+        "combine": {"bytes_per_rank": comb_bytes,
+                    "achieved_gbs": comb_bytes / (per_rank["combine"] / 1e3) / 1e9,
+                    "frac_of_hbm": comb_bytes / (per_rank["combine"] / 1e3) / 1e9 / hbm},
+        "nvlink": {"max_rank_bytes_per_exchange": link_bytes,
+                   "projected_ms_per_exchange": link_bytes / (NVLINK_GBS * 1e9) * 1e3,
+                   "bandwidth_gbs": NVLINK_GBS, "copies_out": out_copies, "copies_in": in_copies},
+        "note": "all ranks run in sequence on one GPU; peer traffic is local HBM here",
+    }
+    del em
+    return res
+
+
 def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e, touched_experts=None):
     T = sh.T
     ms_step = ms_total / args.steps
@@ -594,6 +688,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--ep-world", type=int, default=8,
+                    help="ranks of the emulated expert-parallel leg (1 = skip)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the router-variant and bias-update timings")
     args = ap.parse_args()

@@ -24,7 +24,11 @@
 //           fp32 multiply-adds in slot order (as the single-GPU combine)
 // recv_x / recv_y are device arrays of `world` device pointers: this GPU's
 // buffers and peers' buffers mapped into its address space; the kernels use
-// plain loads and stores through them.
+// plain loads and stores through them.  Each block first builds in shared
+// memory, per expert, delta[e] = base[e] - offsets[e] and the address of the
+// row delta[e] in owner(e)'s buffer, so a copy's address is that pointer plus
+// inv_perm[t][j] rows: one global load (beside topk_idx) before the row itself,
+// as in the single-GPU gather and combine.
 #include "kernels.h"
 
 namespace moe {
@@ -58,28 +62,59 @@ __global__ void ep_plan_kernel(const int32_t *__restrict__ counts_all, int world
                                                                   col[me * El + El - 1];
 }
 
-__global__ void __launch_bounds__(256)
+constexpr int EP_MAX_E = 1024;
+
+// delta[e] = base[e] - offsets[e] and the address of row delta[e] of
+// owner(e)'s buffer, for every expert, in shared memory
+template <typename P>
+__device__ __forceinline__ void ep_stage_rows(const int32_t *__restrict__ offsets,
+                                              const int32_t *__restrict__ base,
+                                              P const *__restrict__ table, int E, int El,
+                                              int chunks, int32_t *delta_s, P *rowbase_s) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int32_t dl = base[e] - offsets[e];
+        delta_s[e] = dl;
+        rowbase_s[e] = table[e / El] + (int64_t)dl * chunks;
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(256, 4)
 ep_dispatch_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
                    const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
                    const int32_t *__restrict__ base, uint4 *const *__restrict__ recv_x,
-                   int64_t recv_rows, int T, int chunks, int E, int K, int El,
-                   int32_t *status) {
+                   int64_t recv_rows, int T, int chunks, int E, int K, int El, int32_t *status) {
+    __shared__ int32_t delta_s[EP_MAX_E];
+    __shared__ uint4 *rowbase_s[EP_MAX_E];
+    ep_stage_rows(offsets, base, recv_x, E, El, chunks, delta_s, rowbase_s);
     const int64_t total = (int64_t)T * chunks;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t t = i / chunks;
         const int c = (int)(i - t * chunks);
         const uint4 v = __ldg(x + i);
-        for (int j = 0; j < K; ++j) {
-            const int e = __ldg(topk_idx + t * K + j);
-            if (e < 0 || e >= E) continue;  // flagged by the local dispatch plan
-            const int64_t row = (int64_t)__ldg(base + e) + __ldg(inv_perm + t * K + j) -
-                                __ldg(offsets + e);
-            if (row < 0 || row >= recv_rows) {
-                if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
-                continue;
+        for (int j0 = 0; j0 < K; j0 += 8) {
+            int e8[8], r8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int j = j0 + q;
+                e8[q] = -1;
+                if (j < K) {
+                    e8[q] = __ldg(topk_idx + t * K + j);
+                    r8[q] = __ldg(inv_perm + t * K + j);
+                }
             }
-            recv_x[e / El][row * chunks + c] = v;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = e8[q];
+                if (e < 0 || e >= E) continue;  // flagged by the local dispatch plan
+                const int64_t row = (int64_t)delta_s[e] + r8[q];
+                if (row < 0 || row >= recv_rows) {
+                    if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                    continue;
+                }
+                rowbase_s[e][(int64_t)r8[q] * chunks + c] = v;
+            }
         }
     }
 }
@@ -91,12 +126,15 @@ __device__ __forceinline__ void ep_acc_row(float (&acc)[8], float wj, const uint
     acc[6] = fmaf(wj, bf16_lo(v.w), acc[6]); acc[7] = fmaf(wj, bf16_hi(v.w), acc[7]);
 }
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 ep_combine_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
                   const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
                   const int32_t *__restrict__ base, const uint4 *const *__restrict__ recv_y,
                   int64_t recv_rows, const uint4 *__restrict__ y_shared, int T, int chunks,
                   int E, int K, int El, uint4 *__restrict__ out, int32_t *status) {
+    __shared__ int32_t delta_s[EP_MAX_E];
+    __shared__ const uint4 *rowbase_s[EP_MAX_E];
+    ep_stage_rows(offsets, base, recv_y, E, El, chunks, delta_s, rowbase_s);
     const int64_t total = (int64_t)T * chunks;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -126,14 +164,14 @@ ep_combine_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict_
                 if (j >= K) continue;
                 w[q] = __ldg(topk_w + t * K + j);
                 const int e = __ldg(topk_idx + t * K + j);
+                const int r = __ldg(inv_perm + t * K + j);
                 if (e < 0 || e >= E) continue;
-                const int64_t row = (int64_t)__ldg(base + e) + __ldg(inv_perm + t * K + j) -
-                                    __ldg(offsets + e);
+                const int64_t row = (int64_t)delta_s[e] + r;
                 if (row < 0 || row >= recv_rows) {
                     if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
                     continue;
                 }
-                rows[q] = recv_y[e / El][row * chunks + c];
+                rows[q] = rowbase_s[e][(int64_t)r * chunks + c];
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -148,12 +186,13 @@ ep_combine_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict_
     }
 }
 
+// one wave of resident blocks (4 per SM): each block stages its tables once
 int grid_for(int64_t total) {
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t want = (total + 255) / 256;
-    return (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+    return (int)(want < (int64_t)sms * 4 ? want : (int64_t)sms * 4);
 }
 
 }  // namespace

@@ -22,7 +22,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (MoeConfig, alloc_workspace, moe_dispatch, moe_ep_combine, moe_ep_dispatch,
+from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_dispatch,
                moe_ep_expert_ffn, moe_ep_plan, moe_ep_workspace_size, moe_ipc_close_handle,
                moe_ipc_get_handle, moe_ipc_open_handle, moe_route, moe_route_hash,
                MOE_ROUTER_HASH)
@@ -79,46 +79,85 @@ def _local_weights(w, rank, world):
     return w[rank * El:(rank + 1) * El]
 
 
-def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, stream=None):
+class EmulatedEP:
     """All `world` ranks of one EP step on this GPU.  The batch is split into
-    equal contiguous chunks (T % world == 0 and (T / world) % G == 0); returns
-    (out [T, d], per-rank states)."""
-    device = inp["x"].device
-    base_cfg = MoeConfig.of(shape, router=router)
-    T = base_cfg.T
-    if T % world or base_cfg.E % world:
-        raise ValueError("T and E must be multiples of world")
-    Tr = T // world
-    cfg = MoeConfig.of(shape.replace(T=Tr), router=router)
-    ranks = [_RankState(cfg, world, device) for _ in range(world)]
-    x = inp["x"]
-    xs = [x[r * Tr:(r + 1) * Tr] for r in range(world)]
-    ids = [None if token_ids is None else token_ids[r * Tr:(r + 1) * Tr] for r in range(world)]
-    for r, st in enumerate(ranks):
-        st.route_and_plan_local(xs[r], inp["router_w"], inp.get("logit_offset"), inp["bias"],
-                                ids[r], stream)
-    counts_all = torch.stack([st.counts for st in ranks])        # the all-gather
-    recv_x_ptrs = torch.tensor([st.recv_x.data_ptr() for st in ranks], dtype=torch.int64,
-                               device=device)
-    recv_y_ptrs = torch.tensor([st.recv_y.data_ptr() for st in ranks], dtype=torch.int64,
-                               device=device)
-    for r, st in enumerate(ranks):
-        moe_ep_plan(cfg, world, r, counts_all, st.base, st.local_offsets, stream)
-    for r, st in enumerate(ranks):
-        moe_ep_dispatch(cfg, world, xs[r], st.topk_idx, st.offsets, st.inv, st.base,
-                        recv_x_ptrs, st.status, stream)
-    for r, st in enumerate(ranks):                                 # (barrier)
-        moe_ep_expert_ffn(cfg, world, r, st.recv_x, st.local_offsets,
-                          _local_weights(inp["w_gate"], r, world),
-                          _local_weights(inp["w_up"], r, world),
-                          _local_weights(inp["w_down"], r, world), st.recv_y, xs[r],
-                          inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"),
-                          st.y_shared if cfg.n_shared else None, st.ws, stream)
-    for r, st in enumerate(ranks):                                 # (barrier)
-        moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,
-                       recv_y_ptrs, st.y_shared if cfg.n_shared else None, st.out, st.status,
-                       stream)
-    return torch.cat([st.out for st in ranks]), ranks
+    equal contiguous chunks (T % world == 0 and (T / world) % G == 0).  Each
+    stage method runs that stage for every rank in rank order; a stage starts
+    only after the previous one has run for all ranks, which stands in for the
+    barriers between them."""
+
+    def __init__(self, shape, inp: dict, world: int, router=None, token_ids=None, stream=None):
+        self.device = inp["x"].device
+        base_cfg = MoeConfig.of(shape, router=router)
+        T = base_cfg.T
+        if T % world or base_cfg.E % world:
+            raise ValueError("T and E must be multiples of world")
+        Tr = T // world
+        self.world, self.stream, self.inp = world, stream, inp
+        self.cfg = MoeConfig.of(shape.replace(T=Tr), router=router)
+        self.ranks = [_RankState(self.cfg, world, self.device) for _ in range(world)]
+        self.xs = [inp["x"][r * Tr:(r + 1) * Tr] for r in range(world)]
+        self.ids = [None if token_ids is None else token_ids[r * Tr:(r + 1) * Tr]
+                    for r in range(world)]
+        self.recv_x_ptrs = torch.tensor([st.recv_x.data_ptr() for st in self.ranks],
+                                        dtype=torch.int64, device=self.device)
+        self.recv_y_ptrs = torch.tensor([st.recv_y.data_ptr() for st in self.ranks],
+                                        dtype=torch.int64, device=self.device)
+        self.counts_all = torch.empty(world, self.cfg.E, dtype=torch.int32, device=self.device)
+
+    def route_and_plan_local(self):
+        inp = self.inp
+        for r, st in enumerate(self.ranks):
+            st.route_and_plan_local(self.xs[r], inp["router_w"], inp.get("logit_offset"),
+                                    inp["bias"], self.ids[r], self.stream)
+
+    def exchange_counts(self):
+        # the all-gather: row r of counts_all is rank r's counts
+        with torch.cuda.stream(self.stream or torch.cuda.current_stream(self.device)):
+            for r, st in enumerate(self.ranks):
+                self.counts_all[r].copy_(st.counts)
+
+    def plan(self):
+        for r, st in enumerate(self.ranks):
+            moe_ep_plan(self.cfg, self.world, r, self.counts_all, st.base, st.local_offsets,
+                        self.stream)
+
+    def dispatch(self):
+        for r, st in enumerate(self.ranks):
+            moe_ep_dispatch(self.cfg, self.world, self.xs[r], st.topk_idx, st.offsets, st.inv,
+                            st.base, self.recv_x_ptrs, st.status, self.stream)
+
+    def expert_ffn(self):
+        inp, cfg, world = self.inp, self.cfg, self.world
+        for r, st in enumerate(self.ranks):
+            moe_ep_expert_ffn(cfg, world, r, st.recv_x, st.local_offsets,
+                              _local_weights(inp["w_gate"], r, world),
+                              _local_weights(inp["w_up"], r, world),
+                              _local_weights(inp["w_down"], r, world), st.recv_y, self.xs[r],
+                              inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"),
+                              st.y_shared if cfg.n_shared else None, st.ws, self.stream)
+
+    def combine(self):
+        for st in self.ranks:
+            moe_ep_combine(self.cfg, self.world, st.topk_idx, st.topk_w, st.offsets, st.inv,
+                           st.base, self.recv_y_ptrs, st.y_shared if self.cfg.n_shared else None,
+                           st.out, st.status, self.stream)
+
+    def forward(self):
+        self.route_and_plan_local()
+        self.exchange_counts()
+        self.plan()
+        self.dispatch()
+        self.expert_ffn()
+        self.combine()
+        return torch.cat([st.out for st in self.ranks])
+
+
+def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, stream=None):
+    """One EP step of all `world` ranks on this GPU; returns (out [T, d],
+    per-rank states)."""
+    em = EmulatedEP(shape, inp, world, router, token_ids, stream)
+    return em.forward(), em.ranks
 
 
 class EPLayer:

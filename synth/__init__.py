@@ -96,8 +96,12 @@ CONFIGS = {
 # Reduced workloads for profiler captures: the V3 layer's dimensions and rows
 # per expert (T*K/E = 256) with fewer experts, so that a capture holds a few
 # GB on the device; DRAM traffic per token is that of the full layer.
+# v3_ep: the V3 row width and top-8 over 4096 tokens and 32 narrow experts, for
+# captures of the expert-parallel exchange kernels (2 ranks of 2048 tokens: one
+# combine launch reads 235 MB, above L2) within a few GB.
 PROFILE_CONFIGS = {
     "v3_e32": CONFIGS["v3"].replace(name="v3_e32", T=1024, E=32),
+    "v3_ep": CONFIGS["v3"].replace(name="v3_ep", T=4096, E=32, d_ff=512),
 }
 
 # Fixed tensor ids: salt of the counter-based generator.
