@@ -605,6 +605,31 @@ def ep_leg(sh, inp, dev, stream, world, reps=20):
         "note": "all ranks run in sequence on one GPU; peer traffic is local HBM here",
     }
     del em
+    if sh.d % 128 == 0:
+        # the FP8 payload: E4M3 codes + one fp32 scale per 128 channels travel
+        # instead of bf16 rows; the owners' GEMM widens them
+        torch.cuda.empty_cache()
+        em = ep.EmulatedEP(sh, inp, world, stream=stream, payload=moe.MOE_PAYLOAD_FP8)
+        em.forward()
+        torch.cuda.synchronize(dev)
+        graphs = {k: graphed(k) for k in ("dispatch", "expert_ffn")}
+        t8 = {k: timed(graphs[k].replay) / world for k in ("dispatch", "expert_ffn")}
+        for st in em.ranks:
+            if int(st.status.item()) != moe.MOE_OK or \
+                    moe.moe_read_device_status(st.ws) != moe.MOE_OK:
+                raise RuntimeError("device status after the emulated FP8 EP stages")
+        del graphs
+        q_bytes = (2.0 * d + K * (d + d / 32.0) + 8.0 * K) * Tr   # x read, codes + scales
+        q_link = (d + d / 32.0) * max(max(out_copies), max(in_copies))
+        res["fp8_payload"] = {
+            "stage_ms_per_rank": t8,
+            "dispatch": {"bytes_per_rank": q_bytes,
+                         "achieved_gbs": q_bytes / (t8["dispatch"] / 1e3) / 1e9,
+                         "frac_of_hbm": q_bytes / (t8["dispatch"] / 1e3) / 1e9 / hbm},
+            "nvlink": {"max_rank_bytes_dispatch": q_link,
+                       "projected_ms_dispatch": q_link / (NVLINK_GBS * 1e9) * 1e3},
+        }
+        del em
     return res
 
 

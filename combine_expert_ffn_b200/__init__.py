@@ -36,8 +36,9 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_selftest_bounded_wait", "moe_dispatch_noalloc", "moe_route_hash",
            "moe_bias_update", "moe_expert_ffn_gather", "moe_dispatch_fp8",
            "moe_expert_ffn_fp8", "moe_permute", "moe_ep_workspace_size", "moe_ep_plan",
-           "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ipc_get_handle",
-           "moe_ipc_open_handle", "moe_ipc_close_handle")
+           "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_dispatch_fp8",
+           "moe_ep_expert_ffn_fp8", "moe_ipc_get_handle", "moe_ipc_open_handle",
+           "moe_ipc_close_handle")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
 MOE_PAYLOAD_BF16, MOE_PAYLOAD_FP8 = 0, 1
@@ -95,6 +96,9 @@ _sig = {
     "moe_ep_expert_ffn": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P,
                                     _P, _P, _P, _P, _S, _P]),
     "moe_ep_combine": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_dispatch_fp8": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_expert_ffn_fp8": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P, _P, _P, _P, _P,
+                                        _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_ipc_get_handle": (C.c_int, [_P, _P]),
     "moe_ipc_open_handle": (C.c_int, [_P, _P]),
     "moe_ipc_close_handle": (C.c_int, [_P]),
@@ -262,6 +266,27 @@ def moe_ep_expert_ffn(cfg, world, rank, recv_x, local_offsets, w_gate, w_up, w_d
                                _ptr(local_offsets), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                                _ptr(recv_y), _ptr(x), _ptr(ws_gate), _ptr(ws_up),
                                _ptr(ws_down), _ptr(y_shared), wp, wn, _stream(stream)))
+
+
+def moe_ep_dispatch_fp8(cfg, world, x, topk_idx, offsets, inv_perm, base, recv_q_ptrs,
+                        recv_scale_ptrs, device_status=None, stream=None) -> None:
+    """recv_q_ptrs / recv_scale_ptrs: device int64 tensors of `world` device pointers."""
+    _ok("moe_ep_dispatch_fp8",
+        _lib.moe_ep_dispatch_fp8(_cfg(cfg), int(world), _ptr(x), _ptr(topk_idx), _ptr(offsets),
+                                 _ptr(inv_perm), _ptr(base), _ptr(recv_q_ptrs),
+                                 _ptr(recv_scale_ptrs), _ptr(device_status), _stream(stream)))
+
+
+def moe_ep_expert_ffn_fp8(cfg, world, rank, recv_q, recv_scale, local_offsets, w_gate, w_up,
+                          w_down, recv_y, x, ws_gate, ws_up, ws_down, y_shared, ws,
+                          stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_ep_expert_ffn_fp8",
+        _lib.moe_ep_expert_ffn_fp8(_cfg(cfg), int(world), int(rank), _ptr(recv_q),
+                                   _ptr(recv_scale), _ptr(local_offsets), _ptr(w_gate),
+                                   _ptr(w_up), _ptr(w_down), _ptr(recv_y), _ptr(x),
+                                   _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_shared), wp,
+                                   wn, _stream(stream)))
 
 
 def moe_ep_combine(cfg, world, topk_idx, topk_w, offsets, inv_perm, base, recv_y_ptrs, y_shared,

@@ -511,22 +511,46 @@ moe_status moe_ep_dispatch(const moe_config *c, int32_t world, const void *x,
                                           as_stream(stream)));
 }
 
-moe_status moe_ep_expert_ffn(const moe_config *c, int32_t world, int32_t rank, const void *recv_x,
-                             const int32_t *local_offsets, const void *w_gate, const void *w_up,
-                             const void *w_down, void *recv_y, const void *x, const void *ws_gate,
-                             const void *ws_up, const void *ws_down, void *y_shared, void *ws,
-                             size_t ws_bytes, void *stream) {
+moe_status moe_ep_dispatch_fp8(const moe_config *c, int32_t world, const void *x,
+                               const int32_t *topk_idx, const int32_t *offsets,
+                               const int32_t *inv_perm, const int32_t *base, void *const *recv_q,
+                               void *const *recv_scale, int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world) || c->d % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!x || !topk_idx || !offsets || !inv_perm || !base || !recv_q || !recv_scale))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t cap = (int64_t)world * c->T * c->K;
+    return cuda_status(launch_ep_dispatch_fp8(x, topk_idx, offsets, inv_perm, base, recv_q,
+                                              recv_scale, cap, c->T, c->d, c->E, c->K, world,
+                                              device_status, as_stream(stream)));
+}
+
+namespace {
+// the expert FFN of one rank's experts over its receive buffer: bf16 rows
+// (recv_x) or FP8 codes + scales (recv_q, recv_scale)
+moe_status ep_expert_ffn(const moe_config *c, int32_t world, int32_t rank, bool fp8,
+                         const void *recv_x,
+                         const uint8_t *recv_q, const float *recv_scale,
+                         const int32_t *local_offsets, const void *w_gate, const void *w_up,
+                         const void *w_down, void *recv_y, const void *x, const void *ws_gate,
+                         const void *ws_up, const void *ws_down, void *y_shared, void *ws,
+                         size_t ws_bytes, void *stream) {
     moe_status st = moe_check_config(c);
     if (st) return st;
     if (!ep_args_ok(c, world) || rank < 0 || rank >= world) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (fp8 && c->d % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!ws) return MOE_ERR_INVALID_ARG;
     if (c->T > 0) {
-        if (!recv_x || !local_offsets || !w_gate || !w_up || !w_down || !recv_y)
-            return MOE_ERR_INVALID_ARG;
+        if (fp8 ? (!recv_q || !recv_scale || !x) : !recv_x) return MOE_ERR_INVALID_ARG;
+        if (!local_offsets || !w_gate || !w_up || !w_down || !recv_y) return MOE_ERR_INVALID_ARG;
         if (c->n_shared > 0 && (!x || !ws_gate || !ws_up || !ws_down || !y_shared))
             return MOE_ERR_INVALID_ARG;
     }
-    const void *ptrs[] = {recv_x, w_gate, w_up, w_down, recv_y, x, ws_gate, ws_up, ws_down, y_shared};
+    const void *ptrs[] = {recv_x, recv_q, recv_scale, w_gate, w_up, w_down, recv_y, x,
+                          ws_gate, ws_up, ws_down, y_shared};
     for (const void *p : ptrs)
         if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
     const moe_config g = ep_global(c, world);
@@ -541,6 +565,7 @@ moe_status moe_ep_expert_ffn(const moe_config *c, int32_t world, int32_t rank, c
     a.T = c->T; a.d = c->d; a.E = c->E / world; a.K = c->K * world; a.d_ff = c->d_ff;
     a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
     a.x_perm = recv_x; a.perm_token = nullptr; a.offsets = local_offsets;
+    a.x_perm_q = recv_q; a.x_scale = recv_scale;
     a.w_gate = w_gate; a.w_up = w_up; a.w_down = w_down;
     a.h = at<void>(ws, L.h); a.y_perm = recv_y;
     a.x = x; a.ws_gate = ws_gate; a.ws_up = ws_up; a.ws_down = ws_down;
@@ -548,6 +573,28 @@ moe_status moe_ep_expert_ffn(const moe_config *c, int32_t world, int32_t rank, c
     a.status = at<int32_t>(ws, L.status);
     a.timeout_ns = kWaitTimeoutNs;
     return cuda_status(launch_expert_ffn(a, as_stream(stream)));
+}
+}  // namespace
+
+moe_status moe_ep_expert_ffn_fp8(const moe_config *c, int32_t world, int32_t rank,
+                                 const uint8_t *recv_q, const float *recv_scale,
+                                 const int32_t *local_offsets, const void *w_gate,
+                                 const void *w_up, const void *w_down, void *recv_y, const void *x,
+                                 const void *ws_gate, const void *ws_up, const void *ws_down,
+                                 void *y_shared, void *ws, size_t ws_bytes, void *stream) {
+    return ep_expert_ffn(c, world, rank, true, nullptr, recv_q, recv_scale, local_offsets, w_gate,
+                         w_up, w_down, recv_y, x, ws_gate, ws_up, ws_down, y_shared, ws, ws_bytes,
+                         stream);
+}
+
+moe_status moe_ep_expert_ffn(const moe_config *c, int32_t world, int32_t rank, const void *recv_x,
+                             const int32_t *local_offsets, const void *w_gate, const void *w_up,
+                             const void *w_down, void *recv_y, const void *x, const void *ws_gate,
+                             const void *ws_up, const void *ws_down, void *y_shared, void *ws,
+                             size_t ws_bytes, void *stream) {
+    return ep_expert_ffn(c, world, rank, false, recv_x, nullptr, nullptr, local_offsets, w_gate,
+                         w_up, w_down, recv_y, x, ws_gate, ws_up, ws_down, y_shared, ws, ws_bytes,
+                         stream);
 }
 
 moe_status moe_ep_combine(const moe_config *c, int32_t world, const int32_t *topk_idx,

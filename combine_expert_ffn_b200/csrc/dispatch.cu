@@ -16,8 +16,8 @@
 //             offsets = exclusive scan of counts (recomputed per block)
 //   gather  : x_perm[row] = x[t], reading each x row once and writing it K
 //             times with 16-byte vector accesses
-#include <cuda_fp8.h>
 
+#include "fp8_payload.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -230,31 +230,9 @@ dispatch_gather_fp8_kernel(const uint4 *__restrict__ x, const int32_t *__restric
         const bool in = i < total;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (in) v = __ldg(x + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float f[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            f[2 * j] = bf16_lo(w[j]);
-            f[2 * j + 1] = bf16_hi(w[j]);
-        }
-        float amax = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        float sc;
+        const uint2 packed = e4m3_quantize_chunk(v, &sc);
         if (!in) continue;
-        const float sc = __fdiv_rn(amax, 448.0f);
-        uint32_t q[2] = {0u, 0u};
-        if (amax > 0.f) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(
-                    make_float2(__fdiv_rn(f[2 * j], sc), __fdiv_rn(f[2 * j + 1], sc)),
-                    __NV_SATFINITE, __NV_E4M3);
-                q[j >> 1] |= (uint32_t)b << (16 * (j & 1));
-            }
-        }
-        const uint2 packed = make_uint2(q[0], q[1]);
         const int64_t t = i / chunks;
         const int c = (int)(i - t * chunks);
         for (int j = 0; j < K; ++j) {

@@ -22,6 +22,10 @@
 //           among this rank's tokens choosing e]; one load, K peer stores
 // combine:  out[t] = y_shared[t] + sum_j w_j recv_y[owner(e_j)][same row],
 //           fp32 multiply-adds in slot order (as the single-GPU combine)
+// FP8 payload (E4M3 codes + one fp32 scale per 128 channels, quantized once
+// at the source with the single-GPU FP8 gather's quantizer): recv_q [cap, d]
+// bytes and recv_scale [cap, d / 128] fp32 per owner take the place of recv_x,
+// and the owner's expert FFN widens the codes inside its GEMM.
 // recv_x / recv_y are device arrays of `world` device pointers: this GPU's
 // buffers and peers' buffers mapped into its address space; the kernels use
 // plain loads and stores through them.  Each block first builds in shared
@@ -29,6 +33,7 @@
 // row delta[e] in owner(e)'s buffer, so a copy's address is that pointer plus
 // inv_perm[t][j] rows: one global load (beside topk_idx) before the row itself,
 // as in the single-GPU gather and combine.
+#include "fp8_payload.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -115,6 +120,54 @@ ep_dispatch_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ topk
                 }
                 rowbase_s[e][(int64_t)r8[q] * chunks + c] = v;
             }
+        }
+    }
+}
+
+// FP8 payload: one 16-lane group per (token, 128-channel block), as the
+// single-GPU FP8 gather; the codes and the scale go to the K owners' rows.
+__global__ void __launch_bounds__(256, 4)
+ep_dispatch_fp8_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
+                       const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
+                       const int32_t *__restrict__ base, uint2 *const *__restrict__ recv_q,
+                       float *const *__restrict__ recv_scale, int64_t recv_rows, int T, int chunks,
+                       int E, int K, int El, int32_t *status) {
+    __shared__ int32_t delta_s[EP_MAX_E];
+    __shared__ uint2 *rowq_s[EP_MAX_E];
+    __shared__ float *rows_s[EP_MAX_E];
+    const int blocks = chunks >> 4;  // 128-channel blocks per row
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int32_t dl = base[e] - offsets[e];
+        delta_s[e] = dl;
+        rowq_s[e] = recv_q[e / El] + (int64_t)dl * chunks;
+        rows_s[e] = recv_scale[e / El] + (int64_t)dl * blocks;
+    }
+    __syncthreads();
+    const int64_t total = (int64_t)T * chunks;  // a multiple of 16: groups never straddle it
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + (threadIdx.x & ~31); i0 < total;
+         i0 += stride) {
+        const int64_t i = i0 + lane;
+        const bool in = i < total;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (in) v = __ldg(x + i);
+        float sc;
+        const uint2 packed = e4m3_quantize_chunk(v, &sc);
+        if (!in) continue;
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        for (int j = 0; j < K; ++j) {
+            const int e = __ldg(topk_idx + t * K + j);
+            const int r = __ldg(inv_perm + t * K + j);
+            if (e < 0 || e >= E) continue;  // flagged by the local dispatch plan
+            const int64_t row = (int64_t)delta_s[e] + r;
+            if (row < 0 || row >= recv_rows) {
+                if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                continue;
+            }
+            rowq_s[e][(int64_t)r * chunks + c] = packed;
+            if ((c & 15) == 0) rows_s[e][(int64_t)r * blocks + (c >> 4)] = sc;
         }
     }
 }
@@ -213,6 +266,21 @@ cudaError_t launch_ep_dispatch(const void *x, const int32_t *topk_idx, const int
     ep_dispatch_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
         static_cast<const uint4 *>(x), topk_idx, offsets, inv_perm, base,
         reinterpret_cast<uint4 *const *>(recv_x), recv_rows, T, chunks, E, K, E / world, status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_dispatch_fp8(const void *x, const int32_t *topk_idx,
+                                   const int32_t *offsets, const int32_t *inv_perm,
+                                   const int32_t *base, void *const *recv_q,
+                                   void *const *recv_scale, int64_t recv_rows, int T, int d, int E,
+                                   int K, int world, int32_t *status, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_dispatch_fp8_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
+        static_cast<const uint4 *>(x), topk_idx, offsets, inv_perm, base,
+        reinterpret_cast<uint2 *const *>(recv_q), reinterpret_cast<float *const *>(recv_scale),
+        recv_rows, T, chunks, E, K, E / world, status);
     count_launch();
     return cudaGetLastError();
 }

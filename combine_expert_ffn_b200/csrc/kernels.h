@@ -58,6 +58,11 @@ cudaError_t launch_ep_dispatch(const void *x, const int32_t *topk_idx, const int
                                const int32_t *inv_perm, const int32_t *base, void *const *recv_x,
                                int64_t recv_rows, int T, int d, int E, int K, int world,
                                int32_t *status, cudaStream_t st);
+cudaError_t launch_ep_dispatch_fp8(const void *x, const int32_t *topk_idx,
+                                   const int32_t *offsets, const int32_t *inv_perm,
+                                   const int32_t *base, void *const *recv_q,
+                                   void *const *recv_scale, int64_t recv_rows, int T, int d, int E,
+                                   int K, int world, int32_t *status, cudaStream_t st);
 cudaError_t launch_ep_combine(const int32_t *topk_idx, const float *topk_w, const int32_t *offsets,
                               const int32_t *inv_perm, const int32_t *base,
                               const void *const *recv_y, int64_t recv_rows, const void *y_shared,

@@ -6,7 +6,8 @@ A rank owns E / world experts and routes its own tokens.  One step:
     moe_route, moe_dispatch(x_perm=None)     local routing and dispatch plan
     all-gather of the per-expert counts       counts_all [world, E]
     moe_ep_plan                               where this rank's copies go
-    moe_ep_dispatch                           gather + peer stores
+    moe_ep_dispatch                           gather + peer stores (bf16 rows, or
+                                              E4M3 codes + scales: moe_ep_dispatch_fp8)
     barrier                                   every rank's stores are done
     moe_ep_expert_ffn                         this rank's experts, shared experts
     barrier                                   every rank's outputs are done
@@ -22,10 +23,10 @@ from __future__ import annotations
 
 import torch
 
-from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_dispatch,
-               moe_ep_expert_ffn, moe_ep_plan, moe_ep_workspace_size, moe_ipc_close_handle,
-               moe_ipc_get_handle, moe_ipc_open_handle, moe_route, moe_route_hash,
-               MOE_ROUTER_HASH)
+from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_dispatch, moe_ep_dispatch_fp8,
+               moe_ep_expert_ffn, moe_ep_expert_ffn_fp8, moe_ep_plan, moe_ep_workspace_size,
+               moe_ipc_close_handle, moe_ipc_get_handle, moe_ipc_open_handle, moe_route,
+               moe_route_hash, MOE_PAYLOAD_FP8, MOE_ROUTER_HASH)
 
 
 def _i32(n, device):
@@ -46,7 +47,13 @@ class _RankState:
         self.perm, self.inv = _i32(T * K, device), torch.empty(T, K, dtype=torch.int32, device=device)
         self.base, self.local_offsets = _i32(E, device), _i32(E // world + 1, device)
         cap = world * T * K
-        self.recv_x = torch.empty(cap, d, dtype=torch.bfloat16, device=device)
+        self.fp8 = cfg.payload == MOE_PAYLOAD_FP8
+        if self.fp8:   # E4M3 codes + one fp32 scale per 128 channels
+            self.recv_x = None
+            self.recv_q = torch.empty(cap, d, dtype=torch.uint8, device=device)
+            self.recv_scale = torch.empty(cap, d // 128, dtype=torch.float32, device=device)
+        else:
+            self.recv_x = torch.empty(cap, d, dtype=torch.bfloat16, device=device)
         self.recv_y = torch.empty(cap, d, dtype=torch.bfloat16, device=device)
         self.y_shared = torch.empty(T, d, dtype=torch.bfloat16, device=device)
         self.out = torch.empty(T, d, dtype=torch.bfloat16, device=device)
@@ -64,6 +71,29 @@ class _RankState:
                       self.ws, stream)
         moe_dispatch(cfg, x, self.topk_idx, self.counts, self.offsets, self.send, self.send_tok,
                      self.perm, self.inv, None, self.ws, stream)
+
+    def recv_buffers(self):
+        """The buffers the dispatch writes into at this rank as an owner."""
+        return [self.recv_q, self.recv_scale] if self.fp8 else [self.recv_x]
+
+    def dispatch(self, world, x, tables, stream):
+        """tables: one device pointer table per entry of recv_buffers()."""
+        if self.fp8:
+            moe_ep_dispatch_fp8(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
+                                self.base, tables[0], tables[1], self.status, stream)
+        else:
+            moe_ep_dispatch(self.cfg, world, x, self.topk_idx, self.offsets, self.inv, self.base,
+                            tables[0], self.status, stream)
+
+    def expert_ffn(self, world, rank, w, x, w_shared, stream):
+        y_sh = self.y_shared if self.cfg.n_shared else None
+        if self.fp8:
+            moe_ep_expert_ffn_fp8(self.cfg, world, rank, self.recv_q, self.recv_scale,
+                                  self.local_offsets, *w, self.recv_y, x, *w_shared, y_sh,
+                                  self.ws, stream)
+        else:
+            moe_ep_expert_ffn(self.cfg, world, rank, self.recv_x, self.local_offsets, *w,
+                              self.recv_y, x, *w_shared, y_sh, self.ws, stream)
 
 
 def gather_counts(counts, group=None):
@@ -86,7 +116,8 @@ class EmulatedEP:
     only after the previous one has run for all ranks, which stands in for the
     barriers between them."""
 
-    def __init__(self, shape, inp: dict, world: int, router=None, token_ids=None, stream=None):
+    def __init__(self, shape, inp: dict, world: int, router=None, token_ids=None, stream=None,
+                 payload=None):
         self.device = inp["x"].device
         base_cfg = MoeConfig.of(shape, router=router)
         T = base_cfg.T
@@ -94,13 +125,15 @@ class EmulatedEP:
             raise ValueError("T and E must be multiples of world")
         Tr = T // world
         self.world, self.stream, self.inp = world, stream, inp
-        self.cfg = MoeConfig.of(shape.replace(T=Tr), router=router)
+        self.cfg = MoeConfig.of(shape.replace(T=Tr), router=router, payload=payload)
         self.ranks = [_RankState(self.cfg, world, self.device) for _ in range(world)]
         self.xs = [inp["x"][r * Tr:(r + 1) * Tr] for r in range(world)]
         self.ids = [None if token_ids is None else token_ids[r * Tr:(r + 1) * Tr]
                     for r in range(world)]
-        self.recv_x_ptrs = torch.tensor([st.recv_x.data_ptr() for st in self.ranks],
-                                        dtype=torch.int64, device=self.device)
+        n_buf = len(self.ranks[0].recv_buffers())
+        self.recv_tables = [torch.tensor([st.recv_buffers()[i].data_ptr() for st in self.ranks],
+                                         dtype=torch.int64, device=self.device)
+                            for i in range(n_buf)]
         self.recv_y_ptrs = torch.tensor([st.recv_y.data_ptr() for st in self.ranks],
                                         dtype=torch.int64, device=self.device)
         self.counts_all = torch.empty(world, self.cfg.E, dtype=torch.int32, device=self.device)
@@ -124,18 +157,14 @@ class EmulatedEP:
 
     def dispatch(self):
         for r, st in enumerate(self.ranks):
-            moe_ep_dispatch(self.cfg, self.world, self.xs[r], st.topk_idx, st.offsets, st.inv,
-                            st.base, self.recv_x_ptrs, st.status, self.stream)
+            st.dispatch(self.world, self.xs[r], self.recv_tables, self.stream)
 
     def expert_ffn(self):
-        inp, cfg, world = self.inp, self.cfg, self.world
+        inp, world = self.inp, self.world
+        w_shared = (inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"))
         for r, st in enumerate(self.ranks):
-            moe_ep_expert_ffn(cfg, world, r, st.recv_x, st.local_offsets,
-                              _local_weights(inp["w_gate"], r, world),
-                              _local_weights(inp["w_up"], r, world),
-                              _local_weights(inp["w_down"], r, world), st.recv_y, self.xs[r],
-                              inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"),
-                              st.y_shared if cfg.n_shared else None, st.ws, self.stream)
+            w = tuple(_local_weights(inp[k], r, world) for k in ("w_gate", "w_up", "w_down"))
+            st.expert_ffn(world, r, w, self.xs[r], w_shared, self.stream)
 
     def combine(self):
         for st in self.ranks:
@@ -153,10 +182,11 @@ class EmulatedEP:
         return torch.cat([st.out for st in self.ranks])
 
 
-def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, stream=None):
+def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, stream=None,
+                    payload=None):
     """One EP step of all `world` ranks on this GPU; returns (out [T, d],
     per-rank states)."""
-    em = EmulatedEP(shape, inp, world, router, token_ids, stream)
+    em = EmulatedEP(shape, inp, world, router, token_ids, stream, payload)
     return em.forward(), em.ranks
 
 
@@ -171,20 +201,20 @@ class EPLayer:
 
     def __init__(self, shape_local, group, router_w, bias, w_gate_local, w_up_local,
                  w_down_local, ws_gate=None, ws_up=None, ws_down=None, logit_offset=None,
-                 router=None):
+                 router=None, payload=None):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.device = w_gate_local.device
-        self.cfg = MoeConfig.of(shape_local, router=router)
+        self.cfg = MoeConfig.of(shape_local, router=router, payload=payload)
         self.st = _RankState(self.cfg, self.world, self.device)
         self.router_w, self.bias, self.logit_offset = router_w, bias, logit_offset
         self.w = (w_gate_local, w_up_local, w_down_local)
         self.ws_shared = (ws_gate, ws_up, ws_down)
         self._opened = []
-        self.recv_x_ptrs = self._map_peers(self.st.recv_x)
+        self.recv_tables = [self._map_peers(b) for b in self.st.recv_buffers()]
         self.recv_y_ptrs = self._map_peers(self.st.recv_y)
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
 
@@ -212,11 +242,9 @@ class EPLayer:
         counts_all = gather_counts(st.counts, self.group)
         moe_ep_plan(cfg, world, r, counts_all, st.base, st.local_offsets, stream)
         self._barrier()                       # every rank's recv_x is free again
-        moe_ep_dispatch(cfg, world, x, st.topk_idx, st.offsets, st.inv, st.base,
-                        self.recv_x_ptrs, st.status, stream)
+        st.dispatch(world, x, self.recv_tables, stream)
         self._barrier()
-        moe_ep_expert_ffn(cfg, world, r, st.recv_x, st.local_offsets, *self.w, st.recv_y, x,
-                          *self.ws_shared, st.y_shared if cfg.n_shared else None, st.ws, stream)
+        st.expert_ffn(world, r, self.w, x, self.ws_shared, stream)
         self._barrier()
         moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,
                        self.recv_y_ptrs, st.y_shared if cfg.n_shared else None, st.out,

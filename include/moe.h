@@ -411,6 +411,30 @@ MOE_API moe_status moe_ep_expert_ffn(const moe_config *cfg, int32_t world, int32
                                      const void *ws_up, const void *ws_down, void *y_shared,
                                      void *ws, size_t ws_bytes, void *stream);
 
+/* FP8 payload variant of moe_ep_dispatch (moe_dispatch_fp8's format, d % 128
+ * == 0): each copy travels as d E4M3 codes into recv_q[owner] ([world*T*K, d]
+ * bytes) and one fp32 scale per 128-channel block into recv_scale[owner]
+ * ([world*T*K, d/128]), both device arrays of `world` device pointers.  The
+ * quantization is moe_dispatch_fp8's, done once per token at the source: the
+ * codes equal those moe_dispatch_fp8 writes for the same token.  Halves the
+ * bytes of the dispatch exchange ("DeepSeek 8.7 -- communication", section 4). */
+MOE_API moe_status moe_ep_dispatch_fp8(const moe_config *cfg, int32_t world, const void *x,
+                                       const int32_t *topk_idx, const int32_t *offsets,
+                                       const int32_t *inv_perm, const int32_t *base,
+                                       void *const *recv_q, void *const *recv_scale,
+                                       int32_t *device_status, void *stream);
+
+/* moe_ep_expert_ffn over the FP8 payload: recv_q / recv_scale of this rank
+ * (moe_expert_ffn_fp8's operands); x [T, d] is required (shared experts and
+ * the GEMM's operand map). */
+MOE_API moe_status moe_ep_expert_ffn_fp8(const moe_config *cfg, int32_t world, int32_t rank,
+                                         const uint8_t *recv_q, const float *recv_scale,
+                                         const int32_t *local_offsets, const void *w_gate,
+                                         const void *w_up, const void *w_down, void *recv_y,
+                                         const void *x, const void *ws_gate, const void *ws_up,
+                                         const void *ws_down, void *y_shared, void *ws,
+                                         size_t ws_bytes, void *stream);
+
 /* Combine fused with its all-to-all: out[t] = y_shared[t] + sum_j topk_w[t][j]
  * * (row of copy (t, j) in recv_y[owner]), fp32 multiply-adds in slot order,
  * bf16 out [T, d].  recv_y: device array of `world` device pointers. */

@@ -187,6 +187,62 @@ def test_router_variants_validate_before_cuda(moe):
     assert lib.moe_forward(C.byref(cfg), *args, P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_expert_parallel_validates_before_cuda(moe):
+    tiny = synth.config("tiny")                        # E = 16, d = 128
+    cfg = moe.MoeConfig.of(tiny)
+    lib, fake, P = moe._lib, 1 << 20, C.c_void_p
+    # world must divide E, 1 <= world <= 64; the workspace is the global batch's
+    assert moe.moe_ep_workspace_size(cfg, 3) == 0
+    assert moe.moe_ep_workspace_size(cfg, 0) == 0
+    assert moe.moe_ep_workspace_size(cfg, 32) == 0
+    assert moe.moe_ep_workspace_size(cfg, 2) == \
+        moe.moe_workspace_size(moe.MoeConfig.of(tiny.replace(T=2 * tiny.T)))
+    ws_n = moe.moe_ep_workspace_size(cfg, 2)
+    UNS, INV = moe.MOE_ERR_UNSUPPORTED_SHAPE, moe.MOE_ERR_INVALID_ARG
+    c = C.byref(cfg)
+    assert lib.moe_ep_plan(c, 3, 0, P(fake), P(fake), P(fake), None) == UNS
+    assert lib.moe_ep_plan(c, 2, 2, P(fake), P(fake), P(fake), None) == UNS      # rank
+    assert lib.moe_ep_plan(c, 2, 0, None, P(fake), P(fake), None) == INV
+    d_args = [P(fake)] * 6                     # x, topk_idx, offsets, inv_perm, base, recv_x
+    bad = list(d_args)
+    bad[5] = None
+    assert lib.moe_ep_dispatch(c, 2, *bad, None, None) == INV
+    bad = list(d_args)
+    bad[0] = P(fake + 8)                       # misaligned x
+    assert lib.moe_ep_dispatch(c, 2, *bad, None, None) == INV
+    assert lib.moe_ep_dispatch(c, 5, *d_args, None, None) == UNS
+    odd = moe.MoeConfig.of(tiny.replace(d=192))
+    q_args = [P(fake)] * 7                     # ..., recv_q, recv_scale
+    assert lib.moe_ep_dispatch_fp8(C.byref(odd), 2, *q_args, None, None) == UNS
+    bad = list(q_args)
+    bad[6] = None
+    assert lib.moe_ep_dispatch_fp8(c, 2, *bad, None, None) == INV
+    f_args = [P(fake)] * 11                    # recv_x .. y_shared
+    assert lib.moe_ep_expert_ffn(c, 2, 0, *f_args, P(fake), ws_n - 1, None) == \
+        moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert lib.moe_ep_expert_ffn(c, 2, -1, *f_args, P(fake), ws_n, None) == UNS
+    bad = list(f_args)
+    bad[0] = None                              # recv_x
+    assert lib.moe_ep_expert_ffn(c, 2, 0, *bad, P(fake), ws_n, None) == INV
+    assert lib.moe_ep_expert_ffn(c, 2, 0, *f_args, P(fake + 16), ws_n, None) == INV  # ws align
+    g_args = [P(fake)] * 12                    # recv_q, recv_scale, ... y_shared
+    bad = list(g_args)
+    bad[1] = None                              # recv_scale
+    assert lib.moe_ep_expert_ffn_fp8(c, 2, 0, *bad, P(fake), ws_n, None) == INV
+    bad = list(g_args)
+    bad[1] = P(fake + 4)                       # misaligned scales
+    assert lib.moe_ep_expert_ffn_fp8(c, 2, 0, *bad, P(fake), ws_n, None) == INV
+    assert lib.moe_ep_expert_ffn_fp8(C.byref(odd), 2, 0, *g_args, P(fake), ws_n, None) == UNS
+    c_args = [P(fake)] * 7                     # topk_idx .. y_shared, then out
+    assert lib.moe_ep_combine(c, 2, *c_args, None, None, None) == INV         # out
+    bad = list(c_args)
+    bad[6] = P(fake + 2)                       # misaligned y_shared
+    assert lib.moe_ep_combine(c, 2, *bad, P(fake), None, None) == INV
+    assert lib.moe_ipc_get_handle(None, P(fake)) == INV
+    assert lib.moe_ipc_open_handle(None, P(fake)) == INV
+    assert lib.moe_ipc_close_handle(None) == INV
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a GPU")
 def test_no_device_is_reported(moe):
     assert moe._lib.moe_clear_device_status(C.c_void_p(1 << 20), None) == moe.MOE_ERR_NO_DEVICE

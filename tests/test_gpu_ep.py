@@ -9,6 +9,7 @@ the router reduces d in one range on both sides (d < 512); at the V3 sizes
 the output is within the layer's bars of the oracle.
 """
 import gc
+import math
 
 import numpy as np
 import pytest
@@ -35,8 +36,8 @@ def _free_gpu():
     torch.cuda.empty_cache()
 
 
-def _forward(sh, inp, router=None, token_ids=None):
-    cfg = moe.MoeConfig.of(sh, router=router)
+def _forward(sh, inp, router=None, token_ids=None, payload=None):
+    cfg = moe.MoeConfig.of(sh, router=router, payload=payload)
     ws = moe.alloc_workspace(cfg)
     o = moe.forward_outputs(cfg)
     moe.moe_forward(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
@@ -83,6 +84,70 @@ def test_emulated_ep_v3_matches_oracle(orc):
         assert int(st.status.item()) == moe.MOE_OK
     rows = np.unique(np.linspace(0, sh.T - 1, 8).astype(np.int64))
     ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows)
+    gi = torch.cat([st.topk_idx for st in ranks]).cpu().numpy()[rows]
+    keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
+    for r in set(range(len(rows))) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    frob, elem = H.compare_out(out[torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
+# d % 128 == 0 for the FP8 payload, one router range over d, shared experts
+EP_FP8 = synth.MoeShape("ep_fp8", T=256, d=384, E=16, G=4, K=4, M=2, d_ff=192, n_shared=1,
+                        d_ff_shared=128, x_sigma=1.0, e_sigma=1 / math.sqrt(384),
+                        bias_sigma=0.1, seed=11)
+
+
+@pytest.mark.parametrize("name,world", [("ep_fp8", 2), ("ep_fp8", 4), ("noshared", 2),
+                                        ("noshared", 4)])
+def test_emulated_ep_fp8_payload_equals_single_gpu(name, world):
+    """The FP8 dispatch payload across ranks: the codes and scales every owner
+    receives are the rows of the single-GPU FP8 dispatch of the whole batch
+    restricted to its experts, and the layer's output equals moe_forward's
+    with the FP8 payload bit for bit."""
+    sh = EP_FP8 if name == "ep_fp8" else H.shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    fp8 = moe.MOE_PAYLOAD_FP8
+    ref = _forward(sh, inp, payload=fp8)
+    out, ranks = ep.emulate_forward(sh, inp, world, payload=fp8)
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+        assert moe.moe_read_device_status(st.ws) == moe.MOE_OK
+    assert torch.equal(torch.cat([st.topk_idx for st in ranks]), ref["topk_idx"])
+    assert torch.equal(out.view(torch.int16), ref["out"].view(torch.int16))
+    # the single-GPU FP8 dispatch of the whole batch
+    cfg8 = moe.MoeConfig.of(sh, payload=fp8)
+    ws = moe.alloc_workspace(cfg8)
+    T, K, E, G = sh.T, sh.K, sh.E, sh.G
+    i32 = dict(dtype=torch.int32, device=DEV)
+    counts, offsets = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    send, send_tok = torch.empty(G, G, **i32), torch.empty(G, G, **i32)
+    perm, inv = torch.empty(T * K, **i32), torch.empty(T, K, **i32)
+    xq = torch.empty(T * K, sh.d, dtype=torch.uint8, device=DEV)
+    xs = torch.empty(T * K, sh.d // 128, dtype=torch.float32, device=DEV)
+    moe.moe_dispatch_fp8(cfg8, inp["x"], ref["topk_idx"], counts, offsets, send, send_tok, perm,
+                         inv, xq, xs, ws)
+    torch.cuda.synchronize()
+    El = E // world
+    off = offsets.cpu().numpy()
+    for o, st in enumerate(ranks):
+        lo, hi = int(off[o * El]), int(off[(o + 1) * El])
+        n = int(st.local_offsets[El].item())
+        assert n == hi - lo
+        assert torch.equal(st.recv_q[:n], xq[lo:hi])
+        assert torch.equal(st.recv_scale[:n].view(torch.int32), xs[lo:hi].view(torch.int32))
+
+
+def test_emulated_ep_fp8_v3_matches_oracle(orc):
+    sh = H.shape("v3")
+    inp = synth.make_inputs(sh, DEV)
+    out, ranks = ep.emulate_forward(sh, inp, 8, payload=moe.MOE_PAYLOAD_FP8)
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+    rows = np.unique(np.linspace(0, sh.T - 1, 6).astype(np.int64))
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows, payload=1)
     gi = torch.cat([st.topk_idx for st in ranks]).cpu().numpy()[rows]
     keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
     for r in set(range(len(rows))) - set(keep):
