@@ -297,14 +297,17 @@ def moe_ep_combine(cfg, world, topk_idx, topk_w, offsets, inv_perm, base, recv_y
                             _ptr(out), _ptr(device_status), _stream(stream)))
 
 
+MOE_IPC_HANDLE_BYTES = 72
+
+
 def moe_ipc_get_handle(t) -> bytes:
-    h = (C.c_char * 64)()
+    h = (C.c_char * MOE_IPC_HANDLE_BYTES)()
     _ok("moe_ipc_get_handle", _lib.moe_ipc_get_handle(_ptr(t), C.cast(h, C.c_void_p)))
     return bytes(h)
 
 
 def moe_ipc_open_handle(handle: bytes) -> int:
-    buf = (C.c_char * 64).from_buffer_copy(handle)
+    buf = (C.c_char * MOE_IPC_HANDLE_BYTES).from_buffer_copy(handle)
     p = C.c_void_p()
     _ok("moe_ipc_open_handle", _lib.moe_ipc_open_handle(C.cast(buf, C.c_void_p), C.byref(p)))
     return p.value

@@ -7,6 +7,8 @@
 // moe_read_device_status, whose purpose is that copy).
 #include <atomic>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "kernels.h"
 
@@ -99,6 +101,34 @@ cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 }  // namespace moe
 
 using namespace moe;
+
+namespace {
+// cuMemGetAddressRange through the runtime's driver entry point (no
+// link-time libcuda): the allocation that holds a device pointer
+using AddrRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+bool ipc_addr_range(const void *p, CUdeviceptr *base, size_t *bytes) {
+    static AddrRangeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<AddrRangeFn>(f);
+    });
+    return fn && fn(base, bytes, reinterpret_cast<CUdeviceptr>(p)) == CUDA_SUCCESS;
+}
+// pointers handed out by moe_ipc_open_handle -> the mapping they lie in
+std::mutex &ipc_mutex() {
+    static std::mutex m;
+    return m;
+}
+std::unordered_map<void *, void *> &ipc_opened() {
+    static std::unordered_map<void *, void *> m;
+    return m;
+}
+}  // namespace
 
 extern "C" {
 
@@ -618,10 +648,18 @@ moe_status moe_ipc_get_handle(const void *dev_ptr, void *handle) {
     if (!dev_ptr || !handle) return MOE_ERR_INVALID_ARG;
     moe_status st = check_device();
     if (st) return st;
+    // the handle names the whole allocation holding dev_ptr (a caching
+    // allocator may place a buffer inside a larger one): send the offset too
+    CUdeviceptr base = 0;
+    size_t bytes = 0;
+    if (!ipc_addr_range(dev_ptr, &base, &bytes)) return MOE_ERR_CUDA;
     cudaIpcMemHandle_t h;
-    if (cudaIpcGetMemHandle(&h, const_cast<void *>(dev_ptr)) != cudaSuccess) return MOE_ERR_CUDA;
-    static_assert(sizeof(h) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    static_assert(sizeof(h) + sizeof(uint64_t) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+    const uint64_t off = reinterpret_cast<uintptr_t>(dev_ptr) - (uintptr_t)base;
     std::memcpy(handle, &h, sizeof(h));
+    std::memcpy(static_cast<char *>(handle) + sizeof(h), &off, sizeof(off));
     return MOE_OK;
 }
 
@@ -630,15 +668,31 @@ moe_status moe_ipc_open_handle(const void *handle, void **dev_ptr) {
     moe_status st = check_device();
     if (st) return st;
     cudaIpcMemHandle_t h;
+    uint64_t off = 0;
     std::memcpy(&h, handle, sizeof(h));
-    return cuda_status(cudaIpcOpenMemHandle(dev_ptr, h, cudaIpcMemLazyEnablePeerAccess));
+    std::memcpy(&off, static_cast<const char *>(handle) + sizeof(h), sizeof(off));
+    void *base = nullptr;
+    if ((st = cuda_status(cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess))))
+        return st;
+    *dev_ptr = static_cast<char *>(base) + off;
+    std::lock_guard<std::mutex> lock(ipc_mutex());
+    ipc_opened()[*dev_ptr] = base;
+    return MOE_OK;
 }
 
 moe_status moe_ipc_close_handle(void *dev_ptr) {
     if (!dev_ptr) return MOE_ERR_INVALID_ARG;
+    void *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(ipc_mutex());
+        auto it = ipc_opened().find(dev_ptr);
+        if (it == ipc_opened().end()) return MOE_ERR_INVALID_ARG;  // not from open_handle
+        base = it->second;
+        ipc_opened().erase(it);
+    }
     moe_status st = check_device();
     if (st) return st;
-    return cuda_status(cudaIpcCloseMemHandle(dev_ptr));
+    return cuda_status(cudaIpcCloseMemHandle(base));
 }
 
 moe_status moe_selftest_bounded_wait(int64_t timeout_ns, void *ws, void *stream) {

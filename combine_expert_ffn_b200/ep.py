@@ -192,11 +192,15 @@ def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, s
 
 class EPLayer:
     """One rank of an expert-parallel MoE layer in a process group with one
-    process per GPU (NCCL backend).  Holds this rank's experts
-    (w_gate / w_up / w_down [E/world, ...]), the replicated router and shared
-    experts, and the receive buffers, mapped into every rank by CUDA IPC.
+    process per GPU.  Holds this rank's experts (w_gate / w_up / w_down
+    [E/world, ...]), the replicated router and shared experts, and the receive
+    buffers, mapped into every rank by CUDA IPC.
 
-    Not run on more than one GPU here: every GPU run of this build had one GPU.
+    With the NCCL backend the counts exchange and the barriers are
+    stream-ordered collectives (no host synchronisation inside the step).
+    With gloo they run on the host after synchronising the step's stream;
+    that form also lets several processes share one GPU (each maps the
+    others' buffers through IPC on the same device).
     """
 
     def __init__(self, shape_local, group, router_w, bias, w_gate_local, w_up_local,
@@ -208,12 +212,14 @@ class EPLayer:
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.device = w_gate_local.device
+        self.host_sync = dist.get_backend(group) != "nccl"
         self.cfg = MoeConfig.of(shape_local, router=router, payload=payload)
         self.st = _RankState(self.cfg, self.world, self.device)
         self.router_w, self.bias, self.logit_offset = router_w, bias, logit_offset
         self.w = (w_gate_local, w_up_local, w_down_local)
         self.ws_shared = (ws_gate, ws_up, ws_down)
         self._opened = []
+        torch.cuda.synchronize(self.device)   # buffers allocated before peers map them
         self.recv_tables = [self._map_peers(b) for b in self.st.recv_buffers()]
         self.recv_y_ptrs = self._map_peers(self.st.recv_y)
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
@@ -231,27 +237,47 @@ class EPLayer:
                 ptrs.append(p)
         return torch.tensor(ptrs, dtype=torch.int64, device=self.device)
 
-    def _barrier(self):
-        # stream-ordered: completes on every rank only after every rank's
-        # preceding kernels on its stream have completed
-        self.dist.all_reduce(self._flag, group=self.group)
+    def _barrier(self, stream):
+        """Every rank's work issued so far on its step stream has completed
+        before any rank's later work on that stream starts."""
+        if self.host_sync:
+            stream.synchronize()
+            self.dist.barrier(group=self.group)
+        else:
+            self.dist.all_reduce(self._flag, group=self.group)
+
+    def _gather_counts(self, counts, stream):
+        if self.host_sync:
+            stream.synchronize()
+            return gather_counts(counts.cpu(), self.group).to(self.device)
+        return gather_counts(counts, self.group)
 
     def forward(self, x, token_ids=None, stream=None):
+        """This rank's tokens x [T, d] -> out [T, d] (a buffer of the layer,
+        overwritten by the next call)."""
         st, cfg, world, r = self.st, self.cfg, self.world, self.rank
-        st.route_and_plan_local(x, self.router_w, self.logit_offset, self.bias, token_ids, stream)
-        counts_all = gather_counts(st.counts, self.group)
-        moe_ep_plan(cfg, world, r, counts_all, st.base, st.local_offsets, stream)
-        self._barrier()                       # every rank's recv_x is free again
-        st.dispatch(world, x, self.recv_tables, stream)
-        self._barrier()
-        st.expert_ffn(world, r, self.w, x, self.ws_shared, stream)
-        self._barrier()
-        moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,
-                       self.recv_y_ptrs, st.y_shared if cfg.n_shared else None, st.out,
-                       st.status, stream)
+        s = stream or torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):   # the collectives order against this stream
+            st.route_and_plan_local(x, self.router_w, self.logit_offset, self.bias, token_ids, s)
+            counts_all = self._gather_counts(st.counts, s)
+            moe_ep_plan(cfg, world, r, counts_all, st.base, st.local_offsets, s)
+            self._barrier(s)          # every rank's receive buffers are free again
+            st.dispatch(world, x, self.recv_tables, s)
+            self._barrier(s)          # every copy has landed
+            st.expert_ffn(world, r, self.w, x, self.ws_shared, s)
+            self._barrier(s)          # every expert output is written
+            moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,
+                           self.recv_y_ptrs, st.y_shared if cfg.n_shared else None, st.out,
+                           st.status, s)
         return st.out
 
-    def close(self):
+    def close(self, stream=None):
+        """Unmaps the peers' buffers once every rank has finished reading
+        them (a barrier first); every rank calls it."""
+        s = stream or torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            self._barrier(s)
+        s.synchronize()
         for p in self._opened:
             moe_ipc_close_handle(p)
         self._opened = []

@@ -444,11 +444,16 @@ MOE_API moe_status moe_ep_combine(const moe_config *cfg, int32_t world, const in
                                   const void *const *recv_y, const void *y_shared, void *out,
                                   int32_t *device_status, void *stream);
 
-/* CUDA IPC of a device allocation for the peer pointer tables: the handle is
- * MOE_IPC_HANDLE_BYTES opaque bytes to send to the other ranks; open maps a
- * peer's allocation into this GPU's address space (peer access enabled),
- * close unmaps it. */
-#define MOE_IPC_HANDLE_BYTES 64
+/* CUDA IPC of a device buffer for the peer pointer tables.  get_handle writes
+ * MOE_IPC_HANDLE_BYTES opaque bytes (the CUDA IPC handle of the allocation
+ * that holds dev_ptr, and dev_ptr's offset inside it: a caching allocator may
+ * place the buffer inside a larger allocation) to send to the other ranks.
+ * open_handle, in another process, maps that allocation into this GPU's
+ * address space (peer access enabled) and returns the buffer's address in
+ * it; close_handle takes that address and unmaps the allocation
+ * (MOE_ERR_INVALID_ARG for an address open_handle did not return).  A process
+ * cannot open its own handles. */
+#define MOE_IPC_HANDLE_BYTES 72
 MOE_API moe_status moe_ipc_get_handle(const void *dev_ptr, void *handle);
 MOE_API moe_status moe_ipc_open_handle(const void *handle, void **dev_ptr);
 MOE_API moe_status moe_ipc_close_handle(void *dev_ptr);
