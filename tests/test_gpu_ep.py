@@ -43,7 +43,7 @@ def _forward(sh, inp, router=None, token_ids=None, payload=None):
     moe.moe_forward(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
                     inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
                     inp.get("ws_up"), inp.get("ws_down"), o["out"], o["topk_idx"], o["topk_w"],
-                    o["counts"], ws=ws, token_ids=token_ids)
+                    o["counts"], offsets=o["offsets"], ws=ws, token_ids=token_ids)
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
     return o
 
@@ -148,6 +148,75 @@ def test_emulated_ep_fp8_v3_matches_oracle(orc):
         assert int(st.status.item()) == moe.MOE_OK
     rows = np.unique(np.linspace(0, sh.T - 1, 6).astype(np.int64))
     ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows, payload=1)
+    gi = torch.cat([st.topk_idx for st in ranks]).cpu().numpy()[rows]
+    keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
+    for r in set(range(len(rows))) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    frob, elem = H.compare_out(out[torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
+def test_emulated_ep_owner_with_no_rows():
+    """A bias that keeps every token out of rank 1's experts (groups 2 and 3
+    of 4): rank 1 receives no rows, runs only its shared experts, and the
+    layer still equals moe_forward bit for bit."""
+    sh = H.shape("ragged")                       # E 12, G 4, M 2: rank 1 owns groups 2, 3
+    inp = synth.make_inputs(sh, DEV)
+    bias = inp["bias"].clone()
+    bias[sh.E // 2:] = -10.0
+    inp = dict(inp, bias=bias)
+    ref = _forward(sh, inp)
+    assert int(ref["counts"][sh.E // 2:].sum()) == 0
+    out, ranks = ep.emulate_forward(sh, inp, 2)
+    torch.cuda.synchronize()
+    assert int(ranks[1].local_offsets[-1].item()) == 0
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+        assert moe.moe_read_device_status(st.ws) == moe.MOE_OK
+    assert torch.equal(out.view(torch.int16), ref["out"].view(torch.int16))
+
+
+def test_emulated_ep_world_one_is_the_single_gpu_layer():
+    sh = H.shape("ragged")
+    inp = synth.make_inputs(sh, DEV)
+    ref = _forward(sh, inp)
+    out, ranks = ep.emulate_forward(sh, inp, 1)
+    torch.cuda.synchronize()
+    assert int(ranks[0].status.item()) == moe.MOE_OK
+    assert torch.equal(out.view(torch.int16), ref["out"].view(torch.int16))
+    assert torch.equal(ranks[0].local_offsets, ref["offsets"])
+
+
+def test_emulated_ep_empty_batch():
+    sh = H.shape("ragged")
+    inp = synth.make_inputs(sh, DEV)
+    empty = sh.replace(T=0)
+    inp = dict(inp, x=inp["x"][:0])
+    out, ranks = ep.emulate_forward(empty, inp, 2)
+    torch.cuda.synchronize()
+    assert out.shape == (0, sh.d)
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+        assert int(st.local_offsets[-1].item()) == 0
+
+
+def test_emulated_ep_maximum_world(orc):
+    """64 ranks (the largest world) of one expert each on the mid workload
+    (T=4096, d=2048, E=64, K=6): sampled tokens within the layer's bars of the
+    oracle."""
+    sh = H.shape("mid")
+    inp = synth.make_inputs(sh, DEV)
+    out, ranks = ep.emulate_forward(sh, inp, 64)
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+    counts_all = torch.stack([st.counts for st in ranks]).cpu().numpy()
+    base, loff = orc.ep_plan(counts_all)
+    for r, st in enumerate(ranks):
+        np.testing.assert_array_equal(st.base.cpu().numpy(), base[r])
+        np.testing.assert_array_equal(st.local_offsets.cpu().numpy(), loff[r])
+    rows = np.unique(np.linspace(0, sh.T - 1, 8).astype(np.int64))
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows)
     gi = torch.cat([st.topk_idx for st in ranks]).cpu().numpy()[rows]
     keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
     for r in set(range(len(rows))) - set(keep):
