@@ -56,6 +56,8 @@ def lib():
         _lib.oracle_e4m3_encode.restype = C.c_uint8
         _lib.oracle_fp8_quantize_row.argtypes = [i32, P, P, P]
         _lib.oracle_ep_plan.argtypes = [i32, i32, P, P, P]
+        _lib.oracle_ep_token_plan.argtypes = [i32, i32, i32, i32, P, P, P]
+        _lib.oracle_ep_token_base.argtypes = [i32, P, P]
         _lib.oracle_fp8_dequantize_row.argtypes = [i32, P, P, P]
         _lib.oracle_hash_route.argtypes = [i32, P, i32, i32, i32, i32, P, P]
         _lib.oracle_lowbias32.argtypes = [C.c_uint32]
@@ -65,7 +67,8 @@ def lib():
                   "oracle_ffn_row", "oracle_shared_row", "oracle_combine",
                   "oracle_layer_rows", "oracle_router_affinity", "oracle_layer_rows_ex",
                   "oracle_hash_route", "oracle_bias_update", "oracle_fp8_quantize_row",
-                  "oracle_fp8_dequantize_row", "oracle_ep_plan"):
+                  "oracle_fp8_dequantize_row", "oracle_ep_plan", "oracle_ep_token_plan",
+                  "oracle_ep_token_base"):
             getattr(_lib, f).restype = C.c_int
     return _lib
 
@@ -220,6 +223,28 @@ def ep_plan(counts_all):
     loff = np.empty((world, E // world + 1), np.int32)
     _check(lib().oracle_ep_plan(world, E, _p(c), _p(base), _p(loff)), "oracle_ep_plan")
     return base, loff
+
+
+def ep_token_plan(topk_idx, E, world):
+    """Deduplicated dispatch of one rank: (tok_slot [T, world], tok_counts
+    [world]) int32; tok_slot -1 where a token has no expert at that owner."""
+    idx = _np(np.asarray(topk_idx, dtype=np.int32), np.int32)
+    T, K = idx.shape
+    slot = np.empty((T, world), np.int32)
+    cnt = np.empty(world, np.int32)
+    _check(lib().oracle_ep_token_plan(T, K, E, world, _p(idx), _p(slot), _p(cnt)),
+           "oracle_ep_token_plan")
+    return slot, cnt
+
+
+def ep_token_base(tok_counts_all):
+    """tok_base [world, world] from tok_counts_all [world, world] (row r = rank
+    r's per-owner token counts): first row of rank r's tokens at owner o."""
+    c = _np(np.asarray(tok_counts_all, dtype=np.int32), np.int32)
+    world = c.shape[0]
+    base = np.empty((world, world), np.int32)
+    _check(lib().oracle_ep_token_base(world, _p(c), _p(base)), "oracle_ep_token_base")
+    return base
 
 
 def fp8_quantize(x):

@@ -689,3 +689,53 @@ int oracle_ep_plan(int world, int E, const int32_t *counts_all, int32_t *base,
     }
     return ORC_OK;
 }
+
+/* Token-level placement of the deduplicated dispatch.  With node-limited
+ * routing a token's activations need to reach each of its (at most M) nodes
+ * once and fan out to its experts there ("moe-node-limited-routing": the
+ * limit bounds the nodes a token's activations must reach; the send_tok
+ * matrix of the single-GPU dispatch counts exactly these token-node pairs).
+ * For one rank's routing topk_idx [T, K], experts in contiguous blocks of
+ * El = E / world per owner:
+ *   tok_slot [T, world] out: position of token t among this rank's tokens
+ *                            that have an expert at owner o, in token
+ *                            order; -1 when t has none there
+ *   tok_counts [world] out:  this rank's tokens sent to owner o            */
+int oracle_ep_token_plan(int T, int K, int E, int world, const int32_t *topk_idx,
+                         int32_t *tok_slot, int32_t *tok_counts)
+{
+    if (T < 0 || K <= 0 || E <= 0 || world <= 0 || E % world || !tok_counts ||
+        (T > 0 && (!topk_idx || !tok_slot)))
+        return ORC_EBADARG;
+    const int El = E / world;
+    for (int o = 0; o < world; ++o) tok_counts[o] = 0;
+    for (int t = 0; t < T; ++t) {
+        for (int o = 0; o < world; ++o) {
+            int sends = 0;
+            for (int j = 0; j < K; ++j) {
+                const int e = topk_idx[(int64_t)t * K + j];
+                if (e < 0 || e >= E) return ORC_EBADARG;
+                if (e / El == o) sends = 1;
+            }
+            tok_slot[(int64_t)t * world + o] = sends ? tok_counts[o]++ : -1;
+        }
+    }
+    return ORC_OK;
+}
+
+/* Receive rows of the deduplicated dispatch at owner o: the tokens of rank
+ * 0, then rank 1, ..., each rank's in its token order.  From tok_counts_all
+ * [world, world] (row r = rank r's tok_counts): tok_base [world, world] out,
+ * tok_base[r][o] = first row of rank r's tokens at owner o.                */
+int oracle_ep_token_base(int world, const int32_t *tok_counts_all, int32_t *tok_base)
+{
+    if (world <= 0 || !tok_counts_all || !tok_base) return ORC_EBADARG;
+    for (int o = 0; o < world; ++o) {
+        int64_t row = 0;
+        for (int r = 0; r < world; ++r) {
+            tok_base[r * world + o] = (int32_t)row;
+            row += tok_counts_all[r * world + o];
+        }
+    }
+    return ORC_OK;
+}

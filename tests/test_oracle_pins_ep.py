@@ -51,3 +51,70 @@ def test_plan_matches_the_single_gpu_dispatch(orc, world, E, K, T):
         lo, hi = glob["offsets"][o * El], glob["offsets"][(o + 1) * El]
         np.testing.assert_array_equal(recv, glob["perm_token"][lo:hi])
         np.testing.assert_array_equal(loff[o, :El], glob["offsets"][o * El:(o + 1) * El] - lo)
+
+
+def test_hand_worked_token_plan(orc):
+    """world 2, E 4 (owner 0: experts 0, 1; owner 1: 2, 3), K 2.  Rank 0's
+    tokens: t0 -> {0, 1} (owner 0 only), t1 -> {1, 2} (both owners); rank 1's:
+    t2 -> {2, 3} (owner 1), t3 -> {0, 3} (both).  Owner 0 receives rank 0's
+    t0, t1 (rows 0, 1) then rank 1's t3 (row 2); owner 1 receives rank 0's t1
+    (row 0), then rank 1's t2, t3 (rows 1, 2)."""
+    slot0, cnt0 = orc.ep_token_plan(np.array([[0, 1], [1, 2]]), 4, 2)
+    slot1, cnt1 = orc.ep_token_plan(np.array([[2, 3], [0, 3]]), 4, 2)
+    np.testing.assert_array_equal(slot0, [[0, -1], [1, 0]])
+    np.testing.assert_array_equal(cnt0, [2, 1])
+    np.testing.assert_array_equal(slot1, [[-1, 0], [0, 1]])
+    np.testing.assert_array_equal(cnt1, [1, 2])
+    np.testing.assert_array_equal(orc.ep_token_base(np.stack([cnt0, cnt1])), [[0, 0], [2, 1]])
+
+
+@pytest.mark.parametrize("world,E,G,K,M,T", [(2, 8, 2, 2, 1, 16), (4, 16, 4, 4, 2, 64),
+                                             (8, 64, 8, 8, 4, 256), (8, 256, 8, 8, 4, 512),
+                                             (4, 32, 8, 8, 4, 96), (1, 12, 3, 3, 3, 30)])
+def test_token_plan_fans_out_to_the_single_gpu_dispatch(orc, world, E, G, K, M, T):
+    """Each token crosses once to each owner holding one of its experts; the
+    owner's fan-out of those rows, indexed through the copy rows of the expert
+    plan, must reproduce the single-GPU dispatch's perm_token for its experts,
+    and with owners = groups the per-owner token counts are the dispatch's
+    send_tok (both from a separate, pinned oracle function).  Routings are
+    node-limited: M of G groups, K/M experts in each."""
+    rng = np.random.default_rng(world * 7919 + E + K)
+    gsz, kpg = E // G, K // M
+    idx = np.stack([np.concatenate([g * gsz + rng.permutation(gsz)[:kpg]
+                                    for g in rng.permutation(G)[:M]]) for _ in range(T)])
+    idx = idx.astype(np.int32)
+    Tr, El = T // world, E // world
+    plans = [orc.ep_token_plan(idx[r * Tr:(r + 1) * Tr], E, world) for r in range(world)]
+    tok_counts_all = np.stack([p[1] for p in plans])
+    tok_base = orc.ep_token_base(tok_counts_all)
+    counts_all = np.stack([np.bincount(idx[r * Tr:(r + 1) * Tr].ravel(), minlength=E)
+                           for r in range(world)]).astype(np.int32)
+    base, loff = orc.ep_plan(counts_all)
+    glob = orc.dispatch(idx, E, G)
+    if world == G:
+        np.testing.assert_array_equal(tok_counts_all, glob["send_tok"])
+    for o in range(world):
+        n_tok = int(tok_counts_all[:, o].sum())
+        recv_tok = np.full(n_tok, -1, np.int64)          # global token of each row
+        rows = int(loff[o, El])
+        fan = np.full(rows, -1, np.int64)                # copy row -> token row
+        for r in range(world):
+            slot = plans[r][0]
+            seen = np.zeros(E, np.int64)
+            for tl in range(Tr):
+                t = r * Tr + tl
+                if slot[tl, o] >= 0:
+                    row = tok_base[r, o] + slot[tl, o]
+                    assert recv_tok[row] == -1
+                    recv_tok[row] = t
+                else:
+                    assert all(int(e) // El != o for e in idx[t])
+                for e in idx[t]:
+                    if e // El != o:
+                        continue
+                    crow = base[r, e] + seen[e]
+                    seen[e] += 1
+                    fan[crow] = tok_base[r, o] + slot[tl, o]
+        assert (recv_tok >= 0).all() and (fan >= 0).all()
+        lo, hi = glob["offsets"][o * El], glob["offsets"][(o + 1) * El]
+        np.testing.assert_array_equal(recv_tok[fan], glob["perm_token"][lo:hi])
