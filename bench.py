@@ -605,6 +605,41 @@ def ep_leg(sh, inp, dev, stream, world, reps=20):
         "note": "all ranks run in sequence on one GPU; peer traffic is local HBM here",
     }
     del em
+    # the deduplicated dispatch: each token crosses once to each owner holding
+    # one of its experts, plus a 4-byte fan-out index per copy; the owner
+    # rebuilds its copy rows locally
+    torch.cuda.empty_cache()
+    em = ep.EmulatedEP(sh, inp, world, stream=stream, dedup=True)
+    em.forward()
+    torch.cuda.synchronize(dev)
+    graphs = {k: graphed(k) for k in ("dispatch", "fanout")}
+    td = {k: timed(graphs[k].replay) / world for k in ("dispatch", "fanout")}
+    for st in em.ranks:
+        if int(st.status.item()) != moe.MOE_OK or moe.moe_read_device_status(st.ws) != moe.MOE_OK:
+            raise RuntimeError("device status after the emulated deduplicated dispatch")
+    del graphs
+    tca = em.gathered[:, E:].cpu().to(torch.int64)              # [world, world] tokens
+    tok_out = [int(tca[r].sum() - tca[r, r]) for r in range(world)]
+    tok_in = [int(tca[:, o].sum() - tca[o, o]) for o in range(world)]
+    dd_link = 2.0 * d * max(max(tok_out), max(tok_in)) + 4.0 * max(max(out_copies),
+                                                                  max(in_copies))
+    mean_tok_rows = float(tca.sum()) / world
+    dd_bytes = 2.0 * d * (Tr + mean_tok_rows) + 12.0 * K * Tr   # x read, token rows, indices
+    fan_bytes = 4.0 * d * (Tr * K) + 4.0 * Tr * K               # copy rows read + written
+    res["dedup_dispatch"] = {
+        "stage_ms_per_rank": td,
+        "token_rows_per_rank": mean_tok_rows,
+        "dispatch": {"bytes_per_rank": dd_bytes,
+                     "achieved_gbs": dd_bytes / (td["dispatch"] / 1e3) / 1e9,
+                     "frac_of_hbm": dd_bytes / (td["dispatch"] / 1e3) / 1e9 / hbm},
+        "fanout": {"bytes_per_rank": fan_bytes,
+                   "achieved_gbs": fan_bytes / (td["fanout"] / 1e3) / 1e9,
+                   "frac_of_hbm": fan_bytes / (td["fanout"] / 1e3) / 1e9 / hbm},
+        "nvlink": {"max_rank_bytes_dispatch": dd_link,
+                   "projected_ms_dispatch": dd_link / (NVLINK_GBS * 1e9) * 1e3,
+                   "tokens_out": tok_out, "tokens_in": tok_in},
+    }
+    del em
     if sh.d % 128 == 0:
         # the FP8 payload: E4M3 codes + one fp32 scale per 128 channels travel
         # instead of bf16 rows; the owners' GEMM widens them

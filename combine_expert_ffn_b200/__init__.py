@@ -37,8 +37,9 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_bias_update", "moe_expert_ffn_gather", "moe_dispatch_fp8",
            "moe_expert_ffn_fp8", "moe_permute", "moe_ep_workspace_size", "moe_ep_plan",
            "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_dispatch_fp8",
-           "moe_ep_expert_ffn_fp8", "moe_ipc_get_handle", "moe_ipc_open_handle",
-           "moe_ipc_close_handle")
+           "moe_ep_expert_ffn_fp8", "moe_ep_token_plan", "moe_ep_token_base",
+           "moe_ep_dispatch_dedup", "moe_ep_fanout", "moe_ipc_get_handle",
+           "moe_ipc_open_handle", "moe_ipc_close_handle")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
 MOE_PAYLOAD_BF16, MOE_PAYLOAD_FP8 = 0, 1
@@ -96,6 +97,10 @@ _sig = {
     "moe_ep_expert_ffn": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P,
                                     _P, _P, _P, _P, _S, _P]),
     "moe_ep_combine": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_token_plan": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P]),
+    "moe_ep_token_base": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P]),
+    "moe_ep_dispatch_dedup": (C.c_int, [_CP, C.c_int32] + [_P] * 11),
+    "moe_ep_fanout": (C.c_int, [_CP, C.c_int32] + [_P] * 6),
     "moe_ep_dispatch_fp8": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_ep_expert_ffn_fp8": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P, _P, _P, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _S, _P]),
@@ -266,6 +271,36 @@ def moe_ep_expert_ffn(cfg, world, rank, recv_x, local_offsets, w_gate, w_up, w_d
                                _ptr(local_offsets), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                                _ptr(recv_y), _ptr(x), _ptr(ws_gate), _ptr(ws_up),
                                _ptr(ws_down), _ptr(y_shared), wp, wn, _stream(stream)))
+
+
+def moe_ep_token_plan(cfg, world, topk_idx, tok_slot, tok_counts, stream=None) -> None:
+    _ok("moe_ep_token_plan",
+        _lib.moe_ep_token_plan(_cfg(cfg), int(world), _ptr(topk_idx), _ptr(tok_slot),
+                               _ptr(tok_counts), _stream(stream)))
+
+
+def moe_ep_token_base(cfg, world, rank, tok_counts_all, tok_base, stream=None) -> None:
+    _ok("moe_ep_token_base",
+        _lib.moe_ep_token_base(_cfg(cfg), int(world), int(rank), _ptr(tok_counts_all),
+                               _ptr(tok_base), _stream(stream)))
+
+
+def moe_ep_dispatch_dedup(cfg, world, x, topk_idx, offsets, inv_perm, base, tok_slot, tok_base,
+                          recv_tok_ptrs, recv_idx_ptrs, device_status=None, stream=None) -> None:
+    """recv_tok_ptrs / recv_idx_ptrs: device int64 tensors of `world` device pointers."""
+    _ok("moe_ep_dispatch_dedup",
+        _lib.moe_ep_dispatch_dedup(_cfg(cfg), int(world), _ptr(x), _ptr(topk_idx), _ptr(offsets),
+                                   _ptr(inv_perm), _ptr(base), _ptr(tok_slot), _ptr(tok_base),
+                                   _ptr(recv_tok_ptrs), _ptr(recv_idx_ptrs), _ptr(device_status),
+                                   _stream(stream)))
+
+
+def moe_ep_fanout(cfg, world, recv_tok, recv_idx, local_offsets, recv_x, device_status=None,
+                  stream=None) -> None:
+    _ok("moe_ep_fanout",
+        _lib.moe_ep_fanout(_cfg(cfg), int(world), _ptr(recv_tok), _ptr(recv_idx),
+                           _ptr(local_offsets), _ptr(recv_x), _ptr(device_status),
+                           _stream(stream)))
 
 
 def moe_ep_dispatch_fp8(cfg, world, x, topk_idx, offsets, inv_perm, base, recv_q_ptrs,

@@ -558,6 +558,66 @@ moe_status moe_ep_dispatch_fp8(const moe_config *c, int32_t world, const void *x
                                               device_status, as_stream(stream)));
 }
 
+moe_status moe_ep_token_plan(const moe_config *c, int32_t world, const int32_t *topk_idx,
+                             int32_t *tok_slot, int32_t *tok_counts, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!tok_counts || (c->T > 0 && (!topk_idx || !tok_slot))) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_ep_token_plan(topk_idx, c->T, c->E, c->K, world, tok_slot,
+                                            tok_counts, as_stream(stream)));
+}
+
+moe_status moe_ep_token_base(const moe_config *c, int32_t world, int32_t rank,
+                             const int32_t *tok_counts_all, int32_t *tok_base, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world) || rank < 0 || rank >= world) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!tok_counts_all || !tok_base) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_ep_token_base(tok_counts_all, world, rank, tok_base,
+                                            as_stream(stream)));
+}
+
+moe_status moe_ep_dispatch_dedup(const moe_config *c, int32_t world, const void *x,
+                                 const int32_t *topk_idx, const int32_t *offsets,
+                                 const int32_t *inv_perm, const int32_t *base,
+                                 const int32_t *tok_slot, const int32_t *tok_base,
+                                 void *const *recv_tok, int32_t *const *recv_idx,
+                                 int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!x || !topk_idx || !offsets || !inv_perm || !base || !tok_slot ||
+                     !tok_base || !recv_tok || !recv_idx))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t tok_rows = (int64_t)world * c->T;
+    const int64_t cap = tok_rows * c->K;
+    return cuda_status(launch_ep_dispatch_dedup(x, topk_idx, offsets, inv_perm, base, tok_slot,
+                                                tok_base, recv_tok, recv_idx, tok_rows, cap, c->T,
+                                                c->d, c->E, c->K, world, device_status,
+                                                as_stream(stream)));
+}
+
+moe_status moe_ep_fanout(const moe_config *c, int32_t world, const void *recv_tok,
+                         const int32_t *recv_idx, const int32_t *local_offsets, void *recv_x,
+                         int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!recv_tok || !recv_idx || !local_offsets || !recv_x))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(recv_tok) || !aligned16(recv_x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t tok_rows = (int64_t)world * c->T;
+    return cuda_status(launch_ep_fanout(recv_tok, recv_idx, local_offsets, c->E / world, tok_rows,
+                                        tok_rows * c->K, c->d, recv_x, device_status,
+                                        as_stream(stream)));
+}
+
 namespace {
 // the expert FFN of one rank's experts over its receive buffer: bf16 rows
 // (recv_x) or FP8 codes + scales (recv_q, recv_scale)

@@ -26,6 +26,15 @@
 // at the source with the single-GPU FP8 gather's quantizer): recv_q [cap, d]
 // bytes and recv_scale [cap, d / 128] fp32 per owner take the place of recv_x,
 // and the owner's expert FFN widens the codes inside its GEMM.
+// Deduplicated dispatch ("moe-node-limited-routing": the node limit bounds the
+// nodes a token's activations must reach): a token's row crosses to each owner
+// holding one of its experts once, into recv_tok[owner] (rows: rank 0's
+// tokens, then rank 1's, ..., each in token order; tok_base[o] = this rank's
+// first row there, tok_slot[t][o] = t's position among this rank's tokens
+// for o), and each copy (t, j) writes only its 4-byte index
+// recv_idx[owner][copy row] = token row.  The owner's fan-out then builds
+// recv_x[r] = recv_tok[recv_idx[r]] locally: the same rows, so the same GEMM
+// input as without deduplication.
 // recv_x / recv_y are device arrays of `world` device pointers: this GPU's
 // buffers and peers' buffers mapped into its address space; the kernels use
 // plain loads and stores through them.  Each block first builds in shared
@@ -67,7 +76,7 @@ __global__ void ep_plan_kernel(const int32_t *__restrict__ counts_all, int world
                                                                   col[me * El + El - 1];
 }
 
-constexpr int EP_MAX_E = 1024;
+constexpr int EP_MAX_E = 1024, EP_MAX_WORLD = 64;
 
 // delta[e] = base[e] - offsets[e] and the address of row delta[e] of
 // owner(e)'s buffer, for every expert, in shared memory
@@ -169,6 +178,161 @@ ep_dispatch_fp8_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ 
             rowq_s[e][(int64_t)r * chunks + c] = packed;
             if ((c & 15) == 0) rows_s[e][(int64_t)r * blocks + (c >> 4)] = sc;
         }
+    }
+}
+
+// tok_slot / tok_counts of one owner o = blockIdx.x: a block-wide exclusive
+// scan over this rank's tokens of "t has an expert at o", in token order.
+__global__ void __launch_bounds__(1024)
+ep_token_plan_kernel(const int32_t *__restrict__ topk_idx, int T, int K, int E, int El, int world,
+                     int32_t *__restrict__ tok_slot, int32_t *__restrict__ tok_counts) {
+    __shared__ int warp_excl[32];
+    __shared__ int total_s, carry_s;
+    const int o = blockIdx.x;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    if (threadIdx.x == 0) carry_s = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+        const int t = t0 + threadIdx.x;
+        int flag = 0;
+        if (t < T) {
+            for (int j = 0; j < K; ++j) {
+                const int e = __ldg(topk_idx + (int64_t)t * K + j);
+                if (e >= 0 && e < E && e / El == o) flag = 1;
+            }
+        }
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, flag);
+        const int in_warp = __popc(bal & ((1u << lane) - 1u));
+        if (lane == 0) warp_excl[wid] = __popc(bal);
+        __syncthreads();
+        if (wid == 0) {
+            const int v = lane < nwarps ? warp_excl[lane] : 0;
+            int incl = v;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int n = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                if (lane >= d) incl += n;
+            }
+            if (lane < nwarps) warp_excl[lane] = incl - v;
+            if (lane == 31) total_s = incl;
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        if (t < T) tok_slot[(int64_t)t * world + o] = flag ? carry + warp_excl[wid] + in_warp : -1;
+        __syncthreads();  // every thread has read carry_s and warp_excl
+        if (threadIdx.x == 0) carry_s = carry + total_s;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) tok_counts[o] = carry_s;
+}
+
+// tok_base[o] = sum over ranks r < me of tok_counts_all[r][o]
+__global__ void ep_token_base_kernel(const int32_t *__restrict__ tok_counts_all, int world, int me,
+                                     int32_t *__restrict__ tok_base) {
+    const int o = threadIdx.x;
+    if (o >= world) return;
+    int s = 0;
+    for (int r = 0; r < me; ++r) s += tok_counts_all[r * world + o];
+    tok_base[o] = s;
+}
+
+// Thread per 16-byte chunk of an x row: one store per (token, owner) of the
+// row, one 4-byte index store per copy (by the chunk-0 thread).
+__global__ void __launch_bounds__(256, 4)
+ep_dispatch_dedup_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
+                         const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
+                         const int32_t *__restrict__ base, const int32_t *__restrict__ tok_slot,
+                         const int32_t *__restrict__ tok_base, uint4 *const *__restrict__ recv_tok,
+                         int32_t *const *__restrict__ recv_idx, int64_t tok_rows,
+                         int64_t recv_rows, int T, int chunks, int E, int K, int El, int world,
+                         int32_t *status) {
+    __shared__ int32_t delta_s[EP_MAX_E];
+    __shared__ int32_t tokbase_s[EP_MAX_WORLD];
+    __shared__ uint4 *tok_tab_s[EP_MAX_WORLD];
+    __shared__ int32_t *idx_tab_s[EP_MAX_WORLD];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) delta_s[e] = base[e] - offsets[e];
+    for (int o = threadIdx.x; o < world; o += blockDim.x) {
+        tokbase_s[o] = tok_base[o];
+        tok_tab_s[o] = recv_tok[o];
+        idx_tab_s[o] = recv_idx[o];
+    }
+    __syncthreads();
+    const int64_t total = (int64_t)T * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        const uint4 v = __ldg(x + i);
+        const int32_t *idx_t = topk_idx + t * K;
+        uint64_t sent = 0;  // owners this token's row has gone to (world <= 64)
+        for (int j0 = 0; j0 < K; j0 += 8) {
+            int o8[8], s8[8], r8[8];
+            int e8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {  // independent loads first
+                const int j = j0 + q;
+                e8[q] = -1;
+                r8[q] = 0;
+                if (j < K) {
+                    e8[q] = __ldg(idx_t + j);
+                    if (c == 0) r8[q] = __ldg(inv_perm + t * K + j);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = e8[q];
+                o8[q] = e >= 0 && e < E ? e / El : -1;  // invalid ids: flagged by the local plan
+                s8[q] = o8[q] >= 0 ? __ldg(tok_slot + t * world + o8[q]) : -1;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int o = o8[q];
+                if (o < 0) continue;
+                const int64_t trow = (int64_t)tokbase_s[o] + s8[q];
+                if (s8[q] < 0 || trow >= tok_rows) {
+                    if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                    continue;
+                }
+                if (!((sent >> o) & 1ull)) {  // the token's first slot at owner o
+                    sent |= 1ull << o;
+                    tok_tab_s[o][trow * chunks + c] = v;
+                }
+                if (c == 0) {
+                    const int64_t row = (int64_t)delta_s[e8[q]] + r8[q];
+                    if (row < 0 || row >= recv_rows) {
+                        if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                        continue;
+                    }
+                    idx_tab_s[o][row] = (int32_t)trow;
+                }
+            }
+        }
+    }
+}
+
+// The owner's fan-out: recv_x[r] = recv_tok[recv_idx[r]] for the rows it
+// received (local_offsets[El] of them).
+__global__ void __launch_bounds__(256, 4)
+ep_fanout_kernel(const uint4 *__restrict__ recv_tok, const int32_t *__restrict__ recv_idx,
+                 const int32_t *__restrict__ local_offsets, int El, int64_t tok_rows,
+                 int64_t recv_rows, int chunks, uint4 *__restrict__ recv_x, int32_t *status) {
+    int64_t n = local_offsets[El];
+    if (n < 0 || n > recv_rows) {
+        if (status && blockIdx.x == 0 && threadIdx.x == 0) record_status(status, MOE_ERR_DEVICE_FAULT);
+        n = n < 0 ? 0 : recv_rows;
+    }
+    const int64_t total = n * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / chunks;
+        const int c = (int)(i - r * chunks);
+        const int64_t src = __ldg(recv_idx + r);
+        if (src < 0 || src >= tok_rows) {
+            if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+            continue;
+        }
+        recv_x[i] = __ldg(recv_tok + src * chunks + c);
     }
 }
 
@@ -281,6 +445,50 @@ cudaError_t launch_ep_dispatch_fp8(const void *x, const int32_t *topk_idx,
         static_cast<const uint4 *>(x), topk_idx, offsets, inv_perm, base,
         reinterpret_cast<uint2 *const *>(recv_q), reinterpret_cast<float *const *>(recv_scale),
         recv_rows, T, chunks, E, K, E / world, status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_token_plan(const int32_t *topk_idx, int T, int E, int K, int world,
+                                  int32_t *tok_slot, int32_t *tok_counts, cudaStream_t st) {
+    ep_token_plan_kernel<<<world, 1024, 0, st>>>(topk_idx, T, K, E, E / world, world, tok_slot,
+                                                 tok_counts);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_token_base(const int32_t *tok_counts_all, int world, int me,
+                                 int32_t *tok_base, cudaStream_t st) {
+    ep_token_base_kernel<<<1, 64, 0, st>>>(tok_counts_all, world, me, tok_base);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_dispatch_dedup(const void *x, const int32_t *topk_idx, const int32_t *offsets,
+                                     const int32_t *inv_perm, const int32_t *base,
+                                     const int32_t *tok_slot, const int32_t *tok_base,
+                                     void *const *recv_tok, int32_t *const *recv_idx,
+                                     int64_t tok_rows, int64_t recv_rows, int T, int d, int E, int K,
+                                     int world, int32_t *status, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_dispatch_dedup_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
+        static_cast<const uint4 *>(x), topk_idx, offsets, inv_perm, base, tok_slot, tok_base,
+        reinterpret_cast<uint4 *const *>(recv_tok), recv_idx, tok_rows, recv_rows, T, chunks, E,
+        K, E / world, world, status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_fanout(const void *recv_tok, const int32_t *recv_idx,
+                             const int32_t *local_offsets, int El, int64_t tok_rows,
+                             int64_t recv_rows, int d, void *recv_x, int32_t *status,
+                             cudaStream_t st) {
+    if (recv_rows == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_fanout_kernel<<<grid_for(recv_rows * chunks), 256, 0, st>>>(
+        static_cast<const uint4 *>(recv_tok), recv_idx, local_offsets, El, tok_rows, recv_rows,
+        chunks, static_cast<uint4 *>(recv_x), status);
     count_launch();
     return cudaGetLastError();
 }

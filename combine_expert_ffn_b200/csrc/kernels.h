@@ -63,6 +63,20 @@ cudaError_t launch_ep_dispatch_fp8(const void *x, const int32_t *topk_idx,
                                    const int32_t *base, void *const *recv_q,
                                    void *const *recv_scale, int64_t recv_rows, int T, int d, int E,
                                    int K, int world, int32_t *status, cudaStream_t st);
+cudaError_t launch_ep_token_plan(const int32_t *topk_idx, int T, int E, int K, int world,
+                                  int32_t *tok_slot, int32_t *tok_counts, cudaStream_t st);
+cudaError_t launch_ep_token_base(const int32_t *tok_counts_all, int world, int me,
+                                 int32_t *tok_base, cudaStream_t st);
+cudaError_t launch_ep_dispatch_dedup(const void *x, const int32_t *topk_idx, const int32_t *offsets,
+                                     const int32_t *inv_perm, const int32_t *base,
+                                     const int32_t *tok_slot, const int32_t *tok_base,
+                                     void *const *recv_tok, int32_t *const *recv_idx,
+                                     int64_t tok_rows, int64_t recv_rows, int T, int d, int E, int K,
+                                     int world, int32_t *status, cudaStream_t st);
+cudaError_t launch_ep_fanout(const void *recv_tok, const int32_t *recv_idx,
+                             const int32_t *local_offsets, int El, int64_t tok_rows,
+                             int64_t recv_rows, int d, void *recv_x, int32_t *status,
+                             cudaStream_t st);
 cudaError_t launch_ep_combine(const int32_t *topk_idx, const float *topk_w, const int32_t *offsets,
                               const int32_t *inv_perm, const int32_t *base,
                               const void *const *recv_y, int64_t recv_rows, const void *y_shared,

@@ -7,7 +7,9 @@ A rank owns E / world experts and routes its own tokens.  One step:
     all-gather of the per-expert counts       counts_all [world, E]
     moe_ep_plan                               where this rank's copies go
     moe_ep_dispatch                           gather + peer stores (bf16 rows, or
-                                              E4M3 codes + scales: moe_ep_dispatch_fp8)
+                                              E4M3 codes + scales: moe_ep_dispatch_fp8;
+                                              or one row per token and owner plus a
+                                              fan-out index per copy: dedup)
     barrier                                   every rank's stores are done
     moe_ep_expert_ffn                         this rank's experts, shared experts
     barrier                                   every rank's outputs are done
@@ -23,8 +25,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_dispatch, moe_ep_dispatch_fp8,
-               moe_ep_expert_ffn, moe_ep_expert_ffn_fp8, moe_ep_plan, moe_ep_workspace_size,
+from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_dispatch, moe_ep_dispatch_dedup,
+               moe_ep_dispatch_fp8, moe_ep_expert_ffn, moe_ep_expert_ffn_fp8, moe_ep_fanout,
+               moe_ep_plan, moe_ep_token_base, moe_ep_token_plan, moe_ep_workspace_size,
                moe_ipc_close_handle, moe_ipc_get_handle, moe_ipc_open_handle, moe_route,
                moe_route_hash, MOE_PAYLOAD_FP8, MOE_ROUTER_HASH)
 
@@ -36,9 +39,9 @@ def _i32(n, device):
 class _RankState:
     """Per-rank buffers of one EP step."""
 
-    def __init__(self, cfg: MoeConfig, world: int, device):
+    def __init__(self, cfg: MoeConfig, world: int, device, dedup: bool = False):
         T, K, E, G, d = cfg.T, cfg.K, cfg.E, cfg.G, cfg.d
-        self.cfg = cfg
+        self.cfg, self.world, self.dedup = cfg, world, dedup
         self.topk_idx = torch.empty(T, K, dtype=torch.int32, device=device)
         self.topk_w = torch.empty(T, K, dtype=torch.float32, device=device)
         self.counts, self.offsets = _i32(E, device), _i32(E + 1, device)
@@ -48,6 +51,13 @@ class _RankState:
         self.base, self.local_offsets = _i32(E, device), _i32(E // world + 1, device)
         cap = world * T * K
         self.fp8 = cfg.payload == MOE_PAYLOAD_FP8
+        if dedup and self.fp8:
+            raise ValueError("the deduplicated dispatch carries bf16 rows")
+        if dedup:      # one row per (token, owner); the owner fans out locally
+            self.recv_tok = torch.empty(world * T, d, dtype=torch.bfloat16, device=device)
+            self.recv_idx = torch.empty(cap, dtype=torch.int32, device=device)
+            self.tok_slot = torch.empty(T, world, dtype=torch.int32, device=device)
+            self.tok_counts, self.tok_base = _i32(world, device), _i32(world, device)
         if self.fp8:   # E4M3 codes + one fp32 scale per 128 channels
             self.recv_x = None
             self.recv_q = torch.empty(cap, d, dtype=torch.uint8, device=device)
@@ -71,14 +81,43 @@ class _RankState:
                       self.ws, stream)
         moe_dispatch(cfg, x, self.topk_idx, self.counts, self.offsets, self.send, self.send_tok,
                      self.perm, self.inv, None, self.ws, stream)
+        if self.dedup:
+            moe_ep_token_plan(cfg, self.world, self.topk_idx, self.tok_slot, self.tok_counts,
+                              stream)
+
+    def exchanged(self):
+        """What every rank sends in the all-gather: the per-expert copy counts
+        (and, deduplicating, the per-owner token counts), one int32 vector."""
+        return torch.cat([self.counts, self.tok_counts]) if self.dedup else self.counts
+
+    def plan(self, world, rank, gathered, stream):
+        """gathered [world, len(exchanged())]: every rank's exchanged vector."""
+        E = self.cfg.E
+        moe_ep_plan(self.cfg, world, rank, gathered[:, :E].contiguous(), self.base,
+                    self.local_offsets, stream)
+        if self.dedup:
+            moe_ep_token_base(self.cfg, world, rank, gathered[:, E:].contiguous(), self.tok_base,
+                              stream)
 
     def recv_buffers(self):
         """The buffers the dispatch writes into at this rank as an owner."""
+        if self.dedup:
+            return [self.recv_tok, self.recv_idx]
         return [self.recv_q, self.recv_scale] if self.fp8 else [self.recv_x]
+
+    def fanout(self, stream):
+        """Deduplicating: this owner's copy rows from its token rows."""
+        if self.dedup:
+            moe_ep_fanout(self.cfg, self.world, self.recv_tok, self.recv_idx, self.local_offsets,
+                          self.recv_x, self.status, stream)
 
     def dispatch(self, world, x, tables, stream):
         """tables: one device pointer table per entry of recv_buffers()."""
-        if self.fp8:
+        if self.dedup:
+            moe_ep_dispatch_dedup(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
+                                  self.base, self.tok_slot, self.tok_base, tables[0], tables[1],
+                                  self.status, stream)
+        elif self.fp8:
             moe_ep_dispatch_fp8(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
                                 self.base, tables[0], tables[1], self.status, stream)
         else:
@@ -117,7 +156,7 @@ class EmulatedEP:
     barriers between them."""
 
     def __init__(self, shape, inp: dict, world: int, router=None, token_ids=None, stream=None,
-                 payload=None):
+                 payload=None, dedup=False):
         self.device = inp["x"].device
         base_cfg = MoeConfig.of(shape, router=router)
         T = base_cfg.T
@@ -126,7 +165,7 @@ class EmulatedEP:
         Tr = T // world
         self.world, self.stream, self.inp = world, stream, inp
         self.cfg = MoeConfig.of(shape.replace(T=Tr), router=router, payload=payload)
-        self.ranks = [_RankState(self.cfg, world, self.device) for _ in range(world)]
+        self.ranks = [_RankState(self.cfg, world, self.device, dedup) for _ in range(world)]
         self.xs = [inp["x"][r * Tr:(r + 1) * Tr] for r in range(world)]
         self.ids = [None if token_ids is None else token_ids[r * Tr:(r + 1) * Tr]
                     for r in range(world)]
@@ -136,7 +175,8 @@ class EmulatedEP:
                             for i in range(n_buf)]
         self.recv_y_ptrs = torch.tensor([st.recv_y.data_ptr() for st in self.ranks],
                                         dtype=torch.int64, device=self.device)
-        self.counts_all = torch.empty(world, self.cfg.E, dtype=torch.int32, device=self.device)
+        n_ex = self.ranks[0].exchanged().numel()
+        self.gathered = torch.empty(world, n_ex, dtype=torch.int32, device=self.device)
 
     def route_and_plan_local(self):
         inp = self.inp
@@ -144,20 +184,27 @@ class EmulatedEP:
             st.route_and_plan_local(self.xs[r], inp["router_w"], inp.get("logit_offset"),
                                     inp["bias"], self.ids[r], self.stream)
 
+    @property
+    def counts_all(self):
+        return self.gathered[:, :self.cfg.E]
+
     def exchange_counts(self):
-        # the all-gather: row r of counts_all is rank r's counts
+        # the all-gather: row r is rank r's exchanged vector
         with torch.cuda.stream(self.stream or torch.cuda.current_stream(self.device)):
             for r, st in enumerate(self.ranks):
-                self.counts_all[r].copy_(st.counts)
+                self.gathered[r].copy_(st.exchanged())
 
     def plan(self):
         for r, st in enumerate(self.ranks):
-            moe_ep_plan(self.cfg, self.world, r, self.counts_all, st.base, st.local_offsets,
-                        self.stream)
+            st.plan(self.world, r, self.gathered, self.stream)
 
     def dispatch(self):
         for r, st in enumerate(self.ranks):
             st.dispatch(self.world, self.xs[r], self.recv_tables, self.stream)
+
+    def fanout(self):
+        for st in self.ranks:
+            st.fanout(self.stream)
 
     def expert_ffn(self):
         inp, world = self.inp, self.world
@@ -177,16 +224,17 @@ class EmulatedEP:
         self.exchange_counts()
         self.plan()
         self.dispatch()
+        self.fanout()
         self.expert_ffn()
         self.combine()
         return torch.cat([st.out for st in self.ranks])
 
 
 def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, stream=None,
-                    payload=None):
+                    payload=None, dedup=False):
     """One EP step of all `world` ranks on this GPU; returns (out [T, d],
     per-rank states)."""
-    em = EmulatedEP(shape, inp, world, router, token_ids, stream, payload)
+    em = EmulatedEP(shape, inp, world, router, token_ids, stream, payload, dedup)
     return em.forward(), em.ranks
 
 
@@ -205,7 +253,7 @@ class EPLayer:
 
     def __init__(self, shape_local, group, router_w, bias, w_gate_local, w_up_local,
                  w_down_local, ws_gate=None, ws_up=None, ws_down=None, logit_offset=None,
-                 router=None, payload=None):
+                 router=None, payload=None, dedup=False):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -214,7 +262,7 @@ class EPLayer:
         self.device = w_gate_local.device
         self.host_sync = dist.get_backend(group) != "nccl"
         self.cfg = MoeConfig.of(shape_local, router=router, payload=payload)
-        self.st = _RankState(self.cfg, self.world, self.device)
+        self.st = _RankState(self.cfg, self.world, self.device, dedup)
         self.router_w, self.bias, self.logit_offset = router_w, bias, logit_offset
         self.w = (w_gate_local, w_up_local, w_down_local)
         self.ws_shared = (ws_gate, ws_up, ws_down)
@@ -246,7 +294,7 @@ class EPLayer:
         else:
             self.dist.all_reduce(self._flag, group=self.group)
 
-    def _gather_counts(self, counts, stream):
+    def _gather(self, counts, stream):
         if self.host_sync:
             stream.synchronize()
             return gather_counts(counts.cpu(), self.group).to(self.device)
@@ -259,11 +307,11 @@ class EPLayer:
         s = stream or torch.cuda.current_stream(self.device)
         with torch.cuda.stream(s):   # the collectives order against this stream
             st.route_and_plan_local(x, self.router_w, self.logit_offset, self.bias, token_ids, s)
-            counts_all = self._gather_counts(st.counts, s)
-            moe_ep_plan(cfg, world, r, counts_all, st.base, st.local_offsets, s)
+            st.plan(world, r, self._gather(st.exchanged(), s), s)
             self._barrier(s)          # every rank's receive buffers are free again
             st.dispatch(world, x, self.recv_tables, s)
             self._barrier(s)          # every copy has landed
+            st.fanout(s)
             st.expert_ffn(world, r, self.w, x, self.ws_shared, s)
             self._barrier(s)          # every expert output is written
             moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,

@@ -435,6 +435,46 @@ MOE_API moe_status moe_ep_expert_ffn_fp8(const moe_config *cfg, int32_t world, i
                                          const void *ws_down, void *y_shared, void *ws,
                                          size_t ws_bytes, void *stream);
 
+/* Deduplicated dispatch: with node-limited routing a token's row needs to
+ * reach each owner holding one of its experts once ("moe-node-limited-
+ * routing": the node limit bounds the nodes a token's activations reach; the
+ * single-GPU send_tok matrix counts these pairs), then fans out to its
+ * experts there.  Steps of a rank, replacing moe_ep_dispatch:
+ *   moe_ep_token_plan  (local)  tok_slot [T, world] int32 out: position of
+ *                      token t among this rank's tokens with an expert at
+ *                      owner o (token order), -1 if none; tok_counts [world]
+ *                      int32 out: this rank's tokens per owner
+ *   (caller) all-gather tok_counts into tok_counts_all [world, world]
+ *   moe_ep_token_base  tok_base [world] int32 out: this rank's first row in
+ *                      each owner's token buffer (sum over lower ranks)
+ *   moe_ep_dispatch_dedup  one store of each token row per owner into
+ *                      recv_tok[o] (rows: rank 0's tokens, then rank 1's,
+ *                      each in token order; capacity world * T rows of d
+ *                      bf16) and, per copy (t, j), the 4-byte token row into
+ *                      recv_idx[o][copy row] (capacity world * T * K int32);
+ *                      recv_tok / recv_idx: device arrays of `world` pointers
+ *   barrier, then at every owner: moe_ep_fanout  recv_x[r] = recv_tok
+ *                      [recv_idx[r]] for its local_offsets[E/world] rows
+ * recv_x then holds exactly what moe_ep_dispatch writes, so the rest of the
+ * step (moe_ep_expert_ffn, moe_ep_combine) is unchanged and the layer's
+ * output is the same bit for bit.  Rows or slots outside the buffers are
+ * skipped and flagged MOE_ERR_DEVICE_FAULT in *device_status (may be NULL). */
+MOE_API moe_status moe_ep_token_plan(const moe_config *cfg, int32_t world,
+                                     const int32_t *topk_idx, int32_t *tok_slot,
+                                     int32_t *tok_counts, void *stream);
+MOE_API moe_status moe_ep_token_base(const moe_config *cfg, int32_t world, int32_t rank,
+                                     const int32_t *tok_counts_all, int32_t *tok_base,
+                                     void *stream);
+MOE_API moe_status moe_ep_dispatch_dedup(const moe_config *cfg, int32_t world, const void *x,
+                                         const int32_t *topk_idx, const int32_t *offsets,
+                                         const int32_t *inv_perm, const int32_t *base,
+                                         const int32_t *tok_slot, const int32_t *tok_base,
+                                         void *const *recv_tok, int32_t *const *recv_idx,
+                                         int32_t *device_status, void *stream);
+MOE_API moe_status moe_ep_fanout(const moe_config *cfg, int32_t world, const void *recv_tok,
+                                 const int32_t *recv_idx, const int32_t *local_offsets,
+                                 void *recv_x, int32_t *device_status, void *stream);
+
 /* Combine fused with its all-to-all: out[t] = y_shared[t] + sum_j topk_w[t][j]
  * * (row of copy (t, j) in recv_y[owner]), fp32 multiply-adds in slot order,
  * bf16 out [T, d].  recv_y: device array of `world` device pointers. */

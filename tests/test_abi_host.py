@@ -238,6 +238,20 @@ def test_expert_parallel_validates_before_cuda(moe):
     bad = list(c_args)
     bad[6] = P(fake + 2)                       # misaligned y_shared
     assert lib.moe_ep_combine(c, 2, *bad, P(fake), None, None) == INV
+    assert lib.moe_ep_token_plan(c, 3, P(fake), P(fake), P(fake), None) == UNS
+    assert lib.moe_ep_token_plan(c, 2, None, P(fake), P(fake), None) == INV
+    assert lib.moe_ep_token_base(c, 2, 2, P(fake), P(fake), None) == UNS
+    assert lib.moe_ep_token_base(c, 2, 0, P(fake), None, None) == INV
+    dd_args = [P(fake)] * 9                    # x .. tok_base, recv_tok, recv_idx
+    bad = list(dd_args)
+    bad[8] = None                              # recv_idx
+    assert lib.moe_ep_dispatch_dedup(c, 2, *bad, None, None) == INV
+    bad = list(dd_args)
+    bad[0] = P(fake + 8)                       # misaligned x
+    assert lib.moe_ep_dispatch_dedup(c, 2, *bad, None, None) == INV
+    assert lib.moe_ep_fanout(c, 2, P(fake), P(fake), None, P(fake), None, None) == INV
+    assert lib.moe_ep_fanout(c, 2, P(fake + 4), P(fake), P(fake), P(fake), None, None) == INV
+    assert lib.moe_ep_fanout(c, 3, P(fake), P(fake), P(fake), P(fake), None, None) == UNS
     assert lib.moe_ipc_get_handle(None, P(fake)) == INV
     assert lib.moe_ipc_open_handle(None, P(fake)) == INV
     assert lib.moe_ipc_close_handle(None) == INV

@@ -223,3 +223,32 @@ def test_emulated_ep_maximum_world(orc):
         assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
     frob, elem = H.compare_out(out[torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
     assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
+@pytest.mark.parametrize("name,world", [("ragged", 2), ("noshared", 4), ("ragged2", 5),
+                                        ("ragged", 3)])
+def test_emulated_ep_dedup_dispatch(orc, name, world):
+    """One row per (token, owner) and a fan-out index per copy: the token
+    plans and bases equal the oracle's bit for bit, every owner's fanned-out
+    rows equal what the per-copy dispatch stores, and the layer equals
+    moe_forward bit for bit."""
+    sh = H.shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    ref = _forward(sh, inp)
+    out, ranks = ep.emulate_forward(sh, inp, world, dedup=True)
+    _, plain = ep.emulate_forward(sh, inp, world)
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+        assert moe.moe_read_device_status(st.ws) == moe.MOE_OK
+    assert torch.equal(out.view(torch.int16), ref["out"].view(torch.int16))
+    plans = [orc.ep_token_plan(st.topk_idx.cpu().numpy(), sh.E, world) for st in ranks]
+    tok_counts_all = np.stack([p[1] for p in plans])
+    tok_base = orc.ep_token_base(tok_counts_all)
+    El = sh.E // world
+    for r, st in enumerate(ranks):
+        np.testing.assert_array_equal(st.tok_slot.cpu().numpy(), plans[r][0])
+        np.testing.assert_array_equal(st.tok_counts.cpu().numpy(), plans[r][1])
+        np.testing.assert_array_equal(st.tok_base.cpu().numpy(), tok_base[r])
+        n = int(st.local_offsets[El].item())
+        assert torch.equal(st.recv_x[:n].view(torch.int16), plain[r].recv_x[:n].view(torch.int16))

@@ -29,7 +29,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, name, payload, q):
+def _rank_main(rank, world, port, name, payload, dedup, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -47,7 +47,8 @@ def _rank_main(rank, world, port, name, payload, q):
         sl = slice(rank * El, (rank + 1) * El)
         layer = EPLayer(sh.replace(T=Tr), None, inp["router_w"], inp["bias"], inp["w_gate"][sl],
                         inp["w_up"][sl], inp["w_down"][sl], inp.get("ws_gate"), inp.get("ws_up"),
-                        inp.get("ws_down"), logit_offset=inp.get("logit_offset"), payload=payload)
+                        inp.get("ws_down"), logit_offset=inp.get("logit_offset"), payload=payload,
+                        dedup=dedup)
         x = inp["x"][rank * Tr:(rank + 1) * Tr]
         outs = []
         for _ in range(2):
@@ -65,16 +66,18 @@ def _rank_main(rank, world, port, name, payload, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("name,world,payload", [("ragged", 2, 0), ("ragged", 3, 0),
-                                                ("noshared", 2, 1)])
-def test_ep_layer_processes_on_one_gpu_equal_single_gpu_forward(name, world, payload):
+@pytest.mark.parametrize("name,world,payload,dedup", [("ragged", 2, 0, False),
+                                                      ("ragged", 3, 0, False),
+                                                      ("noshared", 2, 1, False),
+                                                      ("ragged", 3, 0, True)])
+def test_ep_layer_processes_on_one_gpu_equal_single_gpu_forward(name, world, payload, dedup):
     import synth
     from tests import harness as H
     import combine_expert_ffn_b200 as moe
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, name, payload, q))
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, name, payload, dedup, q))
              for r in range(world)]
     for p in procs:
         p.start()
