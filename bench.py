@@ -609,11 +609,12 @@ def ep_leg(sh, inp, dev, stream, world, reps=20):
     # one of its experts, plus a 4-byte fan-out index per copy; the owner
     # rebuilds its copy rows locally
     torch.cuda.empty_cache()
-    em = ep.EmulatedEP(sh, inp, world, stream=stream, dedup=True)
+    em = ep.EmulatedEP(sh, inp, world, stream=stream, dedup=True, dedup_combine=True)
     em.forward()
     torch.cuda.synchronize(dev)
-    graphs = {k: graphed(k) for k in ("dispatch", "fanout")}
-    td = {k: timed(graphs[k].replay) / world for k in ("dispatch", "fanout")}
+    dd_stages = ("dispatch", "fanout", "precombine", "combine")
+    graphs = {k: graphed(k) for k in dd_stages}
+    td = {k: timed(graphs[k].replay) / world for k in dd_stages}
     for st in em.ranks:
         if int(st.status.item()) != moe.MOE_OK or moe.moe_read_device_status(st.ws) != moe.MOE_OK:
             raise RuntimeError("device status after the emulated deduplicated dispatch")
@@ -626,6 +627,7 @@ def ep_leg(sh, inp, dev, stream, world, reps=20):
     mean_tok_rows = float(tca.sum()) / world
     dd_bytes = 2.0 * d * (Tr + mean_tok_rows) + 12.0 * K * Tr   # x read, token rows, indices
     fan_bytes = 4.0 * d * (Tr * K) + 4.0 * Tr * K               # copy rows read + written
+    dd_comb_link = 2.0 * d * max(max(tok_out), max(tok_in))     # one partial row per pair
     res["dedup_dispatch"] = {
         "stage_ms_per_rank": td,
         "token_rows_per_rank": mean_tok_rows,
@@ -637,7 +639,11 @@ def ep_leg(sh, inp, dev, stream, world, reps=20):
                    "frac_of_hbm": fan_bytes / (td["fanout"] / 1e3) / 1e9 / hbm},
         "nvlink": {"max_rank_bytes_dispatch": dd_link,
                    "projected_ms_dispatch": dd_link / (NVLINK_GBS * 1e9) * 1e3,
+                   "max_rank_bytes_combine": dd_comb_link,
+                   "projected_ms_combine": dd_comb_link / (NVLINK_GBS * 1e9) * 1e3,
                    "tokens_out": tok_out, "tokens_in": tok_in},
+        "note": "dispatch stage includes the combine's list plan; combine = one partial row "
+                "per (token, owner), summed by the owner (precombine) before the exchange",
     }
     del em
     if sh.d % 128 == 0:

@@ -38,7 +38,8 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_expert_ffn_fp8", "moe_permute", "moe_ep_workspace_size", "moe_ep_plan",
            "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_dispatch_fp8",
            "moe_ep_expert_ffn_fp8", "moe_ep_token_plan", "moe_ep_token_base",
-           "moe_ep_dispatch_dedup", "moe_ep_fanout", "moe_ipc_get_handle",
+           "moe_ep_dispatch_dedup", "moe_ep_fanout", "moe_ep_combine_plan",
+           "moe_ep_precombine", "moe_ep_combine_dedup", "moe_ipc_get_handle",
            "moe_ipc_open_handle", "moe_ipc_close_handle")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
@@ -101,6 +102,9 @@ _sig = {
     "moe_ep_token_base": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P]),
     "moe_ep_dispatch_dedup": (C.c_int, [_CP, C.c_int32] + [_P] * 11),
     "moe_ep_fanout": (C.c_int, [_CP, C.c_int32] + [_P] * 6),
+    "moe_ep_combine_plan": (C.c_int, [_CP, C.c_int32] + [_P] * 12),
+    "moe_ep_precombine": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
+    "moe_ep_combine_dedup": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
     "moe_ep_dispatch_fp8": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_ep_expert_ffn_fp8": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P, _P, _P, _P, _P,
                                         _P, _P, _P, _P, _P, _P, _S, _P]),
@@ -301,6 +305,31 @@ def moe_ep_fanout(cfg, world, recv_tok, recv_idx, local_offsets, recv_x, device_
         _lib.moe_ep_fanout(_cfg(cfg), int(world), _ptr(recv_tok), _ptr(recv_idx),
                            _ptr(local_offsets), _ptr(recv_x), _ptr(device_status),
                            _stream(stream)))
+
+
+def moe_ep_combine_plan(cfg, world, topk_idx, topk_w, offsets, inv_perm, base, tok_slot, tok_base,
+                        list_ptrs, lw_ptrs, lcnt_ptrs, device_status=None, stream=None) -> None:
+    _ok("moe_ep_combine_plan",
+        _lib.moe_ep_combine_plan(_cfg(cfg), int(world), _ptr(topk_idx), _ptr(topk_w),
+                                 _ptr(offsets), _ptr(inv_perm), _ptr(base), _ptr(tok_slot),
+                                 _ptr(tok_base), _ptr(list_ptrs), _ptr(lw_ptrs), _ptr(lcnt_ptrs),
+                                 _ptr(device_status), _stream(stream)))
+
+
+def moe_ep_precombine(cfg, world, recv_y, lst, lw, lcnt, tok_base, partial, device_status=None,
+                      stream=None) -> None:
+    _ok("moe_ep_precombine",
+        _lib.moe_ep_precombine(_cfg(cfg), int(world), _ptr(recv_y), _ptr(lst), _ptr(lw),
+                               _ptr(lcnt), _ptr(tok_base), _ptr(partial), _ptr(device_status),
+                               _stream(stream)))
+
+
+def moe_ep_combine_dedup(cfg, world, topk_idx, tok_slot, tok_base, partial_ptrs, y_shared, out,
+                         device_status=None, stream=None) -> None:
+    _ok("moe_ep_combine_dedup",
+        _lib.moe_ep_combine_dedup(_cfg(cfg), int(world), _ptr(topk_idx), _ptr(tok_slot),
+                                  _ptr(tok_base), _ptr(partial_ptrs), _ptr(y_shared), _ptr(out),
+                                  _ptr(device_status), _stream(stream)))
 
 
 def moe_ep_dispatch_fp8(cfg, world, x, topk_idx, offsets, inv_perm, base, recv_q_ptrs,

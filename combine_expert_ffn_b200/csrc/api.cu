@@ -618,6 +618,59 @@ moe_status moe_ep_fanout(const moe_config *c, int32_t world, const void *recv_to
                                         as_stream(stream)));
 }
 
+moe_status moe_ep_combine_plan(const moe_config *c, int32_t world, const int32_t *topk_idx,
+                               const float *topk_w, const int32_t *offsets,
+                               const int32_t *inv_perm, const int32_t *base,
+                               const int32_t *tok_slot, const int32_t *tok_base,
+                               int32_t *const *list, float *const *lw, int32_t *const *lcnt,
+                               int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!topk_idx || !topk_w || !offsets || !inv_perm || !base || !tok_slot ||
+                     !tok_base || !list || !lw || !lcnt))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t tok_rows = (int64_t)world * c->T;
+    return cuda_status(launch_ep_combine_plan(topk_idx, topk_w, offsets, inv_perm, base, tok_slot,
+                                              tok_base, list, lw, lcnt, tok_rows,
+                                              tok_rows * c->K, c->T, c->E, c->K, world,
+                                              device_status, as_stream(stream)));
+}
+
+moe_status moe_ep_precombine(const moe_config *c, int32_t world, const void *recv_y,
+                             const int32_t *list, const float *lw, const int32_t *lcnt,
+                             const int32_t *tok_base, void *partial, int32_t *device_status,
+                             void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!recv_y || !list || !lw || !lcnt || !tok_base || !partial))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(recv_y) || !aligned16(partial)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t tok_rows = (int64_t)world * c->T;
+    return cuda_status(launch_ep_precombine(recv_y, list, lw, lcnt, tok_base, world, tok_rows,
+                                            tok_rows * c->K, c->d, c->K, partial, device_status,
+                                            as_stream(stream)));
+}
+
+moe_status moe_ep_combine_dedup(const moe_config *c, int32_t world, const int32_t *topk_idx,
+                                const int32_t *tok_slot, const int32_t *tok_base,
+                                const void *const *partial, const void *y_shared, void *out,
+                                int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!topk_idx || !tok_slot || !tok_base || !partial || !out))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_shared) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_ep_combine_dedup(topk_idx, tok_slot, tok_base, partial, y_shared,
+                                               (int64_t)world * c->T, c->T, c->d, c->E, c->K,
+                                               world, out, device_status, as_stream(stream)));
+}
+
 namespace {
 // the expert FFN of one rank's experts over its receive buffer: bf16 rows
 // (recv_x) or FP8 codes + scales (recv_q, recv_scale)

@@ -227,14 +227,20 @@ ep_token_plan_kernel(const int32_t *__restrict__ topk_idx, int T, int K, int E, 
     if (threadIdx.x == 0) tok_counts[o] = carry_s;
 }
 
-// tok_base[o] = sum over ranks r < me of tok_counts_all[r][o]
+// tok_base[o] = sum over ranks r < me of tok_counts_all[r][o]; tok_base[world]
+// = the token rows this rank receives as an owner
 __global__ void ep_token_base_kernel(const int32_t *__restrict__ tok_counts_all, int world, int me,
                                      int32_t *__restrict__ tok_base) {
     const int o = threadIdx.x;
-    if (o >= world) return;
-    int s = 0;
-    for (int r = 0; r < me; ++r) s += tok_counts_all[r * world + o];
-    tok_base[o] = s;
+    if (o < world) {
+        int s = 0;
+        for (int r = 0; r < me; ++r) s += tok_counts_all[r * world + o];
+        tok_base[o] = s;
+    } else if (o == world) {
+        int s = 0;
+        for (int r = 0; r < world; ++r) s += tok_counts_all[r * world + me];
+        tok_base[world] = s;
+    }
 }
 
 // Thread per 16-byte chunk of an x row: one store per (token, owner) of the
@@ -311,6 +317,184 @@ ep_dispatch_dedup_kernel(const uint4 *__restrict__ x, const int32_t *__restrict_
     }
 }
 
+__device__ __forceinline__ void ep_acc_row(float (&acc)[8], float wj, const uint4 &v) {
+    acc[0] = fmaf(wj, bf16_lo(v.x), acc[0]); acc[1] = fmaf(wj, bf16_hi(v.x), acc[1]);
+    acc[2] = fmaf(wj, bf16_lo(v.y), acc[2]); acc[3] = fmaf(wj, bf16_hi(v.y), acc[3]);
+    acc[4] = fmaf(wj, bf16_lo(v.z), acc[4]); acc[5] = fmaf(wj, bf16_hi(v.z), acc[5]);
+    acc[6] = fmaf(wj, bf16_lo(v.w), acc[6]); acc[7] = fmaf(wj, bf16_hi(v.w), acc[7]);
+}
+
+// Deduplicated combine, source side, before the exchange: for every token t
+// and owner o holding cnt of its copies, the owner's list entry of token row
+// trow = tok_base[o] + tok_slot[t][o]: copy rows and gates of those copies in
+// slot order (list[trow * K + k], lw[trow * K + k], k < cnt = lcnt[trow]).
+// Thread per token.
+__global__ void __launch_bounds__(256)
+ep_combine_plan_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
+                       const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
+                       const int32_t *__restrict__ base, const int32_t *__restrict__ tok_slot,
+                       const int32_t *__restrict__ tok_base, int32_t *const *__restrict__ list,
+                       float *const *__restrict__ lw, int32_t *const *__restrict__ lcnt,
+                       int64_t tok_rows, int64_t recv_rows, int T, int E, int K, int El, int world,
+                       int32_t *status) {
+    __shared__ int32_t delta_s[EP_MAX_E];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) delta_s[e] = base[e] - offsets[e];
+    __syncthreads();
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    const int32_t *idx_t = topk_idx + (int64_t)t * K;
+    for (int j = 0; j < K; ++j) {
+        const int e = idx_t[j];
+        if (e < 0 || e >= E) continue;  // flagged by the local dispatch plan
+        const int o = e / El;
+        int k = 0, cnt = 0;  // earlier slots at o; all slots at o
+        for (int q = 0; q < K; ++q) {
+            const int eq = idx_t[q];
+            if (eq >= 0 && eq < E && eq / El == o) {
+                if (q < j) ++k;
+                ++cnt;
+            }
+        }
+        const int slot = tok_slot[(int64_t)t * world + o];
+        const int64_t trow = (int64_t)tok_base[o] + slot;
+        const int64_t row = (int64_t)delta_s[e] + inv_perm[(int64_t)t * K + j];
+        if (slot < 0 || trow >= tok_rows || row < 0 || row >= recv_rows) {
+            if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+            continue;
+        }
+        list[o][trow * K + k] = (int32_t)row;
+        lw[o][trow * K + k] = topk_w[(int64_t)t * K + j];
+        if (k == 0) lcnt[o][trow] = cnt;
+    }
+}
+
+// Deduplicated combine, owner side: partial[trow] = bf16(sum over k < cnt of
+// lw[k] * recv_y[list[k]]), fp32 multiply-adds in slot order, for the token
+// rows this rank received (tok_base[world] of them).
+__global__ void __launch_bounds__(256, 4)
+ep_precombine_kernel(const uint4 *__restrict__ recv_y, const int32_t *__restrict__ list,
+                     const float *__restrict__ lw, const int32_t *__restrict__ lcnt,
+                     const int32_t *__restrict__ tok_base, int world, int64_t tok_rows,
+                     int64_t recv_rows, int chunks, int K, uint4 *__restrict__ partial,
+                     int32_t *status) {
+    int64_t n = tok_base[world];
+    if (n < 0 || n > tok_rows) {
+        if (status && blockIdx.x == 0 && threadIdx.x == 0) record_status(status, MOE_ERR_DEVICE_FAULT);
+        n = n < 0 ? 0 : tok_rows;
+    }
+    const int64_t total = n * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tr = i / chunks;
+        const int c = (int)(i - tr * chunks);
+        int cnt = __ldg(lcnt + tr);
+        if (cnt < 1 || cnt > K) {
+            if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+            cnt = 0;
+        }
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        for (int k0 = 0; k0 < cnt; k0 += 8) {
+            uint4 rows[8];
+            float w[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int k = k0 + q;
+                rows[q] = make_uint4(0u, 0u, 0u, 0u);
+                w[q] = 0.f;
+                if (k >= cnt) continue;
+                const int64_t row = __ldg(list + tr * K + k);
+                w[q] = __ldg(lw + tr * K + k);
+                if (row < 0 || row >= recv_rows) {
+                    if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                    continue;
+                }
+                rows[q] = __ldg(recv_y + row * chunks + c);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (k0 + q < cnt) ep_acc_row(acc, w[q], rows[q]);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        partial[i] = o;
+    }
+}
+
+// Deduplicated combine, source side, after the exchange: out[t] = y_shared[t]
+// + the partial rows of t's owners (one peer load per owner), added in fp32 in
+// the order of each owner's first slot.
+__global__ void __launch_bounds__(256, 4)
+ep_combine_dedup_kernel(const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ tok_slot,
+                        const int32_t *__restrict__ tok_base,
+                        const uint4 *const *__restrict__ partial, const uint4 *__restrict__ y_shared,
+                        int64_t tok_rows, int T, int chunks, int E, int K, int El, int world,
+                        uint4 *__restrict__ out, int32_t *status) {
+    __shared__ int32_t tokbase_s[EP_MAX_WORLD];
+    __shared__ const uint4 *tab_s[EP_MAX_WORLD];
+    for (int o = threadIdx.x; o < world; o += blockDim.x) {
+        tokbase_s[o] = tok_base[o];
+        tab_s[o] = partial[o];
+    }
+    __syncthreads();
+    const int64_t total = (int64_t)T * chunks;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        float acc[8];
+        if (y_shared) {
+            const uint4 v = __ldg(y_shared + i);
+            acc[0] = bf16_lo(v.x); acc[1] = bf16_hi(v.x);
+            acc[2] = bf16_lo(v.y); acc[3] = bf16_hi(v.y);
+            acc[4] = bf16_lo(v.z); acc[5] = bf16_hi(v.z);
+            acc[6] = bf16_lo(v.w); acc[7] = bf16_hi(v.w);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        }
+        const int32_t *idx_t = topk_idx + t * K;
+        uint64_t seen = 0;
+        for (int j0 = 0; j0 < K; j0 += 8) {
+            uint4 rows[8];
+            bool use[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int j = j0 + q;
+                rows[q] = make_uint4(0u, 0u, 0u, 0u);
+                use[q] = false;
+                if (j >= K) continue;
+                const int e = __ldg(idx_t + j);
+                if (e < 0 || e >= E) continue;
+                const int o = e / El;
+                if ((seen >> o) & 1ull) continue;  // this owner's partial is counted once
+                seen |= 1ull << o;
+                const int slot = __ldg(tok_slot + t * world + o);
+                const int64_t trow = (int64_t)tokbase_s[o] + slot;
+                if (slot < 0 || trow >= tok_rows) {
+                    if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                    continue;
+                }
+                rows[q] = tab_s[o][trow * chunks + c];
+                use[q] = true;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (use[q]) ep_acc_row(acc, 1.0f, rows[q]);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        out[i] = o;
+    }
+}
+
 // The owner's fan-out: recv_x[r] = recv_tok[recv_idx[r]] for the rows it
 // received (local_offsets[El] of them).
 __global__ void __launch_bounds__(256, 4)
@@ -336,12 +520,6 @@ ep_fanout_kernel(const uint4 *__restrict__ recv_tok, const int32_t *__restrict__
     }
 }
 
-__device__ __forceinline__ void ep_acc_row(float (&acc)[8], float wj, const uint4 &v) {
-    acc[0] = fmaf(wj, bf16_lo(v.x), acc[0]); acc[1] = fmaf(wj, bf16_hi(v.x), acc[1]);
-    acc[2] = fmaf(wj, bf16_lo(v.y), acc[2]); acc[3] = fmaf(wj, bf16_hi(v.y), acc[3]);
-    acc[4] = fmaf(wj, bf16_lo(v.z), acc[4]); acc[5] = fmaf(wj, bf16_hi(v.z), acc[5]);
-    acc[6] = fmaf(wj, bf16_lo(v.w), acc[6]); acc[7] = fmaf(wj, bf16_hi(v.w), acc[7]);
-}
 
 __global__ void __launch_bounds__(256, 4)
 ep_combine_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
@@ -459,7 +637,7 @@ cudaError_t launch_ep_token_plan(const int32_t *topk_idx, int T, int E, int K, i
 
 cudaError_t launch_ep_token_base(const int32_t *tok_counts_all, int world, int me,
                                  int32_t *tok_base, cudaStream_t st) {
-    ep_token_base_kernel<<<1, 64, 0, st>>>(tok_counts_all, world, me, tok_base);
+    ep_token_base_kernel<<<1, 96, 0, st>>>(tok_counts_all, world, me, tok_base);
     count_launch();
     return cudaGetLastError();
 }
@@ -489,6 +667,49 @@ cudaError_t launch_ep_fanout(const void *recv_tok, const int32_t *recv_idx,
     ep_fanout_kernel<<<grid_for(recv_rows * chunks), 256, 0, st>>>(
         static_cast<const uint4 *>(recv_tok), recv_idx, local_offsets, El, tok_rows, recv_rows,
         chunks, static_cast<uint4 *>(recv_x), status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_combine_plan(const int32_t *topk_idx, const float *topk_w,
+                                   const int32_t *offsets, const int32_t *inv_perm,
+                                   const int32_t *base, const int32_t *tok_slot,
+                                   const int32_t *tok_base, int32_t *const *list,
+                                   float *const *lw, int32_t *const *lcnt, int64_t tok_rows,
+                                   int64_t recv_rows, int T, int E, int K, int world,
+                                   int32_t *status, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    ep_combine_plan_kernel<<<(T + 255) / 256, 256, 0, st>>>(
+        topk_idx, topk_w, offsets, inv_perm, base, tok_slot, tok_base, list, lw, lcnt, tok_rows,
+        recv_rows, T, E, K, E / world, world, status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_precombine(const void *recv_y, const int32_t *list, const float *lw,
+                                 const int32_t *lcnt, const int32_t *tok_base, int world,
+                                 int64_t tok_rows, int64_t recv_rows, int d, int K, void *partial,
+                                 int32_t *status, cudaStream_t st) {
+    if (tok_rows == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_precombine_kernel<<<grid_for(tok_rows * chunks), 256, 0, st>>>(
+        static_cast<const uint4 *>(recv_y), list, lw, lcnt, tok_base, world, tok_rows, recv_rows,
+        chunks, K, static_cast<uint4 *>(partial), status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_combine_dedup(const int32_t *topk_idx, const int32_t *tok_slot,
+                                    const int32_t *tok_base, const void *const *partial,
+                                    const void *y_shared, int64_t tok_rows, int T, int d, int E,
+                                    int K, int world, void *out, int32_t *status,
+                                    cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_combine_dedup_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
+        topk_idx, tok_slot, tok_base, reinterpret_cast<const uint4 *const *>(partial),
+        static_cast<const uint4 *>(y_shared), tok_rows, T, chunks, E, K, E / world, world,
+        static_cast<uint4 *>(out), status);
     count_launch();
     return cudaGetLastError();
 }

@@ -77,6 +77,22 @@ cudaError_t launch_ep_fanout(const void *recv_tok, const int32_t *recv_idx,
                              const int32_t *local_offsets, int El, int64_t tok_rows,
                              int64_t recv_rows, int d, void *recv_x, int32_t *status,
                              cudaStream_t st);
+cudaError_t launch_ep_combine_plan(const int32_t *topk_idx, const float *topk_w,
+                                   const int32_t *offsets, const int32_t *inv_perm,
+                                   const int32_t *base, const int32_t *tok_slot,
+                                   const int32_t *tok_base, int32_t *const *list,
+                                   float *const *lw, int32_t *const *lcnt, int64_t tok_rows,
+                                   int64_t recv_rows, int T, int E, int K, int world,
+                                   int32_t *status, cudaStream_t st);
+cudaError_t launch_ep_precombine(const void *recv_y, const int32_t *list, const float *lw,
+                                 const int32_t *lcnt, const int32_t *tok_base, int world,
+                                 int64_t tok_rows, int64_t recv_rows, int d, int K, void *partial,
+                                 int32_t *status, cudaStream_t st);
+cudaError_t launch_ep_combine_dedup(const int32_t *topk_idx, const int32_t *tok_slot,
+                                    const int32_t *tok_base, const void *const *partial,
+                                    const void *y_shared, int64_t tok_rows, int T, int d, int E,
+                                    int K, int world, void *out, int32_t *status,
+                                    cudaStream_t st);
 cudaError_t launch_ep_combine(const int32_t *topk_idx, const float *topk_w, const int32_t *offsets,
                               const int32_t *inv_perm, const int32_t *base,
                               const void *const *recv_y, int64_t recv_rows, const void *y_shared,

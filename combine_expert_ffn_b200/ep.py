@@ -25,8 +25,10 @@ from __future__ import annotations
 
 import torch
 
-from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_dispatch, moe_ep_dispatch_dedup,
+from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_combine_dedup,
+               moe_ep_combine_plan, moe_ep_dispatch, moe_ep_dispatch_dedup,
                moe_ep_dispatch_fp8, moe_ep_expert_ffn, moe_ep_expert_ffn_fp8, moe_ep_fanout,
+               moe_ep_precombine,
                moe_ep_plan, moe_ep_token_base, moe_ep_token_plan, moe_ep_workspace_size,
                moe_ipc_close_handle, moe_ipc_get_handle, moe_ipc_open_handle, moe_route,
                moe_route_hash, MOE_PAYLOAD_FP8, MOE_ROUTER_HASH)
@@ -39,9 +41,12 @@ def _i32(n, device):
 class _RankState:
     """Per-rank buffers of one EP step."""
 
-    def __init__(self, cfg: MoeConfig, world: int, device, dedup: bool = False):
+    def __init__(self, cfg: MoeConfig, world: int, device, dedup: bool = False,
+                 dedup_combine: bool = False):
         T, K, E, G, d = cfg.T, cfg.K, cfg.E, cfg.G, cfg.d
-        self.cfg, self.world, self.dedup = cfg, world, dedup
+        if dedup_combine and not dedup:
+            raise ValueError("the deduplicated combine runs on the deduplicated dispatch")
+        self.cfg, self.world, self.dedup, self.dedup_combine = cfg, world, dedup, dedup_combine
         self.topk_idx = torch.empty(T, K, dtype=torch.int32, device=device)
         self.topk_w = torch.empty(T, K, dtype=torch.float32, device=device)
         self.counts, self.offsets = _i32(E, device), _i32(E + 1, device)
@@ -57,7 +62,12 @@ class _RankState:
             self.recv_tok = torch.empty(world * T, d, dtype=torch.bfloat16, device=device)
             self.recv_idx = torch.empty(cap, dtype=torch.int32, device=device)
             self.tok_slot = torch.empty(T, world, dtype=torch.int32, device=device)
-            self.tok_counts, self.tok_base = _i32(world, device), _i32(world, device)
+            self.tok_counts, self.tok_base = _i32(world, device), _i32(world + 1, device)
+        if dedup_combine:  # per (token, owner): copy rows + gates; one partial row back
+            self.recv_list = _i32(world * T * K, device)
+            self.recv_lw = torch.empty(world * T * K, dtype=torch.float32, device=device)
+            self.recv_lcnt = _i32(world * T, device)
+            self.partial = torch.empty(world * T, d, dtype=torch.bfloat16, device=device)
         if self.fp8:   # E4M3 codes + one fp32 scale per 128 channels
             self.recv_x = None
             self.recv_q = torch.empty(cap, d, dtype=torch.uint8, device=device)
@@ -102,8 +112,29 @@ class _RankState:
     def recv_buffers(self):
         """The buffers the dispatch writes into at this rank as an owner."""
         if self.dedup:
-            return [self.recv_tok, self.recv_idx]
+            extra = [self.recv_list, self.recv_lw, self.recv_lcnt] if self.dedup_combine else []
+            return [self.recv_tok, self.recv_idx] + extra
         return [self.recv_q, self.recv_scale] if self.fp8 else [self.recv_x]
+
+    def combine_buffer(self):
+        """The buffer the other ranks' combines read at this rank."""
+        return self.partial if self.dedup_combine else self.recv_y
+
+    def precombine(self, stream):
+        """Deduplicated combine: this owner's partial rows."""
+        if self.dedup_combine:
+            moe_ep_precombine(self.cfg, self.world, self.recv_y, self.recv_list, self.recv_lw,
+                              self.recv_lcnt, self.tok_base, self.partial, self.status, stream)
+
+    def combine(self, world, table, stream):
+        """table: device pointer table of the ranks' combine_buffer()."""
+        y_sh = self.y_shared if self.cfg.n_shared else None
+        if self.dedup_combine:
+            moe_ep_combine_dedup(self.cfg, world, self.topk_idx, self.tok_slot, self.tok_base,
+                                 table, y_sh, self.out, self.status, stream)
+        else:
+            moe_ep_combine(self.cfg, world, self.topk_idx, self.topk_w, self.offsets, self.inv,
+                           self.base, table, y_sh, self.out, self.status, stream)
 
     def fanout(self, stream):
         """Deduplicating: this owner's copy rows from its token rows."""
@@ -117,6 +148,10 @@ class _RankState:
             moe_ep_dispatch_dedup(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
                                   self.base, self.tok_slot, self.tok_base, tables[0], tables[1],
                                   self.status, stream)
+            if self.dedup_combine:
+                moe_ep_combine_plan(self.cfg, world, self.topk_idx, self.topk_w, self.offsets,
+                                    self.inv, self.base, self.tok_slot, self.tok_base, tables[2],
+                                    tables[3], tables[4], self.status, stream)
         elif self.fp8:
             moe_ep_dispatch_fp8(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
                                 self.base, tables[0], tables[1], self.status, stream)
@@ -156,7 +191,7 @@ class EmulatedEP:
     barriers between them."""
 
     def __init__(self, shape, inp: dict, world: int, router=None, token_ids=None, stream=None,
-                 payload=None, dedup=False):
+                 payload=None, dedup=False, dedup_combine=False):
         self.device = inp["x"].device
         base_cfg = MoeConfig.of(shape, router=router)
         T = base_cfg.T
@@ -165,7 +200,8 @@ class EmulatedEP:
         Tr = T // world
         self.world, self.stream, self.inp = world, stream, inp
         self.cfg = MoeConfig.of(shape.replace(T=Tr), router=router, payload=payload)
-        self.ranks = [_RankState(self.cfg, world, self.device, dedup) for _ in range(world)]
+        self.ranks = [_RankState(self.cfg, world, self.device, dedup, dedup_combine)
+                      for _ in range(world)]
         self.xs = [inp["x"][r * Tr:(r + 1) * Tr] for r in range(world)]
         self.ids = [None if token_ids is None else token_ids[r * Tr:(r + 1) * Tr]
                     for r in range(world)]
@@ -173,7 +209,7 @@ class EmulatedEP:
         self.recv_tables = [torch.tensor([st.recv_buffers()[i].data_ptr() for st in self.ranks],
                                          dtype=torch.int64, device=self.device)
                             for i in range(n_buf)]
-        self.recv_y_ptrs = torch.tensor([st.recv_y.data_ptr() for st in self.ranks],
+        self.recv_y_ptrs = torch.tensor([st.combine_buffer().data_ptr() for st in self.ranks],
                                         dtype=torch.int64, device=self.device)
         n_ex = self.ranks[0].exchanged().numel()
         self.gathered = torch.empty(world, n_ex, dtype=torch.int32, device=self.device)
@@ -213,11 +249,13 @@ class EmulatedEP:
             w = tuple(_local_weights(inp[k], r, world) for k in ("w_gate", "w_up", "w_down"))
             st.expert_ffn(world, r, w, self.xs[r], w_shared, self.stream)
 
+    def precombine(self):
+        for st in self.ranks:
+            st.precombine(self.stream)
+
     def combine(self):
         for st in self.ranks:
-            moe_ep_combine(self.cfg, self.world, st.topk_idx, st.topk_w, st.offsets, st.inv,
-                           st.base, self.recv_y_ptrs, st.y_shared if self.cfg.n_shared else None,
-                           st.out, st.status, self.stream)
+            st.combine(self.world, self.recv_y_ptrs, self.stream)
 
     def forward(self):
         self.route_and_plan_local()
@@ -226,15 +264,16 @@ class EmulatedEP:
         self.dispatch()
         self.fanout()
         self.expert_ffn()
+        self.precombine()
         self.combine()
         return torch.cat([st.out for st in self.ranks])
 
 
 def emulate_forward(shape, inp: dict, world: int, router=None, token_ids=None, stream=None,
-                    payload=None, dedup=False):
+                    payload=None, dedup=False, dedup_combine=False):
     """One EP step of all `world` ranks on this GPU; returns (out [T, d],
     per-rank states)."""
-    em = EmulatedEP(shape, inp, world, router, token_ids, stream, payload, dedup)
+    em = EmulatedEP(shape, inp, world, router, token_ids, stream, payload, dedup, dedup_combine)
     return em.forward(), em.ranks
 
 
@@ -253,7 +292,7 @@ class EPLayer:
 
     def __init__(self, shape_local, group, router_w, bias, w_gate_local, w_up_local,
                  w_down_local, ws_gate=None, ws_up=None, ws_down=None, logit_offset=None,
-                 router=None, payload=None, dedup=False):
+                 router=None, payload=None, dedup=False, dedup_combine=False):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -262,14 +301,14 @@ class EPLayer:
         self.device = w_gate_local.device
         self.host_sync = dist.get_backend(group) != "nccl"
         self.cfg = MoeConfig.of(shape_local, router=router, payload=payload)
-        self.st = _RankState(self.cfg, self.world, self.device, dedup)
+        self.st = _RankState(self.cfg, self.world, self.device, dedup, dedup_combine)
         self.router_w, self.bias, self.logit_offset = router_w, bias, logit_offset
         self.w = (w_gate_local, w_up_local, w_down_local)
         self.ws_shared = (ws_gate, ws_up, ws_down)
         self._opened = []
         torch.cuda.synchronize(self.device)   # buffers allocated before peers map them
         self.recv_tables = [self._map_peers(b) for b in self.st.recv_buffers()]
-        self.recv_y_ptrs = self._map_peers(self.st.recv_y)
+        self.recv_y_ptrs = self._map_peers(self.st.combine_buffer())
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
 
     def _map_peers(self, buf):
@@ -313,10 +352,9 @@ class EPLayer:
             self._barrier(s)          # every copy has landed
             st.fanout(s)
             st.expert_ffn(world, r, self.w, x, self.ws_shared, s)
+            st.precombine(s)
             self._barrier(s)          # every expert output is written
-            moe_ep_combine(cfg, world, st.topk_idx, st.topk_w, st.offsets, st.inv, st.base,
-                           self.recv_y_ptrs, st.y_shared if cfg.n_shared else None, st.out,
-                           st.status, s)
+            st.combine(world, self.recv_y_ptrs, s)
         return st.out
 
     def close(self, stream=None):

@@ -445,8 +445,9 @@ MOE_API moe_status moe_ep_expert_ffn_fp8(const moe_config *cfg, int32_t world, i
  *                      owner o (token order), -1 if none; tok_counts [world]
  *                      int32 out: this rank's tokens per owner
  *   (caller) all-gather tok_counts into tok_counts_all [world, world]
- *   moe_ep_token_base  tok_base [world] int32 out: this rank's first row in
- *                      each owner's token buffer (sum over lower ranks)
+ *   moe_ep_token_base  tok_base [world + 1] int32 out: this rank's first row
+ *                      in each owner's token buffer (sum over lower ranks);
+ *                      tok_base[world] = token rows this rank receives
  *   moe_ep_dispatch_dedup  one store of each token row per owner into
  *                      recv_tok[o] (rows: rank 0's tokens, then rank 1's,
  *                      each in token order; capacity world * T rows of d
@@ -474,6 +475,44 @@ MOE_API moe_status moe_ep_dispatch_dedup(const moe_config *cfg, int32_t world, c
 MOE_API moe_status moe_ep_fanout(const moe_config *cfg, int32_t world, const void *recv_tok,
                                  const int32_t *recv_idx, const int32_t *local_offsets,
                                  void *recv_x, int32_t *device_status, void *stream);
+
+/* Deduplicated combine (with the deduplicated dispatch): each owner sums the
+ * gate-weighted outputs of its copies of a token into one bf16 partial row,
+ * and only that row crosses back.
+ *   moe_ep_combine_plan  (source, before the dispatch barrier) for every token
+ *                      t and owner o holding cnt of its copies: the copy rows
+ *                      and gates in slot order into list[o] / lw[o]
+ *                      ([world*T*K] int32 / fp32, entry trow*K + k) and cnt
+ *                      into lcnt[o] ([world*T] int32), trow = t's token row
+ *                      at o; list / lw / lcnt: device arrays of `world`
+ *                      pointers
+ *   moe_ep_precombine    (owner, after its expert FFN) partial [world*T, d]
+ *                      bf16: partial[trow] = bf16(sum_k lw[k] * recv_y
+ *                      [list[k]]), fp32 multiply-adds in slot order, for its
+ *                      tok_base[world] token rows
+ *   barrier, then moe_ep_combine_dedup (source) out[t] = bf16(y_shared[t] +
+ *                      the partial rows of t's owners in the order of their
+ *                      first slots, fp32), partial: device array of `world`
+ *                      pointers
+ * The partial sums are rounded to bf16 once more than in moe_ep_combine, so
+ * the output equals the single-GPU layer within its tolerances, not bit for
+ * bit. */
+MOE_API moe_status moe_ep_combine_plan(const moe_config *cfg, int32_t world,
+                                       const int32_t *topk_idx, const float *topk_w,
+                                       const int32_t *offsets, const int32_t *inv_perm,
+                                       const int32_t *base, const int32_t *tok_slot,
+                                       const int32_t *tok_base, int32_t *const *list,
+                                       float *const *lw, int32_t *const *lcnt,
+                                       int32_t *device_status, void *stream);
+MOE_API moe_status moe_ep_precombine(const moe_config *cfg, int32_t world, const void *recv_y,
+                                     const int32_t *list, const float *lw, const int32_t *lcnt,
+                                     const int32_t *tok_base, void *partial,
+                                     int32_t *device_status, void *stream);
+MOE_API moe_status moe_ep_combine_dedup(const moe_config *cfg, int32_t world,
+                                        const int32_t *topk_idx, const int32_t *tok_slot,
+                                        const int32_t *tok_base, const void *const *partial,
+                                        const void *y_shared, void *out, int32_t *device_status,
+                                        void *stream);
 
 /* Combine fused with its all-to-all: out[t] = y_shared[t] + sum_j topk_w[t][j]
  * * (row of copy (t, j) in recv_y[owner]), fp32 multiply-adds in slot order,

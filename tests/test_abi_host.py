@@ -252,6 +252,25 @@ def test_expert_parallel_validates_before_cuda(moe):
     assert lib.moe_ep_fanout(c, 2, P(fake), P(fake), None, P(fake), None, None) == INV
     assert lib.moe_ep_fanout(c, 2, P(fake + 4), P(fake), P(fake), P(fake), None, None) == INV
     assert lib.moe_ep_fanout(c, 3, P(fake), P(fake), P(fake), P(fake), None, None) == UNS
+    cp_args = [P(fake)] * 10                   # topk_idx .. lcnt
+    bad = list(cp_args)
+    bad[9] = None                              # lcnt
+    assert lib.moe_ep_combine_plan(c, 2, *bad, None, None) == INV
+    assert lib.moe_ep_combine_plan(c, 3, *cp_args, None, None) == UNS
+    pc_args = [P(fake)] * 6                    # recv_y, list, lw, lcnt, tok_base, partial
+    bad = list(pc_args)
+    bad[5] = P(fake + 8)                       # misaligned partial
+    assert lib.moe_ep_precombine(c, 2, *bad, None, None) == INV
+    bad = list(pc_args)
+    bad[1] = None                              # list
+    assert lib.moe_ep_precombine(c, 2, *bad, None, None) == INV
+    cd_args = [P(fake)] * 6                    # topk_idx, tok_slot, tok_base, partial, y_sh, out
+    bad = list(cd_args)
+    bad[5] = None                              # out
+    assert lib.moe_ep_combine_dedup(c, 2, *bad, None, None) == INV
+    bad = list(cd_args)
+    bad[4] = P(fake + 2)                       # misaligned y_shared
+    assert lib.moe_ep_combine_dedup(c, 2, *bad, None, None) == INV
     assert lib.moe_ipc_get_handle(None, P(fake)) == INV
     assert lib.moe_ipc_open_handle(None, P(fake)) == INV
     assert lib.moe_ipc_close_handle(None) == INV

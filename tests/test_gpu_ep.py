@@ -249,6 +249,52 @@ def test_emulated_ep_dedup_dispatch(orc, name, world):
     for r, st in enumerate(ranks):
         np.testing.assert_array_equal(st.tok_slot.cpu().numpy(), plans[r][0])
         np.testing.assert_array_equal(st.tok_counts.cpu().numpy(), plans[r][1])
-        np.testing.assert_array_equal(st.tok_base.cpu().numpy(), tok_base[r])
+        np.testing.assert_array_equal(st.tok_base[:world].cpu().numpy(), tok_base[r])
+        assert int(st.tok_base[world].item()) == int(tok_counts_all[:, r].sum())
         n = int(st.local_offsets[El].item())
         assert torch.equal(st.recv_x[:n].view(torch.int16), plain[r].recv_x[:n].view(torch.int16))
+
+
+
+@pytest.mark.parametrize("name,world", [("ragged", 2), ("ragged", 3), ("noshared", 4),
+                                        ("ragged2", 5)])
+def test_emulated_ep_dedup_combine(orc, name, world):
+    """Both exchanges at (token, owner) granularity: each owner sums its
+    copies of a token into one bf16 partial row.  One more bf16 rounding than
+    the single-GPU combine, so: every token within the layer's bars of the
+    oracle, and close to the per-copy EP path."""
+    sh = H.shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    out, ranks = ep.emulate_forward(sh, inp, world, dedup=True, dedup_combine=True)
+    plain, _ = ep.emulate_forward(sh, inp, world)
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+        assert moe.moe_read_device_status(st.ws) == moe.MOE_OK
+    rows = np.arange(sh.T)
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows)
+    gi = torch.cat([st.topk_idx for st in ranks]).cpu().numpy()
+    keep = [r for r in rows if np.array_equal(gi[r], ref_idx[r])]
+    for r in set(rows.tolist()) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    frob, elem = H.compare_out(out[torch.as_tensor(keep, device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+    a, b = out.float(), plain.float()
+    assert float((a - b).norm() / b.norm()) <= H.TOL_FROB
+
+
+def test_emulated_ep_dedup_combine_v3_matches_oracle(orc):
+    sh = H.shape("v3")
+    inp = synth.make_inputs(sh, DEV)
+    out, ranks = ep.emulate_forward(sh, inp, 8, dedup=True, dedup_combine=True)
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+    rows = np.unique(np.linspace(0, sh.T - 1, 6).astype(np.int64))
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows)
+    gi = torch.cat([st.topk_idx for st in ranks]).cpu().numpy()[rows]
+    keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
+    for r in set(range(len(rows))) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    frob, elem = H.compare_out(out[torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
