@@ -662,7 +662,25 @@ def ep_leg(sh, inp, dev, stream, world, reps=20):
         del graphs
         q_bytes = (2.0 * d + K * (d + d / 32.0) + 8.0 * K) * Tr   # x read, codes + scales
         q_link = (d + d / 32.0) * max(max(out_copies), max(in_copies))
+        del em
+        torch.cuda.empty_cache()
+        # ... and sent once per (token, owner), fanned out at the owner
+        em = ep.EmulatedEP(sh, inp, world, stream=stream, payload=moe.MOE_PAYLOAD_FP8,
+                           dedup=True)
+        em.forward()
+        torch.cuda.synchronize(dev)
+        graphs = {k: graphed(k) for k in ("dispatch", "fanout")}
+        t8d = {k: timed(graphs[k].replay) / world for k in ("dispatch", "fanout")}
+        for st in em.ranks:
+            if int(st.status.item()) != moe.MOE_OK:
+                raise RuntimeError("device status after the emulated FP8 deduplicated dispatch")
+        del graphs
+        q_dd_link = (d + d / 32.0) * max(max(tok_out), max(tok_in)) + \
+            4.0 * max(max(out_copies), max(in_copies))
         res["fp8_payload"] = {
+            "dedup": {"stage_ms_per_rank": t8d,
+                      "nvlink": {"max_rank_bytes_dispatch": q_dd_link,
+                                 "projected_ms_dispatch": q_dd_link / (NVLINK_GBS * 1e9) * 1e3}},
             "stage_ms_per_rank": t8,
             "dispatch": {"bytes_per_rank": q_bytes,
                          "achieved_gbs": q_bytes / (t8["dispatch"] / 1e3) / 1e9,

@@ -38,7 +38,8 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_expert_ffn_fp8", "moe_permute", "moe_ep_workspace_size", "moe_ep_plan",
            "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_dispatch_fp8",
            "moe_ep_expert_ffn_fp8", "moe_ep_token_plan", "moe_ep_token_base",
-           "moe_ep_dispatch_dedup", "moe_ep_fanout", "moe_ep_combine_plan",
+           "moe_ep_dispatch_dedup", "moe_ep_fanout", "moe_ep_dispatch_dedup_fp8",
+           "moe_ep_fanout_fp8", "moe_ep_combine_plan",
            "moe_ep_precombine", "moe_ep_combine_dedup", "moe_ipc_get_handle",
            "moe_ipc_open_handle", "moe_ipc_close_handle")
 
@@ -102,6 +103,8 @@ _sig = {
     "moe_ep_token_base": (C.c_int, [_CP, C.c_int32, C.c_int32, _P, _P, _P]),
     "moe_ep_dispatch_dedup": (C.c_int, [_CP, C.c_int32] + [_P] * 11),
     "moe_ep_fanout": (C.c_int, [_CP, C.c_int32] + [_P] * 6),
+    "moe_ep_dispatch_dedup_fp8": (C.c_int, [_CP, C.c_int32] + [_P] * 12),
+    "moe_ep_fanout_fp8": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
     "moe_ep_combine_plan": (C.c_int, [_CP, C.c_int32] + [_P] * 12),
     "moe_ep_precombine": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
     "moe_ep_combine_dedup": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
@@ -305,6 +308,24 @@ def moe_ep_fanout(cfg, world, recv_tok, recv_idx, local_offsets, recv_x, device_
         _lib.moe_ep_fanout(_cfg(cfg), int(world), _ptr(recv_tok), _ptr(recv_idx),
                            _ptr(local_offsets), _ptr(recv_x), _ptr(device_status),
                            _stream(stream)))
+
+
+def moe_ep_dispatch_dedup_fp8(cfg, world, x, topk_idx, offsets, inv_perm, base, tok_slot,
+                              tok_base, recv_tq_ptrs, recv_ts_ptrs, recv_idx_ptrs,
+                              device_status=None, stream=None) -> None:
+    _ok("moe_ep_dispatch_dedup_fp8",
+        _lib.moe_ep_dispatch_dedup_fp8(_cfg(cfg), int(world), _ptr(x), _ptr(topk_idx),
+                                       _ptr(offsets), _ptr(inv_perm), _ptr(base), _ptr(tok_slot),
+                                       _ptr(tok_base), _ptr(recv_tq_ptrs), _ptr(recv_ts_ptrs),
+                                       _ptr(recv_idx_ptrs), _ptr(device_status), _stream(stream)))
+
+
+def moe_ep_fanout_fp8(cfg, world, recv_tq, recv_ts, recv_idx, local_offsets, recv_q, recv_scale,
+                      device_status=None, stream=None) -> None:
+    _ok("moe_ep_fanout_fp8",
+        _lib.moe_ep_fanout_fp8(_cfg(cfg), int(world), _ptr(recv_tq), _ptr(recv_ts),
+                               _ptr(recv_idx), _ptr(local_offsets), _ptr(recv_q),
+                               _ptr(recv_scale), _ptr(device_status), _stream(stream)))
 
 
 def moe_ep_combine_plan(cfg, world, topk_idx, topk_w, offsets, inv_perm, base, tok_slot, tok_base,

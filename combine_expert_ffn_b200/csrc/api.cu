@@ -618,6 +618,48 @@ moe_status moe_ep_fanout(const moe_config *c, int32_t world, const void *recv_to
                                         as_stream(stream)));
 }
 
+moe_status moe_ep_dispatch_dedup_fp8(const moe_config *c, int32_t world, const void *x,
+                                     const int32_t *topk_idx, const int32_t *offsets,
+                                     const int32_t *inv_perm, const int32_t *base,
+                                     const int32_t *tok_slot, const int32_t *tok_base,
+                                     void *const *recv_tq, void *const *recv_ts,
+                                     int32_t *const *recv_idx, int32_t *device_status,
+                                     void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world) || c->d % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!x || !topk_idx || !offsets || !inv_perm || !base || !tok_slot ||
+                     !tok_base || !recv_tq || !recv_ts || !recv_idx))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t tok_rows = (int64_t)world * c->T;
+    return cuda_status(launch_ep_dispatch_dedup_fp8(x, topk_idx, offsets, inv_perm, base,
+                                                    tok_slot, tok_base, recv_tq, recv_ts,
+                                                    recv_idx, tok_rows, tok_rows * c->K, c->T,
+                                                    c->d, c->E, c->K, world, device_status,
+                                                    as_stream(stream)));
+}
+
+moe_status moe_ep_fanout_fp8(const moe_config *c, int32_t world, const uint8_t *recv_tq,
+                             const float *recv_ts, const int32_t *recv_idx,
+                             const int32_t *local_offsets, uint8_t *recv_q, float *recv_scale,
+                             int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world) || c->d % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!recv_tq || !recv_ts || !recv_idx || !local_offsets || !recv_q ||
+                     !recv_scale))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(recv_tq) || !aligned16(recv_q)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t tok_rows = (int64_t)world * c->T;
+    return cuda_status(launch_ep_fanout_fp8(recv_tq, recv_ts, recv_idx, local_offsets,
+                                            c->E / world, tok_rows, tok_rows * c->K, c->d,
+                                            recv_q, recv_scale, device_status,
+                                            as_stream(stream)));
+}
+
 moe_status moe_ep_combine_plan(const moe_config *c, int32_t world, const int32_t *topk_idx,
                                const float *topk_w, const int32_t *offsets,
                                const int32_t *inv_perm, const int32_t *base,

@@ -495,6 +495,107 @@ ep_combine_dedup_kernel(const int32_t *__restrict__ topk_idx, const int32_t *__r
     }
 }
 
+// Deduplicated dispatch of the FP8 payload: codes and scale of a token go
+// once to each owner holding one of its experts (recv_tq / recv_ts token rows),
+// plus the 4-byte fan-out index per copy.  One 16-lane group per (token,
+// 128-channel block), as the FP8 gather.
+__global__ void __launch_bounds__(256, 4)
+ep_dispatch_dedup_fp8_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ topk_idx,
+                             const int32_t *__restrict__ offsets,
+                             const int32_t *__restrict__ inv_perm,
+                             const int32_t *__restrict__ base, const int32_t *__restrict__ tok_slot,
+                             const int32_t *__restrict__ tok_base, uint2 *const *__restrict__ recv_tq,
+                             float *const *__restrict__ recv_ts,
+                             int32_t *const *__restrict__ recv_idx, int64_t tok_rows,
+                             int64_t recv_rows, int T, int chunks, int E, int K, int El, int world,
+                             int32_t *status) {
+    __shared__ int32_t delta_s[EP_MAX_E];
+    __shared__ int32_t tokbase_s[EP_MAX_WORLD];
+    __shared__ uint2 *tq_s[EP_MAX_WORLD];
+    __shared__ float *ts_s[EP_MAX_WORLD];
+    __shared__ int32_t *idx_tab_s[EP_MAX_WORLD];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) delta_s[e] = base[e] - offsets[e];
+    for (int o = threadIdx.x; o < world; o += blockDim.x) {
+        tokbase_s[o] = tok_base[o];
+        tq_s[o] = recv_tq[o];
+        ts_s[o] = recv_ts[o];
+        idx_tab_s[o] = recv_idx[o];
+    }
+    __syncthreads();
+    const int blocks = chunks >> 4;
+    const int64_t total = (int64_t)T * chunks;  // a multiple of 16: groups never straddle it
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + (threadIdx.x & ~31); i0 < total;
+         i0 += stride) {
+        const int64_t i = i0 + lane;
+        const bool in = i < total;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (in) v = __ldg(x + i);
+        float sc;
+        const uint2 packed = e4m3_quantize_chunk(v, &sc);
+        if (!in) continue;
+        const int64_t t = i / chunks;
+        const int c = (int)(i - t * chunks);
+        const int32_t *idx_t = topk_idx + t * K;
+        uint64_t sent = 0;
+        for (int j = 0; j < K; ++j) {
+            const int e = __ldg(idx_t + j);
+            if (e < 0 || e >= E) continue;  // flagged by the local dispatch plan
+            const int o = e / El;
+            const int slot = __ldg(tok_slot + t * world + o);
+            const int64_t trow = (int64_t)tokbase_s[o] + slot;
+            if (slot < 0 || trow >= tok_rows) {
+                if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                continue;
+            }
+            if (!((sent >> o) & 1ull)) {
+                sent |= 1ull << o;
+                tq_s[o][trow * chunks + c] = packed;
+                if ((c & 15) == 0) ts_s[o][trow * blocks + (c >> 4)] = sc;
+            }
+            if (c == 0) {
+                const int64_t row = (int64_t)delta_s[e] + __ldg(inv_perm + t * K + j);
+                if (row < 0 || row >= recv_rows) {
+                    if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+                    continue;
+                }
+                idx_tab_s[o][row] = (int32_t)trow;
+            }
+        }
+    }
+}
+
+// The owner's fan-out of the FP8 payload: codes (16-byte units) and scales of
+// token row recv_idx[r] into copy row r.
+__global__ void __launch_bounds__(256, 4)
+ep_fanout_fp8_kernel(const uint4 *__restrict__ recv_tq, const float *__restrict__ recv_ts,
+                     const int32_t *__restrict__ recv_idx, const int32_t *__restrict__ local_offsets,
+                     int El, int64_t tok_rows, int64_t recv_rows, int units, int blocks,
+                     uint4 *__restrict__ recv_q, float *__restrict__ recv_scale, int32_t *status) {
+    int64_t n = local_offsets[El];
+    if (n < 0 || n > recv_rows) {
+        if (status && blockIdx.x == 0 && threadIdx.x == 0) record_status(status, MOE_ERR_DEVICE_FAULT);
+        n = n < 0 ? 0 : recv_rows;
+    }
+    const int per_row = units + blocks;
+    const int64_t total = n * per_row;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / per_row;
+        const int u = (int)(i - r * per_row);
+        const int64_t src = __ldg(recv_idx + r);
+        if (src < 0 || src >= tok_rows) {
+            if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+            continue;
+        }
+        if (u < units)
+            recv_q[r * units + u] = __ldg(recv_tq + src * units + u);
+        else
+            recv_scale[r * blocks + (u - units)] = __ldg(recv_ts + src * blocks + (u - units));
+    }
+}
+
 // The owner's fan-out: recv_x[r] = recv_tok[recv_idx[r]] for the rows it
 // received (local_offsets[El] of them).
 __global__ void __launch_bounds__(256, 4)
@@ -710,6 +811,36 @@ cudaError_t launch_ep_combine_dedup(const int32_t *topk_idx, const int32_t *tok_
         topk_idx, tok_slot, tok_base, reinterpret_cast<const uint4 *const *>(partial),
         static_cast<const uint4 *>(y_shared), tok_rows, T, chunks, E, K, E / world, world,
         static_cast<uint4 *>(out), status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_dispatch_dedup_fp8(const void *x, const int32_t *topk_idx,
+                                         const int32_t *offsets, const int32_t *inv_perm,
+                                         const int32_t *base, const int32_t *tok_slot,
+                                         const int32_t *tok_base, void *const *recv_tq,
+                                         void *const *recv_ts, int32_t *const *recv_idx,
+                                         int64_t tok_rows, int64_t recv_rows, int T, int d, int E,
+                                         int K, int world, int32_t *status, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int chunks = d / 8;
+    ep_dispatch_dedup_fp8_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
+        static_cast<const uint4 *>(x), topk_idx, offsets, inv_perm, base, tok_slot, tok_base,
+        reinterpret_cast<uint2 *const *>(recv_tq), reinterpret_cast<float *const *>(recv_ts),
+        recv_idx, tok_rows, recv_rows, T, chunks, E, K, E / world, world, status);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ep_fanout_fp8(const void *recv_tq, const float *recv_ts,
+                                 const int32_t *recv_idx, const int32_t *local_offsets, int El,
+                                 int64_t tok_rows, int64_t recv_rows, int d, void *recv_q,
+                                 float *recv_scale, int32_t *status, cudaStream_t st) {
+    if (recv_rows == 0) return cudaSuccess;
+    const int units = d / 16, blocks = d / 128;
+    ep_fanout_fp8_kernel<<<grid_for(recv_rows * (units + blocks)), 256, 0, st>>>(
+        static_cast<const uint4 *>(recv_tq), recv_ts, recv_idx, local_offsets, El, tok_rows,
+        recv_rows, units, blocks, static_cast<uint4 *>(recv_q), recv_scale, status);
     count_launch();
     return cudaGetLastError();
 }

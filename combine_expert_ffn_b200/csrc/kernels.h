@@ -77,6 +77,17 @@ cudaError_t launch_ep_fanout(const void *recv_tok, const int32_t *recv_idx,
                              const int32_t *local_offsets, int El, int64_t tok_rows,
                              int64_t recv_rows, int d, void *recv_x, int32_t *status,
                              cudaStream_t st);
+cudaError_t launch_ep_dispatch_dedup_fp8(const void *x, const int32_t *topk_idx,
+                                         const int32_t *offsets, const int32_t *inv_perm,
+                                         const int32_t *base, const int32_t *tok_slot,
+                                         const int32_t *tok_base, void *const *recv_tq,
+                                         void *const *recv_ts, int32_t *const *recv_idx,
+                                         int64_t tok_rows, int64_t recv_rows, int T, int d, int E,
+                                         int K, int world, int32_t *status, cudaStream_t st);
+cudaError_t launch_ep_fanout_fp8(const void *recv_tq, const float *recv_ts,
+                                 const int32_t *recv_idx, const int32_t *local_offsets, int El,
+                                 int64_t tok_rows, int64_t recv_rows, int d, void *recv_q,
+                                 float *recv_scale, int32_t *status, cudaStream_t st);
 cudaError_t launch_ep_combine_plan(const int32_t *topk_idx, const float *topk_w,
                                    const int32_t *offsets, const int32_t *inv_perm,
                                    const int32_t *base, const int32_t *tok_slot,

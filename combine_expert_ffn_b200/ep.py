@@ -27,7 +27,8 @@ import torch
 
 from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_combine_dedup,
                moe_ep_combine_plan, moe_ep_dispatch, moe_ep_dispatch_dedup,
-               moe_ep_dispatch_fp8, moe_ep_expert_ffn, moe_ep_expert_ffn_fp8, moe_ep_fanout,
+               moe_ep_dispatch_dedup_fp8, moe_ep_dispatch_fp8, moe_ep_expert_ffn,
+               moe_ep_expert_ffn_fp8, moe_ep_fanout, moe_ep_fanout_fp8,
                moe_ep_precombine,
                moe_ep_plan, moe_ep_token_base, moe_ep_token_plan, moe_ep_workspace_size,
                moe_ipc_close_handle, moe_ipc_get_handle, moe_ipc_open_handle, moe_route,
@@ -56,10 +57,13 @@ class _RankState:
         self.base, self.local_offsets = _i32(E, device), _i32(E // world + 1, device)
         cap = world * T * K
         self.fp8 = cfg.payload == MOE_PAYLOAD_FP8
-        if dedup and self.fp8:
-            raise ValueError("the deduplicated dispatch carries bf16 rows")
         if dedup:      # one row per (token, owner); the owner fans out locally
-            self.recv_tok = torch.empty(world * T, d, dtype=torch.bfloat16, device=device)
+            if self.fp8:   # codes + scales per token row
+                self.recv_tq = torch.empty(world * T, d, dtype=torch.uint8, device=device)
+                self.recv_ts = torch.empty(world * T, d // 128, dtype=torch.float32,
+                                           device=device)
+            else:
+                self.recv_tok = torch.empty(world * T, d, dtype=torch.bfloat16, device=device)
             self.recv_idx = torch.empty(cap, dtype=torch.int32, device=device)
             self.tok_slot = torch.empty(T, world, dtype=torch.int32, device=device)
             self.tok_counts, self.tok_base = _i32(world, device), _i32(world + 1, device)
@@ -113,7 +117,8 @@ class _RankState:
         """The buffers the dispatch writes into at this rank as an owner."""
         if self.dedup:
             extra = [self.recv_list, self.recv_lw, self.recv_lcnt] if self.dedup_combine else []
-            return [self.recv_tok, self.recv_idx] + extra
+            rows = [self.recv_tq, self.recv_ts] if self.fp8 else [self.recv_tok]
+            return rows + [self.recv_idx] + extra
         return [self.recv_q, self.recv_scale] if self.fp8 else [self.recv_x]
 
     def combine_buffer(self):
@@ -138,20 +143,31 @@ class _RankState:
 
     def fanout(self, stream):
         """Deduplicating: this owner's copy rows from its token rows."""
-        if self.dedup:
+        if self.dedup and self.fp8:
+            moe_ep_fanout_fp8(self.cfg, self.world, self.recv_tq, self.recv_ts, self.recv_idx,
+                              self.local_offsets, self.recv_q, self.recv_scale, self.status,
+                              stream)
+        elif self.dedup:
             moe_ep_fanout(self.cfg, self.world, self.recv_tok, self.recv_idx, self.local_offsets,
                           self.recv_x, self.status, stream)
 
     def dispatch(self, world, x, tables, stream):
         """tables: one device pointer table per entry of recv_buffers()."""
         if self.dedup:
-            moe_ep_dispatch_dedup(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
-                                  self.base, self.tok_slot, self.tok_base, tables[0], tables[1],
-                                  self.status, stream)
+            if self.fp8:
+                moe_ep_dispatch_dedup_fp8(self.cfg, world, x, self.topk_idx, self.offsets,
+                                          self.inv, self.base, self.tok_slot, self.tok_base,
+                                          tables[0], tables[1], tables[2], self.status, stream)
+                lists = tables[3:]
+            else:
+                moe_ep_dispatch_dedup(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
+                                      self.base, self.tok_slot, self.tok_base, tables[0],
+                                      tables[1], self.status, stream)
+                lists = tables[2:]
             if self.dedup_combine:
                 moe_ep_combine_plan(self.cfg, world, self.topk_idx, self.topk_w, self.offsets,
-                                    self.inv, self.base, self.tok_slot, self.tok_base, tables[2],
-                                    tables[3], tables[4], self.status, stream)
+                                    self.inv, self.base, self.tok_slot, self.tok_base, lists[0],
+                                    lists[1], lists[2], self.status, stream)
         elif self.fp8:
             moe_ep_dispatch_fp8(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
                                 self.base, tables[0], tables[1], self.status, stream)

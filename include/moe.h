@@ -476,6 +476,24 @@ MOE_API moe_status moe_ep_fanout(const moe_config *cfg, int32_t world, const voi
                                  const int32_t *recv_idx, const int32_t *local_offsets,
                                  void *recv_x, int32_t *device_status, void *stream);
 
+/* The deduplicated dispatch of the FP8 payload (d % 128 == 0): codes and
+ * scales of a token go once to each owner, recv_tq[o] ([world*T, d] bytes)
+ * and recv_ts[o] ([world*T, d/128] fp32), quantized once at the source as by
+ * moe_dispatch_fp8, plus the fan-out index per copy into recv_idx[o];
+ * moe_ep_fanout_fp8 then builds the owner's recv_q / recv_scale (the operands
+ * of moe_ep_expert_ffn_fp8), byte for byte what moe_ep_dispatch_fp8 writes. */
+MOE_API moe_status moe_ep_dispatch_dedup_fp8(const moe_config *cfg, int32_t world, const void *x,
+                                             const int32_t *topk_idx, const int32_t *offsets,
+                                             const int32_t *inv_perm, const int32_t *base,
+                                             const int32_t *tok_slot, const int32_t *tok_base,
+                                             void *const *recv_tq, void *const *recv_ts,
+                                             int32_t *const *recv_idx, int32_t *device_status,
+                                             void *stream);
+MOE_API moe_status moe_ep_fanout_fp8(const moe_config *cfg, int32_t world, const uint8_t *recv_tq,
+                                     const float *recv_ts, const int32_t *recv_idx,
+                                     const int32_t *local_offsets, uint8_t *recv_q,
+                                     float *recv_scale, int32_t *device_status, void *stream);
+
 /* Deduplicated combine (with the deduplicated dispatch): each owner sums the
  * gate-weighted outputs of its copies of a token into one bf16 partial row,
  * and only that row crosses back.

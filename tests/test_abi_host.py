@@ -252,6 +252,16 @@ def test_expert_parallel_validates_before_cuda(moe):
     assert lib.moe_ep_fanout(c, 2, P(fake), P(fake), None, P(fake), None, None) == INV
     assert lib.moe_ep_fanout(c, 2, P(fake + 4), P(fake), P(fake), P(fake), None, None) == INV
     assert lib.moe_ep_fanout(c, 3, P(fake), P(fake), P(fake), P(fake), None, None) == UNS
+    dq_args = [P(fake)] * 10                   # x .. tok_base, recv_tq, recv_ts, recv_idx
+    assert lib.moe_ep_dispatch_dedup_fp8(C.byref(odd), 2, *dq_args, None, None) == UNS
+    bad = list(dq_args)
+    bad[8] = None                              # recv_ts
+    assert lib.moe_ep_dispatch_dedup_fp8(c, 2, *bad, None, None) == INV
+    fq_args = [P(fake)] * 6                    # recv_tq, recv_ts, recv_idx, loff, recv_q, scale
+    assert lib.moe_ep_fanout_fp8(C.byref(odd), 2, *fq_args, None, None) == UNS
+    bad = list(fq_args)
+    bad[4] = P(fake + 8)                       # misaligned recv_q
+    assert lib.moe_ep_fanout_fp8(c, 2, *bad, None, None) == INV
     cp_args = [P(fake)] * 10                   # topk_idx .. lcnt
     bad = list(cp_args)
     bad[9] = None                              # lcnt

@@ -298,3 +298,27 @@ def test_emulated_ep_dedup_combine_v3_matches_oracle(orc):
         assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
     frob, elem = H.compare_out(out[torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
     assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
+@pytest.mark.parametrize("name,world", [("ep_fp8", 2), ("ep_fp8", 4), ("noshared", 4)])
+def test_emulated_ep_dedup_fp8_payload(name, world):
+    """The FP8 payload sent once per (token, owner): every owner's fanned-out
+    codes and scales equal what the per-copy FP8 dispatch stores, and the
+    layer equals moe_forward with the FP8 payload bit for bit."""
+    sh = EP_FP8 if name == "ep_fp8" else H.shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    fp8 = moe.MOE_PAYLOAD_FP8
+    ref = _forward(sh, inp, payload=fp8)
+    out, ranks = ep.emulate_forward(sh, inp, world, payload=fp8, dedup=True)
+    _, plain = ep.emulate_forward(sh, inp, world, payload=fp8)
+    torch.cuda.synchronize()
+    for st in ranks:
+        assert int(st.status.item()) == moe.MOE_OK
+        assert moe.moe_read_device_status(st.ws) == moe.MOE_OK
+    assert torch.equal(out.view(torch.int16), ref["out"].view(torch.int16))
+    El = sh.E // world
+    for r, st in enumerate(ranks):
+        n = int(st.local_offsets[El].item())
+        assert torch.equal(st.recv_q[:n], plain[r].recv_q[:n])
+        assert torch.equal(st.recv_scale[:n].view(torch.int32),
+                           plain[r].recv_scale[:n].view(torch.int32))

@@ -69,7 +69,7 @@ def _rank_main(rank, world, port, name, payload, dedup, q, dedup_combine=False):
 @pytest.mark.parametrize("name,world,payload,dedup,dedup_combine",
                          [("ragged", 2, 0, False, False), ("ragged", 3, 0, False, False),
                           ("noshared", 2, 1, False, False), ("ragged", 3, 0, True, False),
-                          ("ragged", 3, 0, True, True)])
+                          ("ragged", 3, 0, True, True), ("noshared", 2, 1, True, False)])
 def test_ep_layer_processes_on_one_gpu_equal_single_gpu_forward(name, world, payload, dedup,
                                                                 dedup_combine):
     """Bit for bit except with the deduplicated combine (one more bf16
