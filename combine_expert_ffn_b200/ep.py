@@ -4,16 +4,22 @@ points of libmoe (argument marshalling and the collectives that order them).
 A rank owns E / world experts and routes its own tokens.  One step:
 
     moe_route, moe_dispatch(x_perm=None)     local routing and dispatch plan
+      (+ moe_ep_token_plan, dedup)            tokens per owner
     all-gather of the per-expert counts       counts_all [world, E]
-    moe_ep_plan                               where this rank's copies go
+      (+ the per-owner token counts)
+    moe_ep_plan (+ moe_ep_token_base)         where this rank's copies go
     moe_ep_dispatch                           gather + peer stores (bf16 rows, or
                                               E4M3 codes + scales: moe_ep_dispatch_fp8;
                                               or one row per token and owner plus a
                                               fan-out index per copy: dedup)
+      (+ moe_ep_combine_plan, dedup_combine)  copy rows and gates per token, owner
     barrier                                   every rank's stores are done
+    (moe_ep_fanout, dedup)                    the owner's copy rows from token rows
     moe_ep_expert_ffn                         this rank's experts, shared experts
+    (moe_ep_precombine, dedup_combine)        one partial row per token, owner
     barrier                                   every rank's outputs are done
     moe_ep_combine                            peer loads + gate-weighted sum
+      (moe_ep_combine_dedup)                  or one partial row per owner
 
 `EPLayer` runs that step in a process group of one process per GPU, with the
 receive buffers mapped into every rank by CUDA IPC and the barriers as
@@ -28,9 +34,8 @@ import torch
 from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_combine_dedup,
                moe_ep_combine_plan, moe_ep_dispatch, moe_ep_dispatch_dedup,
                moe_ep_dispatch_dedup_fp8, moe_ep_dispatch_fp8, moe_ep_expert_ffn,
-               moe_ep_expert_ffn_fp8, moe_ep_fanout, moe_ep_fanout_fp8,
-               moe_ep_precombine,
-               moe_ep_plan, moe_ep_token_base, moe_ep_token_plan, moe_ep_workspace_size,
+               moe_ep_expert_ffn_fp8, moe_ep_fanout, moe_ep_fanout_fp8, moe_ep_plan,
+               moe_ep_precombine, moe_ep_token_base, moe_ep_token_plan, moe_ep_workspace_size,
                moe_ipc_close_handle, moe_ipc_get_handle, moe_ipc_open_handle, moe_route,
                moe_route_hash, MOE_PAYLOAD_FP8, MOE_ROUTER_HASH)
 
@@ -300,7 +305,8 @@ class EPLayer:
     buffers, mapped into every rank by CUDA IPC.
 
     With the NCCL backend the counts exchange and the barriers are
-    stream-ordered collectives (no host synchronisation inside the step).
+    stream-ordered collectives (no host synchronisation inside the step);
+    call torch.cuda.set_device for this rank's GPU before constructing it.
     With gloo they run on the host after synchronising the step's stream;
     that form also lets several processes share one GPU (each maps the
     others' buffers through IPC on the same device).
