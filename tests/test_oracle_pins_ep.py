@@ -118,3 +118,86 @@ def test_token_plan_fans_out_to_the_single_gpu_dispatch(orc, world, E, G, K, M, 
         assert (recv_tok >= 0).all() and (fan >= 0).all()
         lo, hi = glob["offsets"][o * El], glob["offsets"][(o + 1) * El]
         np.testing.assert_array_equal(recv_tok[fan], glob["perm_token"][lo:hi])
+
+
+def _node_limited(rng, T, E, G, K, M):
+    gsz, kpg = E // G, K // M
+    return np.stack([np.concatenate([g * gsz + rng.permutation(gsz)[:kpg]
+                                     for g in rng.permutation(G)[:M]])
+                     for _ in range(T)]).astype(np.int32)
+
+
+def _fanout_reproduces_dispatch(orc, idx, E, G, world, plans, tok_base, base, loff):
+    """True when the owners' fan-out of the token rows, placed by (plans,
+    tok_base) and indexed through the copy rows of (base, loff), reproduces
+    the single-GPU dispatch's perm_token for every owner."""
+    T = idx.shape[0]
+    Tr, El = T // world, E // world
+    glob = orc.dispatch(idx, E, G)
+    for o in range(world):
+        n_tok = int(sum(int(p[1][o]) for p in plans))
+        recv_tok = np.full(n_tok, -1, np.int64)
+        rows = int(loff[o, El])
+        fan = np.full(rows, -1, np.int64)
+        for r in range(world):
+            slot = plans[r][0]
+            seen = np.zeros(E, np.int64)
+            for tl in range(Tr):
+                t = r * Tr + tl
+                mine = [int(e) for e in idx[t] if int(e) // El == o]
+                if (slot[tl, o] >= 0) != bool(mine):
+                    return False
+                if not mine:
+                    continue
+                row = int(tok_base[r, o] + slot[tl, o])
+                if not 0 <= row < n_tok or recv_tok[row] != -1:
+                    return False
+                recv_tok[row] = t
+                for e in mine:
+                    crow = int(base[r, e] + seen[e])
+                    seen[e] += 1
+                    if not 0 <= crow < rows:
+                        return False
+                    fan[crow] = row
+        if (recv_tok < 0).any() or (fan < 0).any():
+            return False
+        lo, hi = glob["offsets"][o * El], glob["offsets"][(o + 1) * El]
+        if not np.array_equal(recv_tok[fan], glob["perm_token"][lo:hi]):
+            return False
+    return True
+
+
+def test_planted_mistakes_in_the_placements_are_caught(orc):
+    """The fan-out property accepts the oracle's placements and rejects each
+    of these planted mistakes: ranks swapped in the copy placement, a token
+    slot off by one, a token counted at an owner it has no expert at, the
+    token bases taken from the wrong rank."""
+    world, E, G, K, M, T = 4, 16, 4, 4, 2, 64
+    idx = _node_limited(np.random.default_rng(3), T, E, G, K, M)
+    Tr = T // world
+    plans = [orc.ep_token_plan(idx[r * Tr:(r + 1) * Tr], E, world) for r in range(world)]
+    tok_base = orc.ep_token_base(np.stack([p[1] for p in plans]))
+    counts_all = np.stack([np.bincount(idx[r * Tr:(r + 1) * Tr].ravel(), minlength=E)
+                           for r in range(world)]).astype(np.int32)
+    base, loff = orc.ep_plan(counts_all)
+    assert _fanout_reproduces_dispatch(orc, idx, E, G, world, plans, tok_base, base, loff)
+    # ranks 0 and 1 swapped in the copy placement
+    swapped = base.copy()
+    swapped[[0, 1]] = swapped[[1, 0]]
+    assert not _fanout_reproduces_dispatch(orc, idx, E, G, world, plans, tok_base, swapped, loff)
+    # one token's slot at an owner off by one
+    slot0 = plans[0][0].copy()
+    o = int(idx[0][0]) // (E // world)
+    slot0[0, o] += 1
+    bad = [(slot0, plans[0][1])] + plans[1:]
+    assert not _fanout_reproduces_dispatch(orc, idx, E, G, world, bad, tok_base, base, loff)
+    # a token sent to an owner holding none of its experts
+    slot0 = plans[0][0].copy()
+    t_none, o_none = next((t, o) for t in range(Tr) for o in range(world) if slot0[t, o] < 0)
+    slot0[t_none, o_none] = 0
+    bad = [(slot0, plans[0][1])] + plans[1:]
+    assert not _fanout_reproduces_dispatch(orc, idx, E, G, world, bad, tok_base, base, loff)
+    # token bases of rank 1 used for rank 2
+    tb = tok_base.copy()
+    tb[2] = tb[1]
+    assert not _fanout_reproduces_dispatch(orc, idx, E, G, world, plans, tb, base, loff)
