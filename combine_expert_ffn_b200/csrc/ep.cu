@@ -328,7 +328,7 @@ __device__ __forceinline__ void ep_acc_row(float (&acc)[8], float wj, const uint
 // and owner o holding cnt of its copies, the owner's list entry of token row
 // trow = tok_base[o] + tok_slot[t][o]: copy rows and gates of those copies in
 // slot order (list[trow * K + k], lw[trow * K + k], k < cnt = lcnt[trow]).
-// Thread per token.
+// Thread per copy (t, j).
 __global__ void __launch_bounds__(256)
 ep_combine_plan_kernel(const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_w,
                        const int32_t *__restrict__ offsets, const int32_t *__restrict__ inv_perm,
@@ -340,32 +340,32 @@ ep_combine_plan_kernel(const int32_t *__restrict__ topk_idx, const float *__rest
     __shared__ int32_t delta_s[EP_MAX_E];
     for (int e = threadIdx.x; e < E; e += blockDim.x) delta_s[e] = base[e] - offsets[e];
     __syncthreads();
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
-    const int32_t *idx_t = topk_idx + (int64_t)t * K;
-    for (int j = 0; j < K; ++j) {
-        const int e = idx_t[j];
-        if (e < 0 || e >= E) continue;  // flagged by the local dispatch plan
-        const int o = e / El;
-        int k = 0, cnt = 0;  // earlier slots at o; all slots at o
-        for (int q = 0; q < K; ++q) {
-            const int eq = idx_t[q];
-            if (eq >= 0 && eq < E && eq / El == o) {
-                if (q < j) ++k;
-                ++cnt;
-            }
+    const int64_t copy = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (copy >= (int64_t)T * K) return;
+    const int64_t t = copy / K;
+    const int j = (int)(copy - t * K);
+    const int32_t *idx_t = topk_idx + t * K;
+    const int e = idx_t[j];
+    if (e < 0 || e >= E) return;  // flagged by the local dispatch plan
+    const int o = e / El;
+    int k = 0, cnt = 0;  // earlier slots at o; all slots at o
+    for (int q = 0; q < K; ++q) {
+        const int eq = idx_t[q];
+        if (eq >= 0 && eq < E && eq / El == o) {
+            if (q < j) ++k;
+            ++cnt;
         }
-        const int slot = tok_slot[(int64_t)t * world + o];
-        const int64_t trow = (int64_t)tok_base[o] + slot;
-        const int64_t row = (int64_t)delta_s[e] + inv_perm[(int64_t)t * K + j];
-        if (slot < 0 || trow >= tok_rows || row < 0 || row >= recv_rows) {
-            if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
-            continue;
-        }
-        list[o][trow * K + k] = (int32_t)row;
-        lw[o][trow * K + k] = topk_w[(int64_t)t * K + j];
-        if (k == 0) lcnt[o][trow] = cnt;
     }
+    const int slot = tok_slot[(int64_t)t * world + o];
+    const int64_t trow = (int64_t)tok_base[o] + slot;
+    const int64_t row = (int64_t)delta_s[e] + inv_perm[(int64_t)t * K + j];
+    if (slot < 0 || trow >= tok_rows || row < 0 || row >= recv_rows) {
+        if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
+        return;
+    }
+    list[o][trow * K + k] = (int32_t)row;
+    lw[o][trow * K + k] = topk_w[(int64_t)t * K + j];
+    if (k == 0) lcnt[o][trow] = cnt;
 }
 
 // Deduplicated combine, owner side: partial[trow] = bf16(sum over k < cnt of
@@ -780,7 +780,8 @@ cudaError_t launch_ep_combine_plan(const int32_t *topk_idx, const float *topk_w,
                                    int64_t recv_rows, int T, int E, int K, int world,
                                    int32_t *status, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    ep_combine_plan_kernel<<<(T + 255) / 256, 256, 0, st>>>(
+    const int64_t copies = (int64_t)T * K;
+    ep_combine_plan_kernel<<<(unsigned)((copies + 255) / 256), 256, 0, st>>>(
         topk_idx, topk_w, offsets, inv_perm, base, tok_slot, tok_base, list, lw, lcnt, tok_rows,
         recv_rows, T, E, K, E / world, world, status);
     count_launch();
