@@ -201,3 +201,38 @@ def test_planted_mistakes_in_the_placements_are_caught(orc):
     tb = tok_base.copy()
     tb[2] = tb[1]
     assert not _fanout_reproduces_dispatch(orc, idx, E, G, world, plans, tb, base, loff)
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover - hypothesis ships with the test environment
+    given = None
+
+if given is not None:
+    @st.composite
+    def _ep_case(draw):
+        world = draw(st.sampled_from([1, 2, 3, 4]))
+        groups_per_rank = draw(st.integers(1, 2))
+        G = world * groups_per_rank
+        gsz = draw(st.integers(1, 4))
+        E = G * gsz
+        M = draw(st.integers(1, G))
+        kpg = draw(st.integers(1, gsz))
+        Tr = G * draw(st.integers(1, 4))
+        seed = draw(st.integers(0, 2**31 - 1))
+        return world, E, G, M * kpg, M, Tr * world, seed
+
+    @settings(max_examples=40, deadline=None)
+    @given(_ep_case())
+    def test_random_placements_fan_out_to_the_single_gpu_dispatch(orc, case):
+        """Random node-limited routings, worlds and group layouts: the expert
+        and token placements together reproduce the single-GPU dispatch."""
+        world, E, G, K, M, T, seed = case
+        idx = _node_limited(np.random.default_rng(seed), T, E, G, K, M)
+        Tr = T // world
+        plans = [orc.ep_token_plan(idx[r * Tr:(r + 1) * Tr], E, world) for r in range(world)]
+        tok_base = orc.ep_token_base(np.stack([p[1] for p in plans]))
+        counts_all = np.stack([np.bincount(idx[r * Tr:(r + 1) * Tr].ravel(), minlength=E)
+                               for r in range(world)]).astype(np.int32)
+        base, loff = orc.ep_plan(counts_all)
+        assert _fanout_reproduces_dispatch(orc, idx, E, G, world, plans, tok_base, base, loff)
