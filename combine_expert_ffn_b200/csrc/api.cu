@@ -498,7 +498,10 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
 // ----------------------------------------------------------------- expert parallelism
 namespace {
 bool ep_args_ok(const moe_config *c, int32_t world) {
-    return world >= 1 && world <= 64 && c->E % world == 0;
+    // every rank's copies may land on one owner: world * T * K rows there,
+    // indexed in int32 like the single-GPU x_perm
+    return world >= 1 && world <= 64 && c->E % world == 0 &&
+           (int64_t)world * c->T * c->K < (1LL << 31);
 }
 moe_config ep_global(const moe_config *c, int32_t world) {
     moe_config g = *c;

@@ -360,7 +360,8 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
  * dominates MoE step time", and the expert placement of deepnotes "The real
  * cluster, and the mesh DeepSeek actually disclosed").  Rank r owns experts
  * [r*E/world, (r+1)*E/world) and routes its own T tokens (cfg is the
- * per-rank configuration, cfg->T its token count; E % world == 0, world <= 64).
+ * per-rank configuration, cfg->T its token count; E % world == 0, world <= 64,
+ * world * T * K < 2^31; otherwise MOE_ERR_UNSUPPORTED_SHAPE).
  * A rank's step: moe_route and moe_dispatch(x_perm = NULL) on its tokens; an
  * all-gather of the dispatch counts into counts_all [world, E] (the caller's
  * collective); moe_ep_plan; moe_ep_dispatch; a barrier (every rank's stores

@@ -187,6 +187,11 @@ def test_router_variants_validate_before_cuda(moe):
     assert lib.moe_forward(C.byref(cfg), *args, P(fake), ws_n, None) == moe.MOE_ERR_INVALID_ARG
 
 
+def lib_ep_plan_status(moe, cfg, world):
+    P = C.c_void_p
+    return moe._lib.moe_ep_plan(C.byref(cfg), world, 0, P(1 << 20), P(1 << 20), P(1 << 20), None)
+
+
 def test_expert_parallel_validates_before_cuda(moe):
     tiny = synth.config("tiny")                        # E = 16, d = 128
     cfg = moe.MoeConfig.of(tiny)
@@ -195,6 +200,11 @@ def test_expert_parallel_validates_before_cuda(moe):
     assert moe.moe_ep_workspace_size(cfg, 3) == 0
     assert moe.moe_ep_workspace_size(cfg, 0) == 0
     assert moe.moe_ep_workspace_size(cfg, 32) == 0
+    # world * T * K copies must stay below 2^31 rows at one owner
+    big = moe.MoeConfig.of(tiny.replace(T=(1 << 28) - 4))   # T * K just below 2^30
+    assert moe.moe_check_config(big) == moe.MOE_OK
+    assert lib_ep_plan_status(moe, big, 4) == moe.MOE_ERR_UNSUPPORTED_SHAPE  # 4 T K >= 2^31
+    assert moe.moe_ep_workspace_size(big, 4) == 0
     assert moe.moe_ep_workspace_size(cfg, 2) == \
         moe.moe_workspace_size(moe.MoeConfig.of(tiny.replace(T=2 * tiny.T)))
     ws_n = moe.moe_ep_workspace_size(cfg, 2)
