@@ -182,49 +182,104 @@ def job_tokens_per_s(tokens_per_rank, world, steps, ms_max):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def oracle_tokens_per_s(sh, inp, n_tokens, seed_offset=0):
-    """Times the oracle (single thread) on `n_tokens` sampled tokens; returns (tok/s, seconds)."""
-    import numpy as np
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
+
+class OracleHost:
+    """Host copies of one workload's inputs for the CPU oracle.
+
+    The routed experts' weights are copied from the device once, as the sampled
+    tokens first need them, and reused by later samples."""
+
+    def __init__(self, sh, inp):
+        import oracle
+        oracle.build()
+        self.oracle, self.sh, self.inp = oracle, sh, inp
+        self.x, self.e, self.b = inp["x"].cpu(), inp["router_w"].cpu(), inp["bias"].cpu()
+        off = inp.get("logit_offset")
+        self.off = off.cpu() if off is not None else None
+        self.g, self.u, self.d = [None] * sh.E, [None] * sh.E, [None] * sh.E
+        self.sg, self.su, self.sd = (inp["ws_gate"].cpu(), inp["ws_up"].cpu(),
+                                     inp["ws_down"].cpu())
+
+    def tokens_per_s(self, n_tokens, seed_offset=0, threads=1):
+        """Times the oracle's whole layer on `n_tokens` spread tokens over `threads`
+        host threads; returns (tokens/s, seconds)."""
+        import numpy as np
+        sh, orc = self.sh, self.oracle
+        rows = (np.linspace(0, sh.T - 1, n_tokens).astype(np.int64) + seed_offset) % sh.T
+        scores = orc.router_scores(self.x, self.e, self.off, rows=rows)
+        idx, _ = orc.select(scores, self.b, sh.G, sh.K, sh.M)
+        for ex in sorted(set(int(v) for v in idx.ravel())):
+            if self.g[ex] is None:
+                self.g[ex] = self.inp["w_gate"][ex].cpu()
+                self.u[ex] = self.inp["w_up"][ex].cpu()
+                self.d[ex] = self.inp["w_down"][ex].cpu()
+        t0 = time.perf_counter()
+        orc.layer_rows(rows, sh, self.x, self.e, self.b, self.g, self.u, self.d, self.sg,
+                       self.su, self.sd, logit_offset=self.off, threads=threads)
+        dt = time.perf_counter() - t0
+        return n_tokens / dt, dt
+
+
+def cpu_baseline_leg(args, sh, inp):
+    """The oracle as it stands on this machine's host cores: one thread over
+    `--cpu-tokens` tokens, then every core over `--cpu-tokens-per-core` tokens
+    per core (a bounded sample of the same workload, the tokens spread over the
+    batch).  The all-core rate is the reported value."""
     import oracle
-    oracle.build()
-    rows = (np.linspace(0, sh.T - 1, n_tokens).astype(np.int64) + seed_offset) % sh.T
-    x_h, e_h, b_h = inp["x"].cpu(), inp["router_w"].cpu(), inp["bias"].cpu()
-    off = inp.get("logit_offset")
-    off_h = off.cpu() if off is not None else None
-    scores = oracle.router_scores(x_h, e_h, off_h, rows=rows)
-    idx, _ = oracle.select(scores, b_h, sh.G, sh.K, sh.M)
-    g, u, d = [None] * sh.E, [None] * sh.E, [None] * sh.E
-    for e in sorted(set(int(v) for v in idx.ravel())):
-        g[e], u[e], d[e] = inp["w_gate"][e].cpu(), inp["w_up"][e].cpu(), inp["w_down"][e].cpu()
-    sg, su, sd = inp["ws_gate"].cpu(), inp["ws_up"].cpu(), inp["ws_down"].cpu()
-    t0 = time.perf_counter()
-    oracle.layer_rows(rows, sh, x_h, e_h, b_h, g, u, d, sg, su, sd, logit_offset=off_h)
-    dt = time.perf_counter() - t0
-    return n_tokens / dt, dt
+    host = OracleHost(sh, inp)
+    cores = oracle.all_cores()
+    v1, dt1 = host.tokens_per_s(args.cpu_tokens, threads=1)
+    n_all = max(args.cpu_tokens, args.cpu_tokens_per_core * cores)
+    va, dta = host.tokens_per_s(n_all, seed_offset=1, threads=cores)
+    return {
+        "value": va, "unit": UNIT, "cores": cores, "kind": "oracle",
+        "sample": f"{n_all} tokens of the {sh.name} workload spread over the batch, whole layer "
+                  f"per token (routing, {sh.K} routed + {sh.n_shared} shared SwiGLU FFNs, combine), "
+                  f"{cores} threads, {dta:.1f} s",
+        "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+        "single_core": {"value": v1, "unit": UNIT, "cores": 1,
+                        "sample": f"{args.cpu_tokens} tokens, one thread, {dt1:.1f} s"},
+        "all_core": {"value": va, "unit": UNIT, "cores": cores,
+                     "sample": f"{n_all} tokens, {cores} threads, {dta:.1f} s"},
+    }
 
 
 def run_reference(args, sh, world, rank):
     if rank != 0:
         return 0
+    import oracle
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = synth.make_inputs(sh, dev)
-    n = args.ref_tokens
+    host = OracleHost(sh, inp)
+    cores = oracle.all_cores()
+    n = args.ref_tokens_per_core * cores
     vals, total = [], 0.0
     for i in range(args.warmup + args.steps):
-        v, dt = oracle_tokens_per_s(sh, inp, n, seed_offset=i)
+        v, dt = host.tokens_per_s(n, seed_offset=i, threads=cores)
         if i >= args.warmup:
             vals.append(v)
             total += dt
     value = n * args.steps / total
-    sample = f"{n} tokens per step of the {sh.name} workload (routing + {sh.K} routed + {sh.n_shared} shared SwiGLU FFN per token), single thread"
+    sample = (f"{n} tokens per step of the {sh.name} workload (routing + {sh.K} routed + "
+              f"{sh.n_shared} shared SwiGLU FFN per token), {cores} threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator)",
         "config": {"workload": sh.name, **sh.as_dict(), "tokens_per_step": n},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample, "nproc": os.cpu_count(), "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -310,6 +365,8 @@ def run_ours(args, sh, world, rank, local):
             stage_ms[k] += ev[j].elapsed_time(ev[j + 1])
     stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
     stage_ms["dispatch"] = stage_ms["dispatch_plan"] + stage_ms["permute"]
+    # per-step device times (first stage event to last), for the median and minimum
+    step_ms = [ev[0].elapsed_time(ev[5]) for ev in evs]
     status = moe.moe_read_device_status(ws)
     if status != moe.MOE_OK:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -320,7 +377,7 @@ def run_ours(args, sh, world, rank, local):
         return 0
     counts = o["counts"].cpu()
     line = report(args, sh, world, ms_total, stage_ms, launches, clk, e2e,
-                  touched_experts=int((counts > 0).sum()))
+                  touched_experts=int((counts > 0).sum()), step_ms=step_ms)
     # the routing of the timed batch: expert loads and the group-to-group send matrices
     line["routing"] = {
         "max_over_mean_expert_load": float(counts.max()) / (T * K / E),
@@ -333,11 +390,7 @@ def run_ours(args, sh, world, rank, local):
     if args.ep_world > 1:
         line["expert_parallel"] = ep_leg(sh, inp, dev, stream, args.ep_world)
     if world == 1 and not args.no_cpu_baseline:
-        n = args.cpu_tokens
-        v, dt = oracle_tokens_per_s(sh, inp, n)
-        line["cpu_baseline"] = {
-            "value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens of the {sh.name} workload, whole layer per token, single thread, {dt:.1f} s"}
+        line["cpu_baseline"] = cpu_baseline_leg(args, sh, inp)
     print(json.dumps(line), flush=True)
     return 0
 
@@ -692,15 +745,18 @@ def ep_leg(sh, inp, dev, stream, world, reps=20):
     return res
 
 
-def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e, touched_experts=None):
+def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e, touched_experts=None,
+           step_ms=None):
     T = sh.T
     ms_step = ms_total / args.steps
+    step_ms = step_ms or [ms_step]
     value = job_tokens_per_s(T, world, args.steps, ms_total)
     peaks = load_peaks()
     alg = algorithmic(sh)
     ffn_s = stage_ms["expert_ffn"] / 1e3
     ffn_tflops = alg["ffn_flop"] * T / ffn_s / 1e12
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # the timed region is a fraction of a second of short steps: the burst peak applies
+    tensor_peak = peaks["bf16_tflops"]
     hbm = peaks["hbm_gbs"]
     clock_for_alu = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
     route_tflops = alg["route_flop"] * T / (stage_ms["route"] / 1e3) / 1e12
@@ -728,8 +784,9 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e, touched_expe
         "roofline": ({"bound": "tensor", "kernel": "expert FFN: grouped_ffn_gemm_kernel<SwiGLU> + <store> (2 launches)",
                       "achieved": ffn_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
                       "frac": ffn_tflops / tensor_peak,
-                      "peak_kind": f"{peaks['source']} bf16 sustained (burst {peaks['bf16_tflops']})",
-                      "frac_of_burst": ffn_tflops / peaks["bf16_tflops"],
+                      "peak_kind": f"{peaks['source']} bf16 burst",
+                      "frac_of_sustained": ffn_tflops / peaks.get("bf16_tflops_sustained",
+                                                                  peaks["bf16_tflops"]),
                       "traffic": traffic}
                      if not weight_bound else
                      {"bound": "hbm", "kernel": "expert FFN: grouped_ffn_gemm_kernel<SwiGLU> + <store> (2 launches)",
@@ -758,6 +815,20 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e, touched_expe
         "e2e": e2e,
         "clocks": clk,
     }
+    line["ms_per_step_median"] = statistics.median(step_ms)
+    line["ms_per_step_min"] = min(step_ms)
+    # a compact copy of the per-stage times and fractions next to the dominant kernel's line
+    st = line["stages"]
+    line["roofline"]["step_ms"] = {"mean": ms_step, "median": line["ms_per_step_median"],
+                                   "min": line["ms_per_step_min"]}
+    line["roofline"]["other_stages"] = {
+        "route": {"ms": stage_ms["route"], "tflops": route_tflops,
+                  "frac_of_bf16_peak": st["route"]["frac"]},
+        "dispatch": {"ms": stage_ms["dispatch"], "gbs": disp_gbs, "frac_of_hbm": disp_gbs / hbm},
+        "permute": {"ms": stage_ms["permute"], "gbs": perm_gbs, "frac_of_hbm": perm_gbs / hbm},
+        "combine": {"ms": stage_ms["combine"], "gbs": comb_gbs, "frac_of_hbm": comb_gbs / hbm},
+        "hbm_peak_gbs": hbm, "peaks": peaks["source"],
+    }
     return line
 
 
@@ -768,8 +839,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="v3", choices=sorted(synth.CONFIGS) + sorted(synth.PROFILE_CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=24)
-    ap.add_argument("--ref-tokens", type=int, default=2)
+    ap.add_argument("--cpu-tokens", type=int, default=24,
+                    help="tokens of the single-thread oracle sample")
+    ap.add_argument("--cpu-tokens-per-core", type=int, default=8,
+                    help="tokens per host core of the all-core oracle sample")
+    ap.add_argument("--ref-tokens-per-core", type=int, default=1,
+                    help="tokens per host core in each step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--ep-world", type=int, default=8,

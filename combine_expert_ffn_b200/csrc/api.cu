@@ -119,13 +119,19 @@ bool ipc_addr_range(const void *p, CUdeviceptr *base, size_t *bytes) {
     });
     return fn && fn(base, bytes, reinterpret_cast<CUdeviceptr>(p)) == CUDA_SUCCESS;
 }
-// pointers handed out by moe_ipc_open_handle -> the mapping they lie in
+// pointers handed out by moe_ipc_open_handle -> the mapping they lie in and
+// how many successful opens returned them (the runtime hands back the same
+// mapping, reference counted, when one handle is opened twice in a process)
+struct IpcOpened {
+    void *base;
+    int opens;
+};
 std::mutex &ipc_mutex() {
     static std::mutex m;
     return m;
 }
-std::unordered_map<void *, void *> &ipc_opened() {
-    static std::unordered_map<void *, void *> m;
+std::unordered_map<void *, IpcOpened> &ipc_opened() {
+    static std::unordered_map<void *, IpcOpened> m;
     return m;
 }
 }  // namespace
@@ -834,7 +840,11 @@ moe_status moe_ipc_open_handle(const void *handle, void **dev_ptr) {
         return st;
     *dev_ptr = static_cast<char *>(base) + off;
     std::lock_guard<std::mutex> lock(ipc_mutex());
-    ipc_opened()[*dev_ptr] = base;
+    auto it = ipc_opened().find(*dev_ptr);
+    if (it == ipc_opened().end())
+        ipc_opened().emplace(*dev_ptr, IpcOpened{base, 1});
+    else
+        ++it->second.opens;
     return MOE_OK;
 }
 
@@ -845,8 +855,8 @@ moe_status moe_ipc_close_handle(void *dev_ptr) {
         std::lock_guard<std::mutex> lock(ipc_mutex());
         auto it = ipc_opened().find(dev_ptr);
         if (it == ipc_opened().end()) return MOE_ERR_INVALID_ARG;  // not from open_handle
-        base = it->second;
-        ipc_opened().erase(it);
+        base = it->second.base;
+        if (--it->second.opens == 0) ipc_opened().erase(it);
     }
     moe_status st = check_device();
     if (st) return st;

@@ -11,8 +11,11 @@
 // there until the process exits.
 //
 // Host code may not hand the array's name to a kernel: on the host it is only
-// a stand-in symbol.  The device address is looked up once per device with
-// cudaGetSymbolAddress, on the first call made with that device current.
+// a stand-in symbol.  The device address is looked up with
+// cudaGetSymbolAddress on the first call made with that device current, and
+// kept once the lookup has succeeded; a lookup that failed (for example one
+// made while the stream was being captured) is not kept, so the next call
+// tries again.
 #include <mutex>
 
 #include "kernels.h"
@@ -25,12 +28,9 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_dispatch_scratch[kNoAllocScratchBytes];
 
-struct DeviceScratch {
-    std::once_flag once;
-    void *ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
-DeviceScratch g_scratch[kMaxDevices];
+// Per device: the array's device address once a lookup has succeeded.
+std::mutex g_scratch_mutex;
+void *g_scratch_ptr[kMaxDevices];
 
 size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -57,10 +57,14 @@ cudaError_t scratch_address(void **out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    DeviceScratch &s = g_scratch[dev];
-    std::call_once(s.once, [&s] { s.err = cudaGetSymbolAddress(&s.ptr, g_dispatch_scratch); });
-    if (s.err != cudaSuccess) return s.err;
-    *out = s.ptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+        if (e != cudaSuccess) return e;  // not cached: the next call looks it up again
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
     return cudaSuccess;
 }
 

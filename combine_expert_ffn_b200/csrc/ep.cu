@@ -72,8 +72,10 @@ __global__ void ep_plan_kernel(const int32_t *__restrict__ counts_all, int world
         base[e] = b;
     }
     __syncthreads();
-    if (e <= El) local_offsets[e] = e < El ? start[me * El + e] : start[me * El + El - 1] +
-                                                                  col[me * El + El - 1];
+    if (e < El) local_offsets[e] = start[me * El + e];
+    // the end of the last local segment; written by thread 0 because El may be 1024,
+    // one past the last thread of the block
+    if (e == 0) local_offsets[El] = start[me * El + El - 1] + col[me * El + El - 1];
 }
 
 constexpr int EP_MAX_E = 1024, EP_MAX_WORLD = 64;

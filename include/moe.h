@@ -236,8 +236,10 @@ MOE_API moe_status moe_permute(const moe_config *cfg, const void *x, const int32
  *   before anything is launched (the five named workloads need at most
  *   0.3 MiB).  It allocates and frees nothing.
  *   First call on a device: it looks up the array's device address with
- *   cudaGetSymbolAddress (once per device, with that device current); make
- *   that first call before any stream capture.
+ *   cudaGetSymbolAddress (with that device current) and keeps it once the
+ *   lookup has succeeded; make that first call before any stream capture.  A
+ *   lookup that fails returns MOE_ERR_CUDA and is not kept, so a later call
+ *   on that device tries again.
  *   Every call uses the same array: nothing in it has to start at zero
  *   (each call writes every scratch word before reading it), but calls whose
  *   kernels overlap on the GPU -- on two streams, or from two threads --
@@ -367,7 +369,14 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
  * collective); moe_ep_plan; moe_ep_dispatch; a barrier (every rank's stores
  * done); moe_ep_expert_ffn; a barrier; moe_ep_combine.
  * Receive buffers: recv_x and recv_y of every rank hold world * T * K rows of
- * d bf16 (every copy of every rank could go to one owner).  The kernels reach
+ * d bf16 (every copy of every rank could go to one owner, and no copy is
+ * dropped).  Per-rank footprint of the exchange, in bytes:
+ *   recv_x + recv_y          2 * (2 * world * T * K * d)
+ *   moe_ep_workspace_size    about 2 * world * T * K * (2 d + d_ff) more
+ *                            (the expert FFN's x_perm / h / y_perm slots)
+ * so it grows linearly with world: at V3 sizes (T = 8192 per rank, K = 8,
+ * d = 7168, d_ff = 2048) and world = 8, recv_x and recv_y are 7.5 GB each.
+ * The kernels reach
  * the other ranks' buffers through device arrays of `world` device pointers
  * (this rank's own and peers' buffers mapped with moe_ipc_open_handle), with
  * plain peer stores (dispatch) and peer loads (combine): the transfer is the

@@ -23,7 +23,7 @@ def build(force: bool = False) -> str:
     """Compile the oracle with plain IEEE semantics (no fast-math, no FMA contraction)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
-               "-shared", "-Wall", "-Wextra", "-o", _LIB + ".tmp", _SRC, "-lm"]
+               "-shared", "-Wall", "-Wextra", "-pthread", "-o", _LIB + ".tmp", _SRC, "-lm"]
         subprocess.check_call(cmd)
         os.replace(_LIB + ".tmp", _LIB)
     return _LIB
@@ -50,6 +50,7 @@ def lib():
         _lib.oracle_layer_rows_ex.argtypes = [i32, P, i32, i32, i32, i32, i32, i32, i32, i32,
                                               P, P, P, P, i32, P, i32, P, P, P, P, P, P, i32, P,
                                               P, P, P]
+        _lib.oracle_layer_rows_mt.argtypes = [i32] + _lib.oracle_layer_rows_ex.argtypes
         _lib.oracle_e4m3_decode.argtypes = [C.c_uint8]
         _lib.oracle_e4m3_decode.restype = C.c_double
         _lib.oracle_e4m3_encode.argtypes = [C.c_float]
@@ -66,6 +67,7 @@ def lib():
         for f in ("oracle_router_scores", "oracle_select", "oracle_dispatch",
                   "oracle_ffn_row", "oracle_shared_row", "oracle_combine",
                   "oracle_layer_rows", "oracle_router_affinity", "oracle_layer_rows_ex",
+                  "oracle_layer_rows_mt",
                   "oracle_hash_route", "oracle_bias_update", "oracle_fp8_quantize_row",
                   "oracle_fp8_dequantize_row", "oracle_ep_plan", "oracle_ep_token_plan",
                   "oracle_ep_token_base"):
@@ -275,14 +277,16 @@ def fp8_dequantize(q, scale):
 
 def layer_rows(rows, shape, x, router_w, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
                logit_offset=None, round_h=False, router=ROUTER_SIGMOID, token_ids=None,
-               payload=0):
+               payload=0, threads=1):
     """The whole layer for the token rows ``rows``.
 
     ``w_gate``/``w_up``/``w_down`` are sequences of per-expert host matrices
     (entries may be None for experts no listed token selects).
     ``router`` is ROUTER_SIGMOID, ROUTER_SQRT_SOFTPLUS or ROUTER_HASH (the
     last keyed by ``token_ids[row]``, or the row index when None); ``payload``
-    1 feeds the routed experts the FP8 round trip of x.
+    1 feeds the routed experts the FP8 round trip of x.  ``threads`` > 1 runs
+    the same per-row definition on that many contiguous row shards in parallel
+    POSIX threads (``all_cores()`` = every host core); the result is the same.
     Returns (out float64 [n,d], topk_idx [n,K], topk_w [n,K], scores [n,E]).
     """
     r = _np(np.asarray(rows, dtype=np.int64), np.int64)
@@ -310,12 +314,21 @@ def layer_rows(rows, shape, x, router_w, bias, w_gate, w_up, w_down, ws_gate, ws
     w = np.empty((n, shape.K), np.float32)
     sc = np.empty((n, shape.E), np.float32)
     sc.fill(np.nan)
-    rc = lib().oracle_layer_rows_ex(n, _p(r), shape.d, shape.E, shape.G, shape.K, shape.M,
+    rc = lib().oracle_layer_rows_mt(int(threads), n, _p(r), shape.d, shape.E, shape.G, shape.K,
+                                    shape.M,
                                     shape.d_ff, shape.n_shared, shape.d_ff_shared,
                                     _p(x), _p(e), _p(off), _p(b), int(router), _p(tid),
                                     int(payload),
                                     C.cast(g, C.c_void_p), C.cast(u, C.c_void_p),
                                     C.cast(dn, C.c_void_p), _p(sg), _p(su), _p(sd),
                                     int(round_h), _p(out), _p(idx), _p(w), _p(sc))
-    _check(rc, "oracle_layer_rows_ex")
+    _check(rc, "oracle_layer_rows_mt")
     return out, idx, w, sc
+
+
+def all_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):  # pragma: no cover
+        return os.cpu_count() or 1

@@ -39,12 +39,18 @@
  * x travel as FP8 E4M3 with one fp32 scale per 128 values; "Compression has a
  * numerical price", shivam2003 section 4).
  *
+ * All-core runs: oracle_layer_rows_mt hands contiguous shards of the token
+ * rows to POSIX threads, each of which calls the unchanged single-threaded
+ * oracle_layer_rows_ex on its shard.  Rows never interact, so the output is
+ * the same bytes as one call over all rows; only the wall time changes.
+ *
  * Arithmetic: dot products accumulate in double from the exact bf16/fp32
  * inputs; sigmoid and SiLU use libm exp() in double.  The selection steps
  * (2-4) and the gate weights are done in fp32 exactly as written above, so
  * that a GPU given the same fp32 affinities must reproduce them bit for bit.
  */
 #include <math.h>
+#include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -455,6 +461,103 @@ done:
     free(xq);
     free(q);
     free(qs);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ all-core driver */
+struct layer_shard {
+    int n_rows;
+    const int64_t *rows;
+    int d, E, G, K, M, d_ff, n_shared, d_ff_s;
+    const uint16_t *x;
+    const float *e, *off, *bias;
+    int router;
+    const int64_t *token_ids;
+    int payload;
+    const uint16_t *const *Wg, *const *Wu, *const *Wd;
+    const uint16_t *Wsg, *Wsu, *Wsd;
+    int round_h;
+    double *out;
+    int32_t *topk_idx;
+    float *topk_w, *scores_out;
+    int rc;
+};
+
+static void *layer_shard_run(void *arg)
+{
+    struct layer_shard *s = arg;
+    s->rc = oracle_layer_rows_ex(s->n_rows, s->rows, s->d, s->E, s->G, s->K, s->M, s->d_ff,
+                                 s->n_shared, s->d_ff_s, s->x, s->e, s->off, s->bias, s->router,
+                                 s->token_ids, s->payload, s->Wg, s->Wu, s->Wd, s->Wsg, s->Wsu,
+                                 s->Wsd, s->round_h, s->out, s->topk_idx, s->topk_w,
+                                 s->scores_out);
+    return NULL;
+}
+
+/* oracle_layer_rows_ex over n_threads contiguous shards of `rows`, one POSIX
+ * thread each (n_threads <= 1: the calling thread alone).  Same arguments and
+ * outputs as oracle_layer_rows_ex; returns the first nonzero shard status. */
+int oracle_layer_rows_mt(int n_threads, int n_rows, const int64_t *rows,
+                         int d, int E, int G, int K, int M, int d_ff,
+                         int n_shared, int d_ff_s,
+                         const uint16_t *x, const float *e, const float *off,
+                         const float *bias, int router, const int64_t *token_ids, int payload,
+                         const uint16_t *const *Wg, const uint16_t *const *Wu,
+                         const uint16_t *const *Wd,
+                         const uint16_t *Wsg, const uint16_t *Wsu, const uint16_t *Wsd,
+                         int round_h, double *out, int32_t *topk_idx, float *topk_w,
+                         float *scores_out)
+{
+    if (n_rows < 0 || !rows || !out || !topk_idx || !topk_w)
+        return ORC_EBADARG;
+    if (n_threads > n_rows)
+        n_threads = n_rows;
+    if (n_threads <= 1)
+        return oracle_layer_rows_ex(n_rows, rows, d, E, G, K, M, d_ff, n_shared, d_ff_s, x, e,
+                                    off, bias, router, token_ids, payload, Wg, Wu, Wd, Wsg, Wsu,
+                                    Wsd, round_h, out, topk_idx, topk_w, scores_out);
+    struct layer_shard *sh = calloc((size_t)n_threads, sizeof(*sh));
+    pthread_t *th = calloc((size_t)n_threads, sizeof(*th));
+    int *started = calloc((size_t)n_threads, sizeof(int));
+    if (!sh || !th || !started) {
+        free(sh);
+        free(th);
+        free(started);
+        return ORC_ENOMEM;
+    }
+    int rc = ORC_OK;
+    for (int i = 0; i < n_threads; ++i) {
+        const int r0 = (int)((int64_t)n_rows * i / n_threads);
+        const int r1 = (int)((int64_t)n_rows * (i + 1) / n_threads);
+        struct layer_shard *s = &sh[i];
+        s->n_rows = r1 - r0;
+        s->rows = rows + r0;
+        s->d = d; s->E = E; s->G = G; s->K = K; s->M = M; s->d_ff = d_ff;
+        s->n_shared = n_shared; s->d_ff_s = d_ff_s;
+        s->x = x; s->e = e; s->off = off; s->bias = bias;
+        s->router = router; s->token_ids = token_ids; s->payload = payload;
+        s->Wg = Wg; s->Wu = Wu; s->Wd = Wd;
+        s->Wsg = Wsg; s->Wsu = Wsu; s->Wsd = Wsd;
+        s->round_h = round_h;
+        s->out = out + (int64_t)r0 * d;
+        s->topk_idx = topk_idx + (int64_t)r0 * K;
+        s->topk_w = topk_w + (int64_t)r0 * K;
+        s->scores_out = scores_out ? scores_out + (int64_t)r0 * E : NULL;
+        s->rc = ORC_OK;
+        if (pthread_create(&th[i], NULL, layer_shard_run, s) == 0)
+            started[i] = 1;
+        else
+            layer_shard_run(s); /* no thread: run the shard here */
+    }
+    for (int i = 0; i < n_threads; ++i) {
+        if (started[i])
+            pthread_join(th[i], NULL);
+        if (!rc && sh[i].rc)
+            rc = sh[i].rc;
+    }
+    free(sh);
+    free(th);
+    free(started);
     return rc;
 }
 

@@ -64,8 +64,55 @@ def expert_mats_host(inp: dict, experts, E: int):
     return g, u, d
 
 
+def copy_rows(topk_idx: np.ndarray, E: int) -> np.ndarray:
+    """x_perm row of every copy (t, j) by the stable counting sort's definition:
+    expert segments in expert order, tokens ascending inside a segment."""
+    T, K = topk_idx.shape
+    flat = topk_idx.ravel().astype(np.int64)
+    order = np.argsort(flat * (T * K) + np.arange(T * K), kind="stable")
+    rows = np.empty(T * K, np.int64)
+    rows[order] = np.arange(T * K)
+    return rows.reshape(T, K)
+
+
+def parity_rows(sh: synth.MoeShape, topk_idx: np.ndarray, n_spread: int = 192,
+                n_heavy: int = 3, per_tile: int = 12, n_high: int = 24) -> np.ndarray:
+    """Token rows for full-size parity, chosen from the routing the GPU produced.
+
+    * ``n_spread`` tokens evenly over the batch;
+    * for each of the ``n_heavy`` most-loaded experts, ``per_tile`` tokens whose
+      copy is in the expert's last 128-row GEMM tile and ``per_tile`` in the
+      tile before it (the longest segments' final tiles);
+    * ``n_high`` tokens with a copy at the highest x_perm rows, and, where the
+      buffer is longer than 2^31 bytes, ``n_high`` more with a copy just above
+      the 2^31-byte offset (64-bit row addressing).
+    """
+    T, K = topk_idx.shape
+    picks = [np.linspace(0, T - 1, min(n_spread, T)).astype(np.int64)]
+    rows = copy_rows(topk_idx, sh.E)
+    counts = np.bincount(topk_idx.ravel(), minlength=sh.E)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    flat_rows = rows.ravel()
+    tok_of_row = np.empty(T * K, np.int64)
+    tok_of_row[flat_rows] = np.repeat(np.arange(T), K)
+    for e in np.argsort(-counts, kind="stable")[:n_heavy]:
+        c = int(counts[e])
+        if c == 0:
+            continue
+        last0 = (c - 1) // 128 * 128
+        for lo in (last0, max(0, last0 - 128)):
+            seg = np.arange(offsets[e] + lo, offsets[e] + min(c, lo + 128))
+            picks.append(tok_of_row[seg[np.linspace(0, len(seg) - 1, min(per_tile, len(seg)))
+                                        .astype(np.int64)]])
+    picks.append(tok_of_row[T * K - min(n_high, T * K):])
+    first_high = -(-(2 ** 31) // (2 * sh.d))  # first row whose byte offset is >= 2^31
+    if first_high < T * K:
+        picks.append(tok_of_row[first_high:first_high + n_high])
+    return np.unique(np.concatenate(picks))
+
+
 def oracle_layer_sample(orc, sh: synth.MoeShape, inp: dict, rows, router: int = 0,
-                        token_ids=None, payload: int = 0):
+                        token_ids=None, payload: int = 0, threads: int = 1):
     """Oracle layer output for the token rows `rows` of device inputs `inp`.
 
     Only the x rows and the experts those tokens choose (by the oracle's own
@@ -90,7 +137,7 @@ def oracle_layer_sample(orc, sh: synth.MoeShape, inp: dict, rows, router: int = 
     Su = inp["ws_up"].cpu() if ns else torch.zeros(1, 64, sh.d, dtype=torch.bfloat16)
     Sd = inp["ws_down"].cpu() if ns else torch.zeros(1, sh.d, 64, dtype=torch.bfloat16)
     return orc.layer_rows(rows, sh, x_h, e_h, b_h, g, u, d, Sg, Su, Sd, logit_offset=off_h,
-                          router=router, token_ids=token_ids, payload=payload)
+                          router=router, token_ids=token_ids, payload=payload, threads=threads)
 
 
 def near_tie_certified(sh: synth.MoeShape, s_orc: np.ndarray, bias: np.ndarray,

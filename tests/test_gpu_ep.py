@@ -322,3 +322,20 @@ def test_emulated_ep_dedup_fp8_payload(name, world):
         assert torch.equal(st.recv_q[:n], plain[r].recv_q[:n])
         assert torch.equal(st.recv_scale[:n].view(torch.int32),
                            plain[r].recv_scale[:n].view(torch.int32))
+
+
+def test_emulated_ep_world_one_maximum_experts():
+    """One rank owning all 1024 experts (the largest E): the last local segment's
+    end (local_offsets[1024], one past the plan kernel's last thread) is written,
+    and the layer equals moe_forward bit for bit."""
+    sh = synth.MoeShape("ep_max_experts", T=512, d=128, E=1024, G=64, K=32, M=16, d_ff=64,
+                        n_shared=1, d_ff_shared=64, x_sigma=1.0, e_sigma=1 / math.sqrt(128),
+                        bias_sigma=0.1, seed=11)
+    inp = synth.make_inputs(sh, DEV)
+    ref = _forward(sh, inp)
+    out, ranks = ep.emulate_forward(sh, inp, 1)
+    torch.cuda.synchronize()
+    assert int(ranks[0].status.item()) == moe.MOE_OK
+    assert torch.equal(ranks[0].local_offsets, ref["offsets"])
+    assert int(ranks[0].local_offsets[-1].item()) == sh.T * sh.K
+    assert torch.equal(out.view(torch.int16), ref["out"].view(torch.int16))
