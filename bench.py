@@ -302,7 +302,6 @@ def run_ours(args, sh, world, rank, local):
     o = moe.forward_outputs(cfg, dev)
     T, K, E, G, d = sh.T, sh.K, sh.E, sh.G, sh.d
     # stage buffers (the same intermediates moe_forward keeps in its workspace)
-    scores = torch.empty(T, E, dtype=torch.float32, device=dev)
     perm_token = torch.empty(T * K, dtype=torch.int32, device=dev)
     inv_perm = torch.empty(T, K, dtype=torch.int32, device=dev)
     y_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
@@ -314,7 +313,7 @@ def run_ours(args, sh, world, rank, local):
         if ev is not None:
             ev[0].record(stream)
         moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
-                      o["topk_idx"], o["topk_w"], scores, ws, stream)
+                      o["topk_idx"], o["topk_w"], None, ws, stream)
         if ev is not None:
             ev[1].record(stream)
         # the dispatch as its two parts: the plan (counting sort of the copies), then

@@ -95,6 +95,31 @@ moe_status check_device() {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Affinity router + node-limited top-K.  Up to 256 experts (G <= 32, K <= 16)
+// one fused kernel keeps the affinities on chip and writes `scores` only when
+// the caller asks for them; larger layers take the tensor-core logits kernel
+// (affinities into `scores` or the workspace) and the warp-per-token select.
+cudaError_t route_affinity(const moe_config &c, const void *x, const float *router_w,
+                           const float *logit_offset, const float *bias, int32_t *topk_idx,
+                           float *topk_w, float *scores, void *ws, const Layout &L,
+                           cudaStream_t s) {
+    int32_t *status = at<int32_t>(ws, L.status);
+    void *e_split = at<void>(ws, L.e_split);
+    if (router_fused_supported(c.E, c.G, c.K)) {
+        cudaError_t err = launch_router_split(router_w, c.E, c.d, e_split, s);
+        if (err != cudaSuccess) return err;
+        return launch_router_select_fused(x, e_split, logit_offset, bias, c.T, c.d, c.E, c.G, c.K,
+                                          c.M, c.router, scores, topk_idx, topk_w, status,
+                                          kWaitTimeoutNs, s);
+    }
+    if (!scores) scores = at<float>(ws, L.scores);
+    cudaError_t err = launch_router_logits_tc(x, router_w, logit_offset, c.T, c.d, c.E, c.router,
+                                              e_split, at<float>(ws, L.router_part), scores,
+                                              status, kWaitTimeoutNs, s);
+    if (err != cudaSuccess) return err;
+    return launch_route_select(scores, bias, c.T, c.E, c.G, c.K, c.M, topk_idx, topk_w, s);
+}
+
 cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
 }  // namespace
@@ -220,15 +245,9 @@ moe_status moe_route(const moe_config *c, const void *x, const float *router_w,
     const Layout L = layout(*c);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
-    if (!scores) scores = at<float>(ws, L.scores);
     if ((st = check_device())) return st;
-    cudaStream_t s = as_stream(stream);
-    if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, c->router,
-                                at<void>(ws, L.e_split), at<float>(ws, L.router_part), scores,
-                                at<int32_t>(ws, L.status), kWaitTimeoutNs, s))
-        return MOE_ERR_CUDA;
-    return cuda_status(
-        launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s));
+    return cuda_status(route_affinity(*c, x, router_w, logit_offset, bias, topk_idx, topk_w,
+                                      scores, ws, L, as_stream(stream)));
 }
 
 moe_status moe_route_hash(const moe_config *c, const int64_t *token_ids, int32_t *topk_idx,
@@ -449,7 +468,6 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
     if (!offsets) offsets = at<int32_t>(ws, L.offsets);
     if (!send) send = at<int32_t>(ws, L.send);
     if (!send_tok) send_tok = at<int32_t>(ws, L.send_tok);
-    float *scores = at<float>(ws, L.scores);
     int32_t *perm_token = at<int32_t>(ws, L.perm_token);
     int32_t *inv_perm = at<int32_t>(ws, L.inv_perm);
     void *y_perm = at<void>(ws, L.y_perm);
@@ -460,11 +478,8 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
         if (launch_hash_route(token_ids, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
             return MOE_ERR_CUDA;
     } else {
-        if (launch_router_logits_tc(x, router_w, logit_offset, c->T, c->d, c->E, c->router,
-                                    at<void>(ws, L.e_split), at<float>(ws, L.router_part), scores,
-                                    status, kWaitTimeoutNs, s))
-            return MOE_ERR_CUDA;
-        if (launch_route_select(scores, bias, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
+        if (route_affinity(*c, x, router_w, logit_offset, bias, topk_idx, topk_w, nullptr, ws, L,
+                           s))
             return MOE_ERR_CUDA;
     }
     DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),

@@ -212,6 +212,86 @@ dispatch_gather_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ 
     }
 }
 
+// Bulk-copy gather: the copy engine moves whole rows.  Each warp owns two row
+// buffers in shared memory; lane 0 loads token t's row (cp.async.bulk, one
+// mbarrier per buffer) while the previous row's stores drain, and lane j < K
+// stores the row to x_perm[inv_perm[t][j]] (cp.async.bulk shared -> global).
+// A buffer is reloaded only after every store that read it has read it.
+constexpr int GB_WARPS = 4;
+
+__device__ __forceinline__ void drain_wait_ns(uint32_t bar, uint32_t parity, int64_t timeout_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity) && (int64_t)(globaltimer_ns() - t0) < timeout_ns) {
+    }
+}
+
+__global__ void __launch_bounds__(GB_WARPS * 32)
+dispatch_gather_bulk_kernel(const char *__restrict__ x, const int32_t *__restrict__ inv_perm,
+                            int T, int row_bytes, int K, int64_t n_rows, char *__restrict__ x_perm,
+                            int32_t *status, int64_t timeout_ns) {
+    extern __shared__ __align__(128) uint8_t gsm[];
+    __shared__ __align__(8) uint64_t lbar[GB_WARPS][2];
+    __shared__ int abort_s[GB_WARPS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t buf0 = smem_u32(gsm) + (uint32_t)(warp * 2 * row_bytes);
+    const uint32_t bar0 = smem_u32(&lbar[warp][0]), bar1 = smem_u32(&lbar[warp][1]);
+    if (lane == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar1, 1);
+        abort_s[warp] = 0;
+        fence_barrier_init();
+    }
+    __syncwarp();
+    const int nw = gridDim.x * GB_WARPS;
+    int t = blockIdx.x * GB_WARPS + warp;
+    uint32_t in_flight = 0;  // lane 0: bit b set while a load into buffer b is not waited for
+    uint32_t ph = 0;         // bit b: phase parity of buffer b's barrier
+    if (t < T && lane == 0) {
+        mbar_arrive_expect_tx(bar0, row_bytes);
+        bulk_load(buf0, x + (size_t)t * row_bytes, row_bytes, bar0);
+        in_flight = 1u;
+    }
+    for (int i = 0; t < T; t += nw, ++i) {
+        const int b = i & 1;
+        const int tn = t + nw;
+        const int row = lane < K ? __ldg(inv_perm + (size_t)t * K + lane) : -1;
+        // the other buffer: every store of the previous row has read it
+        if (lane < K) bulk_wait_group_read<0>();
+        __syncwarp();
+        if (lane == 0 && tn < T) {
+            const uint32_t nb = b ? bar0 : bar1;
+            mbar_arrive_expect_tx(nb, row_bytes);
+            bulk_load(buf0 + (uint32_t)((b ^ 1) * row_bytes), x + (size_t)tn * row_bytes, row_bytes,
+                      nb);
+            in_flight |= 1u << (b ^ 1);
+        }
+        const uint32_t bar = b ? bar1 : bar0, par = (ph >> b) & 1u;
+        int ok = 1;
+        if (lane == 0) {
+            ok = mbar_wait_bounded(bar, par, &abort_s[warp], status, timeout_ns);
+            if (ok) in_flight &= ~(1u << b);
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        ph ^= 1u << b;
+        // the storing lanes observe the completed phase themselves (it has completed:
+        // one probe suffices) before their copies read the buffer
+        if (lane < K) mbar_try_wait(bar, par);
+        if (lane < K) {
+            if (row >= 0 && row < n_rows)
+                bulk_store(x_perm + (size_t)row * row_bytes, buf0 + (uint32_t)(b * row_bytes),
+                           row_bytes);
+            bulk_commit_group();
+        }
+    }
+    bulk_wait_group_all();
+    // after a timeout: wait (bounded) for loads still in flight into this warp's buffers
+    if (lane == 0) {
+        if (in_flight & 1u) drain_wait_ns(bar0, ph & 1u, timeout_ns);
+        if (in_flight & 2u) drain_wait_ns(bar1, (ph >> 1) & 1u, timeout_ns);
+    }
+}
+
 // FP8 payload gather.  One 16-lane group per (token, 128-channel block);
 // lane l of the group holds channels 8l .. 8l+7.  s = amax / 448 in fp32,
 // q = E4M3(x / s) (fp32 division, nearest-even, saturating), all-zero blocks
@@ -262,8 +342,33 @@ cudaError_t launch_gather_fp8(const void *x, const int32_t *inv_perm, int T, int
 }
 
 cudaError_t launch_permute(const void *x, const int32_t *inv_perm, int T, int d, int K,
-                           void *x_perm, cudaStream_t st) {
+                           void *x_perm, cudaStream_t st, int32_t *status, int64_t timeout_ns) {
     if (T == 0) return cudaSuccess;
+    const int row_bytes = d * 2;
+    const size_t gb_smem = (size_t)GB_WARPS * 2 * row_bytes;
+    if (K <= 32 && gb_smem <= 112 * 1024) {
+        // one wave of four-warp CTAs (two per SM at 14 KB rows); every warp walks
+        // about T / (warps resident) rows
+        int sms = 148, dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaError_t err = cudaFuncSetAttribute(dispatch_gather_bulk_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)gb_smem);
+        if (err != cudaSuccess) return err;
+        int per_sm = 1;  // CTAs resident per SM with this shared memory (one wave)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_gather_bulk_kernel,
+                                                          GB_WARPS * 32, gb_smem) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        const int want = (T + GB_WARPS - 1) / GB_WARPS;
+        const int grid = want < per_sm * sms ? want : per_sm * sms;
+        dispatch_gather_bulk_kernel<<<grid, GB_WARPS * 32, gb_smem, st>>>(
+            static_cast<const char *>(x), inv_perm, T, row_bytes, K, (int64_t)T * K,
+            static_cast<char *>(x_perm), status, timeout_ns);
+        count_launch();
+        return cudaGetLastError();
+    }
     const int chunks = d / 8;
     const int64_t total = (int64_t)T * chunks;
     int sms = 148;
@@ -315,7 +420,7 @@ cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d
                                                              offsets, perm_token, inv_perm);
     count_launch();
     if ((err = cudaGetLastError())) return err;
-    if (x_perm) return launch_permute(x, inv_perm, T, d, K, x_perm, st);
+    if (x_perm) return launch_permute(x, inv_perm, T, d, K, x_perm, st, status);
     return cudaSuccess;
 }
 

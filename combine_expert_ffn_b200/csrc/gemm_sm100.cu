@@ -35,6 +35,15 @@
 #include "kernels.h"
 
 
+// Paired row tiles (grouped_ffn_pair_kernel) for the gate/up GEMM and the
+// down GEMM; 0 selects the single-tile kernel with double-buffered TMEM.
+#ifndef MOE_PAIR_GEMM1
+#define MOE_PAIR_GEMM1 0
+#endif
+#ifndef MOE_PAIR_GEMM2
+#define MOE_PAIR_GEMM2 0
+#endif
+
 namespace moe {
 namespace gemm {
 
@@ -102,6 +111,7 @@ struct Params {
     __nv_bfloat16 *out_s;
     int32_t *status;
     int64_t timeout_ns;
+    int *tile_counter;       // paired kernel: next tile to hand out (zero at launch)
 };
 
 struct Tile {
@@ -603,6 +613,401 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
     }
 }
 
+// ---------------------------------------------------------------- paired row tiles
+// The same grouped GEMM with two 128-row tiles of one expert (or of the shared
+// rows) on every weight stage: per k step the MMA thread issues
+// D0 += A0 B^T and D1 += A1 B^T into the two halves of TMEM, so each 32 KB
+// weight tile loaded into shared memory feeds 2 x 128 rows.  Per SM that is
+// 64 bytes of operands per MMA clock instead of 96, and a 3-stage ring of
+// 64 KB stages covers twice the MMA time of the 4-stage ring above, which
+// hides more of the L2 / HBM latency.  An expert with an odd number of row
+// tiles ends with a single tile (one MMA per k step).  Both accumulators use
+// all 512 TMEM columns, so the epilogue of a tile does not overlap the next
+// tile's MMAs; 8 epilogue warps (two per TMEM lane quarter, each half of the
+// columns) drain it.
+// Tiles are handed out dynamically: the producer warp takes the next index
+// from a launch-wide atomic counter (zeroed on the stream before the launch)
+// and passes it to the MMA thread and the epilogue warps through a small ring
+// in shared memory, so CTAs that drew single tiles or ran slower take more
+// tiles and none idles at the end while others still hold a backlog.
+constexpr int P_STAGES = 3;
+constexpr int P_STAGE_BYTES = 2 * A_BYTES + B_BYTES;     // 64 KB
+constexpr int P_EPI_WARPS = 8;
+constexpr int P_THREADS = 64 + P_EPI_WARPS * 32;         // 320
+constexpr int P_SMEM_DYN = P_STAGES * P_STAGE_BYTES + P_EPI_WARPS * STORE_BUF + 1024;
+constexpr int TQ = 4;  // tile indices handed from the producer to the other roles
+
+struct PTile {
+    int row0;     // first A row of the first tile (the second starts 128 rows later)
+    int rv0, rv1; // rows to store of each tile (rv1 == 0: a single tile)
+    int n0;       // first output column
+    int e;        // expert (routed) or -1 (shared)
+    int kblocks;
+};
+
+// Tile idx: routed experts first, each with ceil(ceil(rows/128)/2) row pairs x
+// the column tiles (row pairs fastest, so consecutive tiles share the weight
+// tile), then the shared rows in pairs x the column tiles (columns fastest).
+template <int EPI>
+__device__ __forceinline__ PTile decode_pair(int idx, const int *tile_base, const int *seg,
+                                             const int *segc, const Params &p, int ntr,
+                                             int nt_s) {
+    constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
+    PTile t;
+    int rows, g;
+    if (idx < ntr) {
+        int lo = 0, hi = p.E;  // tile_base[lo] <= idx < tile_base[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tile_base[mid] <= idx) lo = mid; else hi = mid;
+        }
+        rows = segc[lo];
+        const int mg = ((rows + BM - 1) / BM + 1) / 2;
+        const int local = idx - tile_base[lo];
+        const int n = local / mg;
+        g = local - n * mg;
+        t.row0 = seg[lo] + g * 2 * BM;
+        t.n0 = n * BN_OUT;
+        t.e = lo;
+        t.kblocks = p.k_r / BK;
+    } else {
+        const int local = idx - ntr;
+        g = local / nt_s;
+        const int n = local - g * nt_s;
+        rows = p.T;
+        t.row0 = g * 2 * BM;
+        t.n0 = n * BN_OUT;
+        t.e = -1;
+        t.kblocks = p.k_s / BK;
+    }
+    const int left = rows - g * 2 * BM;
+    t.rv0 = min(BM, left);
+    t.rv1 = max(0, min(BM, left - BM));
+    return t;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(P_THREADS, 1)
+grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
+    constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[P_STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[P_STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar, tempty_bar, done_bar;
+    __shared__ __align__(8) uint64_t tq_full[TQ], tq_empty[TQ];
+    __shared__ int tile_q[TQ];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ int tile_base[MAX_E + 1];
+    __shared__ int seg[MAX_E];
+    __shared__ int segc[MAX_E];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t smem0 = smem_u32(smem);
+    volatile int *abort_flag = &abort_s;
+
+    // ---------------------------------------------------------- prologue
+    if (warp == 0) {
+        const int nt_r = (p.n_out_r + BN_OUT - 1) / BN_OUT;
+        int carry = 0;
+        for (int e0 = 0; e0 < p.E; e0 += 32) {
+            const int e = e0 + lane;
+            int lo = 0, cnt = 0;
+            if (e < p.E) {
+                lo = p.offsets[e];
+                cnt = p.offsets[e + 1] - lo;
+                if (lo < 0 || cnt < 0 || lo + cnt > p.rows_r) {
+                    record_status(p.status, MOE_ERR_DEVICE_FAULT);
+                    lo = 0;
+                    cnt = 0;
+                }
+                seg[e] = lo;
+                segc[e] = cnt;
+            }
+            const int v = (((cnt + BM - 1) / BM + 1) / 2) * nt_r;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (e < p.E) tile_base[e] = carry + incl - v;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) {
+            tile_base[p.E] = carry;
+            tma_prefetch_desc(&maps.o_r);
+            tma_prefetch_desc(&maps.a_r);
+            tma_prefetch_desc(&maps.b0_r);
+            if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
+            if (p.T > 0) {
+                tma_prefetch_desc(&maps.a_s);
+                tma_prefetch_desc(&maps.b0_s);
+                if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_s);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < P_STAGES; ++s) {
+                mbar_init(smem_u32(&full_bar[s]), 1);
+                mbar_init(smem_u32(&empty_bar[s]), 1);
+            }
+            mbar_init(smem_u32(&tfull_bar), 1);
+            mbar_init(smem_u32(&tempty_bar), P_EPI_WARPS);
+            mbar_init(smem_u32(&done_bar), 1);
+            for (int s = 0; s < TQ; ++s) {
+                mbar_init(smem_u32(&tq_full[s]), 1);
+                mbar_init(smem_u32(&tq_empty[s]), 1 + P_EPI_WARPS);
+            }
+            abort_s = 0;
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc<TMEM_COLS>(smem_u32(&tmem_base_s));
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_s;
+
+    const int ntr = tile_base[p.E];
+    const int mg_s = p.T > 0 ? ((p.T + BM - 1) / BM + 1) / 2 : 0;
+    const int nt_s = p.T > 0 ? (p.n_out_s + BN_OUT - 1) / BN_OUT : 0;
+    const int total = ntr + mg_s * nt_s;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0, qs = 0;
+            uint32_t phase = 0, n_issued = 0, qph = 0;
+            for (;;) {
+                // hand out the next tile: fetch it from the launch-wide counter and
+                // publish it to the MMA thread and the epilogue warps
+                if (!mbar_wait_bounded(smem_u32(&tq_empty[qs]), qph ^ 1u, abort_flag, p.status,
+                                       p.timeout_ns))
+                    break;
+                const int idx = atomicAdd(p.tile_counter, 1);
+                tile_q[qs] = idx;
+                mbar_arrive(smem_u32(&tq_full[qs]));
+                if (++qs == TQ) { qs = 0; qph ^= 1u; }
+                if (idx >= total) break;
+                const PTile t = decode_pair<EPI>(idx, tile_base, seg, segc, p, ntr, nt_s);
+                const bool two = t.rv1 > 0;
+                const uint32_t tx = Cfg<EPI>::TX + (two ? A_BYTES : 0);
+                bool ok = true;
+                for (int kb = 0; kb < t.kblocks; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
+                                           p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    const uint32_t a0 = smem0 + stage * P_STAGE_BYTES;
+                    const uint32_t b_dst = a0 + 2 * A_BYTES;
+                    const int k = kb * BK;
+                    mbar_arrive_expect_tx(fb, tx);
+                    if (t.e >= 0) {
+                        tma_load_2d(a0, &maps.a_r, fb, k, t.row0);
+                        if (two) tma_load_2d(a0 + A_BYTES, &maps.a_r, fb, k, t.row0 + BM);
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
+                            tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_r, fb, k, t.n0, t.e);
+                        } else {
+                            tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
+                        }
+                    } else {
+                        tma_load_2d(a0, &maps.a_s, fb, k, t.row0);
+                        if (two) tma_load_2d(a0 + A_BYTES, &maps.a_s, fb, k, t.row0 + BM);
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_3d(b_dst, &maps.b0_s, fb, k, t.n0, 0);
+                            tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_s, fb, k, t.n0, 0);
+                        } else {
+                            const int sidx = k / p.kseg_s;
+                            tma_load_3d(b_dst, &maps.b0_s, fb, k - sidx * p.kseg_s, t.n0, sidx);
+                        }
+                    }
+                    ++n_issued;
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            for (int s = 0; s < P_STAGES; ++s) {
+                if (n_issued > (uint32_t)s) {
+                    const uint32_t uses = (n_issued - 1 - s) / P_STAGES + 1;
+                    drain_wait(smem_u32(&full_bar[s]), (uses - 1) & 1u, p.timeout_ns, p.status);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, qs = 0;
+            uint32_t phase = 0, tphase = 0, qph = 0;
+            constexpr uint32_t idesc = idesc_bf16_f32<BM, Cfg<EPI>::BN_MMA>();
+            for (;;) {
+                if (!mbar_wait_bounded(smem_u32(&tq_full[qs]), qph, abort_flag, p.status,
+                                       p.timeout_ns))
+                    break;
+                const int idx = tile_q[qs];
+                mbar_arrive(smem_u32(&tq_empty[qs]));
+                if (++qs == TQ) { qs = 0; qph ^= 1u; }
+                if (idx >= total) break;
+                const PTile t = decode_pair<EPI>(idx, tile_base, seg, segc, p, ntr, nt_s);
+                const bool two = t.rv1 > 0;
+                if (!mbar_wait_bounded(smem_u32(&tempty_bar), tphase ^ 1u, abort_flag, p.status,
+                                       p.timeout_ns))
+                    break;
+                tc_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < t.kblocks; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.status,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem0 + stage * P_STAGE_BYTES;
+                    const uint64_t a0_desc = smem_desc_sw128(a0);
+                    const uint64_t a1_desc = smem_desc_sw128(a0 + A_BYTES);
+                    const uint64_t b_desc = smem_desc_sw128(a0 + 2 * A_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < BK / 16; ++ks) {
+                        const uint32_t accum = (kb | ks) != 0 ? 1u : 0u;
+                        tc_mma_bf16(tmem_base, a0_desc + 2 * ks, b_desc + 2 * ks, idesc, accum);
+                        if (two)
+                            tc_mma_bf16(tmem_base + BN_ACC, a1_desc + 2 * ks, b_desc + 2 * ks, idesc,
+                                        accum);
+                    }
+                    tc_commit(smem_u32(&empty_bar[stage]));
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&tfull_bar));
+                tphase ^= 1u;
+            }
+            tc_commit(smem_u32(&done_bar));
+            drain_wait(smem_u32(&done_bar), 0, p.timeout_ns, p.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue
+        // Warp w drains TMEM lanes 32*(w%4).. (its 32 rows of each tile) for
+        // half of the tile's output columns: full tiles leave through TMA
+        // stores of 32 x 32 boxes staged in this warp's buffer, partial tiles
+        // through masked direct stores (rows past rv belong to the next
+        // expert or to no one).
+        const int q = warp & 3;
+        const int hh = (warp - 2) >> 2;                 // column half
+        const int row = q * 32 + lane;
+        constexpr int HALF = BN_OUT / 2;                // output columns per warp
+        const uint32_t buf = smem0 + P_STAGES * P_STAGE_BYTES + (warp - 2) * STORE_BUF;
+        uint4 *sp = reinterpret_cast<uint4 *>(smem + (buf - smem0)) + lane * 4;
+        uint32_t tphase = 0, qph = 0;
+        int qs = 0;
+        for (;;) {
+            int idx = 0, ok = 1;
+            if (lane == 0) {
+                ok = mbar_wait_bounded(smem_u32(&tq_full[qs]), qph, abort_flag, p.status,
+                                       p.timeout_ns);
+                if (ok) {
+                    idx = tile_q[qs];
+                    mbar_arrive(smem_u32(&tq_empty[qs]));
+                }
+            }
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            idx = __shfl_sync(0xFFFFFFFFu, idx, 0);
+            if (!ok) break;
+            if (++qs == TQ) { qs = 0; qph ^= 1u; }
+            if (idx >= total) break;
+            const PTile t = decode_pair<EPI>(idx, tile_base, seg, segc, p, ntr, nt_s);
+            if (!mbar_wait_bounded(smem_u32(&tfull_bar), tphase, abort_flag, p.status,
+                                   p.timeout_ns))
+                break;
+            tc_fence_after();
+            const bool shared = t.e < 0;
+            const int n_out = shared ? p.n_out_s : p.n_out_r;
+            const CUtensorMap *omap = shared ? &maps.o_s : &maps.o_r;
+            __nv_bfloat16 *obase = shared ? p.out_s : p.out_r;
+            for (int ti = 0; ti < 2; ++ti) {
+                const int rv = ti == 0 ? t.rv0 : t.rv1;
+                if (rv <= 0) break;
+                const int rbase = t.row0 + ti * BM;
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + ti * BN_ACC;
+                const bool full = rv == BM;
+                const bool row_ok = row < rv;
+                __nv_bfloat16 *orow = obase + (size_t)(rbase + row) * n_out;
+#pragma unroll 1
+                for (int c = hh * HALF; c < hh * HALF + HALF; c += 32) {
+                    uint4 o[4];
+                    if (EPI == EPI_SWIGLU) {
+                        uint32_t g[32], u[32];
+                        tmem_ld32(taddr + c, g);
+                        tmem_ld32(taddr + BN_ACC / 2 + c, u);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            o[v].x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
+                                                 silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
+                            o[v].y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
+                                                 silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
+                            o[v].z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
+                                                 silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
+                            o[v].w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
+                                                 silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
+                        }
+                    } else {
+                        uint32_t r[32];
+                        tmem_ld32(taddr + c, r);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            o[v].x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                            o[v].y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                            o[v].z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                            o[v].w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                        }
+                    }
+                    if (t.n0 + c >= n_out) continue;  // whole chunk past the last column
+                    if (full) {
+                        // the staging buffer: the store that last read it must be done
+                        if (lane == 0) bulk_wait_group_read<0>();
+                        __syncwarp();
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) sp[v] = o[v];
+                        fence_proxy_async();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(omap, buf, t.n0 + c, rbase + q * 32);
+                            bulk_commit_group();
+                        }
+                    } else if (row_ok) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + t.n0 + c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[v] = o[v];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&tempty_bar));
+            tphase ^= 1u;
+        }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
+    }
+
+    // ---------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<TMEM_COLS>(tmem_base);
+    }
+}
+
 // Bounded-wait self-test: one thread waits on a barrier that never completes.
 __global__ void bounded_wait_selftest_kernel(int32_t *status, int64_t timeout_ns) {
     __shared__ __align__(8) uint64_t bar;
@@ -637,6 +1042,16 @@ int sm_count() {
     return sms;
 }
 
+template <int EPI>
+cudaError_t launch_pair(const Maps &maps, const Params &p, cudaStream_t st) {
+    cudaError_t err = cudaFuncSetAttribute(grouped_ffn_pair_kernel<EPI>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_DYN);
+    if (err != cudaSuccess) return err;
+    grouped_ffn_pair_kernel<EPI><<<sm_count(), P_THREADS, P_SMEM_DYN, st>>>(maps, p);
+    count_launch();
+    return cudaGetLastError();
+}
+
 template <int EPI, int AMODE>
 cudaError_t launch_one(const Maps &maps, const Params &p, cudaStream_t st) {
     cudaError_t err = cudaFuncSetAttribute(grouped_ffn_gemm_kernel<EPI, AMODE>,
@@ -657,6 +1072,12 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     const bool has_shared = a.n_shared > 0 && a.T > 0;
     const int ffs = a.n_shared * a.d_ff_shared;
     if (rows_r == 0) return cudaSuccess;
+    // tile counters of the paired kernels: words 16 and 17 of the status block
+    int *counters = reinterpret_cast<int *>(a.status) + 16;
+    if (MOE_PAIR_GEMM1 || MOE_PAIR_GEMM2) {
+        cudaError_t e0 = cudaMemsetAsync(counters, 0, 2 * sizeof(int), st);
+        if (e0 != cudaSuccess) return e0;
+    }
 
     // GEMM1: h = SwiGLU(x_perm) per expert; h_shared = SwiGLU(x) for the shared experts
     Maps m1;
@@ -703,8 +1124,10 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p1.out_s = static_cast<__nv_bfloat16 *>(a.h_shared);
     p1.status = a.status;
     p1.timeout_ns = a.timeout_ns;
+    p1.tile_counter = counters;
     cudaError_t err = fp8      ? launch_one<EPI_SWIGLU, A_FP8>(m1, p1, st)
                       : gather ? launch_one<EPI_SWIGLU, A_GATHER>(m1, p1, st)
+                      : MOE_PAIR_GEMM1 ? launch_pair<EPI_SWIGLU>(m1, p1, st)
                                : launch_one<EPI_SWIGLU, A_TMA>(m1, p1, st);
     if (err != cudaSuccess) return err;
 
@@ -736,7 +1159,9 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p2.kseg_s = a.d_ff_shared;
     p2.out_r = static_cast<__nv_bfloat16 *>(a.y_perm);
     p2.out_s = static_cast<__nv_bfloat16 *>(a.y_shared);
-    return launch_one<EPI_STORE, A_TMA>(m2, p2, st);
+    p2.tile_counter = counters + 1;
+    return MOE_PAIR_GEMM2 ? launch_pair<EPI_STORE>(m2, p2, st)
+                          : launch_one<EPI_STORE, A_TMA>(m2, p2, st);
 }
 
 cudaError_t launch_bounded_wait_selftest(int64_t timeout_ns, int32_t *status, cudaStream_t st) {

@@ -44,8 +44,11 @@ cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d
                             void *x_perm, const DispatchWs &ws, int32_t *status, cudaStream_t st);
 
 // dispatch.cu: the gather-permute alone, x_perm[inv_perm[t][j]] = x[t]
+// (rows of up to 14 KB through the copy engine with bounded waits recording into
+// status, which may be null; wider rows by 16-byte thread copies)
 cudaError_t launch_permute(const void *x, const int32_t *inv_perm, int T, int d, int K,
-                           void *x_perm, cudaStream_t st);
+                           void *x_perm, cudaStream_t st, int32_t *status = nullptr,
+                           int64_t timeout_ns = 2000000000LL);
 // dispatch.cu, FP8 payload: x_perm_q[row] = E4M3(x[token] / s) and x_scale[row][b] = s
 // (one scale per 128 channels, s = amax / 448); d % 128 == 0
 cudaError_t launch_gather_fp8(const void *x, const int32_t *inv_perm, int T, int d, int K,
@@ -130,7 +133,8 @@ struct FfnArgs {
     const void *ws_gate, *ws_up, *ws_down;
     void *h_shared; // [T, n_shared*d_ff_shared] bf16 scratch
     void *y_shared; // [T, d]
-    int32_t *status;
+    int32_t *status;   // the workspace's 256-byte status block: word 0 the status,
+                       // words 16 and 17 the grouped GEMMs' tile counters
     int64_t timeout_ns;
 };
 cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st);
@@ -151,6 +155,21 @@ cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *
                                     int E, int affinity, void *e_split, float *partial,
                                     float *scores, int32_t *status, int64_t timeout_ns,
                                     cudaStream_t st);
+
+// router_tc.cu: e (fp32 [E, d]) -> its three exact bf16 parts e_split [3, E, d]
+cudaError_t launch_router_split(const float *e, int E, int d, void *e_split, cudaStream_t st);
+
+// router_fused.cu: affinities and node-limited top-K in one kernel (E <= 256,
+// G <= 32, K <= 16), from the bf16 parts written by launch_router_split;
+// scores (nullable) receives the affinities.  The reduction over d is split
+// over a cluster of router_fused_cluster(T, d) CTAs.
+bool router_fused_supported(int E, int G, int K);
+int router_fused_cluster(int T, int d);
+cudaError_t launch_router_select_fused(const void *x, const void *e_split, const float *off,
+                                       const float *bias, int T, int d, int E, int G, int K,
+                                       int M, int affinity, float *scores, int32_t *topk_idx,
+                                       float *topk_w, int32_t *status, int64_t timeout_ns,
+                                       cudaStream_t st);
 
 // route_variants.cu: the hash router (token ids -> K experts in M groups,
 // gates 1/K; token_ids NULL = row index) and the per-expert bias update.

@@ -1,0 +1,522 @@
+// router_fused.cu -- router affinities and node-limited top-K in one kernel.
+//
+//   s_i = f(x . e_i + o_i),  b_i = s_i + bias_i
+//   keep the M groups (of G contiguous experts) with the largest sum of their
+//   top-(K/M) b; take the K largest b inside them; w_j = s_j / sum_j s_j
+// (top-k gating over expert affinities with per-expert bias balancing, "MoE +
+// Expert-Parallel Overlap (Exp08)", Implemented; a token's experts in at most
+// M groups, "moe-node-limited-routing", opening definition.  f is
+// DeepSeek-V3's sigmoid or the V4 sqrt(softplus).)
+//
+// For E <= 256 one CTA holds a 128-token tile against ALL experts (MMA
+// M = 128, N = E rounded up to 16), so a token's affinities never leave the
+// chip: they go from TMEM to registers to shared memory, where the selection
+// runs, and only topk_idx / topk_w (and, when asked for, the affinities) are
+// written.  The fp32 weights are split into three exact bf16 parts (router
+// split kernel in router_tc.cu); each 64-wide k block's 12 MMAs land in a
+// fresh TMEM buffer whose values the epilogue adds into IEEE fp32 registers,
+// which keeps the affinities within a few 1e-7 of the double-precision
+// definition.
+//
+// The reduction over d is split over a cluster of C CTAs (C = 1, 2, 4 or 8,
+// enough for tiles x C to fill the SMs, at least four k blocks each).  After
+// its k range, CTA r owns the 128/C token rows [r*128/C, (r+1)*128/C) of the
+// tile: every CTA of the cluster writes its partial logits of those rows into
+// r's shared memory (distributed shared memory), and r adds the C partials in
+// rank order, so the result does not depend on timing.
+//
+// One CTA, 320 threads:
+//   warp 0      TMA producer: x tile (128 x 64) into a 3-stage A ring, each
+//               weight part (N x 64) into a B ring of up to 8 stages
+//   warp 1      TMEM owner (2 buffers x 256 columns), single-thread MMA issuer
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
+//               128*((w-2)/4) .. +128 (two warps per lane quarter), adds each
+//               k block into fp32 registers; then the cluster reduction, the
+//               affinity function and the selection (2C threads per token)
+// Every mbarrier wait is bounded; on running out the kernel records
+// MOE_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs and still meets its
+// cluster barriers, so no CTA of the cluster is left waiting.
+#include <cooperative_groups.h>
+
+#include "kernels.h"
+
+namespace moe {
+namespace rfused {
+
+namespace cg = cooperative_groups;
+
+constexpr int BM = 128, BK = 64, PARTS = 3;
+constexpr int A_STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;          // 16 KB
+constexpr int B_RING_BYTES = 160 * 1024;      // B ring budget
+constexpr int MAX_B_STAGES = 8;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_THREADS = 256;
+constexpr int ACC_COLS = 256;                 // TMEM columns per accumulator buffer
+constexpr int TMEM_COLS = 512;
+
+struct Maps {
+    CUtensorMap x;      // [T, d]      box 64 x 128
+    CUtensorMap parts;  // [3, E, d]   box 64 x BN x 1
+};
+
+struct Params {
+    int T, E, d, G, K, M;
+    int BN;            // MMA N = E rounded up to 16
+    int b_stages;      // B ring stages
+    int C;             // CTAs per cluster (k splits)
+    int affinity;      // 0 sigmoid, 1 sqrt(softplus)
+    const float *off;  // [E] or null
+    const float *bias; // [E] or null
+    float *scores;     // [T, E] or null
+    int32_t *topk_idx; // [T, K]
+    float *topk_w;     // [T, K]
+    int32_t *status;
+    int64_t timeout_ns;
+};
+
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int64_t timeout_ns,
+                                           int32_t *status) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if ((int64_t)(globaltimer_ns() - t0) > timeout_ns) {
+            record_status(status, MOE_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ float affinity_fn(float L, int kind) {
+    if (kind == 1) {
+        const float sp = L > 0.f ? L + log1pf(expf(-L)) : log1pf(expf(L));
+        return sqrtf(sp);
+    }
+    return 1.0f / (1.0f + expf(-L));
+}
+
+// Selection key: orderable(b) in the high word, ~index in the low word, so the
+// largest key is the largest b with ties to the lower index.
+__device__ __forceinline__ uint64_t sel_key(float b, int i) {
+    return ((uint64_t)orderable(b) << 32) | (uint32_t)(~(uint32_t)i);
+}
+__device__ __forceinline__ int key_index(uint64_t k) { return (int)(~(uint32_t)k); }
+
+// 32 lanes x 16 consecutive fp32 columns: thread i receives row (lane base + i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Named barrier over the 256 epilogue threads (id 1; 0 is __syncthreads).
+__device__ __forceinline__ void epi_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t afull[A_STAGES], aempty[A_STAGES];
+    __shared__ __align__(8) uint64_t bfull[MAX_B_STAGES], bempty[MAX_B_STAGES];
+    __shared__ __align__(8) uint64_t accfull[2], accempty[2];
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ float bias_s[256], off_s[256];
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = p.C;
+    const int rank = C > 1 ? (int)cluster.block_rank() : 0;
+    const int tile = blockIdx.x / C;
+    const int m0 = tile * BM;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t smem0 = smem_u32(smem);
+    const uint32_t b_ring0 = smem0 + A_STAGES * A_BYTES;
+    const uint32_t b_bytes = (uint32_t)p.BN * BK * 2;
+    volatile int *abort_flag = &abort_s;
+
+    const int kblocks = p.d / BK;
+    const int kb0 = (int)((int64_t)kblocks * rank / C);
+    const int kb1 = (int)((int64_t)kblocks * (rank + 1) / C);
+
+    for (int i = threadIdx.x; i < p.E; i += NUM_THREADS) {
+        bias_s[i] = p.bias ? p.bias[i] : 0.0f;
+        off_s[i] = p.off ? p.off[i] : 0.0f;
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&maps.x);
+        tma_prefetch_desc(&maps.parts);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < A_STAGES; ++s) {
+                mbar_init(smem_u32(&afull[s]), 1);
+                mbar_init(smem_u32(&aempty[s]), 1);
+            }
+            for (int s = 0; s < p.b_stages; ++s) {
+                mbar_init(smem_u32(&bfull[s]), 1);
+                mbar_init(smem_u32(&bempty[s]), 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(smem_u32(&accfull[b]), 1);
+                mbar_init(smem_u32(&accempty[b]), EPI_THREADS / 32);
+            }
+            mbar_init(smem_u32(&done_bar), 1);
+            abort_s = 0;
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc<TMEM_COLS>(smem_u32(&tmem_base_s));
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_s;
+
+    // epilogue thread geometry (warps 2..9)
+    const int et = threadIdx.x - 64;                  // 0..255 for epilogue threads
+    const int q = warp & 3;                           // TMEM lane quarter
+    const int half = (warp - 2) >> 2;                 // column half
+    const int row = q * 32 + lane;                    // tile row of this thread
+    const int col0 = half * 128;
+    float acc[128];
+#pragma unroll
+    for (int c = 0; c < 128; ++c) acc[c] = 0.f;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int as = 0, bs = 0;
+            uint32_t aph = 0, bph = 0, a_issued = 0, b_issued = 0;
+            bool ok = true;
+            for (int kb = kb0; kb < kb1 && ok; ++kb) {
+                if (!mbar_wait_bounded(smem_u32(&aempty[as]), aph ^ 1u, abort_flag, p.status,
+                                       p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(smem_u32(&afull[as]), A_BYTES);
+                tma_load_2d(smem0 + as * A_BYTES, &maps.x, smem_u32(&afull[as]), kb * BK, m0);
+                ++a_issued;
+                if (++as == A_STAGES) { as = 0; aph ^= 1u; }
+                for (int part = PARTS - 1; part >= 0; --part) {
+                    if (!mbar_wait_bounded(smem_u32(&bempty[bs]), bph ^ 1u, abort_flag, p.status,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(smem_u32(&bfull[bs]), b_bytes);
+                    tma_load_3d(b_ring0 + bs * b_bytes, &maps.parts, smem_u32(&bfull[bs]), kb * BK,
+                                0, part);
+                    ++b_issued;
+                    if (++bs == p.b_stages) { bs = 0; bph ^= 1u; }
+                }
+            }
+            // wind down: every load issued into a stage has landed
+            for (int s = 0; s < A_STAGES; ++s)
+                if (a_issued > (uint32_t)s)
+                    drain_wait(smem_u32(&afull[s]), ((a_issued - 1 - s) / A_STAGES) & 1u,
+                               p.timeout_ns, p.status);
+            for (int s = 0; s < p.b_stages; ++s)
+                if (b_issued > (uint32_t)s)
+                    drain_wait(smem_u32(&bfull[s]), ((b_issued - 1 - s) / p.b_stages) & 1u,
+                               p.timeout_ns, p.status);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int as = 0, bs = 0, buf = 0;
+            uint32_t aph = 0, bph = 0, cph = 0;
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                   ((uint32_t)(p.BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+            bool ok = true;
+            for (int kb = kb0; kb < kb1 && ok; ++kb) {
+                if (!mbar_wait_bounded(smem_u32(&accempty[buf]), cph ^ 1u, abort_flag, p.status,
+                                       p.timeout_ns) ||
+                    !mbar_wait_bounded(smem_u32(&afull[as]), aph, abort_flag, p.status,
+                                       p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                const uint64_t a_desc = smem_desc_sw128(smem0 + as * A_BYTES);
+                const uint32_t d_tmem = tmem_base + buf * ACC_COLS;
+                // smallest part first: the fresh accumulator is smallest while
+                // the smallest products are added
+                for (int part = PARTS - 1; part >= 0; --part) {
+                    if (!mbar_wait_bounded(smem_u32(&bfull[bs]), bph, abort_flag, p.status,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t b_desc = smem_desc_sw128(b_ring0 + bs * b_bytes);
+#pragma unroll
+                    for (int ks = 0; ks < BK / 16; ++ks)
+                        tc_mma_bf16(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks, idesc,
+                                    (part == PARTS - 1 && ks == 0) ? 0u : 1u);
+                    tc_commit(smem_u32(&bempty[bs]));
+                    if (++bs == p.b_stages) { bs = 0; bph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&aempty[as]));
+                if (++as == A_STAGES) { as = 0; aph ^= 1u; }
+                tc_commit(smem_u32(&accfull[buf]));
+                if (++buf == 2) { buf = 0; cph ^= 1u; }
+            }
+            tc_commit(smem_u32(&done_bar));
+            drain_wait(smem_u32(&done_bar), 0, p.timeout_ns, p.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue: k blocks
+        int buf = 0;
+        uint32_t cph = 0;
+        const bool has_cols = col0 < p.BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait_bounded(smem_u32(&accfull[buf]), cph, abort_flag, p.status,
+                                   p.timeout_ns))
+                break;
+            tc_fence_after();
+            if (has_cols) {
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(q * 32) << 16) + buf * ACC_COLS + col0;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    if (col0 + ch * 16 < p.BN) {
+                        uint32_t v[16];
+                        tmem_ld16(taddr + ch * 16, v);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            acc[ch * 16 + j] = __fadd_rn(acc[ch * 16 + j], __uint_as_float(v[j]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&accempty[buf]));
+            if (++buf == 2) { buf = 0; cph ^= 1u; }
+        }
+    }
+
+    // ---------------------------------------------------------- cluster reduction
+    // Ring buffers are free once every CTA of the cluster has passed here (its
+    // copies landed, its MMAs done).  Each epilogue thread then stores its
+    // partial logits into red[rank][row - owner*R][col] of the CTA that owns the
+    // row (through distributed shared memory when that is another CTA).
+    tc_fence_before();
+    __syncthreads();
+    const int R = BM / C;                 // token rows owned by each CTA of the cluster
+    const int sp = p.BN + 4;              // floats per row of red
+    float *red = reinterpret_cast<float *>(smem);  // [C][R][sp] in the owner
+    cluster.sync();
+    if (warp >= 2 && col0 < p.BN) {
+        const int owner = row / R;
+        float *base = owner == rank ? red : cluster.map_shared_rank(red, owner);
+        float *dst = base + ((size_t)rank * R + (row - owner * R)) * sp + col0;
+#pragma unroll
+        for (int c = 0; c < 128; c += 4)
+            if (col0 + c < p.BN)
+                *reinterpret_cast<float4 *>(dst + c) =
+                    make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+    }
+    cluster.sync();
+
+    // ---------------------------------------------------------- affinities
+    // L = P_0 + P_1 + ... + P_{C-1} (rank order) + o, s = f(L), written over
+    // red[0] element by element (each element read and written by one thread).
+    const int E = p.E;
+    if (warp >= 2) {
+        for (int i = et; i < R * E; i += EPI_THREADS) {
+            const int rl = i / E, col = i - rl * E;
+            float *e0 = red + (size_t)rl * sp + col;
+            float L = e0[0];
+            for (int r = 1; r < C; ++r) L = __fadd_rn(L, e0[(size_t)r * R * sp]);
+            if (p.off) L += off_s[col];
+            e0[0] = affinity_fn(L, p.affinity);
+        }
+    }
+    const int tpt = EPI_THREADS / R;      // selection threads per token (2C)
+    float *srow = red;                    // s of local token rl at srow[rl * sp + i]
+
+    // ---------------------------------------------------------- selection
+    if (warp >= 2) {
+        epi_sync();
+        const int G = p.G, K = p.K, M = p.M;
+        const int gsz = E / G, kpg = K / M;
+        const int tl = et / tpt, j = et - tl * tpt;
+        const int t = m0 + rank * R + tl;
+        const float *s = srow + (size_t)tl * sp;
+        uint64_t *gkey = reinterpret_cast<uint64_t *>(smem + (size_t)C * R * sp * 4);  // [R][G]
+        uint64_t *lists = gkey + (size_t)R * G;                       // [R][tpt][K]
+        const bool aborted = *abort_flag != 0;
+
+        // step 1: group scores, the sum of each group's top-(K/M) b added in pick order
+        for (int g = j; g < G; g += tpt) {
+            uint64_t prev = ~0ull;
+            float sum = 0.f;
+            for (int r = 0; r < kpg; ++r) {
+                uint64_t best = 0;
+                float bb = 0.f;
+                for (int i = g * gsz; i < (g + 1) * gsz; ++i) {
+                    const float v = __fadd_rn(s[i], bias_s[i]);
+                    const uint64_t k = sel_key(v, i);
+                    if (k < prev && k > best) { best = k; bb = v; }
+                }
+                prev = best;
+                sum = r == 0 ? bb : __fadd_rn(sum, bb);
+            }
+            gkey[(size_t)tl * G + g] = sel_key(sum, g);
+        }
+        epi_sync();
+        // step 2: the M best groups (every thread of the token, same answer)
+        uint64_t keep = 0;
+        {
+            uint64_t prev = ~0ull;
+            for (int r = 0; r < M; ++r) {
+                uint64_t best = 0;
+                for (int g = 0; g < G; ++g) {
+                    const uint64_t k = gkey[(size_t)tl * G + g];
+                    if (k < prev && k > best) best = k;
+                }
+                keep |= 1ull << (key_index(best) & 63);
+                prev = best;
+            }
+        }
+        // step 3: this thread's K best keys among the kept experts i = j (mod tpt),
+        // as a list sorted descending (zero keys past the end)
+        uint64_t *mine = lists + ((size_t)tl * tpt + j) * K;
+        {
+            int n = 0;
+            uint64_t kth = 0;
+            for (int i = j; i < E; i += tpt) {
+                if (!((keep >> (i / gsz)) & 1ull)) continue;
+                const uint64_t k = sel_key(__fadd_rn(s[i], bias_s[i]), i);
+                if (n < K || k > kth) {
+                    int pos = n < K ? n : K - 1;
+                    if (n < K) ++n;
+                    while (pos > 0 && mine[pos - 1] < k) {
+                        mine[pos] = mine[pos - 1];
+                        --pos;
+                    }
+                    mine[pos] = k;
+                    kth = n == K ? mine[K - 1] : 0;
+                }
+            }
+            for (int r = n; r < K; ++r) mine[r] = 0;
+        }
+        epi_sync();
+        // step 4: merge the token's tpt sorted lists; gates over the unbiased s
+        if (j == 0 && t < p.T && !aborted) {
+            const uint64_t *lst = lists + (size_t)tl * tpt * K;
+            int ptr[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) ptr[u] = 0;
+            float denom = 0.f;
+            for (int r = 0; r < K; ++r) {
+                uint64_t best = 0;
+                int bq = 0;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    if (u < tpt && ptr[u] < K) {
+                        const uint64_t k = lst[u * K + ptr[u]];
+                        if (k > best) { best = k; bq = u; }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) ptr[u] += u == bq;
+                int e = key_index(best);
+                e = e < 0 ? 0 : (e >= E ? E - 1 : e);
+                p.topk_idx[(size_t)t * K + r] = e;
+                denom = __fadd_rn(denom, s[e]);
+            }
+            for (int r = 0; r < K; ++r) {
+                const int e = p.topk_idx[(size_t)t * K + r];
+                p.topk_w[(size_t)t * K + r] = __fdiv_rn(s[e], denom);
+            }
+        }
+        // affinities, when the caller asked for them (coalesced row copies)
+        if (p.scores && !aborted) {
+            for (int i = et; i < R * E; i += EPI_THREADS) {
+                const int rl = i / E, col = i - rl * E;
+                const int tt = m0 + rank * R + rl;
+                if (tt < p.T) p.scores[(size_t)tt * E + col] = srow[(size_t)rl * sp + col];
+            }
+        }
+    }
+
+    // ---------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<TMEM_COLS>(tmem_base);
+    }
+}
+
+}  // namespace rfused
+
+bool router_fused_supported(int E, int G, int K) { return E <= 256 && G <= 32 && K <= 16; }
+
+int router_fused_cluster(int T, int d) {
+    const int tiles = (T + rfused::BM - 1) / rfused::BM;
+    const int kblocks = d / rfused::BK;
+    int c = 1;
+    while (c < 8 && tiles * c * 2 <= 148 && kblocks / (c * 2) >= 4) c *= 2;
+    return c;
+}
+
+cudaError_t launch_router_select_fused(const void *x, const void *e_split, const float *off,
+                                       const float *bias, int T, int d, int E, int G, int K,
+                                       int M, int affinity, float *scores, int32_t *topk_idx,
+                                       float *topk_w, int32_t *status, int64_t timeout_ns,
+                                       cudaStream_t st) {
+    using namespace rfused;
+    if (T == 0) return cudaSuccess;
+    const int BN = (E + 15) / 16 * 16;
+    const int C = router_fused_cluster(T, d);
+    const int R = BM / C, tpt = EPI_THREADS / R;
+    const size_t b_bytes = (size_t)BN * BK * 2;
+    int b_stages = (int)(B_RING_BYTES / b_bytes);
+    if (b_stages > MAX_B_STAGES) b_stages = MAX_B_STAGES;
+    const size_t ring = (size_t)A_STAGES * A_BYTES + b_stages * b_bytes;
+    // after the k loop the same bytes hold the received partials, then the
+    // affinity rows, group keys and candidate lists of the selection
+    const size_t post = (size_t)BM * (BN + 4) * 4 + (size_t)R * G * 8 + (size_t)R * tpt * K * 8;
+    size_t dyn = ring > post ? ring : post;
+    dyn += 1024;
+    Maps m;
+    if (!tensor_map_2d_bf16(&m.x, x, T, d, BK, BM) ||
+        !tensor_map_3d_bf16(&m.parts, e_split, PARTS, E, d, BK, BN))
+        return cudaErrorInvalidValue;
+    Params p{T, E, d, G, K, M, BN, b_stages, C, affinity, off, bias, scores, topk_idx, topk_w,
+             status, timeout_ns};
+    cudaError_t err = cudaFuncSetAttribute(router_select_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (err != cudaSuccess) return err;
+    const int tiles = (T + BM - 1) / BM;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(tiles * C);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = dyn;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, router_select_kernel, m, p);
+    count_launch();
+    return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+}  // namespace moe

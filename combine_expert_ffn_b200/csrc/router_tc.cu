@@ -296,6 +296,17 @@ __global__ void router_finish_kernel(const float *__restrict__ partial, int spli
 
 }  // namespace router
 
+cudaError_t launch_router_split(const float *e, int E, int d, void *e_split, cudaStream_t st) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t n = (int64_t)E * d;
+    router::router_split_kernel<<<(int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 8), 256,
+                                  0, st>>>(e, n, static_cast<__nv_bfloat16 *>(e_split));
+    count_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *off, int T, int d,
                                     int E, int affinity, void *e_split, float *partial,
                                     float *scores, int32_t *status, int64_t timeout_ns,
@@ -305,11 +316,7 @@ cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t n = (int64_t)E * d;
-    router_split_kernel<<<(int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 8), 256, 0, st>>>(
-        e, n, static_cast<__nv_bfloat16 *>(e_split));
-    count_launch();
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_router_split(e, E, d, e_split, st);
     if (err != cudaSuccess) return err;
     Maps m;
     if (!tensor_map_2d_bf16(&m.x, x, T, d, BK, BM) ||

@@ -99,8 +99,13 @@ CONFIGS = {
 # v3_ep: the V3 row width and top-8 over 4096 tokens and 32 narrow experts, for
 # captures of the expert-parallel exchange kernels (2 ranks of 2048 tokens: one
 # combine launch reads 235 MB, above L2) within a few GB.
+# v3_ffn64: the V3 batch, router and routing exactly (T=8192, d=7168, E=256,
+# K=8) with 64-wide expert FFNs, for captures of the route, dispatch and
+# combine kernels at full size within a few GB (their work does not depend on
+# d_ff).
 PROFILE_CONFIGS = {
     "v3_e32": CONFIGS["v3"].replace(name="v3_e32", T=1024, E=32),
+    "v3_ffn64": CONFIGS["v3"].replace(name="v3_ffn64", d_ff=64, d_ff_shared=64),
     "v3_ep": CONFIGS["v3"].replace(name="v3_ep", T=4096, E=32, d_ff=512),
 }
 

@@ -101,14 +101,30 @@ def test_route_select_exact_ties(orc, E, G, K, M):
 
 
 @pytest.mark.parametrize("name,n_sample", [("tiny", None), ("ragged", None), ("ragged2", None),
-                                           ("mid", 256), ("v3", 64), ("skew", 64)])
+                                           ("mid", 256), ("v3", 64), ("decode", None),
+                                           ("skew", 64)])
 def test_route_affinities_and_selection(orc, name, n_sample):
+    """moe_route: affinities within 1e-5 of the oracle's; the selection equals
+    the oracle's selection on the kernel's own affinities bit for bit (every
+    token), and the oracle's on its own affinities except at certified near
+    ties.  These workloads cover the fused router's cluster sizes 1 (tiny,
+    ragged, skew), 2 (v3), 4 (mid) and 8 (decode)."""
     sh = H.shape(name)
     inp = inputs(name)
     idx, w, s = _i32(sh.T, sh.K), _f32(sh.T, sh.K), _f32(sh.T, sh.E)
     cfg = moe.MoeConfig.of(sh)
+    ws = moe.alloc_workspace(cfg)
     moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"], idx, w,
-                  scores=s, ws=moe.alloc_workspace(cfg))
+                  scores=s, ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    own_idx, own_w = orc.select(s.cpu(), inp["bias"].cpu(), sh.G, sh.K, sh.M)
+    np.testing.assert_array_equal(idx.cpu().numpy(), own_idx)
+    np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), own_w.view(np.uint32))
+    # without the affinities output the routing is the same
+    idx2, w2 = _i32(sh.T, sh.K), _f32(sh.T, sh.K)
+    moe.moe_route(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"], idx2, w2,
+                  scores=None, ws=ws)
+    assert torch.equal(idx, idx2) and torch.equal(w.view(torch.int32), w2.view(torch.int32))
     rows = np.arange(sh.T) if n_sample is None else \
         np.unique(np.linspace(0, sh.T - 1, n_sample).astype(np.int64))
     ref_s = orc.router_scores(inp["x"].cpu(), inp["router_w"].cpu(), H.host(inp.get("logit_offset")),
@@ -133,6 +149,32 @@ def test_route_affinities_and_selection(orc, name, n_sample):
         assert len({int(e) // gsz for e in all_idx[t]}) <= sh.M
     wsum = w.double().sum(dim=1).cpu().numpy()
     assert np.abs(wsum - 1).max() < 1e-6 and (w > 0).all()
+
+
+@pytest.mark.parametrize("E,G,K,M,T", [(16, 4, 4, 2, 512), (64, 8, 8, 4, 512),
+                                       (256, 8, 8, 4, 512), (96, 32, 4, 4, 512),
+                                       (256, 8, 8, 4, 128)])
+def test_fused_route_exact_ties(orc, E, G, K, M, T):
+    """Exact ties inside the fused router: experts share router rows in pairs
+    (bit-identical logits) and the bias takes four levels, so biased affinities
+    and group scores tie exactly; the kernel's selection must still equal the
+    oracle's on the kernel's own affinities, bit for bit."""
+    d = 512
+    x = synth.normal(5, 1, (T, d), 1.0, torch.bfloat16, DEV)
+    base = synth.normal(5, 2, (E // 2, d), d ** -0.5, torch.float32, DEV)
+    router_w = base.repeat_interleave(2, dim=0).contiguous()
+    levels = torch.tensor([0.0, 0.125, 0.25, 0.375], device=DEV)
+    bias = levels[(synth.uniform01(5, 3, (E,), DEV) * 4).long().clamp(max=3)]
+    cfg = moe.MoeConfig(T=T, d=d, E=E, G=G, K=K, M=M, d_ff=64, n_shared=0, d_ff_shared=0)
+    idx, w, s = _i32(T, K), _f32(T, K), _f32(T, E)
+    ws = moe.alloc_workspace(cfg)
+    moe.moe_route(cfg, x, router_w, None, bias, idx, w, scores=s, ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    sh_ = s.cpu()
+    assert torch.equal(sh_[:, 0::2].view(torch.int32), sh_[:, 1::2].view(torch.int32))
+    ref_idx, ref_w = orc.select(sh_, bias.cpu(), G, K, M)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), ref_w.view(np.uint32))
 
 
 # ---------------------------------------------------------------- dispatch
