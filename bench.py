@@ -301,6 +301,14 @@ def run_ours(args, sh, world, rank, local):
     ws = moe.alloc_workspace(cfg, dev)
     o = moe.forward_outputs(cfg, dev)
     T, K, E, G, d = sh.T, sh.K, sh.E, sh.G, sh.d
+    # expert weights in the library's tile-packed layout: transformed once here, at
+    # load time, outside every timed region (the row-major copies stay for the e2e
+    # leg's reference and are not read by the packed path)
+    packed = None
+    if args.weights == "packed":
+        packed = moe.pack_weights(cfg, inp["w_gate"], inp["w_up"], inp["w_down"],
+                                  inp["ws_gate"], inp["ws_up"], inp["ws_down"], device=dev)
+        torch.cuda.synchronize(dev)
     # stage buffers (the same intermediates moe_forward keeps in its workspace)
     perm_token = torch.empty(T * K, dtype=torch.int32, device=dev)
     inv_perm = torch.empty(T, K, dtype=torch.int32, device=dev)
@@ -325,9 +333,13 @@ def run_ours(args, sh, world, rank, local):
         moe.moe_permute(cfg, inp["x"], inv_perm, x_perm, stream)
         if ev is not None:
             ev[3].record(stream)
-        moe.moe_expert_ffn(cfg, x_perm, o["offsets"], inp["w_gate"], inp["w_up"], inp["w_down"],
-                           y_perm, inp["x"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], y_sh,
-                           ws, stream)
+        if packed is not None:
+            moe.moe_expert_ffn_packed(cfg, x_perm, o["offsets"], packed, y_perm, inp["x"], y_sh,
+                                      ws, stream)
+        else:
+            moe.moe_expert_ffn(cfg, x_perm, o["offsets"], inp["w_gate"], inp["w_up"],
+                               inp["w_down"], y_perm, inp["x"], inp["ws_gate"], inp["ws_up"],
+                               inp["ws_down"], y_sh, ws, stream)
         if ev is not None:
             ev[4].record(stream)
         moe.moe_combine(cfg, y_perm, inv_perm, o["topk_w"], y_sh, o["out"], stream)
@@ -371,7 +383,8 @@ def run_ours(args, sh, world, rank, local):
         raise RuntimeError(f"device status {status} after the timed region")
 
     # ---- end to end through moe_forward with pinned host buffers
-    e2e = e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world) if not args.no_e2e else None
+    e2e = e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world, packed) \
+        if not args.no_e2e else None
     if rank != 0:
         return 0
     counts = o["counts"].cpu()
@@ -394,7 +407,7 @@ def run_ours(args, sh, world, rank, local):
     return 0
 
 
-def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world):
+def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world, packed=None):
     """moe_forward on pinned host buffers, every step's H2D of x and D2H of out
     inside the timed region.  Steps are pipelined the way a serving loop runs
     them: x of step i+1 goes up on a copy stream and out of step i-1 comes
@@ -423,9 +436,14 @@ def e2e_leg(args, sh, cfg, inp, ws, o, stream, dev, world):
             stream.wait_event(up_done[b])
             if i >= NB:
                 stream.wait_event(down_done[b])    # step i-NB's out_dev[b] is on the host
-            moe.moe_forward(cfg, x_dev[b], inp["router_w"], inp.get("logit_offset"), inp["bias"],
-                            inp["w_gate"], inp["w_up"], inp["w_down"], inp["ws_gate"],
-                            inp["ws_up"], inp["ws_down"], out_dev[b], ws=ws, stream=stream)
+            if packed is not None:
+                moe.moe_forward_packed(cfg, x_dev[b], inp["router_w"], inp.get("logit_offset"),
+                                       inp["bias"], packed, out_dev[b], ws=ws, stream=stream)
+            else:
+                moe.moe_forward(cfg, x_dev[b], inp["router_w"], inp.get("logit_offset"),
+                                inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"],
+                                inp["ws_gate"], inp["ws_up"], inp["ws_down"], out_dev[b], ws=ws,
+                                stream=stream)
             fwd_done[b].record(stream)
             s_down.wait_event(fwd_done[b])
             with torch.cuda.stream(s_down):
@@ -778,6 +796,9 @@ def report(args, sh, world, ms_total, stage_ms, launches, clk, e2e, touched_expe
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded counter-based generator, random-init weights)",
         "config": {"workload": sh.name, **sh.as_dict(), "parallelism": f"replicas x{world}",
+                   "expert_weights": (
+                       "tile-packed (moe_pack_weights, once at load, outside the timed region)"
+                       if args.weights == "packed" else "row-major"),
                    "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
                          % ((3 * sh.E * sh.d * sh.d_ff + 3 * sh.n_shared * sh.d * sh.d_ff_shared) * 2 / 1e9)},
         "roofline": ({"bound": "tensor", "kernel": "expert FFN: grouped_ffn_gemm_kernel<SwiGLU> + <store> (2 launches)",
@@ -848,6 +869,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--ep-world", type=int, default=8,
                     help="ranks of the emulated expert-parallel leg (1 = skip)")
+    ap.add_argument("--weights", default="packed", choices=["packed", "row-major"],
+                    help="expert weights in the tile-packed layout (packed once at load) or "
+                         "row-major")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the router-variant and bias-update timings")
     args = ap.parse_args()

@@ -41,7 +41,8 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_ep_dispatch_dedup", "moe_ep_fanout", "moe_ep_dispatch_dedup_fp8",
            "moe_ep_fanout_fp8", "moe_ep_combine_plan",
            "moe_ep_precombine", "moe_ep_combine_dedup", "moe_ipc_get_handle",
-           "moe_ipc_open_handle", "moe_ipc_close_handle")
+           "moe_ipc_open_handle", "moe_ipc_close_handle", "moe_packed_weights_size",
+           "moe_pack_weights", "moe_expert_ffn_packed", "moe_forward_packed")
 
 MOE_ROUTER_SIGMOID, MOE_ROUTER_SQRT_SOFTPLUS, MOE_ROUTER_HASH = 0, 1, 2
 MOE_PAYLOAD_BF16, MOE_PAYLOAD_FP8 = 0, 1
@@ -122,6 +123,11 @@ _sig = {
     "moe_bias_update": (C.c_int, [_CP, _P, C.c_float, _P, _P]),
     "moe_selftest_bounded_wait": (C.c_int, [_I64, _P, _P]),
     "moe_dispatch_noalloc": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_packed_weights_size": (_S, [_CP]),
+    "moe_pack_weights": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_expert_ffn_packed": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "moe_forward_packed": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                     _P, _S, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -436,6 +442,48 @@ def moe_forward(cfg, x, router_w, logit_offset, bias, w_gate, w_up, w_down, ws_g
                                         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(out),
                                         _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(offsets),
                                         _ptr(send), _ptr(send_tok), wp, wn, _stream(stream)))
+
+
+def moe_packed_weights_size(cfg) -> int:
+    return int(_lib.moe_packed_weights_size(_cfg(cfg)))
+
+
+def moe_pack_weights(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed,
+                     stream=None) -> None:
+    _ok("moe_pack_weights", _lib.moe_pack_weights(_cfg(cfg), _ptr(w_gate), _ptr(w_up),
+                                                  _ptr(w_down), _ptr(ws_gate), _ptr(ws_up),
+                                                  _ptr(ws_down), _ptr(packed), _stream(stream)))
+
+
+def pack_weights(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, device="cuda",
+                 stream=None):
+    """Allocates the packed-weight buffer (uint8) and fills it with moe_pack_weights."""
+    n = moe_packed_weights_size(cfg)
+    if n == 0:
+        raise MoeError("moe_packed_weights_size", MOE_ERR_UNSUPPORTED_SHAPE)
+    packed = torch.empty(n, dtype=torch.uint8, device=device)
+    moe_pack_weights(cfg, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed, stream)
+    return packed
+
+
+def moe_expert_ffn_packed(cfg, x_perm, offsets, packed, y_perm, x, y_shared, ws,
+                          stream=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_expert_ffn_packed",
+        _lib.moe_expert_ffn_packed(_cfg(cfg), _ptr(x_perm), _ptr(offsets), _ptr(packed),
+                                   _ptr(y_perm), _ptr(x), _ptr(y_shared), wp, wn,
+                                   _stream(stream)))
+
+
+def moe_forward_packed(cfg, x, router_w, logit_offset, bias, packed, out, topk_idx=None,
+                       topk_w=None, counts=None, offsets=None, send=None, send_tok=None, ws=None,
+                       stream=None, token_ids=None) -> None:
+    wp, wn = _ws(ws)
+    _ok("moe_forward_packed",
+        _lib.moe_forward_packed(_cfg(cfg), _ptr(x), _ptr(router_w), _ptr(logit_offset),
+                                _ptr(bias), _ptr(token_ids), _ptr(packed), _ptr(out),
+                                _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(offsets),
+                                _ptr(send), _ptr(send_tok), wp, wn, _stream(stream)))
 
 
 def moe_selftest_bounded_wait(timeout_ns, ws, stream=None) -> None:

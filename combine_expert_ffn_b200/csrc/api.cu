@@ -437,22 +437,29 @@ moe_status moe_combine(const moe_config *c, const void *y_perm, const int32_t *i
                                       (int64_t)c->T * c->K, out, as_stream(stream)));
 }
 
-moe_status moe_forward(const moe_config *c, const void *x, const float *router_w,
-                       const float *logit_offset, const float *bias, const int64_t *token_ids,
-                       const void *w_gate,
-                       const void *w_up, const void *w_down, const void *ws_gate,
-                       const void *ws_up, const void *ws_down, void *out, int32_t *topk_idx,
-                       float *topk_w, int32_t *counts, int32_t *offsets, int32_t *send,
-                       int32_t *send_tok, void *ws, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+// The layer forward over row-major weights (packed == null) or the packed ones.
+static moe_status forward_impl(const moe_config *c, const void *x, const float *router_w,
+                               const float *logit_offset, const float *bias,
+                               const int64_t *token_ids, const void *w_gate, const void *w_up,
+                               const void *w_down, const void *ws_gate, const void *ws_up,
+                               const void *ws_down, const void *packed, void *out,
+                               int32_t *topk_idx, float *topk_w, int32_t *counts,
+                               int32_t *offsets, int32_t *send, int32_t *send_tok, void *ws,
+                               size_t ws_bytes, void *stream) {
     moe_status st = moe_check_config(c);
     if (st) return st;
     if (!ws) return MOE_ERR_INVALID_ARG;
+    if (packed && c->payload == MOE_PAYLOAD_FP8) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->T > 0) {
-        if (!x || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+        if (!x || !out) return MOE_ERR_INVALID_ARG;
+        if (!packed && (!w_gate || !w_up || !w_down)) return MOE_ERR_INVALID_ARG;
         if (c->router != MOE_ROUTER_HASH && !router_w) return MOE_ERR_INVALID_ARG;
-        if (c->n_shared > 0 && (!ws_gate || !ws_up || !ws_down)) return MOE_ERR_INVALID_ARG;
+        if (!packed && c->n_shared > 0 && (!ws_gate || !ws_up || !ws_down))
+            return MOE_ERR_INVALID_ARG;
     }
-    const void *ptrs[] = {x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out};
+    const void *ptrs[] = {x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out, packed};
     for (const void *p : ptrs)
         if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
     const Layout L = layout(*c);
@@ -509,11 +516,92 @@ moe_status moe_forward(const moe_config *c, const void *x, const float *router_w
     a.h = at<void>(ws, L.h); a.y_perm = y_perm;
     a.x = x; a.ws_gate = ws_gate; a.ws_up = ws_up; a.ws_down = ws_down;
     a.h_shared = at<void>(ws, L.h_sh); a.y_shared = y_sh;
+    a.packed = packed;
     a.status = status;
     a.timeout_ns = kWaitTimeoutNs;
     if (launch_expert_ffn(a, s)) return MOE_ERR_CUDA;
     return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_sh, c->T, c->d, c->K,
                                       (int64_t)c->T * c->K, out, s));
+}
+
+extern "C" {
+
+moe_status moe_forward(const moe_config *c, const void *x, const float *router_w,
+                       const float *logit_offset, const float *bias, const int64_t *token_ids,
+                       const void *w_gate,
+                       const void *w_up, const void *w_down, const void *ws_gate,
+                       const void *ws_up, const void *ws_down, void *out, int32_t *topk_idx,
+                       float *topk_w, int32_t *counts, int32_t *offsets, int32_t *send,
+                       int32_t *send_tok, void *ws, size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->T > 0 && (!w_gate || !w_up || !w_down)) return MOE_ERR_INVALID_ARG;
+    return forward_impl(c, x, router_w, logit_offset, bias, token_ids, w_gate, w_up, w_down,
+                        ws_gate, ws_up, ws_down, nullptr, out, topk_idx, topk_w, counts, offsets,
+                        send, send_tok, ws, ws_bytes, stream);
+}
+
+moe_status moe_forward_packed(const moe_config *c, const void *x, const float *router_w,
+                              const float *logit_offset, const float *bias,
+                              const int64_t *token_ids, const void *packed, void *out,
+                              int32_t *topk_idx, float *topk_w, int32_t *counts, int32_t *offsets,
+                              int32_t *send, int32_t *send_tok, void *ws, size_t ws_bytes,
+                              void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (c->T > 0 && !packed) return MOE_ERR_INVALID_ARG;
+    return forward_impl(c, x, router_w, logit_offset, bias, token_ids, nullptr, nullptr, nullptr,
+                        nullptr, nullptr, nullptr, packed, out, topk_idx, topk_w, counts, offsets,
+                        send, send_tok, ws, ws_bytes, stream);
+}
+
+size_t moe_packed_weights_size(const moe_config *c) {
+    if (moe_check_config(c) != MOE_OK) return 0;
+    return packed_layout(c->E, c->d, c->d_ff, c->n_shared, c->d_ff_shared).total;
+}
+
+moe_status moe_pack_weights(const moe_config *c, const void *w_gate, const void *w_up,
+                            const void *w_down, const void *ws_gate, const void *ws_up,
+                            const void *ws_down, void *packed, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!w_gate || !w_up || !w_down || !packed) return MOE_ERR_INVALID_ARG;
+    if (c->n_shared > 0 && (!ws_gate || !ws_up || !ws_down)) return MOE_ERR_INVALID_ARG;
+    const void *ptrs[] = {w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    return cuda_status(launch_pack_weights(c->E, c->d, c->d_ff, c->n_shared, c->d_ff_shared,
+                                           w_gate, w_up, w_down, ws_gate, ws_up, ws_down, packed,
+                                           as_stream(stream)));
+}
+
+moe_status moe_expert_ffn_packed(const moe_config *c, const void *x_perm, const int32_t *offsets,
+                                 const void *packed, void *y_perm, const void *x, void *y_shared,
+                                 void *ws, size_t ws_bytes, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (c->T > 0) {
+        if (!x_perm || !offsets || !packed || !y_perm) return MOE_ERR_INVALID_ARG;
+        if (c->n_shared > 0 && (!x || !y_shared)) return MOE_ERR_INVALID_ARG;
+    }
+    const void *ptrs[] = {x_perm, packed, y_perm, x, y_shared};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout(*c);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    FfnArgs a{};
+    a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
+    a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
+    a.x_perm = x_perm; a.offsets = offsets; a.packed = packed;
+    a.h = at<void>(ws, L.h); a.y_perm = y_perm;
+    a.x = x; a.h_shared = at<void>(ws, L.h_sh); a.y_shared = y_shared;
+    a.status = at<int32_t>(ws, L.status);
+    a.timeout_ns = kWaitTimeoutNs;
+    return cuda_status(launch_expert_ffn(a, as_stream(stream)));
 }
 
 // ----------------------------------------------------------------- expert parallelism

@@ -29,6 +29,8 @@
 // those rows are computed and never stored.  Every wait is bounded; on
 // running out the kernel records MOE_ERR_DEVICE_TIMEOUT, drains its own TMA
 // loads and MMAs, frees TMEM and returns.
+#include <cstring>
+
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -44,9 +46,14 @@
 #define MOE_PAIR_GEMM2 0
 #endif
 
+#ifndef MOE_GEMM_KB_GROUP
+#define MOE_GEMM_KB_GROUP 1
+#endif
+
 namespace moe {
 namespace gemm {
 
+constexpr int KB_GROUP = MOE_GEMM_KB_GROUP;
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int BN_ACC = 256;
@@ -112,7 +119,23 @@ struct Params {
     int32_t *status;
     int64_t timeout_ns;
     int *tile_counter;       // paired kernel: next tile to hand out (zero at launch)
+    // packed weights (pack.cu): the B tile (e, n, kb) is the 32 KB block
+    // ((e * bp_nt_r + n) * k_r/64 + kb) of bp_r (routed) and (n * k_s/64 + kb) of
+    // bp_s (shared); null: tensor-map loads of the row-major weights
+    const uint8_t *bp_r, *bp_s;
+    int bp_nt_r;
 };
+
+// The B tile of (tile, k block kb) from the packed weights: one 32 KB bulk copy.
+template <int EPI>
+__device__ __forceinline__ void load_packed_b(const Params &p, int e, int n0, int kb,
+                                              uint32_t dst, uint32_t bar) {
+    const int n = n0 / Cfg<EPI>::BN_OUT;
+    const uint8_t *src = e >= 0
+        ? p.bp_r + ((((size_t)e * p.bp_nt_r + n) * (p.k_r / BK) + kb) << 15)
+        : p.bp_s + ((((size_t)n) * (p.k_s / BK) + kb) << 15);
+    bulk_load(dst, src, 32768, bar);
+}
 
 struct Tile {
     int row0;        // first A row
@@ -241,12 +264,16 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
             tma_prefetch_desc(&maps.o_r);
             if (AMODE == A_TMA) tma_prefetch_desc(&maps.a_r);
             if (AMODE == A_FP8) tma_prefetch_desc(&maps.a_q);
-            tma_prefetch_desc(&maps.b0_r);
-            if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
+            if (!p.bp_r) {
+                tma_prefetch_desc(&maps.b0_r);
+                if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
+            }
             if (p.T > 0) {
                 tma_prefetch_desc(&maps.a_s);
-                tma_prefetch_desc(&maps.b0_s);
-                if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_s);
+                if (!p.bp_s) {
+                    tma_prefetch_desc(&maps.b0_s);
+                    if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_s);
+                }
             }
         }
     } else if (warp == 1) {
@@ -289,6 +316,20 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                 const bool a_by_tma = AMODE == A_TMA || t.e < 0;
                 bool ok = true;
                 for (int kb = 0; kb < t.kblocks; ++kb) {
+                    // KB_GROUP > 1: wait until the next KB_GROUP stages are free, so that
+                    // the copies of adjacent k blocks (adjacent bytes of the same rows)
+                    // are requested together
+                    if (KB_GROUP > 1 && kb % KB_GROUP == 0) {
+                        int st2 = stage;
+                        uint32_t ph2 = phase;
+                        for (int g = 0; g < KB_GROUP && kb + g < t.kblocks && ok; ++g) {
+                            if (!mbar_wait_bounded(smem_u32(&empty_bar[st2]), ph2 ^ 1u, abort_flag,
+                                                   p.status, p.timeout_ns))
+                                ok = false;
+                            if (++st2 == STAGES) { st2 = 0; ph2 ^= 1u; }
+                        }
+                        if (!ok) break;
+                    }
                     if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
                                            p.status, p.timeout_ns)) {
                         ok = false;
@@ -310,7 +351,9 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                     }
                     if (t.e >= 0) {
                         if (a_by_tma) tma_load_2d(a_dst, &maps.a_r, fb, k, t.row0);
-                        if (EPI == EPI_SWIGLU) {
+                        if (p.bp_r) {
+                            load_packed_b<EPI>(p, t.e, t.n0, kb, b_dst, fb);
+                        } else if (EPI == EPI_SWIGLU) {
                             tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
                             tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_r, fb, k, t.n0, t.e);
                         } else {
@@ -318,7 +361,9 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                         }
                     } else {
                         tma_load_2d(a_dst, &maps.a_s, fb, k, t.row0);
-                        if (EPI == EPI_SWIGLU) {
+                        if (p.bp_s) {
+                            load_packed_b<EPI>(p, -1, t.n0, kb, b_dst, fb);
+                        } else if (EPI == EPI_SWIGLU) {
                             tma_load_3d(b_dst, &maps.b0_s, fb, k, t.n0, 0);
                             tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_s, fb, k, t.n0, 0);
                         } else {
@@ -740,12 +785,16 @@ grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
             tile_base[p.E] = carry;
             tma_prefetch_desc(&maps.o_r);
             tma_prefetch_desc(&maps.a_r);
-            tma_prefetch_desc(&maps.b0_r);
-            if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
+            if (!p.bp_r) {
+                tma_prefetch_desc(&maps.b0_r);
+                if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_r);
+            }
             if (p.T > 0) {
                 tma_prefetch_desc(&maps.a_s);
-                tma_prefetch_desc(&maps.b0_s);
-                if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_s);
+                if (!p.bp_s) {
+                    tma_prefetch_desc(&maps.b0_s);
+                    if (EPI == EPI_SWIGLU) tma_prefetch_desc(&maps.b1_s);
+                }
             }
         }
     } else if (warp == 1) {
@@ -811,7 +860,9 @@ grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
                     if (t.e >= 0) {
                         tma_load_2d(a0, &maps.a_r, fb, k, t.row0);
                         if (two) tma_load_2d(a0 + A_BYTES, &maps.a_r, fb, k, t.row0 + BM);
-                        if (EPI == EPI_SWIGLU) {
+                        if (p.bp_r) {
+                            load_packed_b<EPI>(p, t.e, t.n0, kb, b_dst, fb);
+                        } else if (EPI == EPI_SWIGLU) {
                             tma_load_3d(b_dst, &maps.b0_r, fb, k, t.n0, t.e);
                             tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_r, fb, k, t.n0, t.e);
                         } else {
@@ -820,7 +871,9 @@ grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
                     } else {
                         tma_load_2d(a0, &maps.a_s, fb, k, t.row0);
                         if (two) tma_load_2d(a0 + A_BYTES, &maps.a_s, fb, k, t.row0 + BM);
-                        if (EPI == EPI_SWIGLU) {
+                        if (p.bp_s) {
+                            load_packed_b<EPI>(p, -1, t.n0, kb, b_dst, fb);
+                        } else if (EPI == EPI_SWIGLU) {
                             tma_load_3d(b_dst, &maps.b0_s, fb, k, t.n0, 0);
                             tma_load_3d(b_dst + BN_ACC / 2 * BK * 2, &maps.b1_s, fb, k, t.n0, 0);
                         } else {
@@ -1081,9 +1134,15 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
 
     // GEMM1: h = SwiGLU(x_perm) per expert; h_shared = SwiGLU(x) for the shared experts
     Maps m1;
+    std::memset(&m1, 0, sizeof(m1));
     const bool gather = a.perm_token != nullptr;
-    bool ok = map_3d(&m1.b0_r, a.w_gate, a.E, a.d_ff, a.d, BN_ACC / 2) &&
-              map_3d(&m1.b1_r, a.w_up, a.E, a.d_ff, a.d, BN_ACC / 2);
+    const bool packed = a.packed != nullptr;
+    PackedLayout PL{};
+    if (packed) PL = packed_layout(a.E, a.d, a.d_ff, a.n_shared, a.d_ff_shared);
+    const uint8_t *pk = static_cast<const uint8_t *>(a.packed);
+    // with packed weights the B maps stay unused (zero) and are never touched
+    bool ok = packed || (map_3d(&m1.b0_r, a.w_gate, a.E, a.d_ff, a.d, BN_ACC / 2) &&
+                         map_3d(&m1.b1_r, a.w_up, a.E, a.d_ff, a.d, BN_ACC / 2));
     // routed A: x_perm by tiled loads, x rows gathered by the gatherer warps, or the
     // FP8 payload by byte tiles (a_r then only stands in for the unused map)
     const bool fp8 = a.x_perm_q != nullptr;
@@ -1095,8 +1154,8 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     if (!fp8) m1.a_q = m1.a_r;
     if (has_shared)
         ok = ok && map_2d(&m1.a_s, a.x, a.T, a.d, BM) &&
-             map_3d(&m1.b0_s, a.ws_gate, 1, ffs, a.d, BN_ACC / 2) &&
-             map_3d(&m1.b1_s, a.ws_up, 1, ffs, a.d, BN_ACC / 2);
+             (packed || (map_3d(&m1.b0_s, a.ws_gate, 1, ffs, a.d, BN_ACC / 2) &&
+                         map_3d(&m1.b1_s, a.ws_up, 1, ffs, a.d, BN_ACC / 2)));
     else
         m1.a_s = m1.a_r, m1.b0_s = m1.b0_r, m1.b1_s = m1.b1_r;
     // output maps for the full-tile TMA stores (box 32 x 32, no swizzle)
@@ -1125,6 +1184,11 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p1.status = a.status;
     p1.timeout_ns = a.timeout_ns;
     p1.tile_counter = counters;
+    if (packed) {
+        p1.bp_r = pk + PL.gu;
+        p1.bp_s = has_shared ? pk + PL.gu_s : nullptr;
+        p1.bp_nt_r = PL.nt1;
+    }
     cudaError_t err = fp8      ? launch_one<EPI_SWIGLU, A_FP8>(m1, p1, st)
                       : gather ? launch_one<EPI_SWIGLU, A_GATHER>(m1, p1, st)
                       : MOE_PAIR_GEMM1 ? launch_pair<EPI_SWIGLU>(m1, p1, st)
@@ -1133,11 +1197,12 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
 
     // GEMM2: y_perm = h W_d^T per expert; y_shared = h_shared Ws_d^T (k split per shared expert)
     Maps m2;
+    std::memset(&m2, 0, sizeof(m2));
     ok = map_2d(&m2.a_r, a.h, rows_r, a.d_ff, BM) &&
-         map_3d(&m2.b0_r, a.w_down, a.E, a.d, a.d_ff, BN_ACC);
+         (packed || map_3d(&m2.b0_r, a.w_down, a.E, a.d, a.d_ff, BN_ACC));
     if (has_shared)
         ok = ok && map_2d(&m2.a_s, a.h_shared, a.T, ffs, BM) &&
-             map_3d(&m2.b0_s, a.ws_down, a.n_shared, a.d, a.d_ff_shared, BN_ACC);
+             (packed || map_3d(&m2.b0_s, a.ws_down, a.n_shared, a.d, a.d_ff_shared, BN_ACC));
     else
         m2.a_s = m2.a_r, m2.b0_s = m2.b0_r;
     m2.b1_r = m2.b0_r;
@@ -1160,6 +1225,11 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     p2.out_r = static_cast<__nv_bfloat16 *>(a.y_perm);
     p2.out_s = static_cast<__nv_bfloat16 *>(a.y_shared);
     p2.tile_counter = counters + 1;
+    if (packed) {
+        p2.bp_r = pk + PL.down;
+        p2.bp_s = has_shared ? pk + PL.down_s : nullptr;
+        p2.bp_nt_r = PL.nt2;
+    }
     return MOE_PAIR_GEMM2 ? launch_pair<EPI_STORE>(m2, p2, st)
                           : launch_one<EPI_STORE, A_TMA>(m2, p2, st);
 }

@@ -113,6 +113,18 @@ cudaError_t launch_ep_combine(const int32_t *topk_idx, const float *topk_w, cons
                               int T, int d, int E, int K, int world, void *out, int32_t *status,
                               cudaStream_t st);
 
+// pack.cu: expert weights as tile-contiguous, pre-swizzled 32 KB blocks
+// (byte offsets of the four regions inside the packed buffer)
+struct PackedLayout {
+    int nt1, kb1, nt2, kb2, nt1s, kb2s;  // column tiles / k blocks per region
+    size_t gu, down, gu_s, down_s, total;
+};
+PackedLayout packed_layout(int E, int d, int d_ff, int n_shared, int d_ff_shared);
+cudaError_t launch_pack_weights(int E, int d, int d_ff, int n_shared, int d_ff_shared,
+                                const void *w_gate, const void *w_up, const void *w_down,
+                                const void *ws_gate, const void *ws_up, const void *ws_down,
+                                void *packed, cudaStream_t st);
+
 // combine.cu
 cudaError_t launch_combine(const void *y_perm, const int32_t *inv_perm, const float *topk_w,
                            const void *y_shared, int T, int d, int K, int64_t n_rows, void *out,
@@ -131,6 +143,7 @@ struct FfnArgs {
     void *y_perm;   // [T*K, d] bf16
     const void *x;  // [T, d]
     const void *ws_gate, *ws_up, *ws_down;
+    const void *packed;  // weights from launch_pack_weights, or null: the row-major ones above
     void *h_shared; // [T, n_shared*d_ff_shared] bf16 scratch
     void *y_shared; // [T, d]
     int32_t *status;   // the workspace's 256-byte status block: word 0 the status,

@@ -13,10 +13,10 @@
 // chip: they go from TMEM to registers to shared memory, where the selection
 // runs, and only topk_idx / topk_w (and, when asked for, the affinities) are
 // written.  The fp32 weights are split into three exact bf16 parts (router
-// split kernel in router_tc.cu); each 64-wide k block's 12 MMAs land in a
-// fresh TMEM buffer whose values the epilogue adds into IEEE fp32 registers,
-// which keeps the affinities within a few 1e-7 of the double-precision
-// definition.
+// split kernel in router_tc.cu); the 12 MMAs of each 64-wide k block (or of
+// PROMO consecutive k blocks) land in a fresh TMEM buffer whose values the
+// epilogue adds into IEEE fp32 registers, which keeps the affinities within a
+// few 1e-7 of the double-precision definition.
 //
 // The reduction over d is split over a cluster of C CTAs (C = 1, 2, 4 or 8,
 // enough for tiles x C to fill the SMs, at least four k blocks each).  After
@@ -45,7 +45,14 @@ namespace rfused {
 
 namespace cg = cooperative_groups;
 
+#ifndef MOE_ROUTER_PROMO
+#define MOE_ROUTER_PROMO 1
+#endif
+
 constexpr int BM = 128, BK = 64, PARTS = 3;
+// k blocks whose MMAs accumulate in one TMEM buffer before the epilogue adds
+// the buffer into its fp32 registers
+constexpr int PROMO = MOE_ROUTER_PROMO;
 constexpr int A_STAGES = 3;
 constexpr int A_BYTES = BM * BK * 2;          // 16 KB
 constexpr int B_RING_BYTES = 160 * 1024;      // B ring budget
@@ -238,8 +245,10 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
                                    ((uint32_t)(p.BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
             bool ok = true;
             for (int kb = kb0; kb < kb1 && ok; ++kb) {
-                if (!mbar_wait_bounded(smem_u32(&accempty[buf]), cph ^ 1u, abort_flag, p.status,
-                                       p.timeout_ns) ||
+                const bool first = (kb - kb0) % PROMO == 0;
+                const bool last = (kb - kb0) % PROMO == PROMO - 1 || kb + 1 == kb1;
+                if ((first && !mbar_wait_bounded(smem_u32(&accempty[buf]), cph ^ 1u, abort_flag,
+                                                 p.status, p.timeout_ns)) ||
                     !mbar_wait_bounded(smem_u32(&afull[as]), aph, abort_flag, p.status,
                                        p.timeout_ns)) {
                     ok = false;
@@ -260,15 +269,17 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
 #pragma unroll
                     for (int ks = 0; ks < BK / 16; ++ks)
                         tc_mma_bf16(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks, idesc,
-                                    (part == PARTS - 1 && ks == 0) ? 0u : 1u);
+                                    (first && part == PARTS - 1 && ks == 0) ? 0u : 1u);
                     tc_commit(smem_u32(&bempty[bs]));
                     if (++bs == p.b_stages) { bs = 0; bph ^= 1u; }
                 }
                 if (!ok) break;
                 tc_commit(smem_u32(&aempty[as]));
                 if (++as == A_STAGES) { as = 0; aph ^= 1u; }
-                tc_commit(smem_u32(&accfull[buf]));
-                if (++buf == 2) { buf = 0; cph ^= 1u; }
+                if (last) {
+                    tc_commit(smem_u32(&accfull[buf]));
+                    if (++buf == 2) { buf = 0; cph ^= 1u; }
+                }
             }
             tc_commit(smem_u32(&done_bar));
             drain_wait(smem_u32(&done_bar), 0, p.timeout_ns, p.status);
@@ -279,7 +290,7 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
         int buf = 0;
         uint32_t cph = 0;
         const bool has_cols = col0 < p.BN;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += PROMO) {
             if (!mbar_wait_bounded(smem_u32(&accfull[buf]), cph, abort_flag, p.status,
                                    p.timeout_ns))
                 break;

@@ -357,6 +357,47 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const float
                        void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Packed expert weights.  The grouped GEMMs stream every expert weight from
+ * HBM about once per step (6 d d_ff FLOPs per token-expert against 3 d d_ff
+ * weight elements, "MoE + Expert-Parallel Overlap (Exp08)", Implemented /
+ * overlap simulator: at V3 sizes each weight byte feeds only ~2.5 tiles of
+ * 128 token rows), so their speed follows the weights' DRAM access pattern.
+ * moe_pack_weights rewrites the routed and shared expert weights once (at
+ * model load) as contiguous, pre-swizzled 32 KB tiles in the order the GEMMs
+ * read them; moe_expert_ffn_packed and moe_forward_packed then fetch each
+ * tile with one bulk copy.  The arithmetic is unchanged: the packed entry
+ * points return the same bits as moe_expert_ffn / moe_forward.
+ *   moe_packed_weights_size  bytes of the packed buffer (0: unsupported cfg);
+ *                            about the bytes of the six weight tensors
+ *   moe_pack_weights         w_gate, w_up [E, d_ff, d], w_down [E, d, d_ff],
+ *                            ws_gate, ws_up [n_shared, d_ff_shared, d],
+ *                            ws_down [n_shared, d, d_ff_shared] (bf16, the
+ *                            layouts of moe_expert_ffn) -> packed (device,
+ *                            moe_packed_weights_size bytes, 16-byte aligned).
+ *                            Enqueued on `stream`; the inputs are not modified
+ *                            and may be freed once the stream has run it.
+ *   moe_expert_ffn_packed    moe_expert_ffn with `packed` in place of the six
+ *                            weight pointers (bf16 payload only).
+ *   moe_forward_packed       moe_forward likewise; cfg->payload must be bf16
+ *                            (MOE_ERR_UNSUPPORTED_SHAPE otherwise).
+ * The packed buffer depends on E, d, d_ff, n_shared and d_ff_shared only.
+ */
+MOE_API size_t moe_packed_weights_size(const moe_config *cfg);
+MOE_API moe_status moe_pack_weights(const moe_config *cfg, const void *w_gate, const void *w_up,
+                                    const void *w_down, const void *ws_gate, const void *ws_up,
+                                    const void *ws_down, void *packed, void *stream);
+MOE_API moe_status moe_expert_ffn_packed(const moe_config *cfg, const void *x_perm,
+                                         const int32_t *offsets, const void *packed, void *y_perm,
+                                         const void *x, void *y_shared, void *ws, size_t ws_bytes,
+                                         void *stream);
+MOE_API moe_status moe_forward_packed(const moe_config *cfg, const void *x, const float *router_w,
+                                      const float *logit_offset, const float *bias,
+                                      const int64_t *token_ids, const void *packed, void *out,
+                                      int32_t *topk_idx, float *topk_w, int32_t *counts,
+                                      int32_t *offsets, int32_t *send, int32_t *send_tok,
+                                      void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Expert parallelism over `world` ranks, one GPU each (the dispatch and
  * combine all-to-alls of "moe-node-limited-routing", "Why all to all
  * dominates MoE step time", and the expert placement of deepnotes "The real

@@ -1,0 +1,196 @@
+"""Packed expert weights (moe_pack_weights, moe_expert_ffn_packed, moe_forward_packed).
+
+Bars:
+  * the packed buffer equals the tile layout the header defines, restated here
+    independently in numpy (tile (o, n, kb) of 256 rows x 64 columns, 16-byte
+    chunk c of row r at r*128 + ((c ^ (r % 8)) * 16), zero rows past the
+    matrix), byte for byte;
+  * the packed expert FFN and layer forward equal the row-major ones bit for
+    bit (the same bf16 operands meet the same MMAs in the same order), whose
+    parity with the oracle the other tests establish; at V3 sizes the packed
+    layer is also held to the layer's bars against the oracle on sampled
+    tokens.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import combine_expert_ffn_b200 as moe
+else:  # collected on CPU-only machines, skipped by the marker filter
+    moe = None
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _free_gpu():
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def _tile_image(mat: np.ndarray, row0: int, col0: int) -> np.ndarray:
+    """The 32 KB image of rows row0..row0+255, columns col0..col0+63 of the uint16
+    matrix `mat` (rows past the end zero), 128-byte swizzled, as uint16 [256, 64]."""
+    t = np.zeros((256, 64), np.uint16)
+    rows = mat[row0:row0 + 256, col0:col0 + 64]
+    t[:rows.shape[0]] = rows
+    out = np.empty_like(t)
+    for r in range(256):
+        for c in range(8):
+            pos = c ^ (r % 8)
+            out[r, pos * 8:(pos + 1) * 8] = t[r, c * 8:(c + 1) * 8]
+    return out
+
+
+def _expected_packed(sh, wg, wu, wd, sg, su, sd) -> np.ndarray:
+    E, d, ff = sh.E, sh.d, sh.d_ff
+    ffs = sh.n_shared * sh.d_ff_shared
+    nt1, kb1, nt2, kb2 = -(-ff // 128), d // 64, -(-d // 256), ff // 64
+    tiles = []
+    for e in range(E):  # gate/up: rows 0..127 gate, 128..255 up of h columns n*128..
+        for n in range(nt1):
+            gu = np.zeros((256, d), np.uint16)
+            g = wg[e][n * 128:(n + 1) * 128]
+            u = wu[e][n * 128:(n + 1) * 128]
+            gu[:g.shape[0]] = g
+            gu[128:128 + u.shape[0]] = u
+            for kb in range(kb1):
+                tiles.append(_tile_image(gu, 0, kb * 64))
+    for e in range(E):
+        for n in range(nt2):
+            for kb in range(kb2):
+                tiles.append(_tile_image(wd[e], n * 256, kb * 64))
+    if ffs:
+        gcat, ucat = sg.reshape(ffs, d), su.reshape(ffs, d)
+        for n in range(-(-ffs // 128)):
+            gu = np.zeros((256, d), np.uint16)
+            g, u = gcat[n * 128:(n + 1) * 128], ucat[n * 128:(n + 1) * 128]
+            gu[:g.shape[0]] = g
+            gu[128:128 + u.shape[0]] = u
+            for kb in range(kb1):
+                tiles.append(_tile_image(gu, 0, kb * 64))
+        dcat = np.concatenate(list(sd), axis=1)  # [d, ffs]: the shared downs side by side
+        for n in range(nt2):
+            for kb in range(ffs // 64):
+                tiles.append(_tile_image(dcat, n * 256, kb * 64))
+    return np.stack(tiles).reshape(-1)
+
+
+def _u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged2", "noshared"])
+def test_packed_layout_is_the_defined_tile_order(name):
+    sh = H.shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    cfg = moe.MoeConfig.of(sh)
+    packed = moe.pack_weights(cfg, inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                              inp.get("ws_up"), inp.get("ws_down"))
+    torch.cuda.synchronize()
+    ns = sh.n_shared
+    exp = _expected_packed(sh, _u16(inp["w_gate"]), _u16(inp["w_up"]), _u16(inp["w_down"]),
+                           _u16(inp["ws_gate"]) if ns else None,
+                           _u16(inp["ws_up"]) if ns else None,
+                           _u16(inp["ws_down"]) if ns else None)
+    got = packed.cpu().numpy().view(np.uint16)
+    assert got.shape == exp.shape
+    np.testing.assert_array_equal(got, exp)
+
+
+def _forward_pair(sh, inp):
+    cfg = moe.MoeConfig.of(sh)
+    ws = moe.alloc_workspace(cfg)
+    ref = moe.forward_outputs(cfg)
+    moe.moe_forward(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                    inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                    inp.get("ws_up"), inp.get("ws_down"), ref["out"], ref["topk_idx"],
+                    ref["topk_w"], ref["counts"], ref["offsets"], ref["send"], ref["send_tok"],
+                    ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    packed = moe.pack_weights(cfg, inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                              inp.get("ws_up"), inp.get("ws_down"))
+    got = moe.forward_outputs(cfg)
+    moe.moe_forward_packed(cfg, inp["x"], inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                           packed, got["out"], got["topk_idx"], got["topk_w"], got["counts"],
+                           got["offsets"], got["send"], got["send_tok"], ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    return ref, got
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged2", "noshared", "mid"])
+def test_packed_forward_equals_row_major(name):
+    sh = H.shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    ref, got = _forward_pair(sh, inp)
+    for k in ("topk_idx", "counts", "offsets", "send", "send_tok"):
+        assert torch.equal(ref[k], got[k]), k
+    assert torch.equal(ref["topk_w"].view(torch.int32), got["topk_w"].view(torch.int32))
+    assert torch.equal(ref["out"].view(torch.int16), got["out"].view(torch.int16))
+
+
+@pytest.mark.parametrize("counts", [[0, 1, 127, 128, 129, 255, 256, 257, 1000, 7, 0, 0]])
+def test_packed_expert_ffn_segment_edges(counts):
+    """Segments of 0/1/127/128/129/255/256/257/1000 rows: every row and the shared
+    rows of the packed FFN equal the row-major FFN's bits."""
+    sh = H.RAGGED.replace(T=sum(counts) // 4)
+    assert sh.T * sh.K == sum(counts)
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32, device=DEV)
+    n = sh.T * sh.K
+    x_perm = synth.normal(3, 21, (n, sh.d), 1.0, torch.bfloat16, DEV)
+    inp = synth.make_inputs(sh, DEV)
+    cfg = moe.MoeConfig.of(sh)
+    ws = moe.alloc_workspace(cfg)
+    y0 = torch.empty(n, sh.d, dtype=torch.bfloat16, device=DEV)
+    s0 = torch.empty(sh.T, sh.d, dtype=torch.bfloat16, device=DEV)
+    moe.moe_expert_ffn(cfg, x_perm, offsets, inp["w_gate"], inp["w_up"], inp["w_down"], y0,
+                       inp["x"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], s0, ws)
+    packed = moe.pack_weights(cfg, inp["w_gate"], inp["w_up"], inp["w_down"], inp["ws_gate"],
+                              inp["ws_up"], inp["ws_down"])
+    y1 = torch.empty_like(y0)
+    s1 = torch.empty_like(s0)
+    moe.moe_expert_ffn_packed(cfg, x_perm, offsets, packed, y1, inp["x"], s1, ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+    assert torch.equal(s0.view(torch.int16), s1.view(torch.int16))
+
+
+def test_packed_forward_v3_equals_row_major_and_meets_the_oracle(orc):
+    sh = H.shape("v3")
+    inp = synth.make_inputs(sh, DEV)
+    ref, got = _forward_pair(sh, inp)
+    assert torch.equal(ref["topk_idx"], got["topk_idx"])
+    assert torch.equal(ref["out"].view(torch.int16), got["out"].view(torch.int16))
+    rows = H.parity_rows(sh, got["topk_idx"].cpu().numpy(), n_spread=64)
+    ref_out, ref_idx, _, ref_s = H.oracle_layer_sample(orc, sh, inp, rows, threads=orc.all_cores())
+    gi = got["topk_idx"].cpu().numpy()[rows]
+    keep = [r for r in range(len(rows)) if np.array_equal(gi[r], ref_idx[r])]
+    for r in set(range(len(rows))) - set(keep):
+        assert H.near_tie_certified(sh, ref_s[r], inp["bias"].cpu().numpy(), gi[r], ref_idx[r])
+    frob, elem = H.compare_out(got["out"][torch.as_tensor(rows[keep], device=DEV)], ref_out[keep])
+    assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
+
+
+def test_packed_rejects_fp8_payload_and_missing_buffer():
+    sh = H.shape("tiny")
+    cfg = moe.MoeConfig.of(sh, payload=moe.MOE_PAYLOAD_FP8)
+    ws = moe.alloc_workspace(cfg)
+    inp = synth.make_inputs(sh, DEV)
+    out = torch.empty(sh.T, sh.d, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_forward_packed(cfg, inp["x"], inp["router_w"], None, inp["bias"],
+                               torch.empty(16, dtype=torch.uint8, device=DEV), out, ws=ws)
+    assert e.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    cfg = moe.MoeConfig.of(sh)
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_forward_packed(cfg, inp["x"], inp["router_w"], None, inp["bias"], None, out, ws=ws)
+    assert e.value.status == moe.MOE_ERR_INVALID_ARG
