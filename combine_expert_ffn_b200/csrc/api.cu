@@ -95,7 +95,7 @@ moe_status check_device() {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Affinity router + node-limited top-K.  Up to 256 experts (G <= 32, K <= 16)
+// Affinity router + node-limited top-K.  Up to 256 experts (G <= 32, E/G <= 32)
 // one fused kernel keeps the affinities on chip and writes `scores` only when
 // the caller asks for them; larger layers take the tensor-core logits kernel
 // (affinities into `scores` or the workspace) and the warp-per-token select.

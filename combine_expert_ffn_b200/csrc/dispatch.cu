@@ -6,16 +6,18 @@
 // with per-expert counts and offsets and the group-to-group send matrices
 // ("send matrices", shivam2003 "5. Tail latency controls step time").
 //
-// Four kernels, none using global atomics, so every output is deterministic:
+// Kernels, none using global atomics, so every output is deterministic:
 //   count   : per 256-token block, a bitmask per expert (bit = token in the
 //             block chose it) -> block histograms + partial send matrices
-//   scan    : warp per expert, prefix over blocks -> counts, block bases;
-//             block 0 also sums the partial send matrices
+//   scan    : (more than 256 blocks only) warp per expert, prefix over blocks
+//             -> counts, block bases; block 0 also sums the partial send
+//             matrices.  Up to 256 blocks the scatter blocks do this themselves
 //   scatter : per block, rank of a copy = popcount of the expert's mask below
 //             its token; row = offsets[e] + base + rank -> perm, inv_perm;
 //             offsets = exclusive scan of counts (recomputed per block)
-//   gather  : x_perm[row] = x[t], reading each x row once and writing it K
-//             times with 16-byte vector accesses
+//   gather  : x_perm[row] = x[t]: the copy engine moves whole rows (bulk
+//             copies through shared memory), or, for rows wider than 14 KB,
+//             16-byte thread copies reading each x row once
 
 #include "fp8_payload.cuh"
 #include "kernels.h"
@@ -135,24 +137,68 @@ dispatch_scan_kernel(const int32_t *__restrict__ hist_t, int nblk, int E, int G,
     }
 }
 
+// With fused_scan (at most SCAN_FUSE_MAX_BLOCKS blocks) every block sums the
+// block histograms hist_t itself -- counts[e] over all blocks, its base over
+// the blocks before it -- and block 0 writes counts and the send matrices, so
+// no separate scan launch is needed; otherwise counts and base_t come from
+// dispatch_scan_kernel.
+constexpr int SCAN_FUSE_MAX_BLOCKS = 256;
+
 __global__ void __launch_bounds__(BLK)
-dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int K,
-                        const int32_t *__restrict__ counts, const int32_t *__restrict__ base_t,
-                        int32_t *__restrict__ offsets, int32_t *__restrict__ perm_token,
-                        int32_t *__restrict__ inv_perm) {
+dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int G, int K,
+                        int fused_scan, const int32_t *__restrict__ hist_t,
+                        const int32_t *__restrict__ send_part,
+                        const int32_t *__restrict__ sendtok_part, int32_t *__restrict__ counts,
+                        const int32_t *__restrict__ base_t, int32_t *__restrict__ send,
+                        int32_t *__restrict__ send_tok, int32_t *__restrict__ offsets,
+                        int32_t *__restrict__ perm_token, int32_t *__restrict__ inv_perm) {
     extern __shared__ uint32_t dsm[];
     uint32_t *masks = dsm;                                          // [E * WORDS]
     int32_t *offs = reinterpret_cast<int32_t *>(dsm + E * WORDS);   // [E + 1]
     int32_t *wsum = offs + E + 1;                                   // [BLK / 32]
+    int32_t *cnt_s = wsum + BLK / 32;                               // [E]
+    int32_t *base_s = cnt_s + E;                                    // [E]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nblk = gridDim.x, blk = blockIdx.x;
+
+    for (int e = tid; e < E; e += BLK) {
+        int c, b;
+        if (fused_scan) {
+            const int32_t *h = hist_t + (size_t)e * nblk;
+            c = 0;
+            b = 0;
+            for (int q = 0; q < nblk; ++q) {
+                const int v = h[q];
+                c += v;
+                if (q < blk) b += v;
+            }
+            if (blk == 0) counts[e] = c;
+        } else {
+            c = counts[e];
+            b = base_t[(size_t)e * nblk + blk];
+        }
+        cnt_s[e] = c;
+        base_s[e] = b;
+    }
+    if (fused_scan && blk == 0) {
+        for (int i = tid; i < G * G; i += BLK) {
+            int a = 0, c = 0;
+            for (int q = 0; q < nblk; ++q) {
+                a += send_part[(size_t)q * G * G + i];
+                c += sendtok_part[(size_t)q * G * G + i];
+            }
+            send[i] = a;
+            if (send_tok) send_tok[i] = c;
+        }
+    }
+    __syncthreads();
 
     // offsets = exclusive scan of counts: each thread owns a run of experts
     const int per = (E + BLK - 1) / BLK;
     int run = 0;
     for (int i = 0; i < per; ++i) {
         const int e = tid * per + i;
-        if (e < E) run += counts[e];
+        if (e < E) run += cnt_s[e];
     }
     int incl = run;
 #pragma unroll
@@ -169,7 +215,7 @@ dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int 
         const int e = tid * per + i;
         if (e < E) {
             offs[e] = acc;
-            acc += counts[e];
+            acc += cnt_s[e];
         }
     }
     if (tid == BLK - 1) offs[E] = wpre + incl;
@@ -189,7 +235,7 @@ dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int 
         }
         int rank = __popc(masks[e * WORDS + w] & below);
         for (int q = 0; q < w; ++q) rank += __popc(masks[e * WORDS + q]);
-        const int row = offs[e] + base_t[(size_t)e * nblk + blk] + rank;
+        const int row = offs[e] + base_s[e] + rank;
         perm_token[row] = t;
         inv_perm[(size_t)t * K + j] = row;
     }
@@ -398,7 +444,7 @@ cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d
         return cudaSuccess;
     }
     const size_t smem_count = sizeof(uint32_t) * (E * WORDS + 2 * G * G);
-    const size_t smem_scatter = sizeof(uint32_t) * (E * WORDS + E + 1 + BLK / 32);
+    const size_t smem_scatter = sizeof(uint32_t) * (E * WORDS + E + 1 + BLK / 32 + 2 * E);
     if (smem_count > 48 * 1024 &&
         (err = cudaFuncSetAttribute(dispatch_count_kernel,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_count)))
@@ -411,13 +457,17 @@ cudaError_t launch_dispatch(const void *x, const int32_t *topk_idx, int T, int d
                                                          ws.send_part, ws.sendtok_part, status);
     count_launch();
     if ((err = cudaGetLastError())) return err;
-    dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(ws.hist_t, nblk, E, G, ws.send_part,
-                                                      ws.sendtok_part, ws.base_t, counts, send,
-                                                      send_tok);
-    count_launch();
-    if ((err = cudaGetLastError())) return err;
-    dispatch_scatter_kernel<<<nblk, BLK, smem_scatter, st>>>(topk_idx, T, E, K, counts, ws.base_t,
-                                                             offsets, perm_token, inv_perm);
+    const int fused_scan = nblk <= SCAN_FUSE_MAX_BLOCKS;
+    if (!fused_scan) {
+        dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(ws.hist_t, nblk, E, G, ws.send_part,
+                                                          ws.sendtok_part, ws.base_t, counts, send,
+                                                          send_tok);
+        count_launch();
+        if ((err = cudaGetLastError())) return err;
+    }
+    dispatch_scatter_kernel<<<nblk, BLK, smem_scatter, st>>>(
+        topk_idx, T, E, G, K, fused_scan, ws.hist_t, ws.send_part, ws.sendtok_part, counts,
+        ws.base_t, send, send_tok, offsets, perm_token, inv_perm);
     count_launch();
     if ((err = cudaGetLastError())) return err;
     if (x_perm) return launch_permute(x, inv_perm, T, d, K, x_perm, st, status);

@@ -320,15 +320,19 @@ ep_dispatch_dedup_kernel(const uint4 *__restrict__ x, const int32_t *__restrict_
 }
 
 // The deduplicated dispatch on the copy engine.  Warp per token row: lane 0
-// loads the row into one of the warp's two shared-memory buffers
-// (cp.async.bulk, completion on an mbarrier) while the previous row's stores
-// drain; lane o < world (and o + 32) stores it to owner o's token buffer at
+// loads the row into a shared-memory buffer of the warp (cp.async.bulk,
+// completion on an mbarrier); lane o < world (and o + 32) stores it to owner o's token buffer at
 // tok_base[o] + tok_slot[t][o] when the token has an expert there
 // (cp.async.bulk shared -> global, through the owner's pointer); lane j < K
 // writes copy (t, j)'s 4-byte token row into the owner's recv_idx.  The token
 // plan already lists every destination, so no lane walks the copies to find
 // them.
-constexpr int DB_WARPS = 4;
+// NB row buffers per warp: 2 (4 warps per CTA) overlaps a row's load with
+// the previous row's stores when a warp walks several rows; 1 (8 warps per
+// CTA) puts twice as many rows in flight when there are about as many rows as
+// warps (the per-rank batches of an expert-parallel step).
+template <int NB>
+__host__ __device__ constexpr int db_warps() { return NB == 2 ? 4 : 8; }
 
 __device__ __forceinline__ void db_drain(uint32_t bar, uint32_t parity, int64_t timeout_ns) {
     const uint64_t t0 = globaltimer_ns();
@@ -336,7 +340,8 @@ __device__ __forceinline__ void db_drain(uint32_t bar, uint32_t parity, int64_t 
     }
 }
 
-__global__ void __launch_bounds__(DB_WARPS * 32)
+template <int NB>
+__global__ void __launch_bounds__(db_warps<NB>() * 32)
 ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restrict__ topk_idx,
                               const int32_t *__restrict__ offsets,
                               const int32_t *__restrict__ inv_perm,
@@ -345,13 +350,14 @@ ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restr
                               int32_t *const *__restrict__ recv_idx, int64_t tok_rows,
                               int64_t recv_rows, int T, int row_bytes, int E, int K, int El,
                               int world, int32_t *status, int64_t timeout_ns) {
+    constexpr int WARPS = db_warps<NB>();
     extern __shared__ __align__(128) uint8_t dsm_rows[];
     __shared__ int32_t delta_s[EP_MAX_E];
     __shared__ int32_t tokbase_s[EP_MAX_WORLD];
     __shared__ char *tok_tab_s[EP_MAX_WORLD];
     __shared__ int32_t *idx_tab_s[EP_MAX_WORLD];
-    __shared__ __align__(8) uint64_t lbar[DB_WARPS][2];
-    __shared__ int abort_s[DB_WARPS];
+    __shared__ __align__(8) uint64_t lbar[WARPS][2];
+    __shared__ int abort_s[WARPS];
     for (int e = threadIdx.x; e < E; e += blockDim.x) delta_s[e] = base[e] - offsets[e];
     for (int o = threadIdx.x; o < world; o += blockDim.x) {
         tokbase_s[o] = tok_base[o];
@@ -359,7 +365,7 @@ ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restr
         idx_tab_s[o] = recv_idx[o];
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t buf0 = smem_u32(dsm_rows) + (uint32_t)(warp * 2 * row_bytes);
+    const uint32_t buf0 = smem_u32(dsm_rows) + (uint32_t)(warp * NB * row_bytes);
     const uint32_t bar0 = smem_u32(&lbar[warp][0]), bar1 = smem_u32(&lbar[warp][1]);
     if (lane == 0) {
         mbar_init(bar0, 1);
@@ -368,50 +374,56 @@ ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restr
         fence_barrier_init();
     }
     __syncthreads();
-    const int nw = gridDim.x * DB_WARPS;
-    int t = blockIdx.x * DB_WARPS + warp;
+    const int nw = gridDim.x * WARPS;
+    int t = blockIdx.x * WARPS + warp;
     uint32_t in_flight = 0, ph = 0;
-    if (t < T && lane == 0) {
+    if (NB == 2 && t < T && lane == 0) {
         mbar_arrive_expect_tx(bar0, row_bytes);
         bulk_load(buf0, x + (size_t)t * row_bytes, row_bytes, bar0);
         in_flight = 1u;
     }
     for (int i = 0; t < T; t += nw, ++i) {
-        const int b = i & 1;
+        const int b = NB == 2 ? (i & 1) : 0;
         const int tn = t + nw;
         // this token's destinations: owner lane (and lane + 32) and copy lane j < K
         int64_t trow0 = -1, trow1 = -1;
         if (lane < world) {
-            const int s = __ldg(tok_slot + (int64_t)t * world + lane);
-            if (s >= 0) trow0 = (int64_t)tokbase_s[lane] + s;
+            const int sl = __ldg(tok_slot + (int64_t)t * world + lane);
+            if (sl >= 0) trow0 = (int64_t)tokbase_s[lane] + sl;
         }
         if (lane + 32 < world) {
-            const int s = __ldg(tok_slot + (int64_t)t * world + lane + 32);
-            if (s >= 0) trow1 = (int64_t)tokbase_s[lane + 32] + s;
+            const int sl = __ldg(tok_slot + (int64_t)t * world + lane + 32);
+            if (sl >= 0) trow1 = (int64_t)tokbase_s[lane + 32] + sl;
         }
         if (lane < K) {
             const int e = __ldg(topk_idx + (int64_t)t * K + lane);
             if (e >= 0 && e < E) {  // invalid ids: flagged by the local plan
                 const int o = e / El;
-                const int s = __ldg(tok_slot + (int64_t)t * world + o);
-                const int64_t trow = (int64_t)tokbase_s[o] + s;
+                const int sl = __ldg(tok_slot + (int64_t)t * world + o);
+                const int64_t trow = (int64_t)tokbase_s[o] + sl;
                 const int64_t row = (int64_t)delta_s[e] + __ldg(inv_perm + (int64_t)t * K + lane);
-                if (s < 0 || trow >= tok_rows || row < 0 || row >= recv_rows) {
+                if (sl < 0 || trow >= tok_rows || row < 0 || row >= recv_rows) {
                     if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
                 } else {
                     idx_tab_s[o][row] = (int32_t)trow;
                 }
             }
         }
-        // the other buffer: every store of the previous row has read it
+        // the buffer to load next: every store that read it has read it
         bulk_wait_group_read<0>();
         __syncwarp();
-        if (lane == 0 && tn < T) {
-            const uint32_t nb = b ? bar0 : bar1;
-            mbar_arrive_expect_tx(nb, row_bytes);
-            bulk_load(buf0 + (uint32_t)((b ^ 1) * row_bytes), x + (size_t)tn * row_bytes, row_bytes,
-                      nb);
-            in_flight |= 1u << (b ^ 1);
+        if (lane == 0) {
+            if (NB == 1) {  // this row, into the warp's single buffer
+                mbar_arrive_expect_tx(bar0, row_bytes);
+                bulk_load(buf0, x + (size_t)t * row_bytes, row_bytes, bar0);
+                in_flight = 1u;
+            } else if (tn < T) {  // the next row, into the other buffer
+                const uint32_t nb = b ? bar0 : bar1;
+                mbar_arrive_expect_tx(nb, row_bytes);
+                bulk_load(buf0 + (uint32_t)((b ^ 1) * row_bytes), x + (size_t)tn * row_bytes,
+                          row_bytes, nb);
+                in_flight |= 1u << (b ^ 1);
+            }
         }
         const uint32_t bar = b ? bar1 : bar0, par = (ph >> b) & 1u;
         int ok = 1;
@@ -872,27 +884,49 @@ cudaError_t launch_ep_dispatch_dedup(const void *x, const int32_t *topk_idx, con
                                      int world, int32_t *status, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int row_bytes = d * 2;
-    const size_t db_smem = (size_t)DB_WARPS * 2 * row_bytes;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // one buffer per warp when one wave of eight-warp CTAs covers every row
+    const bool one = (int64_t)T <= (int64_t)sms * db_warps<1>();
+    const size_t db_smem = (size_t)(one ? db_warps<1>() : db_warps<2>() * 2) * row_bytes;
     if (db_smem <= 112 * 1024) {
-        // one wave of four-warp CTAs, each warp walking token rows
-        int sms = 148, dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaError_t err = cudaFuncSetAttribute(ep_dispatch_dedup_bulk_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)db_smem);
-        if (err != cudaSuccess) return err;
+        cudaError_t err;
         int per_sm = 1;  // CTAs resident per SM with this shared memory (one wave)
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ep_dispatch_dedup_bulk_kernel,
-                                                          DB_WARPS * 32, db_smem) != cudaSuccess ||
-            per_sm < 1)
-            per_sm = 1;
-        const int want = (T + DB_WARPS - 1) / DB_WARPS;
+        int warps;
+        if (one) {
+            err = cudaFuncSetAttribute(ep_dispatch_dedup_bulk_kernel<1>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)db_smem);
+            if (err == cudaSuccess &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &per_sm, ep_dispatch_dedup_bulk_kernel<1>, 32 * db_warps<1>(), db_smem) !=
+                    cudaSuccess)
+                per_sm = 1;
+            warps = db_warps<1>();
+        } else {
+            err = cudaFuncSetAttribute(ep_dispatch_dedup_bulk_kernel<2>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)db_smem);
+            if (err == cudaSuccess &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &per_sm, ep_dispatch_dedup_bulk_kernel<2>, 32 * db_warps<2>(), db_smem) !=
+                    cudaSuccess)
+                per_sm = 1;
+            warps = db_warps<2>();
+        }
+        if (err != cudaSuccess) return err;
+        if (per_sm < 1) per_sm = 1;
+        const int want = (T + warps - 1) / warps;
         const int grid = want < per_sm * sms ? want : per_sm * sms;
-        ep_dispatch_dedup_bulk_kernel<<<grid, DB_WARPS * 32, db_smem, st>>>(
-            static_cast<const char *>(x), topk_idx, offsets, inv_perm, base, tok_slot, tok_base,
-            reinterpret_cast<char *const *>(recv_tok), recv_idx, tok_rows, recv_rows, T, row_bytes,
-            E, K, E / world, world, status, 2000000000LL);
+        if (one)
+            ep_dispatch_dedup_bulk_kernel<1><<<grid, 32 * warps, db_smem, st>>>(
+                static_cast<const char *>(x), topk_idx, offsets, inv_perm, base, tok_slot,
+                tok_base, reinterpret_cast<char *const *>(recv_tok), recv_idx, tok_rows, recv_rows,
+                T, row_bytes, E, K, E / world, world, status, 2000000000LL);
+        else
+            ep_dispatch_dedup_bulk_kernel<2><<<grid, 32 * warps, db_smem, st>>>(
+                static_cast<const char *>(x), topk_idx, offsets, inv_perm, base, tok_slot,
+                tok_base, reinterpret_cast<char *const *>(recv_tok), recv_idx, tok_rows, recv_rows,
+                T, row_bytes, E, K, E / world, world, status, 2000000000LL);
         count_launch();
         return cudaGetLastError();
     }

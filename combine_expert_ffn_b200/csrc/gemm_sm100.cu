@@ -38,9 +38,16 @@
 
 
 // Paired row tiles (grouped_ffn_pair_kernel) for the gate/up GEMM and the
-// down GEMM; 0 selects the single-tile kernel with double-buffered TMEM.
+// down GEMM; 0 selects the single-tile kernel with double-buffered TMEM.  The
+// gate/up GEMM also takes the paired kernel when the experts average at least
+// MOE_PAIR_MIN_ROWS rows (most row tiles then come in pairs; measured on the
+// skewed V3 workload, 1024 rows per expert on average: 21.4 vs 22.6 ms for the
+// expert FFN, while at 256 rows per expert the single-tile kernel is faster).
 #ifndef MOE_PAIR_GEMM1
 #define MOE_PAIR_GEMM1 0
+#endif
+#ifndef MOE_PAIR_MIN_ROWS
+#define MOE_PAIR_MIN_ROWS 512
 #endif
 #ifndef MOE_PAIR_GEMM2
 #define MOE_PAIR_GEMM2 0
@@ -1127,7 +1134,8 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     if (rows_r == 0) return cudaSuccess;
     // tile counters of the paired kernels: words 16 and 17 of the status block
     int *counters = reinterpret_cast<int *>(a.status) + 16;
-    if (MOE_PAIR_GEMM1 || MOE_PAIR_GEMM2) {
+    const bool pair1 = MOE_PAIR_GEMM1 || rows_r >= (uint64_t)MOE_PAIR_MIN_ROWS * a.E;
+    if (pair1 || MOE_PAIR_GEMM2) {
         cudaError_t e0 = cudaMemsetAsync(counters, 0, 2 * sizeof(int), st);
         if (e0 != cudaSuccess) return e0;
     }
@@ -1191,7 +1199,7 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
     }
     cudaError_t err = fp8      ? launch_one<EPI_SWIGLU, A_FP8>(m1, p1, st)
                       : gather ? launch_one<EPI_SWIGLU, A_GATHER>(m1, p1, st)
-                      : MOE_PAIR_GEMM1 ? launch_pair<EPI_SWIGLU>(m1, p1, st)
+                      : pair1 ? launch_pair<EPI_SWIGLU>(m1, p1, st)
                                : launch_one<EPI_SWIGLU, A_TMA>(m1, p1, st);
     if (err != cudaSuccess) return err;
 

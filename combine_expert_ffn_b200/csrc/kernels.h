@@ -173,7 +173,7 @@ cudaError_t launch_router_logits_tc(const void *x, const float *e, const float *
 cudaError_t launch_router_split(const float *e, int E, int d, void *e_split, cudaStream_t st);
 
 // router_fused.cu: affinities and node-limited top-K in one kernel (E <= 256,
-// G <= 32, K <= 16), from the bf16 parts written by launch_router_split;
+// G <= 32, E/G <= 32), from the bf16 parts written by launch_router_split;
 // scores (nullable) receives the affinities.  The reduction over d is split
 // over a cluster of router_fused_cluster(T, d) CTAs.
 bool router_fused_supported(int E, int G, int K);

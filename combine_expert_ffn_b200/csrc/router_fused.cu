@@ -10,9 +10,9 @@
 //
 // For E <= 256 one CTA holds a 128-token tile against ALL experts (MMA
 // M = 128, N = E rounded up to 16), so a token's affinities never leave the
-// chip: they go from TMEM to registers to shared memory, where the selection
-// runs, and only topk_idx / topk_w (and, when asked for, the affinities) are
-// written.  The fp32 weights are split into three exact bf16 parts (router
+// chip: the logits go from TMEM to registers to shared memory, the selection
+// threads turn them into affinities in their registers, and only topk_idx /
+// topk_w (and, when asked for, the affinities) are written.  The fp32 weights are split into three exact bf16 parts (router
 // split kernel in router_tc.cu); the 12 MMAs of each 64-wide k block (or of
 // PROMO consecutive k blocks) land in a fresh TMEM buffer whose values the
 // epilogue adds into IEEE fp32 registers, which keeps the affinities within a
@@ -31,8 +31,10 @@
 //   warp 1      TMEM owner (2 buffers x 256 columns), single-thread MMA issuer
 //   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
 //               128*((w-2)/4) .. +128 (two warps per lane quarter), adds each
-//               k block into fp32 registers; then the cluster reduction, the
-//               affinity function and the selection (2C threads per token)
+//               k block into fp32 registers; then the cluster reduction and,
+//               with a thread per (token, group), the affinity function and
+//               the selection in registers, warp shuffles between the token's
+//               groups
 // Every mbarrier wait is bounded; on running out the kernel records
 // MOE_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs and still meets its
 // cluster barriers, so no CTA of the cluster is left waiting.
@@ -99,7 +101,9 @@ __device__ __forceinline__ float affinity_fn(float L, int kind) {
         const float sp = L > 0.f ? L + log1pf(expf(-L)) : log1pf(expf(L));
         return sqrtf(sp);
     }
-    return 1.0f / (1.0f + expf(-L));
+    // sigmoid: hardware exp2 and a rounded reciprocal; a few 1e-7 from the
+    // definition, far inside the affinities' 1e-5 bar
+    return __frcp_rn(1.0f + __expf(-L));
 }
 
 // Selection key: orderable(b) in the high word, ~index in the low word, so the
@@ -123,6 +127,142 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 // Named barrier over the 256 epilogue threads (id 1; 0 is __syncthreads).
 __device__ __forceinline__ void epi_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");
+}
+
+// Largest of 32 keys whose slot is below n and whose key is below `below`
+// (0 if none): independent masks, then a depth-5 tree, so the 32 compares
+// overlap instead of forming one dependent chain.
+__device__ __forceinline__ uint64_t tree_best(const uint64_t (&k)[32], int n, uint64_t below) {
+    uint64_t m[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const uint64_t a = (q < n && k[q] < below) ? k[q] : 0ull;
+        const uint64_t b = (q + 16 < n && k[q + 16] < below) ? k[q + 16] : 0ull;
+        m[q] = a > b ? a : b;
+    }
+#pragma unroll
+    for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int q = 0; q < w; ++q) m[q] = m[q] > m[q + w] ? m[q] : m[q + w];
+    return m[0];
+}
+
+// The biased affinity a selection key was made from (orderable() inverted;
+// -0 comes back as +0, which adds and compares the same).
+__device__ __forceinline__ float key_value(uint64_t k) {
+    const uint32_t o = (uint32_t)(k >> 32);
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+
+// Affinities and node-limited top-K of the R token rows this CTA owns, from the
+// C partial logits red[r][row][col] (r = cluster rank).  Thread (token, group
+// g): the token's G groups sit in G consecutive lanes of an epilogue warp, 32
+// / G tokens per warp.  A thread adds its group's gsz <= 32 logits over the C
+// partials in rank order, adds the offset, applies the affinity function and
+// keeps s and the selection key of b = s + bias per expert in registers; then
+//   group score  the sum of the group's K/M best b, added in pick order;
+//   kept groups  the M best group keys (a group is kept when fewer than M of
+//                the token's groups have a larger key);
+//   top-K        K rounds of "largest key below the last pick" over the kept
+//                groups' lanes (tree inside a lane, shuffles across lanes),
+//                the pick's unbiased s travelling with its key.
+// Keys are orderable(b) << 32 | ~index, so ties go to the lower index.
+template <int C>
+__device__ __forceinline__ void select_rows(const Params &p, const float *red, int rs, int R,
+                                            int m0, int rank, int ew, int lane,
+                                            const float *bias_s, const float *off_s,
+                                            bool aborted) {
+    const int E = p.E, G = p.G, K = p.K, M = p.M;
+    const int gsz = E / G, kpg = K / M;
+    const int tpw = 32 / G;                         // tokens per warp
+    const int sub = lane / G, g = lane - (lane / G) * G;
+    const bool pow2 = (G & (G - 1)) == 0;
+    for (int t0 = 0; t0 < R; t0 += 8 * tpw) {
+        const int tl = t0 + ew * tpw + sub;
+        const bool valid = sub < tpw && tl < R;
+        const int t = m0 + rank * R + tl;
+        const float *rg = red + (size_t)(valid ? tl : 0) * rs + g * gsz;
+        float sv[32];
+        uint64_t kv[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            sv[q] = 0.f;
+            kv[q] = 0ull;
+            if (q < gsz) {
+                float L = rg[q];
+#pragma unroll
+                for (int r = 1; r < C; ++r) L = __fadd_rn(L, rg[(size_t)r * R * rs + q]);
+                if (p.off) L += off_s[g * gsz + q];
+                sv[q] = affinity_fn(L, p.affinity);
+                kv[q] = sel_key(__fadd_rn(sv[q], bias_s[g * gsz + q]), g * gsz + q);
+            }
+        }
+        if (valid && p.scores && !aborted && t < p.T) {
+            float *so = p.scores + (size_t)t * E + g * gsz;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                if (q < gsz) so[q] = sv[q];
+        }
+        // group score: the sum of the group's K/M best b, in pick order
+        uint64_t prev = ~0ull;
+        float gsum = 0.f;
+        for (int r = 0; r < kpg; ++r) {
+            const uint64_t best = tree_best(kv, gsz, prev);
+            const float bb = key_value(best);
+            prev = best;
+            gsum = r == 0 ? bb : __fadd_rn(gsum, bb);
+        }
+        const uint64_t gkey = sel_key(gsum, g);
+        // kept: fewer than M of the token's groups have a larger key
+        int above = 0;
+        for (int q = 0; q < G; ++q) {
+            const uint64_t o = __shfl_sync(0xFFFFFFFFu, gkey, sub * G + q < 32 ? sub * G + q : 0);
+            above += o > gkey;
+        }
+        const bool kept = valid && above < M;
+        // top-K over the kept groups, in pick order
+        const bool writer = valid && g == 0 && t < p.T && !aborted;
+        uint64_t last = ~0ull;
+        float denom = 0.f;
+        for (int r = 0; r < K; ++r) {
+            uint64_t best = kept ? tree_best(kv, gsz, last) : 0ull;
+            float bs = 0.f;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                if (q < gsz && kv[q] == best && best != 0ull) bs = sv[q];
+            if (pow2) {  // the token's lanes are an aligned power of two
+                for (int off = G >> 1; off > 0; off >>= 1) {
+                    const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, best, off);
+                    const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, off);
+                    if (o > best) { best = o; bs = os; }
+                }
+            } else {
+                uint64_t mx = best;
+                float ms = bs;
+                for (int q = 0; q < G; ++q) {
+                    const int src = sub * G + q < 32 ? sub * G + q : 0;
+                    const uint64_t o = __shfl_sync(0xFFFFFFFFu, best, src);
+                    const float os = __shfl_sync(0xFFFFFFFFu, bs, src);
+                    if (o > mx) { mx = o; ms = os; }
+                }
+                best = mx;
+                bs = ms;
+            }
+            last = best;
+            if (writer) {
+                int e = key_index(best);
+                e = e < 0 ? 0 : (e >= E ? E - 1 : e);
+                p.topk_idx[(size_t)t * K + r] = e;
+                p.topk_w[(size_t)t * K + r] = bs;  // s for now; divided below
+                denom = __fadd_rn(denom, bs);
+            }
+        }
+        // gates over the chosen unbiased affinities, in slot order
+        if (writer) {
+            for (int r = 0; r < K; ++r)
+                p.topk_w[(size_t)t * K + r] = __fdiv_rn(p.topk_w[(size_t)t * K + r], denom);
+        }
+    }
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -187,7 +327,6 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
     const uint32_t tmem_base = tmem_base_s;
 
     // epilogue thread geometry (warps 2..9)
-    const int et = threadIdx.x - 64;                  // 0..255 for epilogue threads
     const int q = warp & 3;                           // TMEM lane quarter
     const int half = (warp - 2) >> 2;                 // column half
     const int row = q * 32 + lane;                    // tile row of this thread
@@ -319,147 +458,36 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
 
     // ---------------------------------------------------------- cluster reduction
     // Ring buffers are free once every CTA of the cluster has passed here (its
-    // copies landed, its MMAs done).  Each epilogue thread then stores its
-    // partial logits into red[rank][row - owner*R][col] of the CTA that owns the
-    // row (through distributed shared memory when that is another CTA).
+    // copies landed, its MMAs done).  Each epilogue thread stores its partial
+    // logits into red[rank][row - owner*R][col] of the CTA that owns the row
+    // (through distributed shared memory when that is another CTA).
     tc_fence_before();
     __syncthreads();
     const int R = BM / C;                 // token rows owned by each CTA of the cluster
-    const int sp = p.BN + 4;              // floats per row of red
-    float *red = reinterpret_cast<float *>(smem);  // [C][R][sp] in the owner
-    cluster.sync();
+    const int rs = p.BN + 4;              // floats per row of red
+    float *red = reinterpret_cast<float *>(smem);  // [C][R][rs]
+    if (C > 1) cluster.sync();
     if (warp >= 2 && col0 < p.BN) {
         const int owner = row / R;
         float *base = owner == rank ? red : cluster.map_shared_rank(red, owner);
-        float *dst = base + ((size_t)rank * R + (row - owner * R)) * sp + col0;
+        float *dst = base + ((size_t)rank * R + (row - owner * R)) * rs + col0;
 #pragma unroll
         for (int c = 0; c < 128; c += 4)
             if (col0 + c < p.BN)
                 *reinterpret_cast<float4 *>(dst + c) =
                     make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
     }
-    cluster.sync();
+    if (C > 1) cluster.sync();
 
-    // ---------------------------------------------------------- affinities
-    // L = P_0 + P_1 + ... + P_{C-1} (rank order) + o, s = f(L), written over
-    // red[0] element by element (each element read and written by one thread).
-    const int E = p.E;
-    if (warp >= 2) {
-        for (int i = et; i < R * E; i += EPI_THREADS) {
-            const int rl = i / E, col = i - rl * E;
-            float *e0 = red + (size_t)rl * sp + col;
-            float L = e0[0];
-            for (int r = 1; r < C; ++r) L = __fadd_rn(L, e0[(size_t)r * R * sp]);
-            if (p.off) L += off_s[col];
-            e0[0] = affinity_fn(L, p.affinity);
-        }
-    }
-    const int tpt = EPI_THREADS / R;      // selection threads per token (2C)
-    float *srow = red;                    // s of local token rl at srow[rl * sp + i]
-
-    // ---------------------------------------------------------- selection
+    // ---------------------------------------------------------- affinities and selection
     if (warp >= 2) {
         epi_sync();
-        const int G = p.G, K = p.K, M = p.M;
-        const int gsz = E / G, kpg = K / M;
-        const int tl = et / tpt, j = et - tl * tpt;
-        const int t = m0 + rank * R + tl;
-        const float *s = srow + (size_t)tl * sp;
-        uint64_t *gkey = reinterpret_cast<uint64_t *>(smem + (size_t)C * R * sp * 4);  // [R][G]
-        uint64_t *lists = gkey + (size_t)R * G;                       // [R][tpt][K]
         const bool aborted = *abort_flag != 0;
-
-        // step 1: group scores, the sum of each group's top-(K/M) b added in pick order
-        for (int g = j; g < G; g += tpt) {
-            uint64_t prev = ~0ull;
-            float sum = 0.f;
-            for (int r = 0; r < kpg; ++r) {
-                uint64_t best = 0;
-                float bb = 0.f;
-                for (int i = g * gsz; i < (g + 1) * gsz; ++i) {
-                    const float v = __fadd_rn(s[i], bias_s[i]);
-                    const uint64_t k = sel_key(v, i);
-                    if (k < prev && k > best) { best = k; bb = v; }
-                }
-                prev = best;
-                sum = r == 0 ? bb : __fadd_rn(sum, bb);
-            }
-            gkey[(size_t)tl * G + g] = sel_key(sum, g);
-        }
-        epi_sync();
-        // step 2: the M best groups (every thread of the token, same answer)
-        uint64_t keep = 0;
-        {
-            uint64_t prev = ~0ull;
-            for (int r = 0; r < M; ++r) {
-                uint64_t best = 0;
-                for (int g = 0; g < G; ++g) {
-                    const uint64_t k = gkey[(size_t)tl * G + g];
-                    if (k < prev && k > best) best = k;
-                }
-                keep |= 1ull << (key_index(best) & 63);
-                prev = best;
-            }
-        }
-        // step 3: this thread's K best keys among the kept experts i = j (mod tpt),
-        // as a list sorted descending (zero keys past the end)
-        uint64_t *mine = lists + ((size_t)tl * tpt + j) * K;
-        {
-            int n = 0;
-            uint64_t kth = 0;
-            for (int i = j; i < E; i += tpt) {
-                if (!((keep >> (i / gsz)) & 1ull)) continue;
-                const uint64_t k = sel_key(__fadd_rn(s[i], bias_s[i]), i);
-                if (n < K || k > kth) {
-                    int pos = n < K ? n : K - 1;
-                    if (n < K) ++n;
-                    while (pos > 0 && mine[pos - 1] < k) {
-                        mine[pos] = mine[pos - 1];
-                        --pos;
-                    }
-                    mine[pos] = k;
-                    kth = n == K ? mine[K - 1] : 0;
-                }
-            }
-            for (int r = n; r < K; ++r) mine[r] = 0;
-        }
-        epi_sync();
-        // step 4: merge the token's tpt sorted lists; gates over the unbiased s
-        if (j == 0 && t < p.T && !aborted) {
-            const uint64_t *lst = lists + (size_t)tl * tpt * K;
-            int ptr[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) ptr[u] = 0;
-            float denom = 0.f;
-            for (int r = 0; r < K; ++r) {
-                uint64_t best = 0;
-                int bq = 0;
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    if (u < tpt && ptr[u] < K) {
-                        const uint64_t k = lst[u * K + ptr[u]];
-                        if (k > best) { best = k; bq = u; }
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 16; ++u) ptr[u] += u == bq;
-                int e = key_index(best);
-                e = e < 0 ? 0 : (e >= E ? E - 1 : e);
-                p.topk_idx[(size_t)t * K + r] = e;
-                denom = __fadd_rn(denom, s[e]);
-            }
-            for (int r = 0; r < K; ++r) {
-                const int e = p.topk_idx[(size_t)t * K + r];
-                p.topk_w[(size_t)t * K + r] = __fdiv_rn(s[e], denom);
-            }
-        }
-        // affinities, when the caller asked for them (coalesced row copies)
-        if (p.scores && !aborted) {
-            for (int i = et; i < R * E; i += EPI_THREADS) {
-                const int rl = i / E, col = i - rl * E;
-                const int tt = m0 + rank * R + rl;
-                if (tt < p.T) p.scores[(size_t)tt * E + col] = srow[(size_t)rl * sp + col];
-            }
+        switch (C) {
+        case 1: select_rows<1>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
+        case 2: select_rows<2>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
+        case 4: select_rows<4>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
+        default: select_rows<8>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
         }
     }
 
@@ -474,7 +502,9 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
 
 }  // namespace rfused
 
-bool router_fused_supported(int E, int G, int K) { return E <= 256 && G <= 32 && K <= 16; }
+bool router_fused_supported(int E, int G, int K) {
+    return E <= 256 && G <= 32 && E / G <= 32 && K <= 32;
+}
 
 int router_fused_cluster(int T, int d) {
     const int tiles = (T + rfused::BM - 1) / rfused::BM;
@@ -493,14 +523,13 @@ cudaError_t launch_router_select_fused(const void *x, const void *e_split, const
     if (T == 0) return cudaSuccess;
     const int BN = (E + 15) / 16 * 16;
     const int C = router_fused_cluster(T, d);
-    const int R = BM / C, tpt = EPI_THREADS / R;
     const size_t b_bytes = (size_t)BN * BK * 2;
     int b_stages = (int)(B_RING_BYTES / b_bytes);
     if (b_stages > MAX_B_STAGES) b_stages = MAX_B_STAGES;
     const size_t ring = (size_t)A_STAGES * A_BYTES + b_stages * b_bytes;
     // after the k loop the same bytes hold the received partials, then the
     // affinity rows, group keys and candidate lists of the selection
-    const size_t post = (size_t)BM * (BN + 4) * 4 + (size_t)R * G * 8 + (size_t)R * tpt * K * 8;
+    const size_t post = (size_t)BM * (BN + 4) * 4;
     size_t dyn = ring > post ? ring : post;
     dyn += 1024;
     Maps m;

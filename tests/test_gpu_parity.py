@@ -299,6 +299,18 @@ def test_expert_ffn_segment_edges(orc):
     _ffn_case(orc, sh, counts)
 
 
+def test_expert_ffn_paired_tiles(orc):
+    """Experts averaging >= 512 rows take the paired gate/up GEMM (two row tiles
+    per weight stage, tiles handed out dynamically): segments that end in a
+    full pair, a pair with a 1-row second tile, and a trailing single tile,
+    every row against the oracle."""
+    counts = [0, 1, 129, 257, 384, 640, 1000, 1023, 1046, 1386]
+    sh = synth.MoeShape("pairs", T=sum(counts), d=192, E=len(counts), G=1, K=1, M=1, d_ff=192,
+                        n_shared=1, d_ff_shared=192, x_sigma=1, e_sigma=1, bias_sigma=0)
+    assert sh.T * sh.K >= 512 * sh.E
+    _ffn_case(orc, sh, counts)
+
+
 def test_expert_ffn_flags_bad_offsets():
     """Offsets outside the buffer or decreasing are reported; nothing is written out of bounds."""
     sh = H.RAGGED2.replace(T=64, n_shared=0, d_ff_shared=0)
