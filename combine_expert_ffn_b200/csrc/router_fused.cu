@@ -96,14 +96,19 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int64_
     return true;
 }
 
-__device__ __forceinline__ float affinity_fn(float L, int kind) {
-    if (kind == 1) {
+// The affinity function, KIND a compile-time constant so that each instance
+// holds one formula (a runtime branch between the two got both evaluated per
+// element, measured).
+template <int KIND>
+__device__ __forceinline__ float affinity_fn(float L) {
+    if (KIND == 1) {
         const float sp = L > 0.f ? L + log1pf(expf(-L)) : log1pf(expf(L));
         return sqrtf(sp);
     }
-    // sigmoid: hardware exp2 and a rounded reciprocal; a few 1e-7 from the
-    // definition, far inside the affinities' 1e-5 bar
-    return __frcp_rn(1.0f + __expf(-L));
+    // sigmoid: hardware exp2 and reciprocal (a few ulp each), a few 1e-7 from
+    // the definition, far inside the affinities' 1e-5 bar.  (The IEEE-rounded
+    // reciprocal costs about ten times as much here, measured.)
+    return __fdividef(1.0f, 1.0f + __expf(-L));
 }
 
 // Selection key: orderable(b) in the high word, ~index in the low word, so the
@@ -159,15 +164,16 @@ __device__ __forceinline__ float key_value(uint64_t k) {
 // g): the token's G groups sit in G consecutive lanes of an epilogue warp, 32
 // / G tokens per warp.  A thread adds its group's gsz <= 32 logits over the C
 // partials in rank order, adds the offset, applies the affinity function and
-// keeps s and the selection key of b = s + bias per expert in registers; then
+// keeps the selection key of b = s + bias per expert in registers; then
 //   group score  the sum of the group's K/M best b, added in pick order;
 //   kept groups  the M best group keys (a group is kept when fewer than M of
 //                the token's groups have a larger key);
 //   top-K        K rounds of "largest key below the last pick" over the kept
-//                groups' lanes (tree inside a lane, shuffles across lanes),
-//                the pick's unbiased s travelling with its key.
+//                groups' lanes (tree inside a lane, shuffles across lanes);
+//                the token's first lane recomputes each pick's unbiased s
+//                from its logits for the gate.
 // Keys are orderable(b) << 32 | ~index, so ties go to the lower index.
-template <int C>
+template <int C, int KIND>
 __device__ __forceinline__ void select_rows(const Params &p, const float *red, int rs, int R,
                                             int m0, int rank, int ew, int lane,
                                             const float *bias_s, const float *off_s,
@@ -182,26 +188,21 @@ __device__ __forceinline__ void select_rows(const Params &p, const float *red, i
         const bool valid = sub < tpw && tl < R;
         const int t = m0 + rank * R + tl;
         const float *rg = red + (size_t)(valid ? tl : 0) * rs + g * gsz;
-        float sv[32];
         uint64_t kv[32];
+        float *so = (valid && p.scores && !aborted && t < p.T)
+                        ? p.scores + (size_t)t * E + g * gsz : nullptr;
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-            sv[q] = 0.f;
             kv[q] = 0ull;
             if (q < gsz) {
                 float L = rg[q];
 #pragma unroll
                 for (int r = 1; r < C; ++r) L = __fadd_rn(L, rg[(size_t)r * R * rs + q]);
                 if (p.off) L += off_s[g * gsz + q];
-                sv[q] = affinity_fn(L, p.affinity);
-                kv[q] = sel_key(__fadd_rn(sv[q], bias_s[g * gsz + q]), g * gsz + q);
+                const float sq = affinity_fn<KIND>(L);
+                kv[q] = sel_key(__fadd_rn(sq, bias_s[g * gsz + q]), g * gsz + q);
+                if (so) so[q] = sq;
             }
-        }
-        if (valid && p.scores && !aborted && t < p.T) {
-            float *so = p.scores + (size_t)t * E + g * gsz;
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-                if (q < gsz) so[q] = sv[q];
         }
         // group score: the sum of the group's K/M best b, in pick order
         uint64_t prev = ~0ull;
@@ -226,32 +227,32 @@ __device__ __forceinline__ void select_rows(const Params &p, const float *red, i
         float denom = 0.f;
         for (int r = 0; r < K; ++r) {
             uint64_t best = kept ? tree_best(kv, gsz, last) : 0ull;
-            float bs = 0.f;
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-                if (q < gsz && kv[q] == best && best != 0ull) bs = sv[q];
             if (pow2) {  // the token's lanes are an aligned power of two
                 for (int off = G >> 1; off > 0; off >>= 1) {
                     const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, best, off);
-                    const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, off);
-                    if (o > best) { best = o; bs = os; }
+                    best = o > best ? o : best;
                 }
             } else {
                 uint64_t mx = best;
-                float ms = bs;
                 for (int q = 0; q < G; ++q) {
-                    const int src = sub * G + q < 32 ? sub * G + q : 0;
-                    const uint64_t o = __shfl_sync(0xFFFFFFFFu, best, src);
-                    const float os = __shfl_sync(0xFFFFFFFFu, bs, src);
-                    if (o > mx) { mx = o; ms = os; }
+                    const uint64_t o =
+                        __shfl_sync(0xFFFFFFFFu, best, sub * G + q < 32 ? sub * G + q : 0);
+                    mx = o > mx ? o : mx;
                 }
                 best = mx;
-                bs = ms;
             }
             last = best;
             if (writer) {
                 int e = key_index(best);
                 e = e < 0 ? 0 : (e >= E ? E - 1 : e);
+                // the pick's unbiased affinity, recomputed from its logits exactly as
+                // its owner lane computed it
+                const float *re = red + (size_t)tl * rs + e;
+                float L = re[0];
+#pragma unroll
+                for (int c = 1; c < C; ++c) L = __fadd_rn(L, re[(size_t)c * R * rs]);
+                if (p.off) L += off_s[e];
+                const float bs = affinity_fn<KIND>(L);
                 p.topk_idx[(size_t)t * K + r] = e;
                 p.topk_w[(size_t)t * K + r] = bs;  // s for now; divided below
                 denom = __fadd_rn(denom, bs);
@@ -282,8 +283,9 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
     const int tile = blockIdx.x / C;
     const int m0 = tile * BM;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, derived by an offset from the __shared__ array so
+    // that accesses through it stay shared-memory accesses
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t smem0 = smem_u32(smem);
     const uint32_t b_ring0 = smem0 + A_STAGES * A_BYTES;
     const uint32_t b_bytes = (uint32_t)p.BN * BK * 2;
@@ -483,11 +485,21 @@ router_select_kernel(const __grid_constant__ Maps maps, const Params p) {
     if (warp >= 2) {
         epi_sync();
         const bool aborted = *abort_flag != 0;
-        switch (C) {
-        case 1: select_rows<1>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
-        case 2: select_rows<2>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
-        case 4: select_rows<4>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
-        default: select_rows<8>(p, red, rs, R, m0, rank, warp - 2, lane, bias_s, off_s, aborted); break;
+        const int ew = warp - 2;
+        if (p.affinity == 1) {
+            switch (C) {
+            case 1: select_rows<1, 1>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            case 2: select_rows<2, 1>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            case 4: select_rows<4, 1>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            default: select_rows<8, 1>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            }
+        } else {
+            switch (C) {
+            case 1: select_rows<1, 0>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            case 2: select_rows<2, 0>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            case 4: select_rows<4, 0>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            default: select_rows<8, 0>(p, red, rs, R, m0, rank, ew, lane, bias_s, off_s, aborted); break;
+            }
         }
     }
 
