@@ -39,7 +39,7 @@ EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_l
            "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine", "moe_ep_dispatch_fp8",
            "moe_ep_expert_ffn_fp8", "moe_ep_token_plan", "moe_ep_token_base",
            "moe_ep_dispatch_dedup", "moe_ep_fanout", "moe_ep_dispatch_dedup_fp8",
-           "moe_ep_fanout_fp8", "moe_ep_combine_plan",
+           "moe_ep_fanout_fp8", "moe_ep_combine_plan", "moe_ep_dispatch_dedup_plan",
            "moe_ep_precombine", "moe_ep_combine_dedup", "moe_ipc_get_handle",
            "moe_ipc_open_handle", "moe_ipc_close_handle", "moe_packed_weights_size",
            "moe_pack_weights", "moe_expert_ffn_packed", "moe_forward_packed")
@@ -107,6 +107,7 @@ _sig = {
     "moe_ep_dispatch_dedup_fp8": (C.c_int, [_CP, C.c_int32] + [_P] * 12),
     "moe_ep_fanout_fp8": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
     "moe_ep_combine_plan": (C.c_int, [_CP, C.c_int32] + [_P] * 12),
+    "moe_ep_dispatch_dedup_plan": (C.c_int, [_CP, C.c_int32] + [_P] * 15),
     "moe_ep_precombine": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
     "moe_ep_combine_dedup": (C.c_int, [_CP, C.c_int32] + [_P] * 8),
     "moe_ep_dispatch_fp8": (C.c_int, [_CP, C.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -341,6 +342,18 @@ def moe_ep_combine_plan(cfg, world, topk_idx, topk_w, offsets, inv_perm, base, t
                                  _ptr(offsets), _ptr(inv_perm), _ptr(base), _ptr(tok_slot),
                                  _ptr(tok_base), _ptr(list_ptrs), _ptr(lw_ptrs), _ptr(lcnt_ptrs),
                                  _ptr(device_status), _stream(stream)))
+
+
+def moe_ep_dispatch_dedup_plan(cfg, world, x, topk_idx, topk_w, offsets, inv_perm, base,
+                               tok_slot, tok_base, recv_tok_ptrs, recv_idx_ptrs, list_ptrs,
+                               lw_ptrs, lcnt_ptrs, device_status=None, stream=None) -> None:
+    """moe_ep_dispatch_dedup + moe_ep_combine_plan in one launch (same outputs)."""
+    _ok("moe_ep_dispatch_dedup_plan",
+        _lib.moe_ep_dispatch_dedup_plan(_cfg(cfg), int(world), _ptr(x), _ptr(topk_idx),
+                                        _ptr(topk_w), _ptr(offsets), _ptr(inv_perm), _ptr(base),
+                                        _ptr(tok_slot), _ptr(tok_base), _ptr(recv_tok_ptrs),
+                                        _ptr(recv_idx_ptrs), _ptr(list_ptrs), _ptr(lw_ptrs),
+                                        _ptr(lcnt_ptrs), _ptr(device_status), _stream(stream)))
 
 
 def moe_ep_precombine(cfg, world, recv_y, lst, lw, lcnt, tok_base, partial, device_status=None,

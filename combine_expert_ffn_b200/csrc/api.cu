@@ -10,6 +10,8 @@
 #include <mutex>
 #include <unordered_map>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.h"
 
 namespace moe {
@@ -20,6 +22,21 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 namespace {
 
 constexpr int64_t kWaitTimeoutNs = 2000000000LL;  // 2 s per device wait
+
+// NVTX range ("moe.route", "moe.dispatch", ...) around the enqueue of one stage:
+// a timeline profiler shows it over the stage's kernels.  NVTX v3 is header
+// only; without a profiler attached a push or pop is a call to an empty hook.
+class StageRange {
+  public:
+    explicit StageRange(const char *name) { nvtxRangePushA(name); }
+    ~StageRange() { nvtxRangePop(); }
+    void next(const char *name) {  // close this stage's range and open the next one
+        nvtxRangePop();
+        nvtxRangePushA(name);
+    }
+    StageRange(const StageRange &) = delete;
+    StageRange &operator=(const StageRange &) = delete;
+};
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -246,6 +263,7 @@ moe_status moe_route(const moe_config *c, const void *x, const float *router_w,
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
     if ((st = check_device())) return st;
+    StageRange range("moe.route");
     return cuda_status(route_affinity(*c, x, router_w, logit_offset, bias, topk_idx, topk_w,
                                       scores, ws, L, as_stream(stream)));
 }
@@ -282,6 +300,7 @@ moe_status moe_dispatch(const moe_config *c, const void *x, const int32_t *topk_
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
     if ((st = check_device())) return st;
+    StageRange range("moe.dispatch");
     DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),
                   at<int32_t>(ws, L.send_part), at<int32_t>(ws, L.sendtok_part)};
     return cuda_status(launch_dispatch(x, topk_idx, c->T, c->d, c->E, c->G, c->K, counts, offsets,
@@ -296,6 +315,7 @@ moe_status moe_permute(const moe_config *c, const void *x, const int32_t *inv_pe
     if (c->T > 0 && (!x || !inv_perm || !x_perm)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
     if ((st = check_device())) return st;
+    StageRange range("moe.permute");
     return cuda_status(launch_permute(x, inv_perm, c->T, c->d, c->K, x_perm, as_stream(stream)));
 }
 
@@ -379,6 +399,7 @@ moe_status moe_expert_ffn(const moe_config *c, const void *x_perm, const int32_t
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
     if ((st = check_device())) return st;
+    StageRange range("moe.expert_ffn");
     FfnArgs a{};
     a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
     a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
@@ -433,6 +454,7 @@ moe_status moe_combine(const moe_config *c, const void *y_perm, const int32_t *i
     if (c->T > 0 && (!y_perm || !inv_perm || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(y_perm) || !aligned16(y_shared) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
     if ((st = check_device())) return st;
+    StageRange range("moe.combine");
     return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_shared, c->T, c->d, c->K,
                                       (int64_t)c->T * c->K, out, as_stream(stream)));
 }
@@ -481,6 +503,8 @@ static moe_status forward_impl(const moe_config *c, const void *x, const float *
     void *y_sh = c->n_shared > 0 ? at<void>(ws, L.y_sh) : nullptr;
     int32_t *status = at<int32_t>(ws, L.status);
 
+    StageRange layer("moe.forward");
+    StageRange stage("moe.route");
     if (c->router == MOE_ROUTER_HASH) {
         if (launch_hash_route(token_ids, c->T, c->E, c->G, c->K, c->M, topk_idx, topk_w, s))
             return MOE_ERR_CUDA;
@@ -489,6 +513,7 @@ static moe_status forward_impl(const moe_config *c, const void *x, const float *
                            s))
             return MOE_ERR_CUDA;
     }
+    stage.next("moe.dispatch");
     DispatchWs dw{at<int32_t>(ws, L.hist_t), at<int32_t>(ws, L.base_t),
                   at<int32_t>(ws, L.send_part), at<int32_t>(ws, L.sendtok_part)};
     // Two steps: the dispatch writes x_perm, GEMM1 reads it with tiled TMA loads.
@@ -507,6 +532,7 @@ static moe_status forward_impl(const moe_config *c, const void *x, const float *
         return MOE_ERR_CUDA;
     if (fp8 && launch_gather_fp8(x, inv_perm, c->T, c->d, c->K, x_perm_q, x_scale, s))
         return MOE_ERR_CUDA;
+    stage.next("moe.expert_ffn");
     FfnArgs a{};
     a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
     a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
@@ -520,6 +546,7 @@ static moe_status forward_impl(const moe_config *c, const void *x, const float *
     a.status = status;
     a.timeout_ns = kWaitTimeoutNs;
     if (launch_expert_ffn(a, s)) return MOE_ERR_CUDA;
+    stage.next("moe.combine");
     return cuda_status(launch_combine(y_perm, inv_perm, topk_w, y_sh, c->T, c->d, c->K,
                                       (int64_t)c->T * c->K, out, s));
 }
@@ -593,6 +620,7 @@ moe_status moe_expert_ffn_packed(const moe_config *c, const void *x_perm, const 
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
     if ((st = check_device())) return st;
+    StageRange range("moe.expert_ffn");
     FfnArgs a{};
     a.T = c->T; a.d = c->d; a.E = c->E; a.K = c->K; a.d_ff = c->d_ff;
     a.n_shared = c->n_shared; a.d_ff_shared = c->d_ff_shared;
@@ -712,6 +740,30 @@ moe_status moe_ep_dispatch_dedup(const moe_config *c, int32_t world, const void 
                                                 tok_base, recv_tok, recv_idx, tok_rows, cap, c->T,
                                                 c->d, c->E, c->K, world, device_status,
                                                 as_stream(stream)));
+}
+
+moe_status moe_ep_dispatch_dedup_plan(const moe_config *c, int32_t world, const void *x,
+                                      const int32_t *topk_idx, const float *topk_w,
+                                      const int32_t *offsets, const int32_t *inv_perm,
+                                      const int32_t *base, const int32_t *tok_slot,
+                                      const int32_t *tok_base, void *const *recv_tok,
+                                      int32_t *const *recv_idx, int32_t *const *list,
+                                      float *const *lw, int32_t *const *lcnt,
+                                      int32_t *device_status, void *stream) {
+    moe_status st = moe_check_config(c);
+    if (st) return st;
+    if (!ep_args_ok(c, world)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->T > 0 && (!x || !topk_idx || !topk_w || !offsets || !inv_perm || !base ||
+                     !tok_slot || !tok_base || !recv_tok || !recv_idx || !list || !lw || !lcnt))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_device())) return st;
+    const int64_t tok_rows = (int64_t)world * c->T;
+    return cuda_status(launch_ep_dispatch_dedup(x, topk_idx, offsets, inv_perm, base, tok_slot,
+                                                tok_base, recv_tok, recv_idx, tok_rows,
+                                                tok_rows * c->K, c->T, c->d, c->E, c->K, world,
+                                                device_status, as_stream(stream), topk_w, list,
+                                                lw, lcnt));
 }
 
 moe_status moe_ep_fanout(const moe_config *c, int32_t world, const void *recv_tok,

@@ -28,12 +28,21 @@ namespace {
 constexpr int BLK = DISPATCH_BLOCK;       // tokens per block = threads per CTA
 constexpr int WORDS = BLK / 32;           // mask words per expert
 
+constexpr int KMAX = 32;                  // largest K (moe_check_config)
+
+// Token t's K expert ids, all loads issued before any is used; -1 past K or T.
+__device__ __forceinline__ void load_ids(const int32_t *__restrict__ topk_idx, int t, int T, int K,
+                                         int (&ev)[KMAX]) {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+        ev[j] = (t < T && j < K) ? __ldg(topk_idx + (size_t)t * K + j) : -1;
+}
+
 // Rebuilds the block's expert masks in smem: masks[e * WORDS + w] bit l set if
-// token (block * BLK + 32 w + l) chose expert e.  Returns nothing; flags bad
-// ids and repeated experts of a token in `status`.
-__device__ __forceinline__ void build_masks(const int32_t *__restrict__ topk_idx, int T, int E,
-                                            int K, uint32_t *masks, int32_t *status,
-                                            bool flag_errors) {
+// token (block * BLK + 32 w + l) chose expert e (ev: this thread's token's ids).
+// Flags bad ids and repeated experts of a token in `status`.
+__device__ __forceinline__ void build_masks(const int (&ev)[KMAX], int T, int E, int K,
+                                            uint32_t *masks, int32_t *status, bool flag_errors) {
     const int tid = threadIdx.x;
     for (int i = tid; i < E * WORDS; i += BLK) masks[i] = 0u;
     __syncthreads();
@@ -41,8 +50,10 @@ __device__ __forceinline__ void build_masks(const int32_t *__restrict__ topk_idx
     if (t < T) {
         const uint32_t bit = 1u << (tid & 31);
         const int w = tid >> 5;
-        for (int j = 0; j < K; ++j) {
-            const int e = topk_idx[(size_t)t * K + j];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j >= K) break;
+            const int e = ev[j];
             if (e < 0 || e >= E) {
                 if (flag_errors) record_status(status, MOE_ERR_DEVICE_FAULT);
                 continue;
@@ -65,14 +76,18 @@ dispatch_count_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int G,
     int32_t *sendtok_s = send_s + G * G;                     // [G*G]
     const int tid = threadIdx.x, nblk = gridDim.x, blk = blockIdx.x;
     for (int i = tid; i < 2 * G * G; i += BLK) send_s[i] = 0;
-    build_masks(topk_idx, T, E, K, masks, status, true);
-
     const int t = blk * BLK + tid;
+    int ev[KMAX];
+    load_ids(topk_idx, t, T, K, ev);
+    build_masks(ev, T, E, K, masks, status, true);
+
     if (t < T) {
         const int gsz = E / G, src = t / (T / G);
         uint64_t hit = 0;
-        for (int j = 0; j < K; ++j) {
-            const int e = topk_idx[(size_t)t * K + j];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j >= K) break;
+            const int e = ev[j];
             if (e < 0 || e >= E) continue;
             const int g = e / gsz;
             atomicAdd(&send_s[src * G + g], 1);
@@ -160,6 +175,9 @@ dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int 
     int32_t *base_s = cnt_s + E;                                    // [E]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nblk = gridDim.x, blk = blockIdx.x;
+    const int t = blk * BLK + tid;
+    int ev[KMAX];  // issued first: their latency overlaps the histogram reads
+    load_ids(topk_idx, t, T, K, ev);
 
     for (int e = tid; e < E; e += BLK) {
         int c, b;
@@ -167,6 +185,8 @@ dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int 
             const int32_t *h = hist_t + (size_t)e * nblk;
             c = 0;
             b = 0;
+            // independent loads: unrolled so that many are in flight at once
+#pragma unroll 16
             for (int q = 0; q < nblk; ++q) {
                 const int v = h[q];
                 c += v;
@@ -183,6 +203,7 @@ dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int 
     if (fused_scan && blk == 0) {
         for (int i = tid; i < G * G; i += BLK) {
             int a = 0, c = 0;
+#pragma unroll 16
             for (int q = 0; q < nblk; ++q) {
                 a += send_part[(size_t)q * G * G + i];
                 c += sendtok_part[(size_t)q * G * G + i];
@@ -207,7 +228,7 @@ dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int 
         if (lane >= o) incl += n;
     }
     if (lane == 31) wsum[warp] = incl;
-    build_masks(topk_idx, T, E, K, masks, nullptr, false);  // contains __syncthreads
+    build_masks(ev, T, E, K, masks, nullptr, false);  // contains __syncthreads
     int wpre = 0;
     for (int w = 0; w < warp; ++w) wpre += wsum[w];
     int acc = wpre + incl - run;
@@ -223,12 +244,13 @@ dispatch_scatter_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int 
     if (blk == 0)
         for (int e = tid; e <= E; e += BLK) offsets[e] = offs[e];
 
-    const int t = blk * BLK + tid;
     if (t >= T) return;
     const int w = tid >> 5;
     const uint32_t below = (1u << lane) - 1u;
-    for (int j = 0; j < K; ++j) {
-        const int e = topk_idx[(size_t)t * K + j];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        if (j >= K) break;
+        const int e = ev[j];
         if (e < 0 || e >= E) {
             inv_perm[(size_t)t * K + j] = -1;
             continue;

@@ -331,6 +331,10 @@ ep_dispatch_dedup_kernel(const uint4 *__restrict__ x, const int32_t *__restrict_
 // the previous row's stores when a warp walks several rows; 1 (8 warps per
 // CTA) puts twice as many rows in flight when there are about as many rows as
 // warps (the per-rank batches of an expert-parallel step).
+// PLAN: the same launch also writes the deduplicated combine's lists (what
+// ep_combine_plan_kernel writes): lane j < K knows copy (t, j)'s owner, token
+// row and copy row, and its slot k among the token's copies at that owner is
+// the number of lower lanes with the same owner (a warp match).
 template <int NB>
 __host__ __device__ constexpr int db_warps() { return NB == 2 ? 4 : 8; }
 
@@ -340,7 +344,7 @@ __device__ __forceinline__ void db_drain(uint32_t bar, uint32_t parity, int64_t 
     }
 }
 
-template <int NB>
+template <int NB, bool PLAN>
 __global__ void __launch_bounds__(db_warps<NB>() * 32)
 ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restrict__ topk_idx,
                               const int32_t *__restrict__ offsets,
@@ -349,13 +353,18 @@ ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restr
                               const int32_t *__restrict__ tok_base, char *const *__restrict__ recv_tok,
                               int32_t *const *__restrict__ recv_idx, int64_t tok_rows,
                               int64_t recv_rows, int T, int row_bytes, int E, int K, int El,
-                              int world, int32_t *status, int64_t timeout_ns) {
+                              int world, int32_t *status, int64_t timeout_ns,
+                              const float *__restrict__ topk_w, int32_t *const *__restrict__ list,
+                              float *const *__restrict__ lw, int32_t *const *__restrict__ lcnt) {
     constexpr int WARPS = db_warps<NB>();
     extern __shared__ __align__(128) uint8_t dsm_rows[];
     __shared__ int32_t delta_s[EP_MAX_E];
     __shared__ int32_t tokbase_s[EP_MAX_WORLD];
     __shared__ char *tok_tab_s[EP_MAX_WORLD];
     __shared__ int32_t *idx_tab_s[EP_MAX_WORLD];
+    __shared__ int32_t *list_s[PLAN ? EP_MAX_WORLD : 1];
+    __shared__ float *lw_s[PLAN ? EP_MAX_WORLD : 1];
+    __shared__ int32_t *lcnt_s[PLAN ? EP_MAX_WORLD : 1];
     __shared__ __align__(8) uint64_t lbar[WARPS][2];
     __shared__ int abort_s[WARPS];
     for (int e = threadIdx.x; e < E; e += blockDim.x) delta_s[e] = base[e] - offsets[e];
@@ -363,6 +372,11 @@ ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restr
         tokbase_s[o] = tok_base[o];
         tok_tab_s[o] = recv_tok[o];
         idx_tab_s[o] = recv_idx[o];
+        if (PLAN) {
+            list_s[o] = list[o];
+            lw_s[o] = lw[o];
+            lcnt_s[o] = lcnt[o];
+        }
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t buf0 = smem_u32(dsm_rows) + (uint32_t)(warp * NB * row_bytes);
@@ -395,10 +409,13 @@ ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restr
             const int sl = __ldg(tok_slot + (int64_t)t * world + lane + 32);
             if (sl >= 0) trow1 = (int64_t)tokbase_s[lane + 32] + sl;
         }
+        int po = -1;           // owner of copy (t, lane); -1: no copy in this lane
+        int64_t ptrow = -1, prow = -1;  // its token row and copy row there (-1: out of bounds)
         if (lane < K) {
             const int e = __ldg(topk_idx + (int64_t)t * K + lane);
             if (e >= 0 && e < E) {  // invalid ids: flagged by the local plan
                 const int o = e / El;
+                po = o;
                 const int sl = __ldg(tok_slot + (int64_t)t * world + o);
                 const int64_t trow = (int64_t)tokbase_s[o] + sl;
                 const int64_t row = (int64_t)delta_s[e] + __ldg(inv_perm + (int64_t)t * K + lane);
@@ -406,7 +423,18 @@ ep_dispatch_dedup_bulk_kernel(const char *__restrict__ x, const int32_t *__restr
                     if (status) record_status(status, MOE_ERR_DEVICE_FAULT);
                 } else {
                     idx_tab_s[o][row] = (int32_t)trow;
+                    ptrow = trow;
+                    prow = row;
                 }
+            }
+        }
+        if (PLAN) {  // the token's lanes at one owner, in slot order (warp-uniform loop)
+            const unsigned grp = __match_any_sync(0xFFFFFFFFu, po >= 0 ? po : -1 - lane);
+            if (prow >= 0) {
+                const int k = __popc(grp & ((1u << lane) - 1u));
+                list_s[po][ptrow * K + k] = (int32_t)prow;
+                lw_s[po][ptrow * K + k] = __ldg(topk_w + (int64_t)t * K + lane);
+                if (k == 0) lcnt_s[po][ptrow] = __popc(grp);
             }
         }
         // the buffer to load next: every store that read it has read it
@@ -876,13 +904,48 @@ cudaError_t launch_ep_token_base(const int32_t *tok_counts_all, int world, int m
     return cudaGetLastError();
 }
 
+namespace {
+// One wave of the bulk dedup dispatch with NB buffers per warp.
+template <int NB, bool PLAN>
+cudaError_t launch_dedup_bulk(const char *x, const int32_t *topk_idx, const int32_t *offsets,
+                              const int32_t *inv_perm, const int32_t *base,
+                              const int32_t *tok_slot, const int32_t *tok_base,
+                              char *const *recv_tok, int32_t *const *recv_idx, int64_t tok_rows,
+                              int64_t recv_rows, int T, int row_bytes, int E, int K, int world,
+                              int32_t *status, const float *topk_w, int32_t *const *list,
+                              float *const *lw, int32_t *const *lcnt, size_t smem, int sms,
+                              cudaStream_t st) {
+    constexpr int warps = db_warps<NB>();
+    auto kern = ep_dispatch_dedup_bulk_kernel<NB, PLAN>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int per_sm = 1;  // CTAs resident per SM with this shared memory (one wave)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * warps, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int want = (T + warps - 1) / warps;
+    const int grid = want < per_sm * sms ? want : per_sm * sms;
+    kern<<<grid, 32 * warps, smem, st>>>(x, topk_idx, offsets, inv_perm, base, tok_slot, tok_base,
+                                        recv_tok, recv_idx, tok_rows, recv_rows, T, row_bytes, E,
+                                        K, E / world, world, status, 2000000000LL, topk_w, list,
+                                        lw, lcnt);
+    count_launch();
+    return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_ep_dispatch_dedup(const void *x, const int32_t *topk_idx, const int32_t *offsets,
                                      const int32_t *inv_perm, const int32_t *base,
                                      const int32_t *tok_slot, const int32_t *tok_base,
                                      void *const *recv_tok, int32_t *const *recv_idx,
                                      int64_t tok_rows, int64_t recv_rows, int T, int d, int E, int K,
-                                     int world, int32_t *status, cudaStream_t st) {
+                                     int world, int32_t *status, cudaStream_t st,
+                                     const float *topk_w, int32_t *const *list, float *const *lw,
+                                     int32_t *const *lcnt) {
     if (T == 0) return cudaSuccess;
+    const bool plan = list != nullptr;
     const int row_bytes = d * 2;
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -891,52 +954,40 @@ cudaError_t launch_ep_dispatch_dedup(const void *x, const int32_t *topk_idx, con
     const bool one = (int64_t)T <= (int64_t)sms * db_warps<1>();
     const size_t db_smem = (size_t)(one ? db_warps<1>() : db_warps<2>() * 2) * row_bytes;
     if (db_smem <= 112 * 1024) {
-        cudaError_t err;
-        int per_sm = 1;  // CTAs resident per SM with this shared memory (one wave)
-        int warps;
-        if (one) {
-            err = cudaFuncSetAttribute(ep_dispatch_dedup_bulk_kernel<1>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)db_smem);
-            if (err == cudaSuccess &&
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &per_sm, ep_dispatch_dedup_bulk_kernel<1>, 32 * db_warps<1>(), db_smem) !=
-                    cudaSuccess)
-                per_sm = 1;
-            warps = db_warps<1>();
-        } else {
-            err = cudaFuncSetAttribute(ep_dispatch_dedup_bulk_kernel<2>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)db_smem);
-            if (err == cudaSuccess &&
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &per_sm, ep_dispatch_dedup_bulk_kernel<2>, 32 * db_warps<2>(), db_smem) !=
-                    cudaSuccess)
-                per_sm = 1;
-            warps = db_warps<2>();
-        }
-        if (err != cudaSuccess) return err;
-        if (per_sm < 1) per_sm = 1;
-        const int want = (T + warps - 1) / warps;
-        const int grid = want < per_sm * sms ? want : per_sm * sms;
+        const char *xc = static_cast<const char *>(x);
+        char *const *rt = reinterpret_cast<char *const *>(recv_tok);
+        if (one && plan)
+            return launch_dedup_bulk<1, true>(xc, topk_idx, offsets, inv_perm, base, tok_slot,
+                                              tok_base, rt, recv_idx, tok_rows, recv_rows, T,
+                                              row_bytes, E, K, world, status, topk_w, list, lw,
+                                              lcnt, db_smem, sms, st);
         if (one)
-            ep_dispatch_dedup_bulk_kernel<1><<<grid, 32 * warps, db_smem, st>>>(
-                static_cast<const char *>(x), topk_idx, offsets, inv_perm, base, tok_slot,
-                tok_base, reinterpret_cast<char *const *>(recv_tok), recv_idx, tok_rows, recv_rows,
-                T, row_bytes, E, K, E / world, world, status, 2000000000LL);
-        else
-            ep_dispatch_dedup_bulk_kernel<2><<<grid, 32 * warps, db_smem, st>>>(
-                static_cast<const char *>(x), topk_idx, offsets, inv_perm, base, tok_slot,
-                tok_base, reinterpret_cast<char *const *>(recv_tok), recv_idx, tok_rows, recv_rows,
-                T, row_bytes, E, K, E / world, world, status, 2000000000LL);
-        count_launch();
-        return cudaGetLastError();
+            return launch_dedup_bulk<1, false>(xc, topk_idx, offsets, inv_perm, base, tok_slot,
+                                               tok_base, rt, recv_idx, tok_rows, recv_rows, T,
+                                               row_bytes, E, K, world, status, nullptr, nullptr,
+                                               nullptr, nullptr, db_smem, sms, st);
+        if (plan)
+            return launch_dedup_bulk<2, true>(xc, topk_idx, offsets, inv_perm, base, tok_slot,
+                                              tok_base, rt, recv_idx, tok_rows, recv_rows, T,
+                                              row_bytes, E, K, world, status, topk_w, list, lw,
+                                              lcnt, db_smem, sms, st);
+        return launch_dedup_bulk<2, false>(xc, topk_idx, offsets, inv_perm, base, tok_slot,
+                                           tok_base, rt, recv_idx, tok_rows, recv_rows, T,
+                                           row_bytes, E, K, world, status, nullptr, nullptr,
+                                           nullptr, nullptr, db_smem, sms, st);
     }
+    // rows wider than the shared-memory buffers: thread per 16-byte chunk, and the
+    // combine's lists (if asked for) from their own launch
     const int chunks = d / 8;
     ep_dispatch_dedup_kernel<<<grid_for((int64_t)T * chunks), 256, 0, st>>>(
         static_cast<const uint4 *>(x), topk_idx, offsets, inv_perm, base, tok_slot, tok_base,
         reinterpret_cast<uint4 *const *>(recv_tok), recv_idx, tok_rows, recv_rows, T, chunks, E,
         K, E / world, world, status);
     count_launch();
-    return cudaGetLastError();
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess || !plan) return err;
+    return launch_ep_combine_plan(topk_idx, topk_w, offsets, inv_perm, base, tok_slot, tok_base,
+                                  list, lw, lcnt, tok_rows, recv_rows, T, E, K, world, status, st);
 }
 
 cudaError_t launch_ep_fanout(const void *recv_tok, const int32_t *recv_idx,

@@ -75,7 +75,9 @@ cudaError_t launch_ep_dispatch_dedup(const void *x, const int32_t *topk_idx, con
                                      const int32_t *tok_slot, const int32_t *tok_base,
                                      void *const *recv_tok, int32_t *const *recv_idx,
                                      int64_t tok_rows, int64_t recv_rows, int T, int d, int E, int K,
-                                     int world, int32_t *status, cudaStream_t st);
+                                     int world, int32_t *status, cudaStream_t st,
+                                     const float *topk_w = nullptr, int32_t *const *list = nullptr,
+                                     float *const *lw = nullptr, int32_t *const *lcnt = nullptr);
 cudaError_t launch_ep_fanout(const void *recv_tok, const int32_t *recv_idx,
                              const int32_t *local_offsets, int El, int64_t tok_rows,
                              int64_t recv_rows, int d, void *recv_x, int32_t *status,

@@ -13,6 +13,8 @@ A rank owns E / world experts and routes its own tokens.  One step:
                                               or one row per token and owner plus a
                                               fan-out index per copy: dedup)
       (+ moe_ep_combine_plan, dedup_combine)  copy rows and gates per token, owner
+                                              (bf16 dedup: moe_ep_dispatch_dedup_plan,
+                                              one launch for both)
     barrier                                   every rank's stores are done
     (moe_ep_fanout, dedup)                    the owner's copy rows from token rows
     moe_ep_expert_ffn                         this rank's experts, shared experts
@@ -33,11 +35,11 @@ import torch
 
 from . import (MoeConfig, moe_dispatch, moe_ep_combine, moe_ep_combine_dedup,
                moe_ep_combine_plan, moe_ep_dispatch, moe_ep_dispatch_dedup,
-               moe_ep_dispatch_dedup_fp8, moe_ep_dispatch_fp8, moe_ep_expert_ffn,
-               moe_ep_expert_ffn_fp8, moe_ep_fanout, moe_ep_fanout_fp8, moe_ep_plan,
-               moe_ep_precombine, moe_ep_token_base, moe_ep_token_plan, moe_ep_workspace_size,
-               moe_ipc_close_handle, moe_ipc_get_handle, moe_ipc_open_handle, moe_route,
-               moe_route_hash, MOE_PAYLOAD_FP8, MOE_ROUTER_HASH)
+               moe_ep_dispatch_dedup_fp8, moe_ep_dispatch_dedup_plan, moe_ep_dispatch_fp8,
+               moe_ep_expert_ffn, moe_ep_expert_ffn_fp8, moe_ep_fanout, moe_ep_fanout_fp8,
+               moe_ep_plan, moe_ep_precombine, moe_ep_token_base, moe_ep_token_plan,
+               moe_ep_workspace_size, moe_ipc_close_handle, moe_ipc_get_handle,
+               moe_ipc_open_handle, moe_route, moe_route_hash, MOE_PAYLOAD_FP8, MOE_ROUTER_HASH)
 
 
 def _i32(n, device):
@@ -46,6 +48,10 @@ def _i32(n, device):
 
 class _RankState:
     """Per-rank buffers of one EP step."""
+
+    # bf16 dedup with the deduplicated combine: dispatch and combine lists in one
+    # launch (moe_ep_dispatch_dedup_plan); False: the two separate launches
+    fused_plan = True
 
     def __init__(self, cfg: MoeConfig, world: int, device, dedup: bool = False,
                  dedup_combine: bool = False):
@@ -164,6 +170,12 @@ class _RankState:
                                           self.inv, self.base, self.tok_slot, self.tok_base,
                                           tables[0], tables[1], tables[2], self.status, stream)
                 lists = tables[3:]
+            elif self.dedup_combine and self.fused_plan:  # the lists from the same launch
+                moe_ep_dispatch_dedup_plan(self.cfg, world, x, self.topk_idx, self.topk_w,
+                                           self.offsets, self.inv, self.base, self.tok_slot,
+                                           self.tok_base, tables[0], tables[1], tables[2],
+                                           tables[3], tables[4], self.status, stream)
+                return
             else:
                 moe_ep_dispatch_dedup(self.cfg, world, x, self.topk_idx, self.offsets, self.inv,
                                       self.base, self.tok_slot, self.tok_base, tables[0],

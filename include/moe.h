@@ -298,6 +298,15 @@ MOE_API moe_status moe_expert_ffn_fp8(const moe_config *cfg, const uint8_t *x_pe
  *   y_shared  [T, d]               bf16 out: sum of the shared FFNs
  * tcgen05 tensor cores, fp32 accumulation; the intermediate h = SiLU(gate) *
  * up is rounded to bf16 (nearest even) before the down projection.
+ * Passage: "MoE + Expert-Parallel Overlap (Exp08)", Implemented: shared
+ * (always active) plus fine-grained routed experts; its overlap simulator
+ * counts 6*d*d_ff FLOPs per token-expert pair, the work this call does.
+ * No counts argument: a segment's length is offsets[e+1] - offsets[e].
+ * Errors: MOE_ERR_INVALID_ARG (a required pointer NULL or not 16-byte
+ * aligned, ws not 256-byte aligned), MOE_ERR_WORKSPACE_TOO_SMALL,
+ * MOE_ERR_UNSUPPORTED_SHAPE (d or d_ff not a multiple of 64); offsets that
+ * are not monotone or leave [0, T*K] are skipped on the device and flagged
+ * MOE_ERR_DEVICE_FAULT in the status word.
  */
 MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
                           const void *w_gate, const void *w_up, const void *w_down,
@@ -330,6 +339,13 @@ MOE_API moe_status moe_expert_ffn_gather(const moe_config *cfg, const void *x,
 /*
  * Combine: out[t] = y_shared[t] + sum_j topk_w[t,j] * y_perm[inv_perm[t,j]],
  * fp32 accumulation, rounded to bf16.  y_shared may be NULL (treated as 0).
+ * Passage: "moe-node-limited-routing", "Why all to all dominates MoE step
+ * time": the combine all-to-all that returns each expert output to its
+ * token, here a local gather in token order, weighted by the gates.
+ *   y_perm   [T*K, d] bf16, inv_perm [T, K] int32 (row of copy (t, j), -1 for
+ *            none), topk_w [T, K] fp32, out [T, d] bf16; all caller-owned.
+ * Errors: MOE_ERR_INVALID_ARG (a required pointer NULL or not 16-byte
+ * aligned); rows of inv_perm outside [0, T*K) count as 0.
  */
 MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t *inv_perm,
                        const float *topk_w, const void *y_shared, void *out, void *stream);
@@ -526,6 +542,22 @@ MOE_API moe_status moe_ep_dispatch_dedup(const moe_config *cfg, int32_t world, c
 MOE_API moe_status moe_ep_fanout(const moe_config *cfg, int32_t world, const void *recv_tok,
                                  const int32_t *recv_idx, const int32_t *local_offsets,
                                  void *recv_x, int32_t *device_status, void *stream);
+
+/* moe_ep_dispatch_dedup and moe_ep_combine_plan (below) in one launch: the
+ * same recv_tok / recv_idx and the same list / lw / lcnt, bit for bit.  The
+ * lane that writes copy (t, j)'s fan-out index already holds its owner, token
+ * row and copy row, which are what the combine's list entry needs, so the
+ * lists cost no second pass over the copies.  Arguments as in the two calls;
+ * all pointers are required when T > 0; errors as moe_ep_dispatch_dedup. */
+MOE_API moe_status moe_ep_dispatch_dedup_plan(const moe_config *cfg, int32_t world,
+                                              const void *x, const int32_t *topk_idx,
+                                              const float *topk_w, const int32_t *offsets,
+                                              const int32_t *inv_perm, const int32_t *base,
+                                              const int32_t *tok_slot, const int32_t *tok_base,
+                                              void *const *recv_tok, int32_t *const *recv_idx,
+                                              int32_t *const *list, float *const *lw,
+                                              int32_t *const *lcnt, int32_t *device_status,
+                                              void *stream);
 
 /* The deduplicated dispatch of the FP8 payload (d % 128 == 0): codes and
  * scales of a token go once to each owner, recv_tq[o] ([world*T, d] bytes)

@@ -283,6 +283,43 @@ def test_emulated_ep_dedup_combine(orc, name, world):
     assert float((a - b).norm() / b.norm()) <= H.TOL_FROB
 
 
+@pytest.mark.parametrize("name,world", [("ragged", 2), ("ragged", 3), ("noshared", 4),
+                                        ("ragged2", 5)])
+def test_dedup_dispatch_with_plan_equals_two_launches(name, world):
+    """moe_ep_dispatch_dedup_plan (one launch) writes what moe_ep_dispatch_dedup
+    followed by moe_ep_combine_plan write: token rows, fan-out indices and the
+    combine's lists, gates and counts, bit for bit; the counts add up to the
+    copies each owner received."""
+    sh = H.shape(name)
+    inp = synth.make_inputs(sh, DEV)
+    ems = []
+    for fused in (True, False):
+        em = ep.EmulatedEP(sh, inp, world, dedup=True, dedup_combine=True)
+        for st in em.ranks:
+            st.fused_plan = fused
+        em.forward()
+        ems.append(em)
+    torch.cuda.synchronize()
+    K, El = sh.K, sh.E // world
+    for sa, sb in zip(ems[0].ranks, ems[1].ranks):
+        for st in (sa, sb):
+            assert int(st.status.item()) == moe.MOE_OK
+            assert moe.moe_read_device_status(st.ws) == moe.MOE_OK
+        n = int(sa.tok_base[world].item())
+        m = int(sa.local_offsets[El].item())
+        assert n == int(sb.tok_base[world].item()) and m == int(sb.local_offsets[El].item())
+        assert torch.equal(sa.recv_tok[:n].view(torch.int16), sb.recv_tok[:n].view(torch.int16))
+        assert torch.equal(sa.recv_idx[:m], sb.recv_idx[:m])
+        cnt = sa.recv_lcnt[:n]
+        assert torch.equal(cnt, sb.recv_lcnt[:n])
+        assert bool(((cnt >= 1) & (cnt <= K)).all()) and int(cnt.sum()) == m
+        used = (torch.arange(K, device=DEV)[None, :] < cnt[:, None].long()).reshape(-1)
+        assert torch.equal(sa.recv_list[:n * K][used], sb.recv_list[:n * K][used])
+        assert torch.equal(sa.recv_lw[:n * K][used].view(torch.int32),
+                           sb.recv_lw[:n * K][used].view(torch.int32))
+        assert torch.equal(sa.out.view(torch.int16), sb.out.view(torch.int16))
+
+
 def test_emulated_ep_dedup_combine_v3_matches_oracle(orc):
     sh = H.shape("v3")
     inp = synth.make_inputs(sh, DEV)
