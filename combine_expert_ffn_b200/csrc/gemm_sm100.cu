@@ -674,9 +674,11 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
 // 64 KB stages covers twice the MMA time of the 4-stage ring above, which
 // hides more of the L2 / HBM latency.  An expert with an odd number of row
 // tiles ends with a single tile (one MMA per k step).  Both accumulators use
-// all 512 TMEM columns, so the epilogue of a tile does not overlap the next
-// tile's MMAs; 8 epilogue warps (two per TMEM lane quarter, each half of the
-// columns) drain it.
+// all 512 TMEM columns, so there is no second accumulator for the next tile:
+// 8 epilogue warps (two per TMEM lane quarter, each half of the columns) read
+// both accumulators into registers (activated and rounded to bf16: 64 or 128
+// registers a thread), release TMEM, and only then store, so the next tile's
+// MMAs wait for the TMEM reads and the activation but not for the stores.
 // Tiles are handed out dynamically: the producer warp takes the next index
 // from a launch-wide atomic counter (zeroed on the stream before the launch)
 // and passes it to the MMA thread and the epilogue warps through a small ring
@@ -991,18 +993,23 @@ grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
             const int n_out = shared ? p.n_out_s : p.n_out_r;
             const CUtensorMap *omap = shared ? &maps.o_s : &maps.o_r;
             __nv_bfloat16 *obase = shared ? p.out_s : p.out_r;
+            // 1. both accumulators into registers (this warp's rows, its half of the
+            //    columns, already activated and rounded to bf16), then TMEM is
+            //    released: the next tile's MMAs overlap the stores below
+            constexpr int NCH = HALF / 32;  // 32-column chunks per tile and warp
+            uint4 keep[2][NCH][4];
+#pragma unroll
             for (int ti = 0; ti < 2; ++ti) {
                 const int rv = ti == 0 ? t.rv0 : t.rv1;
-                if (rv <= 0) break;
-                const int rbase = t.row0 + ti * BM;
                 const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + ti * BN_ACC;
-                const bool full = rv == BM;
-                const bool row_ok = row < rv;
-                __nv_bfloat16 *orow = obase + (size_t)(rbase + row) * n_out;
-#pragma unroll 1
-                for (int c = hh * HALF; c < hh * HALF + HALF; c += 32) {
-                    uint4 o[4];
-                    if (EPI == EPI_SWIGLU) {
+#pragma unroll
+                for (int cc = 0; cc < NCH; ++cc) {
+                    const int c = hh * HALF + cc * 32;
+                    uint4 *o = keep[ti][cc];
+                    if (rv <= 0) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) o[v] = make_uint4(0u, 0u, 0u, 0u);
+                    } else if (EPI == EPI_SWIGLU) {
                         uint32_t g[32], u[32];
                         tmem_ld32(taddr + c, g);
                         tmem_ld32(taddr + BN_ACC / 2 + c, u);
@@ -1030,6 +1037,25 @@ grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
                             o[v].w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
                         }
                     }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&tempty_bar));
+            tphase ^= 1u;
+            // 2. the stores
+#pragma unroll
+            for (int ti = 0; ti < 2; ++ti) {
+                const int rv = ti == 0 ? t.rv0 : t.rv1;
+                if (rv <= 0) continue;
+                const int rbase = t.row0 + ti * BM;
+                const bool full = rv == BM;
+                const bool row_ok = row < rv;
+                __nv_bfloat16 *orow = obase + (size_t)(rbase + row) * n_out;
+#pragma unroll
+                for (int cc = 0; cc < NCH; ++cc) {
+                    const int c = hh * HALF + cc * 32;
+                    const uint4 *o = keep[ti][cc];
                     if (t.n0 + c >= n_out) continue;  // whole chunk past the last column
                     if (full) {
                         // the staging buffer: the store that last read it must be done
@@ -1050,10 +1076,6 @@ grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&tempty_bar));
-            tphase ^= 1u;
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
