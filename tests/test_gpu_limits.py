@@ -55,10 +55,13 @@ def test_route_select_at_max_sizes(orc, E, G, K, M):
     np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), ref_w.view(np.uint32))
 
 
-@pytest.mark.parametrize("T,E,G,K", [(2048, 1024, 64, 32), (64, 1024, 64, 32), (128, 1024, 1, 1)])
+# 70016 tokens make 274 blocks of 256: more than the scatter kernel sums itself,
+# so the separate block-scan kernel runs
+@pytest.mark.parametrize("T,E,G,K", [(2048, 1024, 64, 32), (64, 1024, 64, 32), (128, 1024, 1, 1),
+                                     (70016, 256, 8, 8)])
 def test_dispatch_at_max_sizes(orc, T, E, G, K):
-    sh = _shape("dmax", T=T, d=128, E=E, G=G, K=K, M=1 if K == 1 else 16, d_ff=64, n_shared=0,
-                d_ff_shared=0)
+    sh = _shape("dmax", T=T, d=128, E=E, G=G, K=K, M=1 if K == 1 else min(16, G), d_ff=64,
+                n_shared=0, d_ff_shared=0)
     topk = synth.random_routing(3, T, E, K, 1.1, DEV)
     x = synth.normal(3, 1, (T, sh.d), 1.0, torch.bfloat16, DEV)
     cfg = moe.MoeConfig.of(sh)
