@@ -57,6 +57,15 @@
 #define MOE_GEMM_KB_GROUP 1
 #endif
 
+// CTA-pair grouped GEMMs (tcgen05.mma.cta_group::2, packed weights only):
+// 0 never (default), 1 always when the weights are packed.  Bit-identical to
+// the one-CTA kernel, but not faster: measured +17 % at the V3 routing (256-row
+// pair tiles pad 19 % more rows than 128-row tiles), +5 % at mid, +1 % at the
+// skewed routing (no padding), +50 % for decode (half as many weight streams).
+#ifndef MOE_GEMM_CTA2
+#define MOE_GEMM_CTA2 0
+#endif
+
 namespace moe {
 namespace gemm {
 
@@ -107,6 +116,7 @@ struct Maps {
     CUtensorMap o_r;   // routed output [rows_r, n_out_r]    box 32 x 32, for full tiles
     CUtensorMap o_s;   // shared output [T, n_out_s]         box 32 x 32
     CUtensorMap a_q;   // routed FP8 payload [rows_r, k_r] bytes, box 64 x 128 (A_FP8)
+    CUtensorMap bpk;   // CTA-pair kernel: the packed weights as rows of 128 bytes, box 64 x 128
 };
 
 struct Params {
@@ -131,6 +141,8 @@ struct Params {
     // bp_s (shared); null: tensor-map loads of the row-major weights
     const uint8_t *bp_r, *bp_s;
     int bp_nt_r;
+    // CTA-pair kernel: first 128-byte row of bp_r / bp_s in the map bpk
+    int64_t bpk_row_r, bpk_row_s;
 };
 
 // The B tile of (tile, k block kb) from the packed weights: one 32 KB bulk copy.
@@ -1090,6 +1102,342 @@ grouped_ffn_pair_kernel(const __grid_constant__ Maps maps, const Params p) {
     }
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// The grouped GEMM on pairs of SMs (a cluster of 2 CTAs and
+// tcgen05.mma.cta_group::2): a pair tile is 256 token rows of one expert (or
+// of the shared rows) x 256 accumulator columns.  CTA r of the pair holds
+// rows 128 r .. 128 r + 127 of A and rows 128 r .. of the 256-row weight tile
+// (its half of the packed 32 KB tile: one contiguous 16 KB), so per SM a k
+// block brings 32 KB into shared memory instead of 48 KB for the same MMA
+// work; each CTA's TMEM holds the accumulator of its own 128 rows, double
+// buffered, so the epilogue overlaps the next tile as in the one-CTA kernel.
+// The leader (rank 0) issues the MMAs.  Every load of both CTAs completes on
+// the leader's full barrier of its stage; the leader's commits arrive on the
+// empty and TMEM-full barriers of both CTAs (tcgen05.commit to both CTAs of
+// the pair), and both CTAs' epilogue warps arrive on the leader's TMEM-empty
+// barrier.  An
+// expert's last pair tile may hold fewer than 256 valid rows: rows past the
+// segment are computed from whatever the loads bring and never stored.
+// Packed weights only.
+constexpr int C2_STAGES = 6;
+constexpr int C2_STAGE_BYTES = A_BYTES + B_BYTES / 2;             // 32 KB per CTA
+constexpr int C2_THREADS = 192;
+constexpr int C2_SMEM_DYN = C2_STAGES * C2_STAGE_BYTES + 4 * 2 * STORE_BUF + 1024;
+constexpr int C2_ROWS = 2 * BM;                                    // rows per pair tile
+
+struct C2Tile {
+    int row0;        // first A row of the pair tile
+    int rows_valid;  // valid rows of the pair tile (may exceed 128, at most 256)
+    int n0;          // first output column
+    int e;           // expert or -1 (shared)
+    int kblocks;
+};
+
+template <int EPI>
+__device__ __forceinline__ C2Tile decode_c2(int idx, const int *tile_base, const int *seg,
+                                            const int *segc, const Params &p, int ntr,
+                                            int nt_s) {
+    constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
+    C2Tile t;
+    if (idx < ntr) {
+        int lo = 0, hi = p.E;  // tile_base[lo] <= idx < tile_base[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tile_base[mid] <= idx) lo = mid; else hi = mid;
+        }
+        const int cnt = segc[lo];
+        const int mt = (cnt + C2_ROWS - 1) / C2_ROWS;
+        const int local = idx - tile_base[lo];
+        const int n = local / mt, m = local - n * mt;
+        t.row0 = seg[lo] + m * C2_ROWS;
+        t.rows_valid = min(C2_ROWS, cnt - m * C2_ROWS);
+        t.n0 = n * BN_OUT;
+        t.e = lo;
+        t.kblocks = p.k_r / BK;
+    } else {
+        const int local = idx - ntr;
+        const int m = local / nt_s, n = local - m * nt_s;
+        t.row0 = m * C2_ROWS;
+        t.rows_valid = min(C2_ROWS, p.T - m * C2_ROWS);
+        t.n0 = n * BN_OUT;
+        t.e = -1;
+        t.kblocks = p.k_s / BK;
+    }
+    return t;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(C2_THREADS, 1)
+grouped_ffn_cta2_kernel(const __grid_constant__ Maps maps, const Params p) {
+    constexpr int BN_OUT = Cfg<EPI>::BN_OUT;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[C2_STAGES];   // used in the leader
+    __shared__ __align__(8) uint64_t empty_bar[C2_STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];          // used in the leader
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ int tile_base[MAX_E + 1];
+    __shared__ int seg[MAX_E];
+    __shared__ int segc[MAX_E];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t smem0 = smem_u32(smem);
+    volatile int *abort_flag = &abort_s;
+
+    // ---------------------------------------------------------- prologue
+    if (warp == 0) {
+        const int nt_r = (p.n_out_r + BN_OUT - 1) / BN_OUT;
+        int carry = 0;
+        for (int e0 = 0; e0 < p.E; e0 += 32) {
+            const int e = e0 + lane;
+            int lo = 0, cnt = 0;
+            if (e < p.E) {
+                lo = p.offsets[e];
+                cnt = p.offsets[e + 1] - lo;
+                if (lo < 0 || cnt < 0 || lo + cnt > p.rows_r) {
+                    record_status(p.status, MOE_ERR_DEVICE_FAULT);
+                    lo = 0;
+                    cnt = 0;
+                }
+                seg[e] = lo;
+                segc[e] = cnt;
+            }
+            const int v = ((cnt + C2_ROWS - 1) / C2_ROWS) * nt_r;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (e < p.E) tile_base[e] = carry + incl - v;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) {
+            tile_base[p.E] = carry;
+            tma_prefetch_desc(&maps.o_r);
+            tma_prefetch_desc(&maps.a_r);
+            tma_prefetch_desc(&maps.bpk);
+            if (p.T > 0) tma_prefetch_desc(&maps.a_s);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < C2_STAGES; ++s) {
+                mbar_init(smem_u32(&full_bar[s]), 1);
+                mbar_init(smem_u32(&empty_bar[s]), 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(smem_u32(&tfull_bar[b]), 1);
+                mbar_init(smem_u32(&tempty_bar[b]), 2 * 4);  // 4 epilogue warps per CTA
+            }
+            mbar_init(smem_u32(&done_bar), 1);
+            abort_s = 0;
+            fence_barrier_init();
+        }
+        __syncwarp();
+        tmem_alloc_pair<TMEM_COLS>(smem_u32(&tmem_base_s));
+        tc_fence_before();
+    }
+    __syncthreads();
+    // both CTAs' barriers are initialised and both TMEM allocations done
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_s;
+
+    const int ntr = tile_base[p.E];
+    const int mt_s = p.T > 0 ? (p.T + C2_ROWS - 1) / C2_ROWS : 0;
+    const int nt_s = p.T > 0 ? (p.n_out_s + BN_OUT - 1) / BN_OUT : 0;
+    const int total = ntr + mt_s * nt_s;
+    const int pair_id = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t n_issued = 0;
+            for (int idx = pair_id; idx < total; idx += n_pairs) {
+                const C2Tile t = decode_c2<EPI>(idx, tile_base, seg, segc, p, ntr, nt_s);
+                const int kb_total = t.e >= 0 ? p.k_r / BK : p.k_s / BK;
+                // first 128-byte row of this CTA's half of the (n, kb = 0) weight tile
+                const int64_t brow0 =
+                    (t.e >= 0 ? p.bpk_row_r + ((int64_t)t.e * p.bp_nt_r + t.n0 / BN_OUT) * kb_total * 256
+                              : p.bpk_row_s + (int64_t)(t.n0 / BN_OUT) * kb_total * 256) +
+                    rank * BM;
+                bool ok = true;
+                for (int kb = 0; kb < t.kblocks; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag,
+                                           p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                    const uint32_t a_dst = smem0 + stage * C2_STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + A_BYTES;
+                    if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[stage]), 2 * C2_STAGE_BYTES);
+                    const CUtensorMap *am = t.e >= 0 ? &maps.a_r : &maps.a_s;
+                    tma_load_2d_pair(a_dst, am, fb, kb * BK, t.row0 + (int)rank * BM);
+                    tma_load_2d_pair(b_dst, &maps.bpk, fb, 0, (int32_t)(brow0 + (int64_t)kb * 256));
+                    ++n_issued;
+                    if (++stage == C2_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            // wind down (leader): every load of both CTAs has landed
+            if (leader) {
+                for (int s = 0; s < C2_STAGES; ++s) {
+                    if (n_issued > (uint32_t)s) {
+                        const uint32_t uses = (n_issued - 1 - s) / C2_STAGES + 1;
+                        drain_wait(smem_u32(&full_bar[s]), (uses - 1) & 1u, p.timeout_ns, p.status);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            constexpr uint32_t idesc = idesc_bf16_f32<C2_ROWS, Cfg<EPI>::BN_MMA>();
+            for (int idx = pair_id; idx < total; idx += n_pairs) {
+                const C2Tile t = decode_c2<EPI>(idx, tile_base, seg, segc, p, ntr, nt_s);
+                if (!mbar_wait_bounded(smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, abort_flag,
+                                       p.status, p.timeout_ns))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN_ACC;
+                bool ok = true;
+                for (int kb = 0; kb < t.kblocks; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.status,
+                                           p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem0 + stage * C2_STAGE_BYTES;
+                    const uint64_t a_desc = smem_desc_sw128(a_addr);
+                    const uint64_t b_desc = smem_desc_sw128(a_addr + A_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < BK / 16; ++ks)
+                        tc_mma_bf16_pair(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks, idesc,
+                                         (kb | ks) != 0 ? 1u : 0u);
+                    tc_commit_pair_both(smem_u32(&empty_bar[stage]));
+                    if (++stage == C2_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit_pair_both(smem_u32(&tfull_bar[acc]));
+                if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+            }
+            // wind down: every MMA issued has completed (both CTAs' TMEM written)
+            tc_commit_pair(smem_u32(&done_bar));
+            drain_wait(smem_u32(&done_bar), 0, p.timeout_ns, p.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue (both CTAs)
+        // as in the one-CTA kernel, for this CTA's 128 rows of the pair tile
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t stage_buf0 = smem0 + C2_STAGES * C2_STAGE_BYTES + (warp - 2) * 2 * STORE_BUF;
+        int sb = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int idx = pair_id; idx < total; idx += n_pairs) {
+            const C2Tile t = decode_c2<EPI>(idx, tile_base, seg, segc, p, ntr, nt_s);
+            if (!mbar_wait_bounded(smem_u32(&tfull_bar[acc]), acc_phase, abort_flag, p.status,
+                                   p.timeout_ns))
+                break;
+            tc_fence_after();
+            const int rv = min(BM, t.rows_valid - (int)rank * BM);  // this CTA's valid rows
+            const int row0 = t.row0 + (int)rank * BM;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
+            const bool shared = t.e < 0;
+            const int n_out = shared ? p.n_out_s : p.n_out_r;
+            __nv_bfloat16 *orow = (shared ? p.out_s : p.out_r) + (size_t)(row0 + row) * n_out;
+            const CUtensorMap *omap = shared ? &maps.o_s : &maps.o_r;
+            const bool full = rv == BM;
+            const bool row_ok = row < rv;
+#pragma unroll 1
+            for (int c = 0; c < BN_OUT && rv > 0; c += 32) {
+                uint4 o[4];
+                if (EPI == EPI_SWIGLU) {
+                    uint32_t g[32], u[32];
+                    tmem_ld32(taddr + c, g);
+                    tmem_ld32(taddr + BN_ACC / 2 + c, u);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        o[v].x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
+                                             silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
+                        o[v].y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
+                                             silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
+                        o[v].z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
+                                             silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
+                        o[v].w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
+                                             silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
+                    }
+                } else {
+                    uint32_t r[32];
+                    tmem_ld32(taddr + c, r);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        o[v].x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                        o[v].y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                        o[v].z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                        o[v].w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                    }
+                }
+                if (t.n0 + c >= n_out) continue;     // whole chunk past the last column
+                if (full) {
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    const uint32_t buf = stage_buf0 + sb * STORE_BUF;
+                    uint4 *sp = reinterpret_cast<uint4 *>(smem + (buf - smem0)) + lane * 4;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) sp[v] = o[v];
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(omap, buf, t.n0 + c, row0 + q * 32);
+                        bulk_commit_group();
+                    }
+                    sb ^= 1;
+                } else if (row_ok) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + t.n0 + c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = o[v];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[acc]), 0));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+        if (lane == 0) bulk_wait_group_all();  // every staged store has landed
+        __syncwarp();
+    }
+
+    // ---------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    // the leader's MMAs into this CTA's TMEM and every load into this CTA's
+    // shared memory are done before either CTA frees TMEM or exits
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair<TMEM_COLS>(tmem_base);
+    }
+}
+
 // Bounded-wait self-test: one thread waits on a barrier that never completes.
 __global__ void bounded_wait_selftest_kernel(int32_t *status, int64_t timeout_ns) {
     __shared__ __align__(8) uint64_t bar;
@@ -1131,6 +1479,36 @@ cudaError_t launch_pair(const Maps &maps, const Params &p, cudaStream_t st) {
     if (err != cudaSuccess) return err;
     grouped_ffn_pair_kernel<EPI><<<sm_count(), P_THREADS, P_SMEM_DYN, st>>>(maps, p);
     count_launch();
+    return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_cta2(const Maps &maps, const Params &p, cudaStream_t st) {
+    auto kern = grouped_ffn_cta2_kernel<EPI>;
+    cudaError_t err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2_SMEM_DYN);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(C2_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C2_SMEM_DYN;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // one wave of pairs: as many clusters as fit at once, at most one CTA per SM
+    int pairs = sm_count() / 2;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    int fit = 0;
+    if (cudaOccupancyMaxActiveClusters(&fit, kern, &cfg) == cudaSuccess && fit > 0 && fit < pairs)
+        pairs = fit;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    err = cudaLaunchKernelEx(&cfg, kern, maps, p);
+    count_launch();
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
@@ -1219,9 +1597,18 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
         p1.bp_s = has_shared ? pk + PL.gu_s : nullptr;
         p1.bp_nt_r = PL.nt1;
     }
+    // the CTA-pair kernels read the packed weights through one 2-D map of 128-byte rows
+    const bool cta2 = MOE_GEMM_CTA2 && packed && !fp8 && !gather;
+    if (cta2) {
+        if (!tensor_map_2d_bf16(&m1.bpk, pk, PL.total / 128, BK, BK, BM, 0))
+            return cudaErrorInvalidValue;
+        p1.bpk_row_r = (int64_t)(PL.gu / 128);
+        p1.bpk_row_s = (int64_t)(PL.gu_s / 128);
+    }
     cudaError_t err = fp8      ? launch_one<EPI_SWIGLU, A_FP8>(m1, p1, st)
                       : gather ? launch_one<EPI_SWIGLU, A_GATHER>(m1, p1, st)
-                      : pair1 ? launch_pair<EPI_SWIGLU>(m1, p1, st)
+                      : cta2   ? launch_cta2<EPI_SWIGLU>(m1, p1, st)
+                      : pair1  ? launch_pair<EPI_SWIGLU>(m1, p1, st)
                                : launch_one<EPI_SWIGLU, A_TMA>(m1, p1, st);
     if (err != cudaSuccess) return err;
 
@@ -1259,6 +1646,12 @@ cudaError_t launch_expert_ffn(const FfnArgs &a, cudaStream_t st) {
         p2.bp_r = pk + PL.down;
         p2.bp_s = has_shared ? pk + PL.down_s : nullptr;
         p2.bp_nt_r = PL.nt2;
+    }
+    if (cta2) {
+        m2.bpk = m1.bpk;
+        p2.bpk_row_r = (int64_t)(PL.down / 128);
+        p2.bpk_row_s = (int64_t)(PL.down_s / 128);
+        return launch_cta2<EPI_STORE>(m2, p2, st);
     }
     return MOE_PAIR_GEMM2 ? launch_pair<EPI_STORE>(m2, p2, st)
                           : launch_one<EPI_STORE, A_TMA>(m2, p2, st);
