@@ -277,6 +277,17 @@ def test_expert_parallel_validates_before_cuda(moe):
     bad[9] = None                              # lcnt
     assert lib.moe_ep_combine_plan(c, 2, *bad, None, None) == INV
     assert lib.moe_ep_combine_plan(c, 3, *cp_args, None, None) == UNS
+    # dispatch + combine lists in one launch: x, topk_idx, topk_w, offsets, inv_perm, base,
+    # tok_slot, tok_base, recv_tok, recv_idx, list, lw, lcnt
+    dp_args = [P(fake)] * 13
+    for i in (2, 10, 12):                      # topk_w, list, lcnt
+        bad = list(dp_args)
+        bad[i] = None
+        assert lib.moe_ep_dispatch_dedup_plan(c, 2, *bad, None, None) == INV
+    bad = list(dp_args)
+    bad[0] = P(fake + 8)                       # misaligned x
+    assert lib.moe_ep_dispatch_dedup_plan(c, 2, *bad, None, None) == INV
+    assert lib.moe_ep_dispatch_dedup_plan(c, 3, *dp_args, None, None) == UNS
     pc_args = [P(fake)] * 6                    # recv_y, list, lw, lcnt, tok_base, partial
     bad = list(pc_args)
     bad[5] = P(fake + 8)                       # misaligned partial
