@@ -138,10 +138,17 @@ def test_packed_forward_equals_row_major(name):
     assert torch.equal(ref["out"].view(torch.int16), got["out"].view(torch.int16))
 
 
-@pytest.mark.parametrize("counts", [[0, 1, 127, 128, 129, 255, 256, 257, 1000, 7, 0, 0]])
+@pytest.mark.parametrize("counts", [
+    [0, 1, 127, 128, 129, 255, 256, 257, 1000, 7, 0, 0],
+    # >= 512 rows per expert on average: the paired-row-tile GEMMs, whose packed
+    # weight stages come from the same 32 KB blocks (full pairs, a 1-row second
+    # tile, trailing single tiles)
+    [0, 1, 129, 257, 384, 640, 1000, 1023, 1046, 1386, 1280, 1046],
+])
 def test_packed_expert_ffn_segment_edges(counts):
-    """Segments of 0/1/127/128/129/255/256/257/1000 rows: every row and the shared
-    rows of the packed FFN equal the row-major FFN's bits."""
+    """Segments of 0/1/127/128/129/255/256/257/1000 rows (and a set averaging
+    more than 512): every row and the shared rows of the packed FFN equal the
+    row-major FFN's bits."""
     sh = H.RAGGED.replace(T=sum(counts) // 4)
     assert sh.T * sh.K == sum(counts)
     offsets = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32, device=DEV)
