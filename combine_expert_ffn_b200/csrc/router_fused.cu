@@ -225,6 +225,7 @@ __device__ __forceinline__ void select_rows(const Params &p, const float *red, i
         const bool writer = valid && g == 0 && t < p.T && !aborted;
         uint64_t last = ~0ull;
         float denom = 0.f;
+        float sv[32];  // the picks' unbiased affinities, slot order (K <= 32)
         for (int r = 0; r < K; ++r) {
             uint64_t best = kept ? tree_best(kv, gsz, last) : 0ull;
             if (pow2) {  // the token's lanes are an aligned power of two
@@ -254,14 +255,13 @@ __device__ __forceinline__ void select_rows(const Params &p, const float *red, i
                 if (p.off) L += off_s[e];
                 const float bs = affinity_fn<KIND>(L);
                 p.topk_idx[(size_t)t * K + r] = e;
-                p.topk_w[(size_t)t * K + r] = bs;  // s for now; divided below
+                sv[r] = bs;
                 denom = __fadd_rn(denom, bs);
             }
         }
         // gates over the chosen unbiased affinities, in slot order
         if (writer) {
-            for (int r = 0; r < K; ++r)
-                p.topk_w[(size_t)t * K + r] = __fdiv_rn(p.topk_w[(size_t)t * K + r], denom);
+            for (int r = 0; r < K; ++r) p.topk_w[(size_t)t * K + r] = __fdiv_rn(sv[r], denom);
         }
     }
 }
