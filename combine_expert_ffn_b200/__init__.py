@@ -31,7 +31,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_WORKSPACE_TOO_SM
     MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_FAULT, MOE_ERR_NO_DEVICE = range(8)
 
 EXPORTS = ("moe_check_config", "moe_workspace_size", "moe_status_string", "moe_launch_count",
-           "moe_read_device_status", "moe_clear_device_status", "moe_route", "moe_route_select",
+           "moe_read_device_status", "moe_last_device_status", "moe_clear_device_status",
+           "moe_route", "moe_route_select",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_selftest_bounded_wait", "moe_dispatch_noalloc", "moe_route_hash",
            "moe_bias_update", "moe_expert_ffn_gather", "moe_dispatch_fp8",
@@ -84,6 +85,7 @@ _sig = {
     "moe_status_string": (C.c_char_p, [C.c_int]),
     "moe_launch_count": (C.c_uint64, []),
     "moe_read_device_status": (C.c_int, [_P, _P, _P]),
+    "moe_last_device_status": (C.c_int, [_P, _P]),
     "moe_clear_device_status": (C.c_int, [_P, _P]),
     "moe_route": (C.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_route_select": (C.c_int, [_CP, _P, _P, _P, _P, _P]),
@@ -195,6 +197,11 @@ def moe_read_device_status(ws, stream=None) -> int:
     out = C.c_int32(-1)
     _ok("moe_read_device_status", _lib.moe_read_device_status(_ptr(ws), C.byref(out), _stream(stream)))
     return out.value
+
+
+def moe_last_device_status(ws, stream=None) -> int:
+    """The device status word (synchronises the stream); host-side read errors as codes."""
+    return int(_lib.moe_last_device_status(_ptr(ws), _stream(stream)))
 
 
 def moe_clear_device_status(ws, stream=None) -> None:

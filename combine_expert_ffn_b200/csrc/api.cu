@@ -233,6 +233,12 @@ moe_status moe_read_device_status(const void *ws, int32_t *host_status, void *st
     return cuda_status(cudaStreamSynchronize(s));
 }
 
+moe_status moe_last_device_status(const void *ws, void *stream) {
+    int32_t word = MOE_OK;
+    const moe_status st = moe_read_device_status(ws, &word, stream);
+    return st != MOE_OK ? st : static_cast<moe_status>(word);
+}
+
 moe_status moe_clear_device_status(void *ws, void *stream) {
     if (!ws) return MOE_ERR_INVALID_ARG;
     moe_status st = check_device();

@@ -124,6 +124,11 @@ MOE_API uint64_t moe_launch_count(void);
  * recorded a fault since the last moe_clear_device_status(). */
 MOE_API moe_status moe_read_device_status(const void *ws, int32_t *host_status, void *stream);
 
+/* The same read, returning the device status word itself: MOE_OK, or the
+ * MOE_ERR_DEVICE_* code a kernel recorded; a host-side failure of the read
+ * (ws NULL, no device, a CUDA error) is returned in its place. */
+MOE_API moe_status moe_last_device_status(const void *ws, void *stream);
+
 /* Enqueues a reset of the workspace status word to MOE_OK. */
 MOE_API moe_status moe_clear_device_status(void *ws, void *stream);
 

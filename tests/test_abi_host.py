@@ -310,3 +310,5 @@ def test_expert_parallel_validates_before_cuda(moe):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a GPU")
 def test_no_device_is_reported(moe):
     assert moe._lib.moe_clear_device_status(C.c_void_p(1 << 20), None) == moe.MOE_ERR_NO_DEVICE
+    assert moe._lib.moe_last_device_status(C.c_void_p(1 << 20), None) == moe.MOE_ERR_NO_DEVICE
+    assert moe._lib.moe_last_device_status(None, None) == moe.MOE_ERR_INVALID_ARG

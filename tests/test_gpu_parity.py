@@ -65,8 +65,10 @@ def test_bounded_wait_times_out_and_context_survives():
     ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
     moe.moe_selftest_bounded_wait(5_000_000, ws)          # 5 ms limit
     assert moe.moe_read_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    assert moe.moe_last_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
     moe.moe_clear_device_status(ws)
     assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    assert moe.moe_last_device_status(ws) == moe.MOE_OK
     a = torch.arange(10, device=DEV)
     assert int((a * 2).sum()) == 90                        # context still usable
 
