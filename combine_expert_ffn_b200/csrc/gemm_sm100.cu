@@ -57,6 +57,12 @@
 #define MOE_GEMM_KB_GROUP 1
 #endif
 
+// One-CTA kernel: a tile with at most 64 valid rows issues M = 64 MMAs (1 on,
+// 0 off).  Its accumulator rows then sit in TMEM lanes (i % 16) + 32 (i / 16).
+#ifndef MOE_GEMM_TAIL64
+#define MOE_GEMM_TAIL64 1
+#endif
+
 // CTA-pair grouped GEMMs (tcgen05.mma.cta_group::2, packed weights only):
 // 0 never (default), 1 always when the weights are packed.  Bit-identical to
 // the one-CTA kernel, but not faster: measured +17 % at the V3 routing (256-row
@@ -418,6 +424,10 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN_ACC;
+                // a tail tile of at most 64 rows: M = 64 MMAs over the first 64 A rows
+                const uint32_t idesc = MOE_GEMM_TAIL64 && t.rows_valid <= BM / 2
+                                           ? idesc_bf16_f32<BM / 2, Cfg<EPI>::BN_MMA>()
+                                           : idesc_bf16_f32<BM, Cfg<EPI>::BN_MMA>();
                 bool ok = true;
                 for (int kb = 0; kb < t.kblocks; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.status,
@@ -432,8 +442,7 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                     const uint64_t b_desc = smem_desc_sw128(a_addr + A_BYTES);
 #pragma unroll
                     for (int ks = 0; ks < BK / 16; ++ks)
-                        tc_mma_bf16(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks,
-                                    idesc_bf16_f32<BM, Cfg<EPI>::BN_MMA>(),
+                        tc_mma_bf16(d_tmem, a_desc + 2 * ks, b_desc + 2 * ks, idesc,
                                     (kb | ks) != 0 ? 1u : 0u);
                     tc_commit(smem_u32(&empty_bar[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -589,7 +598,6 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
         // pieces.  Rows of a partial tile that belong to the next expert must
         // not be written, so partial tiles use masked direct stores.
         const int q = warp & 3;            // TMEM lane quarter this warp may access
-        const int row = q * 32 + lane;     // accumulator row = tile row
         const uint32_t stage_buf0 = smem0 + STAGES * STAGE_BYTES + (warp - 2) * 2 * STORE_BUF;
         int sb = 0;                        // staging buffer toggle
         int acc = 0;
@@ -601,12 +609,16 @@ grouped_ffn_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
                 break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN_ACC;
+            // accumulator row of this lane: lane of quarter q for M = 128; for an
+            // M = 64 tail tile lanes 0..15 of the quarter hold rows 16 q .. 16 q + 15
+            const bool m64 = MOE_GEMM_TAIL64 && t.rows_valid <= BM / 2;
+            const int row = m64 ? q * 16 + (lane & 15) : q * 32 + lane;
             const bool shared = t.e < 0;
             const int n_out = shared ? p.n_out_s : p.n_out_r;
             __nv_bfloat16 *orow = (shared ? p.out_s : p.out_r) + (size_t)(t.row0 + row) * n_out;
             const CUtensorMap *omap = shared ? &maps.o_s : &maps.o_r;
             const bool full = t.rows_valid == BM;
-            const bool row_ok = row < t.rows_valid;
+            const bool row_ok = (!m64 || lane < 16) && row < t.rows_valid;
 #pragma unroll 1
             for (int c = 0; c < BN_OUT; c += 32) {
                 uint4 o[4];
