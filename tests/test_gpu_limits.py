@@ -3,7 +3,8 @@
 Maximum routing sizes (E = 1024 experts, G = 64 groups, K = 32, M up to 32),
 no node limit (M = G), every expert chosen (K = E), the smallest batch
 (T = G), and many tiny expert segments.  Bars as in the main parity tests:
-selection and dispatch bit-exact, layer output within the output bars.
+selection and dispatch bit-exact, layer output within the output bars; the
+layers through the tile-packed weights bit-identical to the row-major ones.
 """
 import gc
 
@@ -115,6 +116,16 @@ def test_forward_degenerate_and_max_layers(orc, sh):
     assert frob <= H.TOL_FROB and elem <= H.TOL_ELEM, (frob, elem)
     if sh.K == sh.E:
         assert (np.sort(gi, axis=1) == np.arange(sh.E)).all()
+    # the tile-packed weights give the same layer bit for bit
+    packed = moe.pack_weights(cfg, inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                              inp.get("ws_up"), inp.get("ws_down"))
+    o2 = moe.forward_outputs(cfg)
+    moe.moe_forward_packed(cfg, inp["x"], inp["router_w"], None, inp["bias"], packed, o2["out"],
+                           o2["topk_idx"], o2["topk_w"], o2["counts"], o2["offsets"], o2["send"],
+                           o2["send_tok"], ws=ws)
+    assert moe.moe_read_device_status(ws) == moe.MOE_OK
+    assert torch.equal(o2["topk_idx"], o["topk_idx"])
+    assert torch.equal(o2["out"].view(torch.int16), o["out"].view(torch.int16))
 
 
 # Router work split over d (small batches): decode has 2 tiles and 28 k ranges;
