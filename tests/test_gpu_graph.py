@@ -3,7 +3,7 @@
 The forward only enqueues kernels on the caller's stream (no allocation, no
 synchronisation, no host read-back), so it can be captured once and replayed:
 the replay must give the eager forward's bits, also after the input buffer is
-refilled with another batch.
+refilled with another batch.  With row-major and with tile-packed weights.
 """
 import gc
 
@@ -30,18 +30,30 @@ def _free_gpu():
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name,router,payload", [("tiny", 0, 0), ("ragged2", 1, 0),
-                                                 ("noshared", 0, 1), ("mid", 2, 0)])
-def test_forward_replays_from_a_cuda_graph(name, router, payload):
-    sh = H.shape(name)
+@pytest.mark.parametrize("name,router,payload,packed", [
+    ("tiny", 0, 0, False), ("ragged2", 1, 0, False), ("noshared", 0, 1, False),
+    ("mid", 2, 0, False),
+    # the tile-packed weights; ragged at 2048 tokens averages 683 rows per expert, so
+    # its GEMMs are the paired-row-tile kernels whose tile counters a memset resets
+    ("tiny", 0, 0, True), ("mid", 0, 0, True), ("ragged_2048", 0, 0, True)])
+def test_forward_replays_from_a_cuda_graph(name, router, payload, packed):
+    sh = H.RAGGED.replace(name=name, T=2048) if name == "ragged_2048" else H.shape(name)
     inp = synth.make_inputs(sh, DEV)
     cfg = moe.MoeConfig.of(sh, router=router, payload=payload)
     ws = moe.alloc_workspace(cfg)
     o = moe.forward_outputs(cfg)
     ids = synth.token_ids(sh.seed, sh.T, device=DEV)
     x = inp["x"].clone()
+    pw = moe.pack_weights(cfg, inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
+                          inp.get("ws_up"), inp.get("ws_down")) if packed else None
 
     def forward(stream=None):
+        if packed:
+            moe.moe_forward_packed(cfg, x, inp["router_w"], inp.get("logit_offset"), inp["bias"],
+                                   pw, o["out"], o["topk_idx"], o["topk_w"], o["counts"],
+                                   o["offsets"], o["send"], o["send_tok"], ws=ws, stream=stream,
+                                   token_ids=ids)
+            return
         moe.moe_forward(cfg, x, inp["router_w"], inp.get("logit_offset"), inp["bias"],
                         inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("ws_gate"),
                         inp.get("ws_up"), inp.get("ws_down"), o["out"], o["topk_idx"],
