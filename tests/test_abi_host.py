@@ -124,6 +124,55 @@ def test_entry_points_validate_before_cuda(moe):
     assert lib.moe_selftest_bounded_wait(10, P(fake), None) == moe.MOE_ERR_INVALID_ARG
 
 
+def _packed_bytes(E, d, d_ff, n_shared, d_ff_shared):
+    """The packed layout's size, restated from its definition in moe.h: 32 KB
+    tiles of 256 weight rows x 64 k values; gate/up tiles hold 128 columns of
+    h, down tiles 256 output columns."""
+    up = lambda a, b: -(-a // b)  # noqa: E731
+    ffs = n_shared * d_ff_shared
+    tiles = E * up(d_ff, 128) * (d // 64) + E * up(d, 256) * (d_ff // 64)
+    if ffs:
+        tiles += up(ffs, 128) * (d // 64) + up(d, 256) * (ffs // 64)
+    return tiles * 32768
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged2", "noshared", "mid", "v3"])
+def test_packed_weights_size_and_validation(moe, name):
+    sh = H.shape(name)
+    cfg = moe.MoeConfig.of(sh)
+    assert moe.moe_packed_weights_size(cfg) == _packed_bytes(sh.E, sh.d, sh.d_ff, sh.n_shared,
+                                                             sh.d_ff_shared)
+    assert moe.moe_packed_weights_size(moe.MoeConfig.of(sh.replace(E=sh.E + 1))) == 0
+    lib, fake, P = moe._lib, 1 << 20, C.c_void_p
+    c = C.byref(cfg)
+    INV, UNS = moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_UNSUPPORTED_SHAPE
+    w = [P(fake)] * 6                                  # w_gate .. ws_down
+    assert lib.moe_pack_weights(c, *w, None, None) == INV               # packed
+    bad = list(w)
+    bad[1] = P(fake + 8)                               # misaligned w_up
+    assert lib.moe_pack_weights(c, *bad, P(fake), None) == INV
+    if sh.n_shared:
+        bad = list(w)
+        bad[3] = None                                  # ws_gate
+        assert lib.moe_pack_weights(c, *bad, P(fake), None) == INV
+    ws_n = moe.moe_workspace_size(cfg)
+    # x_perm, offsets, packed, y_perm, x, y_shared
+    f = [P(fake)] * 6
+    assert lib.moe_expert_ffn_packed(c, *f, P(fake), ws_n - 1, None) == \
+        moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    bad = list(f)
+    bad[2] = None                                      # packed
+    assert lib.moe_expert_ffn_packed(c, *bad, P(fake), ws_n, None) == INV
+    assert lib.moe_expert_ffn_packed(c, *f, P(fake + 64), ws_n, None) == INV   # ws alignment
+    # x, router_w, logit_offset, bias, token_ids, packed, out, then 6 optional outputs
+    fw = [P(fake), P(fake), None, None, None, None, P(fake)] + [None] * 6
+    assert lib.moe_forward_packed(c, *fw, P(fake), ws_n, None) == INV          # packed
+    fw[5] = P(fake)
+    fp8 = moe.MoeConfig.of(sh, payload=moe.MOE_PAYLOAD_FP8)
+    if moe.moe_check_config(fp8) == moe.MOE_OK:
+        assert lib.moe_forward_packed(C.byref(fp8), *fw, P(fake), ws_n, None) == UNS
+
+
 def test_fused_gather_validates_before_cuda(moe):
     cfg = moe.MoeConfig.of(synth.config("tiny"))
     ws_n = moe.moe_workspace_size(cfg)
